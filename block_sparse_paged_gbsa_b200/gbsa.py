@@ -1,0 +1,296 @@
+"""Python binding of libgbsa (argument marshalling only).
+
+Every step of the computation runs in the CUDA kernels behind the C ABI
+declared in ``include/gbsa.h``; this module checks tensor shapes, strides and
+devices, fills the C structs and calls the library on the current CUDA
+stream.  There is no fallback: if ``libgbsa.so`` is missing or no CUDA device
+is present the calls raise.
+
+Function and argument names follow the PyTorch interface of the
+GenericBlockSparseAttention article (cf-1.com/news/4865651), "Calling /
+PyTorch API": ``generic_block_sparse_attention_metadata(sparse_block_idx,
+sparse_block_count, num_heads_q, num_heads_kv, head_dim, block_shape, *,
+cu_seqlens_q, seqused_q, seqused_kv, ...)`` and
+``generic_block_sparse_attention(q, k, v, sparse_block_idx,
+sparse_block_count, block_shape, *, metadata, cu_seqlens_q, seqused_q,
+seqused_kv, block_table, softmax_scale, mask_mode, win_left, win_right,
+return_softmax_lse, ...) -> (attention_out, softmax_lse)``.  The quantisation,
+attention-mask and raw-KV arguments of that interface are not offered: the
+article marks those modes unsupported.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+import threading
+from typing import Optional, Sequence
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_NAME = "libgbsa.so"
+_lock = threading.Lock()
+_lib = None
+
+STATUS_NAMES = {0: "GBSA_OK", 1: "GBSA_ERR_INVALID_ARG", 2: "GBSA_ERR_UNSUPPORTED",
+                3: "GBSA_ERR_SHAPE", 4: "GBSA_ERR_ALIGNMENT", 5: "GBSA_ERR_WORKSPACE_TOO_SMALL",
+                6: "GBSA_ERR_METADATA_TOO_SMALL", 7: "GBSA_ERR_CUDA", 8: "GBSA_ERR_NO_DEVICE"}
+
+DEV_BITS = {0x01: "BAD_SEQLEN", 0x02: "BAD_BLOCK_IDX", 0x04: "BAD_COUNT", 0x08: "BAD_PAGE",
+            0x10: "META_MISMATCH", 0x20: "TIMEOUT", 0x40: "CAPACITY"}
+
+
+class GbsaError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS_NAMES.get(status, status)}")
+
+
+class _Problem(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("T", ctypes.c_int32), ("N1", ctypes.c_int32),
+                ("N2", ctypes.c_int32), ("D", ctypes.c_int32), ("block_x", ctypes.c_int32),
+                ("block_y", ctypes.c_int32), ("total_q_blocks", ctypes.c_int32),
+                ("top_k", ctypes.c_int32), ("max_pages_per_seq", ctypes.c_int32),
+                ("num_pages", ctypes.c_int32), ("kv_page_stride", ctypes.c_int64),
+                ("scale", ctypes.c_double), ("mask_mode", ctypes.c_int32),
+                ("win_left", ctypes.c_int32), ("win_right", ctypes.c_int32),
+                ("is_packed_gqa", ctypes.c_int32), ("return_lse", ctypes.c_int32),
+                ("has_seqused_q", ctypes.c_int32), ("num_ctas", ctypes.c_int32),
+                ("max_blocks_per_split", ctypes.c_int32)]
+
+
+class _Tensors(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("q", "k", "v", "sparse_idx", "sparse_count", "cu_seqlens_q", "seqused_q",
+                 "seqused_kv", "block_table", "out", "lse")]
+
+
+@dataclasses.dataclass
+class Problem:
+    """Host-known description of one call (mirrors ``gbsa_problem``)."""
+    B: int
+    T: int
+    N1: int
+    N2: int
+    D: int
+    block_x: int
+    total_q_blocks: int
+    top_k: int
+    max_pages_per_seq: int = 1
+    num_pages: int = 1
+    kv_page_stride: int = 0
+    scale: float = 0.0
+    mask_mode: int = 1
+    win_left: int = -1
+    win_right: int = -1
+    is_packed_gqa: int = 1
+    return_lse: int = 0
+    has_seqused_q: int = 0
+    num_ctas: int = 0
+    max_blocks_per_split: int = 0
+    block_y: int = 128
+
+    def as_c(self) -> _Problem:
+        p = _Problem()
+        for f, _ in _Problem._fields_:
+            setattr(p, f, getattr(self, f))
+        return p
+
+
+def library_path() -> str:
+    return os.path.join(_HERE, _LIB_NAME)
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        path = library_path()
+        if not os.path.exists(path):
+            raise RuntimeError(f"{path} is missing: build it with "
+                               "`python -m block_sparse_paged_gbsa_b200.build`")
+        lib = ctypes.CDLL(path)
+        P, Tn, vp, sz = ctypes.POINTER(_Problem), ctypes.POINTER(_Tensors), ctypes.c_void_p, ctypes.c_size_t
+        lib.gbsa_abi_version.restype = ctypes.c_int32
+        lib.gbsa_status_string.argtypes = [ctypes.c_int]
+        lib.gbsa_status_string.restype = ctypes.c_char_p
+        lib.gbsa_metadata_size.argtypes = [P, ctypes.POINTER(sz)]
+        lib.gbsa_metadata_size.restype = ctypes.c_int
+        lib.gbsa_workspace_size.argtypes = [P, ctypes.POINTER(sz)]
+        lib.gbsa_workspace_size.restype = ctypes.c_int
+        lib.gbsa_metadata.argtypes = [P, Tn, vp, sz, vp, vp]
+        lib.gbsa_metadata.restype = ctypes.c_int
+        lib.gbsa_forward.argtypes = [P, Tn, vp, vp, sz, vp, vp]
+        lib.gbsa_forward.restype = ctypes.c_int
+        if lib.gbsa_abi_version() != 1:
+            raise RuntimeError("libgbsa ABI version mismatch")
+        _lib = lib
+        return lib
+
+
+def lib():
+    """The loaded ctypes library (raises if missing)."""
+    return _load()
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        raise GbsaError(status, what)
+
+
+def metadata_size(problem: Problem) -> int:
+    n = ctypes.c_size_t(0)
+    _check(_load().gbsa_metadata_size(ctypes.byref(problem.as_c()), ctypes.byref(n)),
+           "gbsa_metadata_size")
+    return int(n.value)
+
+
+def workspace_size(problem: Problem) -> int:
+    n = ctypes.c_size_t(0)
+    _check(_load().gbsa_workspace_size(ctypes.byref(problem.as_c()), ctypes.byref(n)),
+           "gbsa_workspace_size")
+    return int(n.value)
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream_handle():
+    import torch
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _need(t, name, dtype, ndim, device=None):
+    import torch
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if not isinstance(t, torch.Tensor) or t.dtype != dtype or t.dim() != ndim:
+        raise ValueError(f"{name}: expected a {ndim}-d {dtype} tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name}: must be a CUDA tensor")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name}: on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous (no silent copies)")
+    return t
+
+
+def _block_shape(block_shape: Sequence[int]):
+    bx, by = (int(x) for x in block_shape)
+    return bx, by
+
+
+def metadata(sparse_block_idx, sparse_block_count, num_heads_q: int, num_heads_kv: int,
+             head_dim: int, block_shape: Sequence[int], *, cu_seqlens_q, seqused_kv,
+             seqused_q=None, num_tokens: int = 0, is_packed_gqa: bool = True, mask_mode: int = 1,
+             win_left: int = -1, win_right: int = -1, num_ctas: int = 0,
+             max_blocks_per_split: int = 0, dev_status=None):
+    """Builds the work list (int32 tensor) on the device of the inputs.
+
+    num_tokens: T if known (enables the device check cu_seqlens_q[B] == T); 0 skips it.
+    """
+    import torch
+    idx = _need(sparse_block_idx, "sparse_block_idx", torch.int32, 3)
+    dev = idx.device
+    cnt = _need(sparse_block_count, "sparse_block_count", torch.int32, 2, dev)
+    cu = _need(cu_seqlens_q, "cu_seqlens_q", torch.int64, 1, dev)
+    sku = _need(seqused_kv, "seqused_kv", torch.int32, 1, dev)
+    squ = None if seqused_q is None else _need(seqused_q, "seqused_q", torch.int32, 1, dev)
+    bx, by = _block_shape(block_shape)
+    N2, tqb, top_k = idx.shape
+    if num_heads_kv != N2 or tuple(cnt.shape) != (N2, tqb):
+        raise ValueError("sparse_block_idx / sparse_block_count shapes disagree with num_heads_kv")
+    prob = Problem(B=cu.shape[0] - 1, T=int(num_tokens), N1=num_heads_q, N2=num_heads_kv,
+                   D=head_dim, block_x=bx, block_y=by, total_q_blocks=tqb, top_k=top_k,
+                   mask_mode=mask_mode, win_left=win_left, win_right=win_right,
+                   is_packed_gqa=int(bool(is_packed_gqa)), has_seqused_q=int(squ is not None),
+                   num_ctas=num_ctas, max_blocks_per_split=max_blocks_per_split)
+    nbytes = metadata_size(prob)
+    with torch.cuda.device(dev):
+        meta = torch.empty((nbytes // 4,), dtype=torch.int32, device=dev)
+        ten = _Tensors(sparse_idx=_ptr(idx), sparse_count=_ptr(cnt), cu_seqlens_q=_ptr(cu),
+                       seqused_q=_ptr(squ), seqused_kv=_ptr(sku))
+        _check(_load().gbsa_metadata(ctypes.byref(prob.as_c()), ctypes.byref(ten),
+                                     meta.data_ptr(), nbytes, _ptr(dev_status), _stream_handle()),
+               "gbsa_metadata")
+    return meta
+
+
+def make_problem(q, k, sparse_block_idx, block_shape, block_table, cu_seqlens_q, *,
+                 softmax_scale=0.0, mask_mode=1, win_left=-1, win_right=-1, is_packed_gqa=True,
+                 return_softmax_lse=False, has_seqused_q=False, num_ctas=0,
+                 max_blocks_per_split=0) -> Problem:
+    """The gbsa_problem a forward call with these tensors describes."""
+    T, N1, D = q.shape
+    num_pages, page, N2, Dk = k.shape
+    N2i, tqb, top_k = sparse_block_idx.shape
+    bx, by = _block_shape(block_shape)
+    return Problem(B=cu_seqlens_q.shape[0] - 1, T=T, N1=N1, N2=N2, D=D, block_x=bx, block_y=by,
+                   total_q_blocks=tqb, top_k=top_k, max_pages_per_seq=block_table.shape[1],
+                   num_pages=num_pages, kv_page_stride=k.stride(0), scale=float(softmax_scale),
+                   mask_mode=mask_mode, win_left=win_left, win_right=win_right,
+                   is_packed_gqa=int(bool(is_packed_gqa)), return_lse=int(bool(return_softmax_lse)),
+                   has_seqused_q=int(bool(has_seqused_q)), num_ctas=num_ctas,
+                   max_blocks_per_split=max_blocks_per_split)
+
+
+def forward(q, k, v, sparse_block_idx, sparse_block_count, block_shape: Sequence[int], *,
+            metadata, cu_seqlens_q, seqused_kv, block_table, seqused_q=None,
+            softmax_scale: float = 0.0, mask_mode: int = 1, win_left: int = -1,
+            win_right: int = -1, is_packed_gqa: bool = True, return_softmax_lse: bool = False,
+            num_ctas: int = 0, max_blocks_per_split: int = 0, out=None, lse=None, workspace=None,
+            dev_status=None):
+    """Block-sparse paged GQA attention.  Returns (out [T,N1,D] bf16,
+    lse [T,N1,1] fp32 -- an empty tensor unless return_softmax_lse)."""
+    import torch
+    q = _need(q, "q", torch.bfloat16, 3)
+    dev = q.device
+    if k is None or v is None or k.dim() != 4 or v.dim() != 4:
+        raise ValueError("k, v: expected [num_pages, 128, N2, D] tensors")
+    for name, t in (("k", k), ("v", v)):
+        if t.dtype != torch.bfloat16 or t.device != dev:
+            raise ValueError(f"{name}: expected bf16 on {dev}")
+        _, page, n2, d = t.shape
+        if t.stride()[1:] != (n2 * d, d, 1):
+            raise ValueError(f"{name}: only dim0 (the page axis) may be strided")
+    if k.shape != v.shape or k.stride() != v.stride():
+        raise ValueError("k and v must have the same shape and strides")
+    idx = _need(sparse_block_idx, "sparse_block_idx", torch.int32, 3, dev)
+    cnt = _need(sparse_block_count, "sparse_block_count", torch.int32, 2, dev)
+    cu = _need(cu_seqlens_q, "cu_seqlens_q", torch.int64, 1, dev)
+    sku = _need(seqused_kv, "seqused_kv", torch.int32, 1, dev)
+    bt = _need(block_table, "block_table", torch.int32, 2, dev)
+    squ = None if seqused_q is None else _need(seqused_q, "seqused_q", torch.int32, 1, dev)
+    meta = _need(metadata, "metadata", torch.int32, 1, dev)
+    prob = make_problem(q, k, idx, block_shape, bt, cu, softmax_scale=softmax_scale,
+                        mask_mode=mask_mode, win_left=win_left, win_right=win_right,
+                        is_packed_gqa=is_packed_gqa, return_softmax_lse=return_softmax_lse,
+                        has_seqused_q=squ is not None, num_ctas=num_ctas,
+                        max_blocks_per_split=max_blocks_per_split)
+    T, N1, D = q.shape
+    with torch.cuda.device(dev):
+        if out is None:
+            out = torch.empty_like(q)
+        if return_softmax_lse:
+            if lse is None:
+                lse = torch.empty((T, N1, 1), dtype=torch.float32, device=dev)
+        else:
+            lse = torch.empty((0,), dtype=torch.float32, device=dev)
+        ws_bytes = workspace_size(prob)
+        if workspace is None:
+            workspace = torch.empty((max(ws_bytes, 16),), dtype=torch.uint8, device=dev)
+        ten = _Tensors(q=_ptr(q), k=_ptr(k), v=_ptr(v), sparse_idx=_ptr(idx),
+                       sparse_count=_ptr(cnt), cu_seqlens_q=_ptr(cu), seqused_q=_ptr(squ),
+                       seqused_kv=_ptr(sku), block_table=_ptr(bt), out=_ptr(out),
+                       lse=_ptr(lse) if return_softmax_lse else None)
+        _check(_load().gbsa_forward(ctypes.byref(prob.as_c()), ctypes.byref(ten),
+                                    meta.data_ptr(), workspace.data_ptr(),
+                                    workspace.numel() * workspace.element_size(),
+                                    _ptr(dev_status), _stream_handle()),
+               "gbsa_forward")
+    return out, lse
+
+
+def decode_dev_status(word: int) -> list:
+    return [name for bit, name in DEV_BITS.items() if word & bit]

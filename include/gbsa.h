@@ -1,0 +1,165 @@
+/*
+ * gbsa.h -- C ABI of libgbsa: block-sparse flash attention over a paged KV
+ * cache with grouped-query heads (forward pass), for NVIDIA B200 (sm_100a).
+ *
+ * Source of the operation: the GenericBlockSparseAttention article
+ * (cf-1.com/news/4865651, "GBSA article" below) and the FlashAttention blog
+ * post on CANN ops-transformer (ai6s.net, "FA blog" below).
+ *
+ *   out = Softmax(scale * Q * K_sparse^T + mask) * V_sparse
+ *       (GBSA article, "Function / sparse attention mechanism", the formula)
+ *
+ * Q is cut into blocks of block_x query tokens; every Q block, per KV head,
+ * attends only to the sparse_count[kvh][qb] KV blocks listed in
+ * sparse_idx[kvh][qb][0:top_k].  A KV block is one 128-token page of the
+ * paged K/V pool, found through block_table (layout PA_BBND).  The scores are
+ * computed tile by tile with an online softmax (FA blog, "three steps"), so
+ * the score matrix never exists; the log-sum-exp can be written out.
+ *
+ * Two-phase use, as in the GBSA article ("two-phase call: metadata first"):
+ *   1. gbsa_metadata()  builds the load-balanced work list on the device;
+ *   2. gbsa_forward()   runs the attention from that work list.
+ * The metadata must be rebuilt for every call whose index/count/length
+ * tensors change, with the same problem description as the forward call.
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the
+ *     library allocates no device memory, never synchronises the stream and
+ *     never reads device values on the host.  Work is enqueued on `stream`
+ *     (a cudaStream_t passed as void*; NULL = the legacy default stream).
+ *   - Host-detectable rule violations return a non-zero gbsa_status before
+ *     anything is launched.  Values inside device tensors are not checked on
+ *     the host (GBSA article, "Constraints": tiling does not check values);
+ *     when `dev_status` is non-NULL the kernels OR GBSA_DEV_* bits into that
+ *     device int32 instead (and skip the offending work; they never trap).
+ *   - Layouts (GBSA article, "Parameters" and the aclnn example call):
+ *       q            [T, N1, D]                 bf16, contiguous   (TND)
+ *       k, v         [num_pages, 128, N2, D]    bf16; only dim0 may be
+ *                    strided: stride0 = kv_page_stride elements  (PA_BBND)
+ *       sparse_idx   [N2, total_q_blocks, top_k] int32, contiguous
+ *       sparse_count [N2, total_q_blocks]        int32, contiguous
+ *       cu_seqlens_q [B+1]                       int64 prefix sums of the
+ *                                                Q storage lengths
+ *       seqused_q    [B] int32 (optional), seqused_kv [B] int32 (required)
+ *       block_table  [B, max_pages_per_seq]      int32 logical->physical page
+ *       out          [T, N1, D] bf16;  lse [T, N1] fp32 (natural log)
+ */
+#ifndef GBSA_H
+#define GBSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define GBSA_ABI_VERSION 1
+
+/* Return codes.  The GBSA article's return-code table did not survive
+ * extraction; these are this library's own. */
+typedef enum gbsa_status {
+  GBSA_OK = 0,
+  GBSA_ERR_INVALID_ARG = 1,         /* NULL pointer, negative size, bad enum value     */
+  GBSA_ERR_UNSUPPORTED = 2,         /* a mode the article lists as unsupported         */
+  GBSA_ERR_SHAPE = 3,               /* a dimension rule of "Constraints" is violated   */
+  GBSA_ERR_ALIGNMENT = 4,           /* a pointer or stride is not 16-byte aligned      */
+  GBSA_ERR_WORKSPACE_TOO_SMALL = 5, /* workspace smaller than gbsa_workspace_size()    */
+  GBSA_ERR_METADATA_TOO_SMALL = 6,  /* metadata smaller than gbsa_metadata_size()      */
+  GBSA_ERR_CUDA = 7,                /* a CUDA runtime/driver call failed               */
+  GBSA_ERR_NO_DEVICE = 8            /* num_ctas = 0 needs a device, and none is usable */
+} gbsa_status;
+
+/* Bits OR-ed into *dev_status by the kernels (device-side validation). */
+#define GBSA_DEV_BAD_SEQLEN 0x01      /* cu_seqlens_q not monotone / not ending at T, seqused_q > storage,
+                                         seqused_kv < 0, or the Q blocks do not add up to total_q_blocks */
+#define GBSA_DEV_BAD_BLOCK_IDX 0x02   /* a listed KV block lies outside [0, ceil(seqused_kv/128)); skipped */
+#define GBSA_DEV_BAD_COUNT 0x04       /* sparse_count outside [0, top_k]; clamped                       */
+#define GBSA_DEV_BAD_PAGE 0x08        /* block_table entry outside [0, num_pages); the page reads as 0  */
+#define GBSA_DEV_META_MISMATCH 0x10   /* metadata built for another problem; forward did nothing         */
+#define GBSA_DEV_TIMEOUT 0x20         /* a pipeline wait gave up (about 1 s); results are not valid       */
+#define GBSA_DEV_CAPACITY 0x40        /* a work-list capacity bound was exceeded; forward did nothing    */
+
+/* Host-known description of one call.  No field is read from the device.
+ * Field names follow the GBSA article's aclnn and PyTorch signatures
+ * ("Calling / aclnn API", "Calling / PyTorch API"). */
+typedef struct gbsa_problem {
+  int32_t B;                  /* number of sequences (batch)                                  */
+  int32_t T;                  /* total query tokens = cu_seqlens_q[B]                         */
+  int32_t N1;                 /* query heads                                                  */
+  int32_t N2;                 /* key/value heads; N1 % N2 == 0, N1/N2 <= 128                  */
+  int32_t D;                  /* head dim; only 128 ("Constraints: dimension")                */
+  int32_t block_x;            /* blockShapeX: query tokens per Q block, >= 1                  */
+  int32_t block_y;            /* blockShapeY: keys per KV block; must equal the page size 128 */
+  int32_t total_q_blocks;     /* sum_b ceil(storage_len_b / block_x)                          */
+  int32_t top_k;              /* last dim of sparse_idx; 1..256                               */
+  int32_t max_pages_per_seq;  /* second dim of block_table                                    */
+  int32_t num_pages;          /* first dim of the K/V pool                                    */
+  int64_t kv_page_stride;     /* elements between pages; >= 128*N2*D and % (N2*D) == 0        */
+  double scale;               /* scale_value; 0.0 selects 1/sqrt(D)                           */
+  int32_t mask_mode;          /* 1 = built-in causal (the only mode the article supports)    */
+  int32_t win_left;           /* -1 = unbounded; else keys >= pos - win_left are kept         */
+  int32_t win_right;          /* -1 = unbounded; else keys <= pos + win_right are kept        */
+  int32_t is_packed_gqa;      /* 1: the G heads of a group share each K/V tile (required)    */
+  int32_t return_lse;         /* 1: write lse                                                 */
+  int32_t has_seqused_q;      /* 1: seqused_q is given; 0: every Q storage token is used      */
+  int32_t num_ctas;           /* persistent CTAs of the forward; 0 = SM count of the device   */
+  int32_t max_blocks_per_split; /* 0 = automatic split-KV length; > 0 forces a smaller one     */
+} gbsa_problem;
+
+/* Device pointers of one call (caller-owned).  Unused optional pointers are NULL. */
+typedef struct gbsa_tensors {
+  const void* q;               /* bf16 [T, N1, D]                                 */
+  const void* k;               /* bf16 [num_pages, 128, N2, D], page stride above */
+  const void* v;               /* same layout and stride as k                     */
+  const int32_t* sparse_idx;   /* [N2, total_q_blocks, top_k]                     */
+  const int32_t* sparse_count; /* [N2, total_q_blocks]                            */
+  const int64_t* cu_seqlens_q; /* [B+1]                                           */
+  const int32_t* seqused_q;    /* [B] or NULL (has_seqused_q = 0)                 */
+  const int32_t* seqused_kv;   /* [B]                                             */
+  const int32_t* block_table;  /* [B, max_pages_per_seq]                          */
+  void* out;                   /* bf16 [T, N1, D]                                 */
+  float* lse;                  /* fp32 [T, N1] or NULL (return_lse = 0)           */
+} gbsa_tensors;
+
+/* Version of this header the library was built from (GBSA_ABI_VERSION). */
+int32_t gbsa_abi_version(void);
+
+/* Human-readable name of a status code; never NULL. */
+const char* gbsa_status_string(gbsa_status status);
+
+/* Bytes of metadata gbsa_metadata() writes for `problem` (a host-known bound:
+ * it does not depend on device values).  Validates `problem` first.
+ * GBSA article, "two-phase call": the metadata records the core split.
+ * Returns GBSA_ERR_NO_DEVICE if num_ctas == 0 and no device can be queried. */
+gbsa_status gbsa_metadata_size(const gbsa_problem* problem, size_t* bytes);
+
+/* Builds the work list for `problem` into the caller's device buffer `meta`
+ * (16-byte aligned, meta_bytes >= gbsa_metadata_size()).  Reads
+ * sparse_idx, sparse_count, cu_seqlens_q, seqused_q and seqused_kv; other
+ * tensor fields may be NULL.  Deterministic: equal inputs give equal bytes.
+ * GBSA article, "two-phase call" step 2 and "Constraints: metadata first". */
+gbsa_status gbsa_metadata(const gbsa_problem* problem, const gbsa_tensors* tensors,
+                          void* meta, size_t meta_bytes, int32_t* dev_status, void* stream);
+
+/* Bytes of scratch the forward needs for split-KV partial results
+ * (fp32 partial outputs and log-sum-exps); may be 0 only if splitting is
+ * impossible.  GBSA article, "aclnn API": first-phase workspace query. */
+gbsa_status gbsa_workspace_size(const gbsa_problem* problem, size_t* bytes);
+
+/* Runs the attention: out (and lse when return_lse) from q, k, v through the
+ * work list in `meta`.  `workspace` (16-byte aligned, ws_bytes >=
+ * gbsa_workspace_size()) is caller-owned scratch, overwritten.  If `meta`
+ * was built for a different problem the kernels set GBSA_DEV_META_MISMATCH
+ * and leave out/lse untouched.  Deterministic for a fixed num_ctas
+ * (GBSA article, "Constraints: determinism").  Rows past seqused_q, and rows
+ * with no visible key, get out = 0 and lse = -inf. */
+gbsa_status gbsa_forward(const gbsa_problem* problem, const gbsa_tensors* tensors,
+                         const void* meta, void* workspace, size_t ws_bytes,
+                         int32_t* dev_status, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GBSA_H */

@@ -1,0 +1,131 @@
+"""fp64 CPU oracle for block-sparse paged GQA attention (forward).
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this package.  It shares no code
+with the CUDA library: the arithmetic lives in ``gbsa_oracle.c`` (plain loops,
+fp64, a two-pass softmax over exactly the selected, unmasked keys), compiled
+here with gcc; ``scheduler.py`` is an independent sequential rebuild of the
+work-list format the metadata kernel writes.
+
+What the oracle computes is stated at the top of ``gbsa_oracle.c``; it follows
+the GenericBlockSparseAttention article (cf-1.com/news/4865651), "Function /
+sparse attention mechanism" and "Constraints", and the FlashAttention blog
+post on CANN ops-transformer (ai6s.net), "three steps" (the online softmax is
+exactly the two-pass softmax).  Pins: tests/test_oracle_pins.py.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "gbsa_oracle.c")
+_BUILD = os.path.join(_HERE, "_build")
+_LIB_PATH = os.path.join(_BUILD, "libgbsa_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compiles gbsa_oracle.c into _build/libgbsa_oracle.so (gcc, -O2)."""
+    os.makedirs(_BUILD, exist_ok=True)
+    stale = (not os.path.exists(_LIB_PATH)
+             or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC))
+    if force or stale:
+        compile_to(_SRC, _LIB_PATH)
+    return _LIB_PATH
+
+
+def compile_to(src: str, dst: str) -> str:
+    """Compiles an oracle C source file into a shared library at ``dst``."""
+    tmp = dst + f".{os.getpid()}.tmp"
+    # -ffp-contract=off keeps every product and sum a separately rounded fp64 op.
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fPIC", "-shared",
+                           "-pthread", src, "-o", tmp, "-lm"])
+    os.replace(tmp, dst)
+    return dst
+
+
+def load_library(path: str):
+    """Loads an oracle shared library and declares its entry point."""
+    lib = ctypes.CDLL(path)
+    f = lib.gbsa_oracle_attention_rows
+    i32, i64, dbl, ptr = ctypes.c_int32, ctypes.c_int64, ctypes.c_double, ctypes.c_void_p
+    f.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, i32, i32, i64, dbl, i32, i32,
+                  ptr, ptr, ptr, ptr, ptr, ptr, ptr, ptr, ptr, ptr, i64, ptr, ptr, i32]
+    f.restype = ctypes.c_int
+    return lib
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            _lib = load_library(build())
+    return _lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data
+
+
+def _as(a, dtype):
+    return None if a is None else np.ascontiguousarray(a, dtype=dtype)
+
+
+def default_threads() -> int:
+    return max(1, len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count())
+
+
+def attention_rows(*, q_bits, k_bits, v_bits, kv_page_stride, num_pages, sparse_idx, sparse_count,
+                   cu_seqlens_q, seqused_q, seqused_kv, block_table, block_x, scale,
+                   win_left=-1, win_right=-1, rows, n_threads=None, lib=None):
+    """Reference out/lse for selected (token, head) rows.
+
+    q_bits:  uint16 [T, N1, D] -- bf16 bit patterns of the queries.
+    k_bits, v_bits: flat uint16 arrays of the page pool; page ``p`` row ``r``
+             head ``h`` starts at ``p*kv_page_stride + (r*N2 + h)*D``.
+    rows:    int64 [n, 2] -- (global token index, query head).
+    Returns (out [n, D] float64, lse [n] float64).  Rows past seqused_q, or
+    with no visible key, give out = 0 and lse = -inf.
+    """
+    q_bits = _as(q_bits, np.uint16)
+    k_bits = _as(k_bits, np.uint16).reshape(-1)
+    v_bits = _as(v_bits, np.uint16).reshape(-1)
+    T, N1, D = q_bits.shape
+    sparse_idx = _as(sparse_idx, np.int32)
+    N2, tqb, top_k = sparse_idx.shape
+    sparse_count = _as(sparse_count, np.int32)
+    cu = _as(cu_seqlens_q, np.int64)
+    squ = _as(seqused_q, np.int32)
+    sku = _as(seqused_kv, np.int32)
+    bt = _as(block_table, np.int32)
+    B = cu.shape[0] - 1
+    need = (num_pages - 1) * kv_page_stride + 128 * N2 * D
+    if k_bits.size < need or v_bits.size < need:
+        raise ValueError("page pool arrays are shorter than num_pages pages")
+    rows = _as(rows, np.int64).reshape(-1, 2)
+    n = rows.shape[0]
+    out = np.zeros((n, D), np.float64)
+    lse = np.full((n,), -np.inf, np.float64)
+    rc = (lib or _load()).gbsa_oracle_attention_rows(
+        B, T, N1, N2, D, block_x, tqb, top_k, bt.shape[1], num_pages, kv_page_stride, float(scale),
+        win_left, win_right, _ptr(q_bits), _ptr(k_bits), _ptr(v_bits), _ptr(sparse_idx),
+        _ptr(sparse_count), _ptr(cu), _ptr(squ), _ptr(sku), _ptr(bt), _ptr(rows), n,
+        _ptr(out), _ptr(lse), n_threads or default_threads())
+    if rc != 0:
+        raise ValueError(f"oracle rejected the inputs (code {rc})")
+    return out, lse
+
+
+def attention(*, q_bits, rows=None, **kw):
+    """Reference out [T, N1, D] and lse [T, N1] (fp64) over every row."""
+    T, N1, D = np.asarray(q_bits).shape
+    tt, hh = np.meshgrid(np.arange(T), np.arange(N1), indexing="ij")
+    all_rows = np.stack([tt.reshape(-1), hh.reshape(-1)], axis=1)
+    out, lse = attention_rows(q_bits=q_bits, rows=all_rows, **kw)
+    return out.reshape(T, N1, D), lse.reshape(T, N1)

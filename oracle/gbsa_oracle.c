@@ -1,0 +1,246 @@
+/*
+ * gbsa_oracle.c -- plain fp64 CPU reference for block-sparse paged GQA
+ * attention (forward).  TEST INFRASTRUCTURE ONLY: the tests, the smoke check
+ * and the benchmark's CPU-baseline leg may call it; the product path never
+ * does.  It shares no code, header or constant with the CUDA library.
+ *
+ * What it computes, for each requested (global token row tg, query head h):
+ *
+ *   b      = the sequence holding tg          (cu_seqlens_q prefix sums)
+ *   t      = tg - cu_seqlens_q[b]             (token index inside b)
+ *   qs, qu = storage and used query length of b; ku = seqused_kv[b]
+ *   G      = N1 / N2, kvh = h / G             (grouped query heads)
+ *   qb     = (Q blocks of the sequences before b) + t / block_x
+ *   n      = sparse_count[kvh][qb] clamped to [0, top_k]
+ *   pos    = t + (ku - qu)                    (query position; bottom-right
+ *                                              aligned causal mask)
+ *   keys   = for every list entry j < n with lb = sparse_idx[kvh][qb][j]
+ *            inside [0, ceil(ku/128)): the positions p = 128*lb + r,
+ *            r in [0,128), that satisfy p < ku, p <= pos,
+ *            (win_left  < 0 or p >= pos - win_left),
+ *            (win_right < 0 or p <= pos + win_right);
+ *            position p is stored in physical page block_table[b][lb], row r.
+ *   s_p    = scale * sum_d q[tg][h][d] * k[page][r][kvh][d]
+ *   out    = sum_p exp(s_p - m) v_p / sum_p exp(s_p - m),  m = max_p s_p
+ *   lse    = m + ln(sum_p exp(s_p - m))
+ *   no key, or t >= qu:  out = 0, lse = -inf
+ *
+ * Sources: GBSA article (cf-1.com/news/4865651), "Function / sparse attention
+ * mechanism" (the formula, the block split along S, selection by
+ * sparseBlockIdx / sparseBlockCount from the paged cache); "Constraints"
+ * (Q blocks counted over storage lengths, seqused dual-length semantics,
+ * GQA N1 % N2 == 0, page size = blockShapeY = 128, PA_BBND stride rule);
+ * "Mask" (maskType 1 = built-in causal); "Return values" (lse shape).
+ * FA blog (ai6s.net), "three steps": the tiled online softmax is exactly
+ * equal to this two-pass softmax, which is why the reference uses the
+ * plain definition.  Readings where the pages are silent (head grouping
+ * kvh = h / G, bottom-right causal alignment, the window's inclusive bounds,
+ * logical block indices, duplicate entries counted twice, out-of-range
+ * entries ignored, empty rows -> 0 / -inf, natural-log lse) are listed in
+ * the design notes.
+ *
+ * Inputs are raw bf16 bit patterns (uint16); each is widened exactly to fp64.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_PAGE 128
+
+typedef struct {
+  int32_t B, T, N1, N2, D, block_x, total_q_blocks, top_k, max_pages_per_seq, num_pages;
+  int64_t kv_page_stride;
+  double scale;
+  int32_t win_left, win_right;
+  const uint16_t *q, *k, *v;
+  const int32_t *sparse_idx, *sparse_count;
+  const int64_t* cu_seqlens_q;
+  const int32_t *seqused_q, *seqused_kv, *block_table;
+  const int64_t* rows; /* pairs (tg, h) */
+  int64_t n_rows;
+  double *out, *lse;
+  int64_t* q_block_base; /* [B]: Q blocks of the sequences before b */
+  int failed;            /* set to a nonzero code by a worker on bad input */
+} oracle_ctx;
+
+static double widen_bf16(uint16_t bits) {
+  uint32_t u = ((uint32_t)bits) << 16;
+  float f;
+  memcpy(&f, &u, sizeof f);
+  return (double)f;
+}
+
+/* Largest b with cu_seqlens_q[b] <= tg (sequences may be empty). */
+static int32_t find_sequence(const oracle_ctx* c, int64_t tg) {
+  int32_t lo = 0, hi = c->B - 1;
+  while (lo < hi) {
+    int32_t mid = (lo + hi + 1) / 2;
+    if (c->cu_seqlens_q[mid] <= tg) lo = mid; else hi = mid - 1;
+  }
+  /* skip empty sequences that share the same start */
+  while (lo + 1 < c->B && c->cu_seqlens_q[lo + 1] <= tg) lo++;
+  return lo;
+}
+
+/* Computes one (tg, h) row; scratch holds room for top_k*128 keys. */
+static int one_row(const oracle_ctx* c, int64_t tg, int32_t h, double* out, double* lse,
+                   double* score, int64_t* key_page, int32_t* key_row) {
+  const int32_t D = c->D;
+  for (int32_t d = 0; d < D; d++) out[d] = 0.0;
+  *lse = -INFINITY;
+  if (tg < 0 || tg >= c->T || h < 0 || h >= c->N1) return 1;
+
+  const int32_t b = find_sequence(c, tg);
+  const int64_t t = tg - c->cu_seqlens_q[b];
+  const int64_t qs = c->cu_seqlens_q[b + 1] - c->cu_seqlens_q[b];
+  const int64_t qu = c->seqused_q ? (int64_t)c->seqused_q[b] : qs;
+  const int64_t ku = c->seqused_kv[b];
+  if (t >= qu) return 0; /* rows past seqused_q: out 0, lse -inf */
+
+  const int32_t G = c->N1 / c->N2;
+  const int32_t kvh = h / G;
+  const int64_t qb = c->q_block_base[b] + t / c->block_x;
+  if (qb < 0 || qb >= c->total_q_blocks) return 2;
+  int64_t n = c->sparse_count[(int64_t)kvh * c->total_q_blocks + qb];
+  if (n < 0) n = 0;
+  if (n > c->top_k) n = c->top_k;
+
+  const int64_t pos = t + (ku - qu);
+  const int64_t blocks_in_seq = (ku + ORACLE_PAGE - 1) / ORACLE_PAGE;
+  const int32_t* list = c->sparse_idx + ((int64_t)kvh * c->total_q_blocks + qb) * c->top_k;
+
+  /* Gather the visible keys, entry by entry, row by row. */
+  int64_t nk = 0;
+  for (int64_t j = 0; j < n; j++) {
+    const int64_t lb = list[j];
+    if (lb < 0 || lb >= blocks_in_seq) continue; /* out-of-range entries add nothing */
+    const int64_t page = c->block_table[(int64_t)b * c->max_pages_per_seq + lb];
+    if (page < 0 || page >= c->num_pages) return 3;
+    for (int32_t r = 0; r < ORACLE_PAGE; r++) {
+      const int64_t p = lb * ORACLE_PAGE + r;
+      if (p >= ku) continue;
+      if (p > pos) continue;
+      if (c->win_left >= 0 && p < pos - c->win_left) continue;
+      if (c->win_right >= 0 && p > pos + c->win_right) continue;
+      key_page[nk] = page;
+      key_row[nk] = r;
+      nk++;
+    }
+  }
+  if (nk == 0) return 0;
+
+  const uint16_t* qrow = c->q + (tg * c->N1 + h) * (int64_t)D;
+  for (int64_t i = 0; i < nk; i++) {
+    const uint16_t* krow =
+        c->k + key_page[i] * c->kv_page_stride + ((int64_t)key_row[i] * c->N2 + kvh) * D;
+    double dot = 0.0;
+    for (int32_t d = 0; d < D; d++) dot += widen_bf16(qrow[d]) * widen_bf16(krow[d]);
+    score[i] = c->scale * dot;
+  }
+
+  /* Two-pass softmax: the maximum first, then the normalised weights. */
+  double m = -INFINITY;
+  for (int64_t i = 0; i < nk; i++) if (score[i] > m) m = score[i];
+  double l = 0.0;
+  for (int64_t i = 0; i < nk; i++) l += exp(score[i] - m);
+  for (int64_t i = 0; i < nk; i++) {
+    const double w = exp(score[i] - m) / l;
+    const uint16_t* vrow =
+        c->v + key_page[i] * c->kv_page_stride + ((int64_t)key_row[i] * c->N2 + kvh) * D;
+    for (int32_t d = 0; d < D; d++) out[d] += w * widen_bf16(vrow[d]);
+  }
+  *lse = m + log(l);
+  return 0;
+}
+
+typedef struct {
+  oracle_ctx* c;
+  int64_t begin, end;
+} oracle_job;
+
+static void* run_job(void* arg) {
+  oracle_job* job = (oracle_job*)arg;
+  oracle_ctx* c = job->c;
+  const int64_t cap = (int64_t)c->top_k * ORACLE_PAGE;
+  double* score = (double*)malloc(sizeof(double) * (size_t)cap);
+  int64_t* key_page = (int64_t*)malloc(sizeof(int64_t) * (size_t)cap);
+  int32_t* key_row = (int32_t*)malloc(sizeof(int32_t) * (size_t)cap);
+  if (!score || !key_page || !key_row) {
+    c->failed = 4;
+  } else {
+    for (int64_t i = job->begin; i < job->end; i++) {
+      const int rc = one_row(c, c->rows[2 * i], (int32_t)c->rows[2 * i + 1], c->out + i * c->D,
+                             c->lse + i, score, key_page, key_row);
+      if (rc) c->failed = rc;
+    }
+  }
+  free(score);
+  free(key_page);
+  free(key_row);
+  return NULL;
+}
+
+/*
+ * Reference attention for n_rows (token, head) pairs given in `rows`
+ * ([n_rows][2] int64: global token index, query head).  Writes out
+ * [n_rows][D] and lse [n_rows] in fp64.  kv_page_stride is in elements.
+ * seqused_q may be NULL (every storage token used).  Returns 0 on success,
+ * nonzero if an argument or a device-style value is outside its range.
+ */
+int gbsa_oracle_attention_rows(int32_t B, int32_t T, int32_t N1, int32_t N2, int32_t D,
+                               int32_t block_x, int32_t total_q_blocks, int32_t top_k,
+                               int32_t max_pages_per_seq, int32_t num_pages,
+                               int64_t kv_page_stride, double scale, int32_t win_left,
+                               int32_t win_right, const uint16_t* q, const uint16_t* k,
+                               const uint16_t* v, const int32_t* sparse_idx,
+                               const int32_t* sparse_count, const int64_t* cu_seqlens_q,
+                               const int32_t* seqused_q, const int32_t* seqused_kv,
+                               const int32_t* block_table, const int64_t* rows, int64_t n_rows,
+                               double* out, double* lse, int32_t n_threads) {
+  if (B < 1 || T < 1 || N2 < 1 || N1 < N2 || N1 % N2 || D < 1 || block_x < 1 || top_k < 1 ||
+      total_q_blocks < 1 || max_pages_per_seq < 1 || num_pages < 1 || n_rows < 0)
+    return 10;
+  oracle_ctx c;
+  memset(&c, 0, sizeof c);
+  c.B = B; c.T = T; c.N1 = N1; c.N2 = N2; c.D = D; c.block_x = block_x;
+  c.total_q_blocks = total_q_blocks; c.top_k = top_k;
+  c.max_pages_per_seq = max_pages_per_seq; c.num_pages = num_pages;
+  c.kv_page_stride = kv_page_stride; c.scale = scale;
+  c.win_left = win_left; c.win_right = win_right;
+  c.q = q; c.k = k; c.v = v; c.sparse_idx = sparse_idx; c.sparse_count = sparse_count;
+  c.cu_seqlens_q = cu_seqlens_q; c.seqused_q = seqused_q; c.seqused_kv = seqused_kv;
+  c.block_table = block_table; c.rows = rows; c.n_rows = n_rows; c.out = out; c.lse = lse;
+
+  /* Q blocks are counted over storage lengths ("Constraints: block split"). */
+  c.q_block_base = (int64_t*)malloc(sizeof(int64_t) * (size_t)B);
+  if (!c.q_block_base) return 11;
+  int64_t acc = 0;
+  for (int32_t b = 0; b < B; b++) {
+    c.q_block_base[b] = acc;
+    const int64_t qs = cu_seqlens_q[b + 1] - cu_seqlens_q[b];
+    if (qs < 0) { free(c.q_block_base); return 12; }
+    acc += (qs + block_x - 1) / block_x;
+  }
+  if (acc != total_q_blocks || cu_seqlens_q[0] != 0 || cu_seqlens_q[B] != T) {
+    free(c.q_block_base);
+    return 13;
+  }
+
+  if (n_threads < 1) n_threads = 1;
+  if (n_threads > 256) n_threads = 256;
+  if (n_rows < n_threads) n_threads = n_rows > 0 ? (int32_t)n_rows : 1;
+  pthread_t tid[256];
+  oracle_job jobs[256];
+  for (int32_t i = 0; i < n_threads; i++) {
+    jobs[i].c = &c;
+    jobs[i].begin = n_rows * i / n_threads;
+    jobs[i].end = n_rows * (i + 1) / n_threads;
+  }
+  for (int32_t i = 1; i < n_threads; i++) pthread_create(&tid[i], NULL, run_job, &jobs[i]);
+  run_job(&jobs[0]);
+  for (int32_t i = 1; i < n_threads; i++) pthread_join(tid[i], NULL);
+  free(c.q_block_base);
+  return c.failed;
+}

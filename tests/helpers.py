@@ -1,0 +1,124 @@
+"""Shared test helpers: oracle calls on a Workload, an independent brute-force
+formulation used to pin the oracle, and tolerance checks."""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+import oracle
+from block_sparse_paged_gbsa_b200.workloads import PAGE, Workload, bf16_bits
+
+
+def oracle_rows(w: Workload, q, kf, vf, rows, n_threads=None, lib=None):
+    return oracle.attention_rows(
+        q_bits=bf16_bits(q), k_bits=bf16_bits(kf), v_bits=bf16_bits(vf),
+        kv_page_stride=w.kv_page_stride, num_pages=w.num_pages, sparse_idx=w.sparse_idx,
+        sparse_count=w.sparse_count, cu_seqlens_q=w.cu_seqlens_q, seqused_q=w.seqused_q,
+        seqused_kv=w.kv_used, block_table=w.block_table, block_x=w.block_x, scale=w.scale,
+        win_left=w.win_left, win_right=w.win_right, rows=rows, n_threads=n_threads, lib=lib)
+
+
+def oracle_all(w: Workload, q, kf, vf, n_threads=None, lib=None):
+    T, N1 = w.T, w.N1
+    tt, hh = np.meshgrid(np.arange(T), np.arange(N1), indexing="ij")
+    rows = np.stack([tt.reshape(-1), hh.reshape(-1)], axis=1)
+    out, lse = oracle_rows(w, q, kf, vf, rows, n_threads, lib=lib)
+    return out.reshape(T, N1, w.D), lse.reshape(T, N1)
+
+
+def to_f64(bits: np.ndarray) -> np.ndarray:
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def logical_kv(w: Workload, pool_bits: np.ndarray, b: int) -> np.ndarray:
+    """[ku, N2, D] fp64 keys (or values) of sequence b in logical order."""
+    ku = int(w.kv_used[b])
+    rows = []
+    for lb in range(-(-ku // PAGE)):
+        page = int(w.block_table[b, lb])
+        start = page * w.kv_page_stride
+        blk = pool_bits[start:start + PAGE * w.N2 * w.D].reshape(PAGE, w.N2, w.D)
+        rows.append(blk)
+    if not rows:
+        return np.zeros((0, w.N2, w.D))
+    return to_f64(np.concatenate(rows, 0)[:ku])
+
+
+def brute_force(w: Workload, q, kf, vf):
+    """A second formulation of the operator: for every (token, head) the
+    multiplicity of every logical key position is found by walking the block
+    list entry by entry, the masks are applied as a dense boolean vector, and
+    a dense fp64 softmax with those multiplicities as weights gives out/lse."""
+    qb_bits, kb, vb = bf16_bits(q), bf16_bits(kf), bf16_bits(vf)
+    qd = to_f64(qb_bits)
+    out = np.zeros((w.T, w.N1, w.D))
+    lse = np.full((w.T, w.N1), -np.inf)
+    G = w.N1 // w.N2
+    qbase = 0
+    for b in range(w.B):
+        qs = int(w.cu_seqlens_q[b + 1] - w.cu_seqlens_q[b])
+        qu = int(w.q_used[b]) if w.has_seqused_q else qs
+        ku = int(w.kv_used[b])
+        K = logical_kv(w, kb, b)
+        V = logical_kv(w, vb, b)
+        keys = np.arange(ku)
+        for t in range(qu):
+            tg = int(w.cu_seqlens_q[b]) + t
+            qb = qbase + t // w.block_x
+            pos = t + ku - qu
+            allowed = keys <= pos
+            if w.win_left >= 0:
+                allowed &= keys >= pos - w.win_left
+            if w.win_right >= 0:
+                allowed &= keys <= pos + w.win_right
+            for h in range(w.N1):
+                kvh = h // G
+                mult = np.zeros(ku)
+                n = min(max(int(w.sparse_count[kvh, qb]), 0), w.top_k)
+                for j in range(n):
+                    lb = int(w.sparse_idx[kvh, qb, j])
+                    if 0 <= lb < -(-ku // PAGE):
+                        mult[lb * PAGE:min(lb * PAGE + PAGE, ku)] += 1
+                wgt = mult * allowed
+                if wgt.sum() == 0:
+                    continue
+                s = w.scale * (K[:, kvh, :] @ qd[tg, h])
+                m = s[wgt > 0].max()
+                e = np.where(wgt > 0, wgt * np.exp(np.where(wgt > 0, s - m, 0.0)), 0.0)
+                out[tg, h] = e @ V[:, kvh, :] / e.sum()
+                lse[tg, h] = m + math.log(e.sum())
+        qbase += -(-qs // w.block_x)
+    return out, lse
+
+
+def bf16_half_ulp(x: np.ndarray) -> np.ndarray:
+    """Half the bf16 spacing at |x| (the representation error of an exact
+    value rounded to bf16)."""
+    a = np.abs(np.asarray(x, np.float64))
+    e = np.floor(np.log2(np.maximum(a, 2.0 ** -126)))
+    return 0.5 * 2.0 ** (e - 7)
+
+
+OUT_TOL = 1e-2     # max abs error on the bf16 output, on top of bf16 representation
+LSE_TOL = 1e-3     # max abs error on the fp32 lse
+
+
+def assert_out_close(gpu_out, ref_out, tol=OUT_TOL, what="out"):
+    g = np.asarray(gpu_out, np.float64)
+    r = np.asarray(ref_out, np.float64)
+    assert g.shape == r.shape, (g.shape, r.shape)
+    assert np.isfinite(g).all(), f"{what}: non-finite values"
+    err = np.abs(g - r) - bf16_half_ulp(r)
+    worst = float(err.max()) if err.size else 0.0
+    assert worst <= tol, f"{what}: max abs error {worst:.4g} beyond bf16 rounding > {tol}"
+
+
+def assert_lse_close(gpu_lse, ref_lse, tol=LSE_TOL):
+    g = np.asarray(gpu_lse, np.float64)
+    r = np.asarray(ref_lse, np.float64)
+    inf_r = np.isneginf(r)
+    assert np.array_equal(np.isneginf(g), inf_r), "lse: -inf pattern differs"
+    if (~inf_r).any():
+        worst = float(np.abs(g[~inf_r] - r[~inf_r]).max())
+        assert worst <= tol, f"lse: max abs error {worst:.4g} > {tol}"

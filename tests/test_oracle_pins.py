@@ -1,0 +1,313 @@
+"""Pins for the fp64 oracle: each test ties it to something other than itself
+(closed forms, hand-derived fixtures, a library routine, brute-force
+enumeration, invariants), so that a dropped term, a wrong sign or index, or a
+transposed operand in the oracle fails at least one of them."""
+import glob
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from block_sparse_paged_gbsa_b200.workloads import PAGE, bf16_bits, generate, make_values, workload
+from tests.helpers import brute_force, oracle_all, oracle_rows, to_f64
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# --------------------------------------------------------------------------
+# golden fixtures: hand-derived closed forms
+# --------------------------------------------------------------------------
+def _fixture_workload(fx):
+    p = fx["problem"]
+    w = generate(name="fixture", seed=5, q_storage=p["q_storage"], q_used=p["q_used"],
+                 kv_used=p["kv_used"], N1=p["N1"], N2=p["N2"], block_x=p["block_x"],
+                 top_k=p["top_k"], selection="random_causal", win_left=p["win_left"],
+                 win_right=p["win_right"], scale=p["scale"])
+    lists = fx["lists"]            # [N2][qb] -> list
+    for kvh, per_qb in enumerate(lists):
+        for qb, lst in enumerate(per_qb):
+            w.sparse_count[kvh, qb] = len(lst)
+            w.sparse_idx[kvh, qb, :len(lst)] = lst
+    q = torch.zeros((w.T, w.N1, w.D), dtype=torch.bfloat16)
+    kf = torch.zeros((w.pool_elems,), dtype=torch.bfloat16)
+    vf = torch.zeros((w.pool_elems,), dtype=torch.bfloat16)
+
+    def place(pool, p_log, kvh, d, val, b=0):
+        page = int(w.block_table[b, p_log // PAGE])
+        pool[page * w.kv_page_stride + ((p_log % PAGE) * w.N2 + kvh) * w.D + d] = val
+
+    for t, h, d, val in fx["q"]:
+        q[t, h, d] = val
+    for p_log, kvh, d, val in fx["k"]:
+        place(kf, p_log, kvh, d, val)
+    if fx["v"] == "ramp":
+        for p_log in range(int(w.kv_used[0])):
+            for kvh in range(w.N2):
+                place(vf, p_log, kvh, 0, float(p_log))
+    else:
+        for p_log, kvh, d, val in fx["v"]:
+            place(vf, p_log, kvh, d, val)
+    return w, q, kf, vf
+
+
+@pytest.mark.parametrize("path", sorted(p for p in glob.glob(os.path.join(GOLDEN, "*.json"))
+                                        if not p.endswith("example_call_shapes.json")))
+def test_golden_fixture(path):
+    fx = json.load(open(path))
+    w, q, kf, vf = _fixture_workload(fx)
+    rows = np.array([[e["t"], e["h"]] for e in fx["expected"]], np.int64)
+    out, lse = oracle_rows(w, q, kf, vf, rows)
+    for i, e in enumerate(fx["expected"]):
+        assert lse[i] == pytest.approx(e["lse"], abs=1e-12), (path, e)
+        for d, val in e["out"].items():
+            assert out[i, int(d)] == pytest.approx(val, abs=1e-12), (path, e, d)
+    # the brute-force formulation agrees on the same fixture
+    bo, bl = brute_force(w, q, kf, vf)
+    for i, e in enumerate(fx["expected"]):
+        assert bl[e["t"], e["h"]] == pytest.approx(e["lse"], abs=1e-12)
+
+
+def test_example_call_shapes():
+    """The pages' Python example: out has q's shape, lse is (T, N1, 1); its
+    randint(0, 2) indices repeat blocks and must be accepted."""
+    fx = json.load(open(os.path.join(GOLDEN, "example_call_shapes.json")))
+    p = fx["problem"]
+    rng = np.random.default_rng(0)
+    w = generate(name="example", seed=11, q_storage=[p["Q_S"]], q_used=[p["Q_S"]],
+                 kv_used=[p["KV_S"]], N1=p["N1"], N2=p["N2"], block_x=p["block_x"],
+                 top_k=p["top_k"], selection="random_any", extra_pages=0)
+    nb = fx["expected"]["num_blocks"]
+    assert w.total_q_blocks == fx["expected"]["total_q_blocks"]
+    assert w.num_pages == nb
+    w.block_table[0, :nb] = np.arange(nb)
+    w.sparse_idx[:] = rng.integers(0, nb, size=w.sparse_idx.shape)
+    w.sparse_count[:] = p["top_k"]
+    q, kf, vf = make_values(w, "cpu")
+    out, lse = oracle_all(w, q, kf, vf)
+    assert list(out.shape) == fx["expected"]["out_shape"]
+    assert list(lse[..., None].shape) == fx["expected"]["lse_shape"]
+    bo, bl = brute_force(w, q, kf, vf)
+    np.testing.assert_allclose(out, bo, atol=1e-12, rtol=0)
+    np.testing.assert_allclose(lse, bl, atol=1e-12, rtol=0)
+
+
+# --------------------------------------------------------------------------
+# brute-force enumeration on tiny random cases
+# --------------------------------------------------------------------------
+TINY_CASES = [
+    dict(q_storage=[200, 77], N1=4, N2=2, block_x=64, top_k=3, selection="random_causal"),
+    dict(q_storage=[300], N1=2, N2=1, block_x=16, top_k=4, selection="random_causal",
+         win_left=70, win_right=0),
+    dict(q_storage=[150, 260], q_used=[140, 200], kv_used=[170, 200], N1=4, N2=4,
+         block_x=32, top_k=3, selection="random_causal", page_stride_factor=1.5),
+    dict(q_storage=[1, 1, 1], q_used=[1, 1, 1], kv_used=[300, 5, 129], N1=4, N2=2,
+         block_x=1, top_k=4, selection="decode", count_range=(1, 4)),
+    dict(q_storage=[90, 130], N1=3, N2=1, block_x=7, top_k=5, selection="random_any"),
+    dict(q_storage=[256], q_used=[250], kv_used=[299], N1=2, N2=2, block_x=128, top_k=3,
+         selection="random_causal", win_left=5, win_right=3),
+]
+
+
+@pytest.mark.parametrize("case", range(len(TINY_CASES)))
+def test_brute_force_matches(case):
+    w = generate(name=f"tiny{case}", seed=100 + case, **TINY_CASES[case])
+    q, kf, vf = make_values(w, "cpu")
+    out, lse = oracle_all(w, q, kf, vf)
+    bo, bl = brute_force(w, q, kf, vf)
+    assert np.isfinite(out).all()
+    np.testing.assert_allclose(out, bo, atol=1e-12, rtol=0)
+    inf = np.isneginf(bl)
+    assert np.array_equal(np.isneginf(lse), inf)
+    np.testing.assert_allclose(lse[~inf], bl[~inf], atol=1e-12, rtol=0)
+
+
+def test_counts_outside_range_and_bad_entries():
+    """count > top_k is clamped, count < 0 is empty, entries outside the
+    sequence's blocks contribute nothing (brute force applies the same reading)."""
+    w = generate(name="bad", seed=3, q_storage=[256, 100], N1=2, N2=1, block_x=32, top_k=4,
+                 selection="random_causal")
+    w.sparse_count[0, 0] = 9
+    w.sparse_count[0, 1] = -2
+    w.sparse_idx[0, 2, 0] = 57
+    w.sparse_idx[0, 3, 0] = -1
+    w.sparse_count[0, 3] = max(w.sparse_count[0, 3], 1)
+    q, kf, vf = make_values(w, "cpu")
+    out, lse = oracle_all(w, q, kf, vf)
+    bo, bl = brute_force(w, q, kf, vf)
+    np.testing.assert_allclose(out, bo, atol=1e-12, rtol=0)
+    assert np.all(np.isneginf(lse[32:64]))          # count < 0 -> no key for that Q block
+
+
+# --------------------------------------------------------------------------
+# special cases that reduce to a library routine or a closed form
+# --------------------------------------------------------------------------
+def test_all_causal_blocks_equal_dense_causal_sdpa():
+    """Every causal block selected => dense causal attention; checked against
+    torch's scaled_dot_product_attention in fp64 with GQA-expanded K/V."""
+    w = generate(name="dense_small", seed=21, q_storage=[384, 256], N1=8, N2=2, block_x=128,
+                 top_k=3, selection="all_causal")
+    q, kf, vf = make_values(w, "cpu")
+    out, lse = oracle_all(w, q, kf, vf)
+    kb, vb = bf16_bits(kf), bf16_bits(vf)
+    for b in range(w.B):
+        t0, t1 = int(w.cu_seqlens_q[b]), int(w.cu_seqlens_q[b + 1])
+        qq = q[t0:t1].double().transpose(0, 1)                       # [N1, S, D]
+        from tests.helpers import logical_kv
+        K = torch.from_numpy(logical_kv(w, kb, b)).transpose(0, 1)   # [N2, S, D]
+        V = torch.from_numpy(logical_kv(w, vb, b)).transpose(0, 1)
+        K = K.repeat_interleave(w.G, dim=0)
+        V = V.repeat_interleave(w.G, dim=0)
+        ref = torch.nn.functional.scaled_dot_product_attention(qq, K, V, is_causal=True,
+                                                               scale=w.scale)
+        np.testing.assert_allclose(out[t0:t1], ref.transpose(0, 1).numpy(), atol=1e-11, rtol=0)
+        s = (qq @ K.transpose(1, 2)) * w.scale
+        s = s.masked_fill(torch.ones_like(s, dtype=torch.bool).triu(1), -math.inf)
+        np.testing.assert_allclose(lse[t0:t1], torch.logsumexp(s, -1).T.numpy(), atol=1e-11)
+
+
+def test_values_all_ones_give_ones():
+    """Softmax weights sum to 1: V = 1 gives out = 1 on every row with a key,
+    V = c gives out = c."""
+    w = workload("ragged", scale_down=16)
+    q, kf, vf = make_values(w, "cpu")
+    for c in (1.0, -2.5):
+        vf2 = torch.where(torch.isnan(vf), vf, torch.full_like(vf, c))
+        out, lse = oracle_all(w, q, kf, vf2)
+        has = np.isfinite(lse)
+        assert has.sum() > 100
+        np.testing.assert_allclose(out[has], c, atol=1e-13, rtol=0)
+        assert np.all(out[~has] == 0)
+
+
+def test_single_key_row_closed_form():
+    """A row with exactly one visible key: out = v exactly, lse = the score."""
+    w = generate(name="single", seed=8, q_storage=[130], N1=2, N2=1, block_x=1, top_k=1,
+                 selection="all_causal")
+    # the first token of the sequence sees only key 0
+    q, kf, vf = make_values(w, "cpu")
+    kb, vb = bf16_bits(kf), bf16_bits(vf)
+    out, lse = oracle_rows(w, q, kf, vf, np.array([[0, 0], [0, 1]]))
+    page = int(w.block_table[0, 0])
+    v0 = to_f64(vb[page * w.kv_page_stride:page * w.kv_page_stride + w.D])
+    np.testing.assert_array_equal(out[0], v0)
+    np.testing.assert_array_equal(out[1], v0)
+    # score from a constructed q/k pair with an exactly known dot product
+    q2 = torch.zeros_like(q)
+    q2[0, 0, 5] = 3.0
+    kf2 = kf.clone()
+    kf2[page * w.kv_page_stride: page * w.kv_page_stride + w.D] = 0
+    kf2[page * w.kv_page_stride + 5] = -0.25
+    _, lse2 = oracle_rows(w, q2, kf2, vf, np.array([[0, 0]]))
+    assert lse2[0] == pytest.approx(w.scale * 3.0 * -0.25, abs=1e-15)
+
+
+def test_zero_queries_give_mean_of_visible_values():
+    """q = 0: uniform weights, out = mean of v over the visible keys and
+    lse = ln(#keys); with every causal block selected the visible keys of
+    token t are 0..t, so out is the running mean of v (np.cumsum)."""
+    w = generate(name="zeroq", seed=13, q_storage=[300], N1=2, N2=1, block_x=64, top_k=3,
+                 selection="all_causal")
+    q, kf, vf = make_values(w, "cpu")
+    out, lse = oracle_all(w, torch.zeros_like(q), kf, vf)
+    from tests.helpers import logical_kv
+    V = logical_kv(w, bf16_bits(vf), 0)[:, 0, :]
+    mean = np.cumsum(V, 0) / np.arange(1, 301)[:, None]
+    for h in range(2):
+        np.testing.assert_allclose(out[:, h], mean, atol=1e-12)
+        np.testing.assert_allclose(lse[:, h], np.log(np.arange(1, 301)), atol=1e-13)
+
+
+# --------------------------------------------------------------------------
+# invariants
+# --------------------------------------------------------------------------
+def test_page_permutation_is_bit_identical():
+    w = workload("tiny", scale_down=2)
+    q, kf, vf = make_values(w, "cpu")
+    out, lse = oracle_all(w, q, kf, vf)
+    rng = np.random.default_rng(4)
+    perm = rng.permutation(w.num_pages)           # physical page p moves to perm[p]
+    k2, v2 = torch.empty_like(kf), torch.empty_like(vf)
+    view = lambda f: f.view(w.num_pages, w.kv_page_stride)
+    view(k2)[torch.as_tensor(perm)] = view(kf)
+    view(v2)[torch.as_tensor(perm)] = view(vf)
+    bt = w.block_table.copy()
+    w.block_table[:] = np.where(bt >= 0, perm[np.maximum(bt, 0)], -1)
+    out2, lse2 = oracle_all(w, q, k2, v2)
+    assert np.array_equal(out, out2) and np.array_equal(lse, lse2)
+    # and the oracle really reads the table: the old table on moved pages differs
+    w.block_table[:] = bt
+    out3, _ = oracle_all(w, q, k2, v2)
+    assert not np.array_equal(out, out3)
+
+
+def test_page_stride_is_bit_identical():
+    a = generate(name="s1", seed=31, q_storage=[256, 200], N1=4, N2=2, block_x=64, top_k=3,
+                 selection="random_causal", page_stride_factor=1.0)
+    b = generate(name="s2", seed=31, q_storage=[256, 200], N1=4, N2=2, block_x=64, top_k=3,
+                 selection="random_causal", page_stride_factor=1.25)
+    assert b.kv_page_stride > a.kv_page_stride
+    q, kf, vf = make_values(a, "cpu")
+    kb = torch.full((b.pool_elems,), float("nan"), dtype=torch.bfloat16)
+    vb = kb.clone()
+    pe = PAGE * a.N2 * a.D
+    kb.view(b.num_pages, -1)[:, :pe] = kf.view(a.num_pages, -1)[:, :pe]
+    vb.view(b.num_pages, -1)[:, :pe] = vf.view(a.num_pages, -1)[:, :pe]
+    o1, l1 = oracle_all(a, q, kf, vf)
+    o2, l2 = oracle_all(b, q, kb, vb)
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+
+
+def test_packed_gqa_equals_replicated_heads():
+    w = generate(name="gqa", seed=41, q_storage=[200, 130], N1=8, N2=2, block_x=32, top_k=4,
+                 selection="random_causal")
+    q, kf, vf = make_values(w, "cpu")
+    out, lse = oracle_all(w, q, kf, vf)
+    G = w.G
+    r = generate(name="gqa_rep", seed=41, q_storage=[200, 130], N1=8, N2=8, block_x=32,
+                 top_k=4, selection="random_causal")
+    r.block_table[:] = w.block_table
+    r.sparse_idx = np.repeat(w.sparse_idx, G, axis=0)
+    r.sparse_count = np.repeat(w.sparse_count, G, axis=0)
+    r.num_pages, r.kv_page_stride = w.num_pages, PAGE * 8 * w.D
+
+    def rep(f):
+        pages = f.view(w.num_pages, w.kv_page_stride)[:, :PAGE * w.N2 * w.D]
+        pages = pages.view(w.num_pages, PAGE, w.N2, w.D).repeat_interleave(G, dim=2)
+        return pages.reshape(-1).contiguous()
+    o2, l2 = oracle_all(r, q, rep(kf), rep(vf))
+    assert np.array_equal(out, o2) and np.array_equal(lse, l2)
+
+
+def test_padding_entries_and_unused_rows_change_nothing():
+    w = workload("ragged", scale_down=16)
+    q, kf, vf = make_values(w, "cpu")
+    out, lse = oracle_all(w, q, kf, vf)
+    rng = np.random.default_rng(9)
+    j = np.arange(w.top_k)[None, None, :]
+    pad = j >= w.sparse_count[:, :, None]
+    w.sparse_idx = np.where(pad, rng.integers(-50, 500, size=w.sparse_idx.shape),
+                            w.sparse_idx).astype(np.int32)
+    q2 = q.clone()
+    for b in range(w.B):                           # garbage in rows past seqused_q
+        t0 = int(w.cu_seqlens_q[b]) + int(w.q_used[b])
+        q2[t0:int(w.cu_seqlens_q[b + 1])] = float("nan")
+    out2, lse2 = oracle_all(w, q2, kf, vf)
+    assert np.array_equal(out, out2) and np.array_equal(lse, lse2)
+    for b in range(w.B):
+        t0 = int(w.cu_seqlens_q[b]) + int(w.q_used[b])
+        t1 = int(w.cu_seqlens_q[b + 1])
+        assert np.all(out[t0:t1] == 0) and np.all(np.isneginf(lse[t0:t1]))
+
+
+def test_oracle_rejects_bad_page():
+    w = workload("tiny", scale_down=4)
+    q, kf, vf = make_values(w, "cpu")
+    w.block_table[0, 0] = w.num_pages + 3
+    w.sparse_idx[0, 0, 0] = 0
+    w.sparse_count[0, 0] = max(int(w.sparse_count[0, 0]), 1)
+    with pytest.raises(ValueError):
+        oracle_all(w, q, kf, vf)
