@@ -1,0 +1,678 @@
+// gbsa_fwd.cu -- forward kernel of block-sparse paged GQA attention for
+// sm_100a, and the split-KV combine kernel.
+//
+// Operation (GBSA article, cf-1.com/news/4865651, "Function / sparse
+// attention mechanism"): out = Softmax(scale * Q * K_sparse^T + mask) *
+// V_sparse, where each Q block of each KV head attends only to the KV blocks
+// of its list, gathered from the paged cache (PA_BBND) through the block
+// table.  Scores are produced tile by tile with the online softmax of the FA
+// blog (ai6s.net), "three steps": running max, running sum and a rescale of
+// the partial output, so the score matrix never exists.
+//
+// Design (one persistent CTA per SM, 384 threads):
+//   warp 0       TMA producer: Q tiles (2 per unit) and, per selected block,
+//                the K and V pages into a 5-stage ring of 32 KiB buffers;
+//   warp 1       MMA issuer: S = Q K^T (SS MMA) and O += P V (TS MMA, P read
+//                from TMEM); zeroes the rows of a last page past seqused_kv
+//                in the V buffer so that stale values cannot reach O;
+//   warps 4..7   softmax + epilogue of tile 0 (TMEM lanes = tile rows);
+//   warps 8..11  softmax + epilogue of tile 1.
+// TMEM (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each; P (bf16,
+// packed in pairs) overwrites the first 64 columns of its S.
+// Units come from the metadata work list, longest first; CTA c takes units
+// c, c + gridDim.x, ...  Every wait is bounded: after ~1 s the kernel sets
+// GBSA_DEV_TIMEOUT, drains its own copies and MMAs, frees TMEM and returns.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "gbsa_internal.cuh"
+#include "sm100.cuh"
+
+namespace gbsa {
+
+using namespace sm100;
+
+namespace {
+
+constexpr int kThreads = 384;
+// Register split: launched with kLaunchRegs per thread (384 threads); the
+// producer/MMA warpgroup gives registers to the two softmax warpgroups.
+constexpr int kLaunchRegs = 168;
+constexpr int kRegsControl = 56;
+constexpr int kRegsSoftmax = 224;
+static_assert(128 * kRegsControl + 256 * kRegsSoftmax <= kLaunchRegs * kThreads,
+              "register split exceeds the launch allocation");
+constexpr int kStages = 5;
+constexpr int kTileBytes = 32768;  // 128 rows x 128 bf16 (two 64-column SW128 boxes)
+constexpr int kHalfBytes = 16384;
+constexpr int kSmemQ = 0;
+constexpr int kSmemRing = 2 * kTileBytes;
+constexpr int kSmemBars = kSmemRing + kStages * kTileBytes;
+constexpr int kSmemBytes = kSmemBars + 1024;
+constexpr int kSmemAlloc = kSmemBytes + 1024;  // slack for the 1024-byte alignment
+constexpr uint64_t kWaitLimitNs = 1000000000ull;
+constexpr float kRescaleThreshold = 8.0f;  // log2 of the largest allowed P (256)
+constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, false, false);
+constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, false, true);
+
+struct FwdParams {
+  const int32_t* meta;
+  const int32_t* block_table;
+  __nv_bfloat16* out;
+  float* lse;
+  float* ws_o;    // [slot_cap][rows_per_unit][128] fp32 partial outputs
+  float* ws_lse;  // [slot_cap][rows_per_unit] fp32 partial lse
+  int32_t* dev_status;
+  uint32_t signature;
+  int32_t N1, N2, G, T, top_k, max_pages, num_pages, tile_tokens, rows_per_unit;
+  int32_t win_left, return_lse;
+  float scale_log2;
+};
+
+struct Bars {
+  uint64_t q_full, q_empty;
+  uint64_t kv_full[kStages], kv_empty[kStages];
+  uint64_t s_full[2], p_full[2], o_done[2], o_free[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int32_t abort;
+};
+
+struct Unit {
+  int32_t item, tp, j0, j1, slot;
+  int32_t b, n_live, n_tiles, tok_begin, n_store, n_used, pos0, ku;
+  int32_t kvh, nt;  // KV head, tiles in this unit (1 or 2)
+};
+
+__device__ __forceinline__ Unit load_unit(const int32_t* meta, int64_t off_unit, int64_t off_item,
+                                          int32_t u, int32_t N2) {
+  Unit x;
+  const int4 rec = *reinterpret_cast<const int4*>(meta + off_unit + 4 * (int64_t)u);
+  x.item = rec.x;
+  x.tp = rec.y;
+  x.j0 = rec.z & 0xffff;
+  x.j1 = (int32_t)((uint32_t)rec.z >> 16);
+  x.slot = rec.w;
+  const int4 a = *reinterpret_cast<const int4*>(meta + off_item + 8 * (int64_t)x.item);
+  const int4 c = *reinterpret_cast<const int4*>(meta + off_item + 8 * (int64_t)x.item + 4);
+  x.b = a.x;
+  x.n_live = a.y;
+  x.n_tiles = a.z;
+  x.tok_begin = a.w;
+  x.n_store = c.x;
+  x.n_used = c.y;
+  x.pos0 = c.z;
+  x.ku = c.w;
+  x.kvh = x.item % N2;
+  x.nt = min(2, x.n_tiles - 2 * x.tp);
+  return x;
+}
+
+// Bounded wait on an mbarrier phase.  Returns false (and raises the CTA's
+// abort flag) after kWaitLimitNs, or at once if another role aborted.
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Bars* bars) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (;;) {
+#pragma unroll 1
+    for (int i = 0; i < 32; i++)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (*reinterpret_cast<volatile int32_t*>(&bars->abort)) return false;
+    if (global_timer_ns() - t0 > kWaitLimitNs) {
+      atomicExch(&bars->abort, 1);
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ uint64_t desc_k_major(uint32_t tile_addr, int kk) {
+  // K step kk covers 16 bf16 (32 bytes); 64-column halves are 16 KiB apart.
+  return smem_desc_sw128(tile_addr + (kk >> 2) * kHalfBytes + (kk & 3) * 32, 16, 1024);
+}
+
+__device__ __forceinline__ uint64_t desc_v_mn_major(uint32_t tile_addr, int kk) {
+  // K step kk covers 16 keys = 16 rows of 128 B; the two 64-column halves
+  // of D are 16 KiB apart (leading byte offset), 8-row groups 1 KiB apart.
+  return smem_desc_sw128(tile_addr + kk * 2048, kHalfBytes, 1024);
+}
+
+// ---------------------------------------------------------------------------
+// producer (one thread)
+// ---------------------------------------------------------------------------
+__device__ void run_producer(const FwdParams& p, const CUtensorMap* map_q, const CUtensorMap* map_k,
+                             const CUtensorMap* map_v, uint8_t* smem, Bars* bars, int32_t n_units,
+                             int64_t off_unit, int64_t off_item, int64_t off_list) {
+  uint32_t kv_iter = 0, q_iter = 0;
+  int32_t bad = 0;
+  bool ok = true;
+  const uint32_t q_box_bytes = 128u * (uint32_t)p.G * (uint32_t)p.tile_tokens;
+  for (int32_t u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+    const Unit x = load_unit(p.meta, off_unit, off_item, u, p.N2);
+    if (x.j1 <= x.j0) continue;
+    if (q_iter > 0 && !(ok = wait_bar(&bars->q_empty, (q_iter - 1) & 1, bars))) break;
+    mbar_arrive_expect_tx(&bars->q_full, (uint32_t)x.nt * 2u * q_box_bytes);
+    for (int s = 0; s < x.nt; s++) {
+      const int32_t tok = x.tok_begin + (2 * x.tp + s) * p.tile_tokens;
+      uint8_t* dst = smem + kSmemQ + s * kTileBytes;
+      tma_load_3d(dst, map_q, &bars->q_full, 0, x.kvh * p.G, tok);
+      tma_load_3d(dst + kHalfBytes, map_q, &bars->q_full, 64, x.kvh * p.G, tok);
+    }
+    q_iter++;
+    const int32_t* list = p.meta + off_list + (int64_t)x.item * p.top_k;
+    const int32_t* bt = p.block_table + (int64_t)x.b * p.max_pages;
+    for (int32_t j = x.j0; j < x.j1 && ok; j++) {
+      const int32_t lb = list[j] & kEntryLbMask;
+      int32_t page = lb < p.max_pages ? bt[lb] : -1;
+      if (page < 0 || page >= p.num_pages) {
+        bad |= kDevBadPage;
+        page = 0;
+      }
+      for (int kv = 0; kv < 2; kv++) {
+        const uint32_t stage = kv_iter % kStages;
+        if (kv_iter >= kStages &&
+            !(ok = wait_bar(&bars->kv_empty[stage], ((kv_iter / kStages) & 1) ^ 1, bars)))
+          break;
+        uint8_t* dst = smem + kSmemRing + stage * kTileBytes;
+        const CUtensorMap* map = kv ? map_v : map_k;
+        mbar_arrive_expect_tx(&bars->kv_full[stage], kTileBytes);
+        tma_load_4d(dst, map, &bars->kv_full[stage], 0, x.kvh, 0, page);
+        tma_load_4d(dst + kHalfBytes, map, &bars->kv_full[stage], 64, x.kvh, 0, page);
+        kv_iter++;
+      }
+    }
+  }
+  if (bad && p.dev_status) atomicOr(p.dev_status, bad);
+  if (!ok) {
+    // drain: wait (bounded) for the copies this thread issued last
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t i = (kv_iter > kStages ? kv_iter - kStages : 0); i < kv_iter; i++) {
+      while (!mbar_try_wait(&bars->kv_full[i % kStages], (i / kStages) & 1) &&
+             global_timer_ns() - t0 < kWaitLimitNs) {
+      }
+    }
+    if (q_iter > 0)
+      while (!mbar_try_wait(&bars->q_full, (q_iter - 1) & 1) &&
+             global_timer_ns() - t0 < kWaitLimitNs) {
+      }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// MMA issuer (warp 1; lane 0 issues, the warp zeroes stale V rows)
+// ---------------------------------------------------------------------------
+__device__ void run_mma(const FwdParams& p, uint8_t* smem, Bars* bars, uint32_t tmem,
+                        int32_t n_units, int64_t off_unit, int64_t off_item, int64_t off_list) {
+  const uint32_t lane = lane_id();
+  uint32_t kv_iter = 0, q_iter = 0;
+  uint32_t blk_iter[2] = {0, 0}, unit_iter[2] = {0, 0};
+  bool ok = true;
+  const uint32_t q_addr = smem_u32(smem + kSmemQ);
+  const uint32_t ring_addr = smem_u32(smem + kSmemRing);
+  for (int32_t u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+    const Unit x = load_unit(p.meta, off_unit, off_item, u, p.N2);
+    const int32_t nblk = x.j1 - x.j0;
+    if (nblk > 0) {
+      if (lane == 0) ok = wait_bar(&bars->q_full, q_iter & 1, bars);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      q_iter++;
+      const int32_t* list = p.meta + off_list + (int64_t)x.item * p.top_k;
+      for (int32_t jb = 0; jb < nblk && ok; jb++) {
+        // ---- S = Q K^T for every tile of the unit
+        uint32_t stage = kv_iter % kStages;
+        if (lane == 0) {
+          ok = wait_bar(&bars->kv_full[stage], (kv_iter / kStages) & 1, bars);
+          tc_fence_after_sync();
+          for (int s = 0; s < x.nt && ok; s++) {
+            if (blk_iter[s] > 0) ok = wait_bar(&bars->o_done[s], (blk_iter[s] - 1) & 1, bars);
+            if (!ok) break;
+            tc_fence_after_sync();
+            const uint32_t qa = q_addr + s * kTileBytes, ka = ring_addr + stage * kTileBytes;
+#pragma unroll
+            for (int kk = 0; kk < 8; kk++)
+              mma_ss(tmem + 128 * s, desc_k_major(qa, kk), desc_k_major(ka, kk), kIdescQK, kk > 0);
+            tc_commit(&bars->s_full[s]);
+          }
+          if (ok) {
+            tc_commit(&bars->kv_empty[stage]);
+            if (jb == nblk - 1) tc_commit(&bars->q_empty);
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        kv_iter++;
+        // ---- O += P V
+        stage = kv_iter % kStages;
+        if (lane == 0) ok = wait_bar(&bars->kv_full[stage], (kv_iter / kStages) & 1, bars);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        const int32_t entry = list[x.j0 + jb];
+        if (entry & kEntryPartial) {
+          // keys >= seqused_kv of the last page: zero those V rows (both halves)
+          const int32_t r0 = min(max(x.ku - (entry & kEntryLbMask) * kPage, 0), kPage);
+          uint8_t* vt = smem + kSmemRing + stage * kTileBytes;
+          const int32_t n16 = (kPage - r0) * 16;
+          for (int32_t i = lane; i < n16; i += 32) {
+            const int32_t row = r0 + (i >> 4), chunk = i & 15;
+            *reinterpret_cast<uint4*>(vt + (chunk >> 3) * kHalfBytes + row * 128 + (chunk & 7) * 16) =
+                make_uint4(0, 0, 0, 0);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+        }
+        if (lane == 0) {
+          tc_fence_after_sync();
+          for (int s = 0; s < x.nt && ok; s++) {
+            if (jb == 0 && unit_iter[s] > 0)
+              ok = wait_bar(&bars->o_free[s], (unit_iter[s] - 1) & 1, bars);
+            if (ok) ok = wait_bar(&bars->p_full[s], blk_iter[s] & 1, bars);
+            if (!ok) break;
+            tc_fence_after_sync();
+            const uint32_t va = ring_addr + stage * kTileBytes;
+            const uint32_t p_tmem = tmem + 128 * s;
+#pragma unroll
+            for (int kk = 0; kk < 8; kk++)
+              mma_ts(tmem + 256 + 128 * s, p_tmem + kk * 8, desc_v_mn_major(va, kk), kIdescPV,
+                     (jb > 0 || kk > 0) ? 1u : 0u);
+            tc_commit(&bars->o_done[s]);
+            blk_iter[s]++;
+          }
+          if (ok) tc_commit(&bars->kv_empty[stage]);
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        blk_iter[0] = __shfl_sync(0xffffffffu, blk_iter[0], 0);
+        blk_iter[1] = __shfl_sync(0xffffffffu, blk_iter[1], 0);
+        kv_iter++;
+      }
+    }
+    for (int s = 0; s < x.nt; s++) unit_iter[s]++;
+  }
+  // all MMAs issued by this thread complete before TMEM is released
+  if (lane == 0) {
+    tc_commit(&bars->drain);
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(&bars->drain, 0) && global_timer_ns() - t0 < kWaitLimitNs) {
+    }
+  }
+  __syncwarp();
+}
+
+// ---------------------------------------------------------------------------
+// softmax + epilogue (one warpgroup per tile slot; thread = tile row)
+// ---------------------------------------------------------------------------
+__device__ void run_softmax(const FwdParams& p, Bars* bars, uint32_t tmem, int slot,
+                            int32_t n_units, int64_t off_unit, int64_t off_item, int64_t off_list) {
+  const int row = (threadIdx.x & 127);            // tile row = TMEM lane
+  const uint32_t lane_sel = (uint32_t)((threadIdx.x & 96)) << 16;  // warp's 32-lane quarter
+  const uint32_t t_s = tmem + 128 * slot + lane_sel;
+  const uint32_t t_o = tmem + 256 + 128 * slot + lane_sel;
+  const int rows_in_tile = p.tile_tokens * p.G;
+  const int tok_in_tile = row / p.G;
+  const int g = row - tok_in_tile * p.G;
+  uint32_t blk_iter = 0;
+  int32_t bad = 0;
+  bool ok = true;
+  for (int32_t u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+    const Unit x = load_unit(p.meta, off_unit, off_item, u, p.N2);
+    if (slot >= x.nt) continue;
+    const int32_t tok_off = (2 * x.tp + slot) * p.tile_tokens + tok_in_tile;
+    const bool row_store = row < rows_in_tile && tok_off < x.n_store;
+    const bool row_used = row_store && tok_off < x.n_used;
+    const int32_t tok = x.tok_begin + tok_off;
+    const int32_t h = x.kvh * p.G + g;
+    const int32_t pos = x.pos0 + tok_off;  // query position (bottom-right aligned)
+    const int32_t key_hi = min(pos, x.ku - 1);
+    const int32_t key_lo = p.win_left >= 0 ? pos - p.win_left : INT32_MIN;
+    const int32_t* list = p.meta + off_list + (int64_t)x.item * p.top_k;
+    float m = -INFINITY, l = 0.f;
+    const int32_t nblk = x.j1 - x.j0;
+    for (int32_t jb = 0; jb < nblk; jb++) {
+      const int32_t entry = list[x.j0 + jb];
+      if (!(ok = wait_bar(&bars->s_full[slot], blk_iter & 1, bars))) break;
+      tc_fence_after_sync();
+      uint32_t r[4][32];
+      tmem_ld_32x32(t_s + 0, r[0]);
+      tmem_ld_32x32(t_s + 32, r[1]);
+      tmem_ld_32x32(t_s + 64, r[2]);
+      tmem_ld_32x32(t_s + 96, r[3]);
+      tmem_wait_ld(r[0]);
+      reg_fence(r[1]);
+      reg_fence(r[2]);
+      reg_fence(r[3]);
+      // visible key columns of this block for this row: [clo, chi]
+      int32_t clo = 0, chi = kPage - 1;
+      if (!row_used) {
+        clo = kPage;
+        chi = -1;
+      } else if (entry & kEntryMask) {
+        const int32_t base = (entry & kEntryLbMask) * kPage;
+        clo = key_lo == INT32_MIN ? 0 : max(key_lo - base, 0);
+        chi = min(key_hi - base, kPage - 1);
+      }
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 128; c++) {
+        const float v = (c >= clo && c <= chi) ? __uint_as_float(r[c >> 5][c & 31]) : -INFINITY;
+        r[c >> 5][c & 31] = __float_as_uint(v);
+        mx = fmaxf(mx, v);
+      }
+      const float m_blk = mx * p.scale_log2;
+      const float m_new = fmaxf(m, m_blk);
+      // lazy rescale: keep the old reference max unless it grew by > 8 (P <= 256)
+      const bool rescale = m_new != -INFINITY && (m == -INFINITY || m_new > m + kRescaleThreshold);
+      const bool fix_o = rescale && m != -INFINITY;
+      const float factor = fix_o ? fast_exp2(m - m_new) : 1.f;
+      if (rescale) {
+        l *= factor;
+        m = m_new;
+      }
+      const float neg_m = (m == -INFINITY) ? 0.f : -m;
+      float sum = 0.f;
+#pragma unroll
+      for (int half = 0; half < 2; half++) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int i = 0; i < 32; i++) {
+          const int c = half * 64 + 2 * i;
+          const float s0 = __uint_as_float(r[c >> 5][c & 31]);
+          const float s1 = __uint_as_float(r[(c + 1) >> 5][(c + 1) & 31]);
+          const float p0 = s0 == -INFINITY ? 0.f : fast_exp2(fmaf(s0, p.scale_log2, neg_m));
+          const float p1 = s1 == -INFINITY ? 0.f : fast_exp2(fmaf(s1, p.scale_log2, neg_m));
+          sum += p0 + p1;
+          pk[i] = pack_bf16x2(p0, p1);
+        }
+        tmem_st_32x32(t_s + 32 * half, pk);
+      }
+      l += sum;
+      if (__any_sync(0xffffffffu, fix_o)) {
+        // O holds the earlier blocks (their PV completed before this S was
+        // committed); bring it to the new reference max.
+#pragma unroll 1
+        for (int c = 0; c < 4; c++) {
+          uint32_t o[32];
+          tmem_ld_32x32(t_o + 32 * c, o);
+          tmem_wait_ld(o);
+#pragma unroll
+          for (int i = 0; i < 32; i++) o[i] = __float_as_uint(__uint_as_float(o[i]) * factor);
+          tmem_st_32x32(t_o + 32 * c, o);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before_sync();
+      mbar_arrive(&bars->p_full[slot]);
+      blk_iter++;
+    }
+    if (!ok) break;
+    // ---- epilogue
+    if (nblk > 0) {
+      if (!(ok = wait_bar(&bars->o_done[slot], (blk_iter - 1) & 1, bars))) break;
+      tc_fence_after_sync();
+    }
+    const bool has = nblk > 0 && row_used && l > 0.f;
+    const float inv_l = has ? 1.f / l : 0.f;
+    const float lse = has ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+    const bool write_row = row_store && tok < p.T;
+    if (row_store && tok >= p.T) bad |= kDevBadSeqlen;
+    if (x.slot < 0) {
+      __nv_bfloat16* dst = p.out + ((int64_t)tok * p.N1 + h) * kHeadDim;
+#pragma unroll 1
+      for (int c = 0; c < 4; c++) {
+        uint32_t o[32];
+        if (nblk > 0) {
+          tmem_ld_32x32(t_o + 32 * c, o);
+          tmem_wait_ld(o);
+        }
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; i++)
+          pk[i] = has ? pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l,
+                                    __uint_as_float(o[2 * i + 1]) * inv_l)
+                      : 0u;
+        if (write_row) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
+#pragma unroll
+          for (int i = 0; i < 4; i++)
+            d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+        }
+      }
+      if (write_row && p.return_lse) p.lse[(int64_t)tok * p.N1 + h] = lse;
+    } else {
+      const int64_t wrow = (int64_t)x.slot * p.rows_per_unit + slot * rows_in_tile + row;
+      float* dst = p.ws_o + wrow * kHeadDim;
+#pragma unroll 1
+      for (int c = 0; c < 4; c++) {
+        uint32_t o[32];
+        if (nblk > 0) {
+          tmem_ld_32x32(t_o + 32 * c, o);
+          tmem_wait_ld(o);
+        }
+        if (row < rows_in_tile) {
+          float4* d4 = reinterpret_cast<float4*>(dst + 32 * c);
+#pragma unroll
+          for (int i = 0; i < 8; i++)
+            d4[i] = has ? make_float4(__uint_as_float(o[4 * i]) * inv_l,
+                                      __uint_as_float(o[4 * i + 1]) * inv_l,
+                                      __uint_as_float(o[4 * i + 2]) * inv_l,
+                                      __uint_as_float(o[4 * i + 3]) * inv_l)
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+      if (row < rows_in_tile) p.ws_lse[wrow] = lse;
+    }
+    tc_fence_before_sync();
+    mbar_arrive(&bars->o_free[slot]);
+  }
+  if (bad && p.dev_status) atomicOr(p.dev_status, bad);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+               const __grid_constant__ CUtensorMap map_v, const FwdParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  Bars* bars = reinterpret_cast<Bars*>(smem + kSmemBars);
+  const int warp = threadIdx.x >> 5;
+
+  // the work list must have been built for this problem
+  const int32_t* meta = p.meta;
+  const bool match = (uint32_t)meta[H_MAGIC] == kMagic && meta[H_VERSION] == kFormatVersion &&
+                     (uint32_t)meta[H_SIGNATURE] == p.signature;
+  if (!match) {
+    if (threadIdx.x == 0 && blockIdx.x == 0 && p.dev_status) atomicOr(p.dev_status, kDevMetaMismatch);
+    return;
+  }
+  const int32_t n_units = meta[H_NUNITS];
+  const int64_t off_unit = meta[H_OFF_UNIT], off_item = meta[H_OFF_ITEM], off_list = meta[H_OFF_LIST];
+  if ((int32_t)blockIdx.x >= n_units) return;  // no work for this CTA (uniform)
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->q_full, 1);
+    mbar_init(&bars->q_empty, 1);
+    for (int i = 0; i < kStages; i++) {
+      mbar_init(&bars->kv_full[i], 1);
+      mbar_init(&bars->kv_empty[i], 1);
+    }
+    for (int s = 0; s < 2; s++) {
+      mbar_init(&bars->s_full[s], 1);
+      mbar_init(&bars->p_full[s], 128);
+      mbar_init(&bars->o_done[s], 1);
+      mbar_init(&bars->o_free[s], 128);
+    }
+    mbar_init(&bars->drain, 1);
+    bars->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp < 4) {
+    setmaxnreg_dec<kRegsControl>();
+    if (warp == 0) {
+      if (lane_id() == 0) {
+        tma_prefetch_map(&map_q);
+        tma_prefetch_map(&map_k);
+        tma_prefetch_map(&map_v);
+        run_producer(p, &map_q, &map_k, &map_v, smem, bars, n_units, off_unit, off_item,
+                     off_list);
+      }
+    } else if (warp == 1) {
+      run_mma(p, smem, bars, tmem, n_units, off_unit, off_item, off_list);
+    }
+  } else {
+    setmaxnreg_inc<kRegsSoftmax>();
+    run_softmax(p, bars, tmem, (warp - 4) >> 2, n_units, off_unit, off_item, off_list);
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  if (threadIdx.x == 0 && bars->abort && p.dev_status) atomicOr(p.dev_status, kDevTimeout);
+  if (warp == 1) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// split-KV combine: one CTA per split (item, tile pair); a warp per row
+// ---------------------------------------------------------------------------
+struct CombineParams {
+  const int32_t* meta;
+  const float* ws_o;
+  const float* ws_lse;
+  __nv_bfloat16* out;
+  float* lse;
+  int32_t* dev_status;
+  uint32_t signature;
+  int32_t N1, N2, G, T, tile_tokens, rows_per_unit, return_lse;
+};
+
+__global__ void __launch_bounds__(256) combine_kernel(const CombineParams p) {
+  const int32_t* meta = p.meta;
+  if ((uint32_t)meta[H_MAGIC] != kMagic || (uint32_t)meta[H_SIGNATURE] != p.signature) return;
+  const int32_t n_comb = meta[H_NCOMB];
+  if ((int32_t)blockIdx.x >= n_comb) return;
+  const int4 rec = *reinterpret_cast<const int4*>(meta + meta[H_OFF_COMB] + 4 * (int64_t)blockIdx.x);
+  const int32_t item = rec.x, tp = rec.y, first = rec.z, k = rec.w;
+  const int32_t* it = meta + meta[H_OFF_ITEM] + 8 * (int64_t)item;
+  const int32_t n_tiles = it[2], tok_begin = it[3], n_store = it[4];
+  const int32_t kvh = item % p.N2;
+  const int rows_in_tile = p.tile_tokens * p.G;
+  const int lane = threadIdx.x & 31;
+  const int nt = min(2, n_tiles - 2 * tp);
+  for (int rr = threadIdx.x >> 5; rr < nt * rows_in_tile; rr += blockDim.x >> 5) {
+    const int s = rr / rows_in_tile, row = rr - s * rows_in_tile;
+    const int32_t tok_off = (2 * tp + s) * p.tile_tokens + row / p.G;
+    if (tok_off >= n_store) continue;
+    const int32_t tok = tok_begin + tok_off;
+    if (tok >= p.T) continue;
+    const int32_t h = kvh * p.G + row % p.G;
+    const int64_t wrow0 = (int64_t)first * p.rows_per_unit + rr;
+    float mx = -INFINITY;
+    for (int j = 0; j < k; j++) mx = fmaxf(mx, p.ws_lse[wrow0 + (int64_t)j * p.rows_per_unit]);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float wsum = 0.f;
+    if (mx != -INFINITY) {
+      for (int j = 0; j < k; j++) {
+        const int64_t wrow = wrow0 + (int64_t)j * p.rows_per_unit;
+        const float lj = p.ws_lse[wrow];
+        const float w = lj == -INFINITY ? 0.f : expf(lj - mx);
+        wsum += w;
+        const float4 o = reinterpret_cast<const float4*>(p.ws_o + wrow * kHeadDim)[lane];
+        acc.x += w * o.x;
+        acc.y += w * o.y;
+        acc.z += w * o.z;
+        acc.w += w * o.w;
+      }
+    }
+    const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+    __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+    __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+    uint2 pk;
+    pk.x = *reinterpret_cast<uint32_t*>(&lo);
+    pk.y = *reinterpret_cast<uint32_t*>(&hi);
+    reinterpret_cast<uint2*>(p.out + ((int64_t)tok * p.N1 + h) * kHeadDim)[lane] = pk;
+    if (lane == 0 && p.return_lse)
+      p.lse[(int64_t)tok * p.N1 + h] = wsum > 0.f ? mx + logf(wsum) : -INFINITY;
+  }
+}
+
+}  // namespace
+
+size_t forward_smem_bytes() { return kSmemAlloc; }
+
+cudaError_t launch_forward(const CUtensorMap& map_q, const CUtensorMap& map_k,
+                           const CUtensorMap& map_v, const int32_t* meta,
+                           const int32_t* block_table, void* out, float* lse, float* ws_o,
+                           float* ws_lse, int32_t* dev_status, uint32_t signature, int32_t N1,
+                           int32_t N2, int32_t T, int32_t top_k, int32_t max_pages,
+                           int32_t num_pages, int32_t tile_tokens, int32_t rows_per_unit,
+                           int32_t win_left, int32_t return_lse, float scale_log2,
+                           int32_t num_ctas, int64_t comb_cap, cudaStream_t stream) {
+  static int configured_device = -1;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (configured_device != dev) {
+    // The register re-split is only safe if the kernel launches with exactly
+    // the registers the split was computed for.
+    cudaFuncAttributes attr;
+    e = cudaFuncGetAttributes(&attr, fwd_kernel);
+    if (e != cudaSuccess) return e;
+    if (attr.numRegs != kLaunchRegs) return cudaErrorInvalidKernelImage;
+    e = cudaFuncSetAttribute(fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
+    if (e != cudaSuccess) return e;
+    configured_device = dev;
+  }
+  FwdParams p;
+  p.meta = meta;
+  p.block_table = block_table;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.ws_o = ws_o;
+  p.ws_lse = ws_lse;
+  p.dev_status = dev_status;
+  p.signature = signature;
+  p.N1 = N1;
+  p.N2 = N2;
+  p.G = N1 / N2;
+  p.T = T;
+  p.top_k = top_k;
+  p.max_pages = max_pages;
+  p.num_pages = num_pages;
+  p.tile_tokens = tile_tokens;
+  p.rows_per_unit = rows_per_unit;
+  p.win_left = win_left;
+  p.return_lse = return_lse;
+  p.scale_log2 = scale_log2;
+  fwd_kernel<<<num_ctas, kThreads, kSmemAlloc, stream>>>(map_q, map_k, map_v, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || comb_cap <= 0) return e;
+  CombineParams c;
+  c.meta = meta;
+  c.ws_o = ws_o;
+  c.ws_lse = ws_lse;
+  c.out = p.out;
+  c.lse = lse;
+  c.dev_status = dev_status;
+  c.signature = signature;
+  c.N1 = N1;
+  c.N2 = N2;
+  c.G = p.G;
+  c.T = T;
+  c.tile_tokens = tile_tokens;
+  c.rows_per_unit = rows_per_unit;
+  c.return_lse = return_lse;
+  combine_kernel<<<(unsigned)comb_cap, 256, 0, stream>>>(c);
+  return cudaGetLastError();
+}
+
+}  // namespace gbsa

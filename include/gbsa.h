@@ -56,6 +56,13 @@ extern "C" {
 
 #define GBSA_ABI_VERSION 1
 
+/* Symbols of the C ABI are exported; everything else in libgbsa is hidden. */
+#if defined(__GNUC__)
+#define GBSA_API __attribute__((visibility("default")))
+#else
+#define GBSA_API
+#endif
+
 /* Return codes.  The GBSA article's return-code table did not survive
  * extraction; these are this library's own. */
 typedef enum gbsa_status {
@@ -123,29 +130,29 @@ typedef struct gbsa_tensors {
 } gbsa_tensors;
 
 /* Version of this header the library was built from (GBSA_ABI_VERSION). */
-int32_t gbsa_abi_version(void);
+GBSA_API int32_t gbsa_abi_version(void);
 
 /* Human-readable name of a status code; never NULL. */
-const char* gbsa_status_string(gbsa_status status);
+GBSA_API const char* gbsa_status_string(gbsa_status status);
 
 /* Bytes of metadata gbsa_metadata() writes for `problem` (a host-known bound:
  * it does not depend on device values).  Validates `problem` first.
  * GBSA article, "two-phase call": the metadata records the core split.
  * Returns GBSA_ERR_NO_DEVICE if num_ctas == 0 and no device can be queried. */
-gbsa_status gbsa_metadata_size(const gbsa_problem* problem, size_t* bytes);
+GBSA_API gbsa_status gbsa_metadata_size(const gbsa_problem* problem, size_t* bytes);
 
 /* Builds the work list for `problem` into the caller's device buffer `meta`
  * (16-byte aligned, meta_bytes >= gbsa_metadata_size()).  Reads
  * sparse_idx, sparse_count, cu_seqlens_q, seqused_q and seqused_kv; other
  * tensor fields may be NULL.  Deterministic: equal inputs give equal bytes.
  * GBSA article, "two-phase call" step 2 and "Constraints: metadata first". */
-gbsa_status gbsa_metadata(const gbsa_problem* problem, const gbsa_tensors* tensors,
+GBSA_API gbsa_status gbsa_metadata(const gbsa_problem* problem, const gbsa_tensors* tensors,
                           void* meta, size_t meta_bytes, int32_t* dev_status, void* stream);
 
 /* Bytes of scratch the forward needs for split-KV partial results
  * (fp32 partial outputs and log-sum-exps); may be 0 only if splitting is
  * impossible.  GBSA article, "aclnn API": first-phase workspace query. */
-gbsa_status gbsa_workspace_size(const gbsa_problem* problem, size_t* bytes);
+GBSA_API gbsa_status gbsa_workspace_size(const gbsa_problem* problem, size_t* bytes);
 
 /* Runs the attention: out (and lse when return_lse) from q, k, v through the
  * work list in `meta`.  `workspace` (16-byte aligned, ws_bytes >=
@@ -154,7 +161,7 @@ gbsa_status gbsa_workspace_size(const gbsa_problem* problem, size_t* bytes);
  * and leave out/lse untouched.  Deterministic for a fixed num_ctas
  * (GBSA article, "Constraints: determinism").  Rows past seqused_q, and rows
  * with no visible key, get out = 0 and lse = -inf. */
-gbsa_status gbsa_forward(const gbsa_problem* problem, const gbsa_tensors* tensors,
+GBSA_API gbsa_status gbsa_forward(const gbsa_problem* problem, const gbsa_tensors* tensors,
                          const void* meta, void* workspace, size_t ws_bytes,
                          int32_t* dev_status, void* stream);
 

@@ -1,0 +1,148 @@
+"""The C-ABI library on the host: it loads without a GPU, exports every
+function include/gbsa.h declares, and rejects every rule of the GBSA
+article's "Constraints" section before anything is launched."""
+import ctypes
+import dataclasses
+import os
+import re
+
+import pytest
+
+import block_sparse_paged_gbsa_b200 as gbsa
+from block_sparse_paged_gbsa_b200 import build as build_mod
+from block_sparse_paged_gbsa_b200.gbsa import Problem, _Tensors
+from block_sparse_paged_gbsa_b200.workloads import workload
+from oracle import scheduler
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include",
+                      "gbsa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_mod.build()
+    return gbsa.gbsa.lib()
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gbsa_[a-z_]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = _declared_functions()
+    assert {"gbsa_metadata", "gbsa_forward", "gbsa_metadata_size",
+            "gbsa_workspace_size"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert lib.gbsa_abi_version() == 1
+    for code in range(0, 9):
+        assert lib.gbsa_status_string(code).decode().startswith("GBSA_")
+
+
+def _problem(**kw):
+    w = workload("tiny")
+    base = dict(B=w.B, T=w.T, N1=w.N1, N2=w.N2, D=128, block_x=w.block_x,
+                total_q_blocks=w.total_q_blocks, top_k=w.top_k,
+                max_pages_per_seq=w.max_pages_per_seq, num_pages=w.num_pages,
+                kv_page_stride=w.kv_page_stride, scale=w.scale, num_ctas=148, return_lse=1)
+    base.update(kw)
+    return Problem(**base), w
+
+
+def test_metadata_size_matches_format(lib):
+    for ctas, forced in ((148, 0), (7, 3)):
+        p, w = _problem(num_ctas=ctas, max_blocks_per_split=forced)
+        g = scheduler.geometry(dict(w.problem_kwargs(), num_ctas=ctas,
+                                    max_blocks_per_split=forced))
+        assert gbsa.metadata_size(p) == 4 * g["total"]
+        ws = gbsa.workspace_size(p)
+        rpu = g["rows_per_unit"]
+        o_bytes = g["slot_cap"] * rpu * 128 * 4
+        assert ws == ((o_bytes + 255) // 256) * 256 + g["slot_cap"] * rpu * 4
+
+
+CASES = [
+    (dict(D=64), "GBSA_ERR_UNSUPPORTED"),
+    (dict(block_y=64), "GBSA_ERR_UNSUPPORTED"),
+    (dict(N1=6, N2=4), "GBSA_ERR_SHAPE"),
+    (dict(N1=2, N2=4), "GBSA_ERR_SHAPE"),
+    (dict(N1=258, N2=2), "GBSA_ERR_UNSUPPORTED"),
+    (dict(top_k=257), "GBSA_ERR_UNSUPPORTED"),
+    (dict(mask_mode=0), "GBSA_ERR_UNSUPPORTED"),
+    (dict(is_packed_gqa=0), "GBSA_ERR_UNSUPPORTED"),
+    (dict(B=0), "GBSA_ERR_SHAPE"),
+    (dict(top_k=0), "GBSA_ERR_SHAPE"),
+    (dict(block_x=0), "GBSA_ERR_SHAPE"),
+    (dict(win_left=-2), "GBSA_ERR_INVALID_ARG"),
+    (dict(scale=-1.0), "GBSA_ERR_INVALID_ARG"),
+]
+
+
+@pytest.mark.parametrize("kw,expected", CASES)
+def test_problem_rules(lib, kw, expected):
+    p, _ = _problem(**kw)
+    with pytest.raises(gbsa.GbsaError) as e:
+        gbsa.metadata_size(p)
+    assert expected in str(e.value)
+
+
+FWD_CASES = [
+    (dict(kv_page_stride=128 * 2 * 128 - 256), "GBSA_ERR_SHAPE"),      # smaller than a page
+    (dict(kv_page_stride=128 * 2 * 128 + 128), "GBSA_ERR_SHAPE"),      # not a multiple of N2*D
+    (dict(num_pages=0), "GBSA_ERR_SHAPE"),
+    (dict(T=0), "GBSA_ERR_SHAPE"),
+]
+
+
+def _call_forward(lib, p, tensors, meta=16, ws=16, ws_bytes=1 << 30):
+    return lib.gbsa_forward(ctypes.byref(p.as_c()), ctypes.byref(tensors), meta, ws, ws_bytes,
+                            None, None)
+
+
+def _fake_tensors(**kw):
+    # addresses that are never dereferenced: every case fails validation first
+    f = dict(q=1 << 20, k=2 << 20, v=3 << 20, sparse_idx=4 << 20, sparse_count=5 << 20,
+             cu_seqlens_q=6 << 20, seqused_kv=7 << 20, block_table=8 << 20, out=9 << 20,
+             lse=10 << 20)
+    f.update(kw)
+    return _Tensors(**f)
+
+
+@pytest.mark.parametrize("kw,expected", FWD_CASES)
+def test_forward_shape_rules(lib, kw, expected):
+    p, _ = _problem(**kw)
+    rc = _call_forward(lib, p, _fake_tensors())
+    assert lib.gbsa_status_string(rc).decode() == expected
+
+
+def test_forward_pointer_rules(lib):
+    p, _ = _problem()
+    assert _call_forward(lib, p, _fake_tensors(q=None)) == 1              # INVALID_ARG
+    assert _call_forward(lib, p, _fake_tensors(lse=None)) == 1            # lse requested
+    p2, _ = _problem(has_seqused_q=1)
+    assert _call_forward(lib, p2, _fake_tensors()) == 1                   # seqused_q missing
+    assert _call_forward(lib, p, _fake_tensors(k=(2 << 20) + 8)) == 4     # ALIGNMENT
+    assert _call_forward(lib, p, _fake_tensors(), meta=24) == 4
+    assert _call_forward(lib, p, _fake_tensors(), ws_bytes=0) == 5        # workspace too small
+
+
+def test_no_device_means_no_default_cta_count(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a device is present")
+    p, _ = _problem(num_ctas=0)
+    with pytest.raises(gbsa.GbsaError) as e:
+        gbsa.metadata_size(p)
+    assert "NO_DEVICE" in str(e.value)
+
+
+def test_metadata_pointer_rules(lib):
+    p, _ = _problem()
+    t = _fake_tensors(sparse_idx=None)
+    rc = lib.gbsa_metadata(ctypes.byref(p.as_c()), ctypes.byref(t), 16, 1 << 30, None, None)
+    assert rc == 1
+    rc = lib.gbsa_metadata(ctypes.byref(p.as_c()), ctypes.byref(_fake_tensors()), 16, 8, None,
+                           None)
+    assert rc == 6                                                        # METADATA_TOO_SMALL
