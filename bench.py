@@ -1,0 +1,442 @@
+#!/usr/bin/env python
+"""Benchmark: block-sparse paged GQA attention forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload dense]
+    python bench.py --impl reference ...    # the fp64 CPU oracle arm
+
+One step = the whole hot path over one batch of synthetic input: the
+metadata (work list) launches, the forward kernel and the split-KV combine,
+through the C ABI.  Inputs are resident in HBM before timing; L2 is flushed
+(a 256 MiB write) between timed steps; every step is timed with CUDA events
+on the launching stream; with N GPUs each rank runs its own seeded batch
+(independent problems, no collective on the data path, weak scaling) and the
+time is the max over ranks.  Prints one JSON line on rank 0.
+
+Metric: effective TFLOPS counted over selected, unmasked (live) blocks, with
+KV-page GB/s and the roofline fraction beside it.  The fp64 oracle is timed
+on the host cores over a bounded sample of rows as the CPU baseline.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "effective TFLOPS + KV GB/s (selected blocks), % of roofline, 1×B200"
+UNIT = "TFLOPS"
+DESCRIPTIONS = {
+    "dense": "dense-equivalent causal prefill: B=4 x 4096 tokens, N1=32, N2=8, D=128, "
+             "block_shape=[128,128], 128-token pages, top_k=32, every causal block selected",
+    "tiny": "tiny block-sparse prefill: B=2 x 512 tokens, N1=8, N2=2, block_shape=[64,128], "
+            "top_k=4 random causal blocks incl. the diagonal",
+    "long": "long-context block-sparse prefill: B=1 x 131072 tokens, N1=32, N2=4, "
+            "block_shape=[128,128], top_k=64 (sink + diagonal + 62 random causal)",
+    "decode": "decode with packed GQA: 64 x 1 query token, KV ~ U[8192,65536], N1=64, N2=8, "
+              "block_shape=[1,128], top_k=256, count ~ U{64..256} incl. last page, split-KV",
+    "ragged": "ragged varlen: 16 sequences lognormal(4096, 1.0) in [512,32768], seqused = "
+              "storage - U[0,127], N1=40, N2=8, block_shape=[64,128], top_k=128, window "
+              "(4096, 0), page stride 1.25x",
+}
+FLUSH_BYTES = 256 << 20
+KERNEL_SOURCES = ["block_sparse_paged_gbsa_b200/csrc/gbsa_fwd.cu",
+                  "block_sparse_paged_gbsa_b200/csrc/sm100.cuh",
+                  "block_sparse_paged_gbsa_b200/csrc/gbsa_internal.cuh"]
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["gbsa", "reference"], default="gbsa")
+    ap.add_argument("--workload", default="dense", choices=sorted(DESCRIPTIONS))
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return dict(hbm_gbs=float(d["hbm_gbs"]), bf16_tflops=float(d["bf16_tflops"]),
+                    bf16_tflops_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    source="measured")
+    except (OSError, KeyError, ValueError):
+        return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0,
+                    source="fallback")
+
+
+def kernel_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per forward launch from the committed ncu summary, if it was
+    taken on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", f"forward_{workload}_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if d.get("kernel_sha") != kernel_hash():
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi sampling (50 ms) around the timed region."""
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=self.file, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self, t0: float, t1: float) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.12)
+        self.proc.terminate()
+        self.proc.wait()
+        self.file.flush()
+        rows = []
+        with open(self.file.name) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 10:
+                    continue
+                try:
+                    ts = time.mktime(time.strptime(parts[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                    frac = float("0." + parts[0].split(".")[1]) if "." in parts[0] else 0.0
+                    rows.append((ts + frac, float(parts[2]), float(parts[3]), parts[6:10]))
+                except ValueError:
+                    continue
+        os.unlink(self.file.name)
+        inside = [r for r in rows if t0 - 0.06 <= r[0] <= t1 + 0.06]
+        if not inside:
+            after = [r for r in rows if r[0] >= t0 - 0.06]
+            inside = after[:1]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in inside for i, v in enumerate(r[3]) if v == "Active"})
+        sm = [r[1] for r in inside]
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": max((r[2] for r in inside), default=None), "reasons": reasons,
+                "samples": len(inside)}
+
+
+def rank_seed(base_seed: int, rank: int) -> int:
+    """Each rank draws its own batch of the same workload (weak scaling)."""
+    return base_seed + 1000 * rank
+
+
+def reduce_max(values, dist, device):
+    """Max over ranks of a list of per-rank timings (host plumbing only)."""
+    import torch
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def reduce_sum(values, dist, device):
+    """Sum over ranks (the work each rank did)."""
+    import torch
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return [float(x) for x in t.tolist()]
+
+
+def job_value(total_flops: float, max_ms: float) -> float:
+    """Whole-job TFLOPS: the work of all ranks over the slowest rank's time."""
+    return total_flops / (max_ms * 1e-3) / 1e12
+
+
+def dist_info():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def cpu_cores() -> int:
+    return len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+
+
+def oracle_sample(w, q, kf, vf, target_s: float, seed: int = 0):
+    """Times the oracle on a bounded random sample of rows sized to about
+    target_s seconds.  Returns (TFLOPS, seconds, rows, description)."""
+    import oracle
+    from block_sparse_paged_gbsa_b200.accounting import row_flops
+    from block_sparse_paged_gbsa_b200.workloads import bf16_bits
+
+    qb, kb, vb = bf16_bits(q), bf16_bits(kf), bf16_bits(vf)
+    rng = np.random.default_rng(seed)
+    threads = cpu_cores()
+
+    def run(n):
+        rows = np.stack([rng.integers(0, w.T, n), rng.integers(0, w.N1, n)], 1).astype(np.int64)
+        t0 = time.perf_counter()
+        oracle.attention_rows(q_bits=qb, k_bits=kb, v_bits=vb, kv_page_stride=w.kv_page_stride,
+                              num_pages=w.num_pages, sparse_idx=w.sparse_idx,
+                              sparse_count=w.sparse_count, cu_seqlens_q=w.cu_seqlens_q,
+                              seqused_q=w.seqused_q, seqused_kv=w.kv_used,
+                              block_table=w.block_table, block_x=w.block_x, scale=w.scale,
+                              win_left=w.win_left, win_right=w.win_right, rows=rows,
+                              n_threads=threads)
+        return time.perf_counter() - t0, rows
+
+    n = 4 * threads
+    dt, rows = run(n)
+    while dt < 0.5:
+        n *= 4
+        dt, rows = run(n)
+    n = max(n, int(n * target_s / max(dt, 1e-6)))
+    dt, rows = run(n)
+    flops = row_flops(w, rows)
+    return flops / dt / 1e12, dt, n, threads
+
+
+def run_reference(args, world, rank):
+    """The CPU oracle arm: each step is the oracle over a bounded random
+    sample of rows of the same workload, on the host cores."""
+    if rank != 0:
+        return
+    from block_sparse_paged_gbsa_b200.workloads import make_values, workload
+
+    w = workload(args.workload)
+    q, kf, vf = make_values(w, "cpu")
+    per_step = max(0.5, min(5.0, 150.0 / max(1, args.steps + args.warmup)))
+    vals = []
+    for i in range(args.warmup + args.steps):
+        tf, dt, n, threads = oracle_sample(w, q, kf, vf, per_step, seed=i)
+        if i >= args.warmup:
+            vals.append((tf, dt, n))
+    tf = float(np.mean([v[0] for v in vals]))
+    sample = (f"{int(np.mean([v[2] for v in vals]))} random (token, head) rows per step, "
+              f"about {per_step:.1f} s of fp64 oracle work each")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(tf, 6), "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * float(np.mean([v[1] for v in vals])), 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": DESCRIPTIONS[args.workload], "sample": sample},
+        "cpu_baseline": {"value": round(tf, 6), "unit": UNIT, "cores": threads,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(tf, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    world, rank, local = dist_info()
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import block_sparse_paged_gbsa_b200 as gbsa
+    from block_sparse_paged_gbsa_b200.accounting import work
+    from block_sparse_paged_gbsa_b200.workloads import make_values, pool_view, workload
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the CPU oracle arm is --impl reference)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    # each rank: its own seeded batch of the same workload (weak scaling)
+    base = workload(args.workload)
+    w = workload(args.workload, seed=rank_seed(base.seed, rank))
+    acc = work(w)
+    q, kf, vf = make_values(w, dev)
+    to = lambda a, dt: torch.as_tensor(np.ascontiguousarray(a), dtype=dt, device=dev)
+    idx, cnt = to(w.sparse_idx, torch.int32), to(w.sparse_count, torch.int32)
+    cu, sku, bt = to(w.cu_seqlens_q, torch.int64), to(w.kv_used, torch.int32), to(w.block_table, torch.int32)
+    squ = to(w.q_used, torch.int32) if w.has_seqused_q else None
+    k, v = pool_view(w, kf), pool_view(w, vf)
+    block_shape = [w.block_x, 128]
+    prob = gbsa.gbsa.make_problem(q, k, idx, block_shape, bt, cu, softmax_scale=w.scale,
+                                  win_left=w.win_left, win_right=w.win_right,
+                                  return_softmax_lse=w.return_lse, has_seqused_q=squ is not None)
+    meta_buf = torch.empty(gbsa.metadata_size(prob) // 4, dtype=torch.int32, device=dev)
+    ws = torch.empty(max(gbsa.workspace_size(prob), 16), dtype=torch.uint8, device=dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((w.T, w.N1, 1), dtype=torch.float32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step(qq=q, kk=k, vv=v, ii=idx, cc=cnt, uu=cu, su=squ, kv=sku, tb=bt, ev=None):
+        if ev is not None:
+            ev[0].record()
+        meta = gbsa.metadata(ii, cc, w.N1, w.N2, w.D, block_shape, cu_seqlens_q=uu, seqused_q=su,
+                             seqused_kv=kv, num_tokens=w.T, win_left=w.win_left,
+                             win_right=w.win_right, dev_status=status, out=meta_buf)
+        if ev is not None:
+            ev[1].record()
+        gbsa.forward(qq, kk, vv, ii, cc, block_shape, metadata=meta, cu_seqlens_q=uu,
+                     seqused_q=su, seqused_kv=kv, block_table=tb, softmax_scale=w.scale,
+                     win_left=w.win_left, win_right=w.win_right,
+                     return_softmax_lse=w.return_lse, out=out, lse=lse, workspace=ws,
+                     dev_status=status)
+        if ev is not None:
+            ev[2].record()
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    meta_host = meta_buf[:32].cpu().numpy()
+    comb_cap = int(meta_host[10])
+    launches_per_step = 3 + 1 + (1 if comb_cap > 0 else 0)
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    for i in range(args.steps):
+        flush.zero_()
+        step(ev=events[i])
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    t_wall1 = time.time()
+    clocks = sampler.stop(t_wall0, t_wall1)
+    step_ms = float(np.mean([e[0].elapsed_time(e[2]) for e in events]))
+    meta_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in events]))
+    fwd_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in events]))
+    dev_bits = int(status.item())
+    total_flops, total_kv = acc["flops_block"], acc["kv_bytes"]
+    if world > 1:
+        step_ms, meta_ms, fwd_ms = reduce_max([step_ms, meta_ms, fwd_ms], dist, dev)
+        total_flops, total_kv = reduce_sum([total_flops, total_kv], dist, dev)
+
+    # end to end through the public API: pinned host inputs -> device -> host output
+    e2e = None
+    if not args.no_e2e:
+        host = {name: t.cpu().pin_memory() for name, t in
+                dict(q=q, kf=kf, vf=vf, idx=idx, cnt=cnt, cu=cu, sku=sku, bt=bt).items()}
+        if squ is not None:
+            host["squ"] = squ.cpu().pin_memory()
+        dev_in = {name: torch.empty_like(t, device=dev) for name, t in host.items()}
+        out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        lse_h = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = out_h.numel() * out_h.element_size() + (lse_h.numel() * 4 if w.return_lse else 0)
+        n_e2e = max(3, min(args.steps, 10))
+        times = []
+        for i in range(n_e2e + 2):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            flush.zero_()
+            e0.record()
+            for name, t in host.items():
+                dev_in[name].copy_(t, non_blocking=True)
+            step(dev_in["q"], pool_view(w, dev_in["kf"]), pool_view(w, dev_in["vf"]),
+                 dev_in["idx"], dev_in["cnt"], dev_in["cu"], dev_in.get("squ"), dev_in["sku"],
+                 dev_in["bt"])
+            out_h.copy_(out, non_blocking=True)
+            if w.return_lse:
+                lse_h.copy_(lse, non_blocking=True)
+            e1.record()
+            torch.cuda.synchronize()
+            if i >= 2:
+                times.append(e0.elapsed_time(e1))
+        e2e_ms = float(np.mean(times))
+        if world > 1:
+            e2e_ms = reduce_max([e2e_ms], dist, dev)[0]
+        e2e = {"value": round(job_value(total_flops, e2e_ms), 4),
+               "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": round(e2e_ms, 4)}
+
+    peaks = load_peaks()
+    flops, nbytes = acc["flops_block"], acc["bytes"]
+    value = job_value(total_flops, step_ms)
+    t_roof = max(flops / (peaks["bf16_tflops"] * 1e12), nbytes / (peaks["hbm_gbs"] * 1e9))
+    bound = "tensor" if flops / (peaks["bf16_tflops"] * 1e12) >= nbytes / (peaks["hbm_gbs"] * 1e9) else "hbm"
+    if bound == "tensor":
+        achieved = flops / (fwd_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": round(achieved, 3), "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4)}
+    else:
+        achieved = nbytes / (fwd_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 3), "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4)}
+    roof["traffic"] = profiled_traffic(args.workload)
+    roof["kernel"] = "gbsa forward (attention + split-KV combine launch)"
+    roof["peak_source"] = peaks["source"] + " (burst)"
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        qc, kc, vc = q.cpu(), kf.cpu(), vf.cpu()
+        tf, dt, n, threads = oracle_sample(w, qc, kc, vc, args.cpu_seconds)
+        cpu = {"value": round(tf, 8), "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": f"{n} random (token, head) rows of the same workload, {dt:.1f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": round(step_ms, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": DESCRIPTIONS[args.workload],
+                       "parallelism": f"dp{world} (independent batches, no collective)",
+                       "l2": "flushed between timed steps (256 MiB write)",
+                       "num_ctas": int(meta_host[7])},
+            "kv_gbs": round(total_kv / (step_ms * 1e-3) / 1e9, 2),
+            "roofline_step": {"time_ms": round(t_roof * 1e3, 5),
+                              "frac": round(t_roof * 1e3 / step_ms, 4),
+                              "flops": flops, "bytes": nbytes},
+            "flops_exact": acc["flops_exact"],
+            "metadata_ms": round(meta_ms, 4), "forward_ms": round(fwd_ms, 4),
+            "roofline": roof, "clocks": clocks, "e2e": e2e, "cpu_baseline": cpu,
+            "gpu_launches": launches_per_step * args.steps,
+            "dev_status": dev_bits,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

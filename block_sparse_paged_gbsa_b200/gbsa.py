@@ -185,10 +185,11 @@ def metadata(sparse_block_idx, sparse_block_count, num_heads_q: int, num_heads_k
              head_dim: int, block_shape: Sequence[int], *, cu_seqlens_q, seqused_kv,
              seqused_q=None, num_tokens: int = 0, is_packed_gqa: bool = True, mask_mode: int = 1,
              win_left: int = -1, win_right: int = -1, num_ctas: int = 0,
-             max_blocks_per_split: int = 0, dev_status=None):
+             max_blocks_per_split: int = 0, dev_status=None, out=None):
     """Builds the work list (int32 tensor) on the device of the inputs.
 
     num_tokens: T if known (enables the device check cu_seqlens_q[B] == T); 0 skips it.
+    out: optional preallocated int32 buffer of at least metadata_size() bytes.
     """
     import torch
     idx = _need(sparse_block_idx, "sparse_block_idx", torch.int32, 3)
@@ -208,7 +209,13 @@ def metadata(sparse_block_idx, sparse_block_count, num_heads_q: int, num_heads_k
                    num_ctas=num_ctas, max_blocks_per_split=max_blocks_per_split)
     nbytes = metadata_size(prob)
     with torch.cuda.device(dev):
-        meta = torch.empty((nbytes // 4,), dtype=torch.int32, device=dev)
+        if out is None:
+            meta = torch.empty((nbytes // 4,), dtype=torch.int32, device=dev)
+        else:
+            meta = _need(out, "out", torch.int32, 1, dev)
+            if meta.numel() * 4 < nbytes:
+                raise ValueError(f"out: needs {nbytes} bytes")
+            nbytes = meta.numel() * 4
         ten = _Tensors(sparse_idx=_ptr(idx), sparse_count=_ptr(cnt), cu_seqlens_q=_ptr(cu),
                        seqused_q=_ptr(squ), seqused_kv=_ptr(sku))
         _check(_load().gbsa_metadata(ctypes.byref(prob.as_c()), ctypes.byref(ten),
