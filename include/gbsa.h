@@ -165,6 +165,35 @@ GBSA_API gbsa_status gbsa_forward(const gbsa_problem* problem, const gbsa_tensor
                          const void* meta, void* workspace, size_t ws_bytes,
                          int32_t* dev_status, void* stream);
 
+/* Size of the device scratch that gbsa_forward_static_scratch() uses. */
+#define GBSA_STATIC_SCRATCH_BYTES ((size_t)32 << 20)
+
+/* gbsa_forward() for callers that cannot allocate device memory (the paper
+ * has no counterpart: this is a library addition).  Some hosts hand out a
+ * fixed device-memory budget at start-up and forbid any allocation later,
+ * and code that runs inside an allocator or a framework hook cannot call
+ * cudaMalloc without risking a deadlock; such callers have no way to provide
+ * the workspace gbsa_forward() asks for.  Here the split-KV scratch is a
+ * GBSA_STATIC_SCRATCH_BYTES array that the library's CUDA module holds on
+ * every GPU that loads it, until the process exits; nothing is allocated,
+ * and the caller still passes inputs, outputs and the metadata.
+ *   - Limit: problems whose gbsa_workspace_size() exceeds
+ *     GBSA_STATIC_SCRATCH_BYTES are rejected with GBSA_ERR_WORKSPACE_TOO_SMALL
+ *     before anything is launched (decode-shaped problems fit; prefill-shaped
+ *     ones need gbsa_forward() with a caller-provided workspace).
+ *   - The first call on a device looks up the array's device address; make
+ *     that first call before any stream capture on that device.
+ *   - Every call on a device shares the one array, which keeps the last
+ *     call's contents (nothing in it needs to start at zero: every partial the
+ *     merge reads is written earlier in the same call).  Calls whose work
+ *     overlaps on the GPU (other streams, other host threads) race on it:
+ *     order them on one stream or with events.
+ * Everything else -- arguments, layouts, errors, dev_status -- is as for
+ * gbsa_forward(). */
+GBSA_API gbsa_status gbsa_forward_static_scratch(const gbsa_problem* problem,
+                                                 const gbsa_tensors* tensors, const void* meta,
+                                                 int32_t* dev_status, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
