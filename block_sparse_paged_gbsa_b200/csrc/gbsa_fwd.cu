@@ -128,17 +128,12 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Bars* b
   }
 }
 
-__device__ __forceinline__ uint64_t desc_k_major(uint32_t tile_addr, int kk) {
-  // K step kk covers 16 bf16 (32 bytes); 64-column halves are 16 KiB apart.
-  return smem_desc_sw128(tile_addr + (kk >> 2) * kHalfBytes + (kk & 3) * 32, 16, 1024);
-}
-
-__device__ __forceinline__ uint64_t desc_v_mn_major(uint32_t tile_addr, int kk) {
-  // K step kk covers 16 keys = 16 rows of 128 B; the two 64-column halves
-  // of D are 16 KiB apart (leading byte offset), 8-row groups 1 KiB apart.
-  return smem_desc_sw128(tile_addr + kk * 2048, kHalfBytes, 1024);
-}
-
+// Operand layouts in shared memory (128-byte swizzle, tiles 1 KiB aligned):
+//   Q and K tiles, K-major: 128 rows x 128 B per 64-column half, halves
+//   16 KiB apart; a K step of 16 bf16 advances 32 B inside the row.
+//   V tile, MN-major (N = D): the two 64-column halves of D 16 KiB apart
+//   (leading byte offset), 8-key groups 1 KiB apart; a K step of 16 keys
+//   advances 2 KiB.
 // ---------------------------------------------------------------------------
 // producer (one thread)
 // ---------------------------------------------------------------------------
@@ -201,93 +196,147 @@ __device__ void run_producer(const FwdParams& p, const CUtensorMap* map_q, const
 }
 
 // ---------------------------------------------------------------------------
-// MMA issuer (warp 1; lane 0 issues, the warp zeroes stale V rows)
+// MMA issuer (warp 1; lane 0 waits and issues, the warp zeroes stale V rows)
+//
+// Issue order for a two-tile unit with blocks 0..n-1 (tcgen05 MMAs of a CTA
+// execute in issue order, so an S written after the PV that reads the P
+// aliased on it needs no wait):
+//     S0_0, S1_0, PV0_0,
+//     for i >= 1:  S0_i, PV1_{i-1}, S1_i, PV0_i,
+//     PV1_{n-1}.
+// While softmax 0 works on S0_i the tensor pipe runs PV1_{i-1} and S1_i, and
+// while softmax 1 works on S1_i it runs PV0_i and S0_{i+1}.  K_i is released
+// after S1_i, V_i after PV1_i, which keeps the ring in fill order.
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Bars* bars) {
+  int ok = 1;
+  if (lane_id() == 0) ok = wait_bar(bar, parity, bars) ? 1 : 0;
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+// Low word of a descriptor holds (address >> 4) in its first 14 bits; tile
+// offsets are added there (addresses stay below 256 KiB, so no carry).
+__device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
+
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint64_t q_desc, uint64_t k_desc) {
+#pragma unroll
+  for (int kk = 0; kk < 8; kk++) {
+    const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+    mma_ss(d_tmem, desc_add(q_desc, off), desc_add(k_desc, off), kIdescQK, kk > 0 ? 1u : 0u);
+  }
+}
+
+__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint64_t v_desc,
+                                         bool accumulate) {
+#pragma unroll
+  for (int kk = 0; kk < 8; kk++)
+    mma_ts(d_tmem, p_tmem + kk * 8, desc_add(v_desc, kk * 2048), kIdescPV,
+           (accumulate || kk > 0) ? 1u : 0u);
+}
+
 __device__ void run_mma(const FwdParams& p, uint8_t* smem, Bars* bars, uint32_t tmem,
                         int32_t n_units, int64_t off_unit, int64_t off_item, int64_t off_list) {
   const uint32_t lane = lane_id();
   uint32_t kv_iter = 0, q_iter = 0;
-  uint32_t blk_iter[2] = {0, 0}, unit_iter[2] = {0, 0};
+  uint32_t blk0 = 0, blk1 = 0;      // blocks processed per tile slot (p_full / o_done phases)
+  uint32_t units0 = 0, units1 = 0;  // units processed per tile slot (o_free phases)
   bool ok = true;
   const uint32_t q_addr = smem_u32(smem + kSmemQ);
   const uint32_t ring_addr = smem_u32(smem + kSmemRing);
+  const uint64_t q0_desc = smem_desc_sw128(q_addr, 16, 1024);
+  const uint64_t q1_desc = smem_desc_sw128(q_addr + kTileBytes, 16, 1024);
+  const uint64_t k_desc0 = smem_desc_sw128(ring_addr, 16, 1024);
+  const uint64_t v_desc0 = smem_desc_sw128(ring_addr, kHalfBytes, 1024);
+  const uint32_t s0 = tmem, s1 = tmem + 128, o0 = tmem + 256, o1 = tmem + 384;
+
   for (int32_t u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
     const Unit x = load_unit(p.meta, off_unit, off_item, u, p.N2);
-    const int32_t nblk = x.j1 - x.j0;
-    if (nblk > 0) {
-      if (lane == 0) ok = wait_bar(&bars->q_full, q_iter & 1, bars);
-      ok = __shfl_sync(0xffffffffu, ok, 0);
+    const int32_t n = x.j1 - x.j0;
+    const bool two = x.nt == 2;
+    if (n > 0) {
+      if (!(ok = warp_wait(&bars->q_full, q_iter & 1, bars))) break;
       q_iter++;
       const int32_t* list = p.meta + off_list + (int64_t)x.item * p.top_k;
-      for (int32_t jb = 0; jb < nblk && ok; jb++) {
-        // ---- S = Q K^T for every tile of the unit
-        uint32_t stage = kv_iter % kStages;
+      const uint32_t kv0 = kv_iter;
+      for (int32_t i = 0; i < n && ok; i++) {
+        const uint32_t ki = kv0 + 2 * i, vi = ki + 1;
+        const uint32_t ks = ki % kStages, vs = vi % kStages;
+        // ---- S0_i
+        if (!(ok = warp_wait(&bars->kv_full[ks], (ki / kStages) & 1, bars))) break;
         if (lane == 0) {
-          ok = wait_bar(&bars->kv_full[stage], (kv_iter / kStages) & 1, bars);
           tc_fence_after_sync();
-          for (int s = 0; s < x.nt && ok; s++) {
-            if (blk_iter[s] > 0) ok = wait_bar(&bars->o_done[s], (blk_iter[s] - 1) & 1, bars);
-            if (!ok) break;
-            tc_fence_after_sync();
-            const uint32_t qa = q_addr + s * kTileBytes, ka = ring_addr + stage * kTileBytes;
-#pragma unroll
-            for (int kk = 0; kk < 8; kk++)
-              mma_ss(tmem + 128 * s, desc_k_major(qa, kk), desc_k_major(ka, kk), kIdescQK, kk > 0);
-            tc_commit(&bars->s_full[s]);
+          issue_qk(s0, q0_desc, desc_add(k_desc0, ks * kTileBytes));
+          tc_commit(&bars->s_full[0]);
+        }
+        if (two) {
+          // ---- PV1_{i-1}
+          if (i > 0) {
+            if (i == 1 && units1 > 0)
+              if (!(ok = warp_wait(&bars->o_free[1], (units1 - 1) & 1, bars))) break;
+            if (!(ok = warp_wait(&bars->p_full[1], blk1 & 1, bars))) break;
+            if (lane == 0) {
+              tc_fence_after_sync();
+              const uint32_t pvs = (vi - 2) % kStages;
+              issue_pv(o1, s1, desc_add(v_desc0, pvs * kTileBytes), i - 1 > 0);
+              tc_commit(&bars->o_done[1]);
+              tc_commit(&bars->kv_empty[pvs]);
+            }
+            blk1++;
           }
-          if (ok) {
-            tc_commit(&bars->kv_empty[stage]);
-            if (jb == nblk - 1) tc_commit(&bars->q_empty);
+          // ---- S1_i
+          if (lane == 0) {
+            issue_qk(s1, q1_desc, desc_add(k_desc0, ks * kTileBytes));
+            tc_commit(&bars->s_full[1]);
           }
         }
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok) break;
-        kv_iter++;
-        // ---- O += P V
-        stage = kv_iter % kStages;
-        if (lane == 0) ok = wait_bar(&bars->kv_full[stage], (kv_iter / kStages) & 1, bars);
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok) break;
-        const int32_t entry = list[x.j0 + jb];
+        if (lane == 0) {
+          tc_commit(&bars->kv_empty[ks]);
+          if (i == n - 1) tc_commit(&bars->q_empty);
+        }
+        // ---- V_i: zero the rows of a last page past seqused_kv
+        if (!(ok = warp_wait(&bars->kv_full[vs], (vi / kStages) & 1, bars))) break;
+        const int32_t entry = list[x.j0 + i];
         if (entry & kEntryPartial) {
-          // keys >= seqused_kv of the last page: zero those V rows (both halves)
           const int32_t r0 = min(max(x.ku - (entry & kEntryLbMask) * kPage, 0), kPage);
-          uint8_t* vt = smem + kSmemRing + stage * kTileBytes;
+          uint8_t* vt = smem + kSmemRing + vs * kTileBytes;
           const int32_t n16 = (kPage - r0) * 16;
-          for (int32_t i = lane; i < n16; i += 32) {
-            const int32_t row = r0 + (i >> 4), chunk = i & 15;
+          for (int32_t t = lane; t < n16; t += 32) {
+            const int32_t row = r0 + (t >> 4), chunk = t & 15;
             *reinterpret_cast<uint4*>(vt + (chunk >> 3) * kHalfBytes + row * 128 + (chunk & 7) * 16) =
                 make_uint4(0, 0, 0, 0);
           }
           fence_proxy_async_smem();
           __syncwarp();
         }
+        // ---- PV0_i
+        if (i == 0 && units0 > 0)
+          if (!(ok = warp_wait(&bars->o_free[0], (units0 - 1) & 1, bars))) break;
+        if (!(ok = warp_wait(&bars->p_full[0], blk0 & 1, bars))) break;
         if (lane == 0) {
           tc_fence_after_sync();
-          for (int s = 0; s < x.nt && ok; s++) {
-            if (jb == 0 && unit_iter[s] > 0)
-              ok = wait_bar(&bars->o_free[s], (unit_iter[s] - 1) & 1, bars);
-            if (ok) ok = wait_bar(&bars->p_full[s], blk_iter[s] & 1, bars);
-            if (!ok) break;
-            tc_fence_after_sync();
-            const uint32_t va = ring_addr + stage * kTileBytes;
-            const uint32_t p_tmem = tmem + 128 * s;
-#pragma unroll
-            for (int kk = 0; kk < 8; kk++)
-              mma_ts(tmem + 256 + 128 * s, p_tmem + kk * 8, desc_v_mn_major(va, kk), kIdescPV,
-                     (jb > 0 || kk > 0) ? 1u : 0u);
-            tc_commit(&bars->o_done[s]);
-            blk_iter[s]++;
-          }
-          if (ok) tc_commit(&bars->kv_empty[stage]);
+          issue_pv(o0, s0, desc_add(v_desc0, vs * kTileBytes), i > 0);
+          tc_commit(&bars->o_done[0]);
+          if (!two) tc_commit(&bars->kv_empty[vs]);
         }
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        blk_iter[0] = __shfl_sync(0xffffffffu, blk_iter[0], 0);
-        blk_iter[1] = __shfl_sync(0xffffffffu, blk_iter[1], 0);
-        kv_iter++;
+        blk0++;
       }
+      // ---- PV1_{n-1}
+      if (ok && two) {
+        if (n == 1 && units1 > 0) ok = warp_wait(&bars->o_free[1], (units1 - 1) & 1, bars);
+        if (ok) ok = warp_wait(&bars->p_full[1], blk1 & 1, bars);
+        if (ok && lane == 0) {
+          tc_fence_after_sync();
+          const uint32_t pvs = (kv0 + 2 * n - 1) % kStages;
+          issue_pv(o1, s1, desc_add(v_desc0, pvs * kTileBytes), n - 1 > 0);
+          tc_commit(&bars->o_done[1]);
+          tc_commit(&bars->kv_empty[pvs]);
+        }
+        blk1++;
+      }
+      kv_iter = kv0 + 2 * n;
     }
-    for (int s = 0; s < x.nt; s++) unit_iter[s]++;
+    units0++;
+    if (two) units1++;
   }
   // all MMAs issued by this thread complete before TMEM is released
   if (lane == 0) {
@@ -341,7 +390,8 @@ __device__ void run_softmax(const FwdParams& p, Bars* bars, uint32_t tmem, int s
       reg_fence(r[1]);
       reg_fence(r[2]);
       reg_fence(r[3]);
-      // visible key columns of this block for this row: [clo, chi]
+      // visible key columns of this block for this row: [clo, chi]; the
+      // element mask runs only in warps that hold a row needing it
       int32_t clo = 0, chi = kPage - 1;
       if (!row_used) {
         clo = kPage;
@@ -351,13 +401,16 @@ __device__ void run_softmax(const FwdParams& p, Bars* bars, uint32_t tmem, int s
         clo = key_lo == INT32_MIN ? 0 : max(key_lo - base, 0);
         chi = min(key_hi - base, kPage - 1);
       }
+      if (__any_sync(0xffffffffu, clo > 0 || chi < kPage - 1)) {
+#pragma unroll
+        for (int c = 0; c < 128; c++)
+          if (c < clo || c > chi) r[c >> 5][c & 31] = __float_as_uint(-INFINITY);
+      }
       float mx = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 128; c++) {
-        const float v = (c >= clo && c <= chi) ? __uint_as_float(r[c >> 5][c & 31]) : -INFINITY;
-        r[c >> 5][c & 31] = __float_as_uint(v);
-        mx = fmaxf(mx, v);
-      }
+      for (int c = 0; c < 128; c += 2)
+        mx = fmaxf(mx, fmaxf(__uint_as_float(r[c >> 5][c & 31]),
+                             __uint_as_float(r[(c + 1) >> 5][(c + 1) & 31])));
       const float m_blk = mx * p.scale_log2;
       const float m_new = fmaxf(m, m_blk);
       // lazy rescale: keep the old reference max unless it grew by > 8 (P <= 256)
@@ -378,8 +431,9 @@ __device__ void run_softmax(const FwdParams& p, Bars* bars, uint32_t tmem, int s
           const int c = half * 64 + 2 * i;
           const float s0 = __uint_as_float(r[c >> 5][c & 31]);
           const float s1 = __uint_as_float(r[(c + 1) >> 5][(c + 1) & 31]);
-          const float p0 = s0 == -INFINITY ? 0.f : fast_exp2(fmaf(s0, p.scale_log2, neg_m));
-          const float p1 = s1 == -INFINITY ? 0.f : fast_exp2(fmaf(s1, p.scale_log2, neg_m));
+          // masked scores are -inf and ex2(-inf) = +0
+          const float p0 = fast_exp2(fmaf(s0, p.scale_log2, neg_m));
+          const float p1 = fast_exp2(fmaf(s1, p.scale_log2, neg_m));
           sum += p0 + p1;
           pk[i] = pack_bf16x2(p0, p1);
         }
