@@ -9,14 +9,14 @@
 // blog (ai6s.net), "three steps": running max, running sum and a rescale of
 // the partial output, so the score matrix never exists.
 //
-// Design (one persistent CTA per SM, 384 threads):
-//   warp 0       TMA producer: Q tiles (2 per unit) and, per selected block,
-//                the K and V pages into a 5-stage ring of 32 KiB buffers;
-//   warp 1       MMA issuer: S = Q K^T (SS MMA) and O += P V (TS MMA, P read
-//                from TMEM); zeroes the rows of a last page past seqused_kv
-//                in the V buffer so that stale values cannot reach O;
-//   warps 4..7   softmax + epilogue of tile 0 (TMEM lanes = tile rows);
-//   warps 8..11  softmax + epilogue of tile 1.
+// Design (one persistent CTA per SM, 512 threads, four warpgroups):
+//   warps 0..3    softmax of tile 0 (TMEM lanes = tile rows)
+//   warps 4..7    softmax of tile 1
+//   warps 8..11   epilogue: O / l -> out (bf16) and lse, or split partials
+//   warp 12       MMA issuer: S = Q K^T (SS MMA), O += P V (TS MMA, P read
+//                 from TMEM); zeroes V rows of a last page past seqused_kv
+//   warp 13       TMA producer: Q tiles and, per live block, the K and V
+//                 pages into a 5-stage ring of 32 KiB buffers
 // TMEM (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each; P (bf16,
 // packed in pairs) overwrites the first 64 columns of its S.
 // Units come from the metadata work list, longest first; CTA c takes units
@@ -37,22 +37,24 @@ using namespace sm100;
 
 namespace {
 
-constexpr int kThreads = 384;
-// Register split: launched with kLaunchRegs per thread (384 threads); the
-// producer/MMA warpgroup gives registers to the two softmax warpgroups.
-constexpr int kLaunchRegs = 168;
-constexpr int kRegsControl = 56;
-constexpr int kRegsSoftmax = 224;
-static_assert(128 * kRegsControl + 256 * kRegsSoftmax <= kLaunchRegs * kThreads,
+constexpr int kThreads = 512;
+// Register split: launched with kLaunchRegs per thread; the epilogue and
+// control warpgroups give registers to the two softmax warpgroups.
+constexpr int kLaunchRegs = 128;
+constexpr int kRegsSoftmax = 184;   // warpgroups 0, 1
+constexpr int kRegsEpilogue = 80;   // warpgroup 2
+constexpr int kRegsControl = 64;    // warpgroup 3 (MMA, producer)
+static_assert(256 * kRegsSoftmax + 128 * kRegsEpilogue + 128 * kRegsControl <=
+                  kLaunchRegs * kThreads,
               "register split exceeds the launch allocation");
+constexpr int kWarpMma = 12;
+constexpr int kWarpProducer = 13;
 constexpr int kStages = 5;
 constexpr int kTileBytes = 32768;  // 128 rows x 128 bf16 (two 64-column SW128 boxes)
 constexpr int kHalfBytes = 16384;
 constexpr int kSmemQ = 0;
 constexpr int kSmemRing = 2 * kTileBytes;
 constexpr int kSmemBars = kSmemRing + kStages * kTileBytes;
-constexpr int kSmemBytes = kSmemBars + 1024;
-constexpr int kSmemAlloc = kSmemBytes + 1024;  // slack for the 1024-byte alignment
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
 constexpr float kRescaleThreshold = 8.0f;  // log2 of the largest allowed P (256)
 constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, false, false);
@@ -73,17 +75,25 @@ struct FwdParams {
 };
 
 struct Bars {
-  uint64_t q_full, q_empty;
+  uint64_t q_full[2], q_empty[2];
   uint64_t kv_full[kStages], kv_empty[kStages];
-  uint64_t s_full[2], p_full[2], o_done[2], o_free[2];
+  uint64_t s_full[2];      // S of a block ready (MMA commit)
+  uint64_t p_full[2];      // P of a block in TMEM, O rescaled (128 softmax threads)
+  uint64_t o_final[2];     // last PV of a unit complete (MMA commit)
+  uint64_t o_free[2];      // epilogue has read O (128 epilogue threads)
+  uint64_t stats_full[2];  // row max / sum of a unit in `stats` (128 softmax threads)
+  uint64_t stats_free[2];  // epilogue has read them (128 epilogue threads)
   uint64_t drain;
   uint32_t tmem_base;
   int32_t abort;
+  float2 stats[2][128];    // (reference max in log2 units, row sum) per tile row
 };
+constexpr int kSmemBytes = kSmemBars + (int)sizeof(Bars);
+static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 struct Unit {
   int32_t item, tp, j0, j1, slot;
-  int32_t b, n_live, n_tiles, tok_begin, n_store, n_used, pos0, ku;
+  int32_t b, n_tiles, tok_begin, n_store, n_used, pos0, ku;
   int32_t kvh, nt;  // KV head, tiles in this unit (1 or 2)
 };
 
@@ -99,7 +109,6 @@ __device__ __forceinline__ Unit load_unit(const int32_t* meta, int64_t off_unit,
   const int4 a = *reinterpret_cast<const int4*>(meta + off_item + 8 * (int64_t)x.item);
   const int4 c = *reinterpret_cast<const int4*>(meta + off_item + 8 * (int64_t)x.item + 4);
   x.b = a.x;
-  x.n_live = a.y;
   x.n_tiles = a.z;
   x.tok_begin = a.w;
   x.n_store = c.x;
@@ -134,30 +143,73 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Bars* b
 //   V tile, MN-major (N = D): the two 64-column halves of D 16 KiB apart
 //   (leading byte offset), 8-key groups 1 KiB apart; a K step of 16 keys
 //   advances 2 KiB.
+
+// Row identity of TMEM lane `row` in tile `slot` of unit x.
+struct RowInfo {
+  bool store;   // row holds a stored query token of this unit (out is written)
+  bool used;    // ... and the token is used (t < seqused_q)
+  int32_t tok;  // global token index
+  int32_t h;    // query head
+  int32_t pos;  // query position (bottom-right aligned causal)
+};
+
+__device__ __forceinline__ RowInfo row_info(const FwdParams& p, const Unit& x, int slot, int row) {
+  RowInfo r;
+  const int rows_in_tile = p.tile_tokens * p.G;
+  const int tok_in_tile = row / p.G;
+  const int32_t tok_off = (2 * x.tp + slot) * p.tile_tokens + tok_in_tile;
+  r.store = row < rows_in_tile && tok_off < x.n_store;
+  r.used = r.store && tok_off < x.n_used;
+  r.tok = x.tok_begin + tok_off;
+  r.h = x.kvh * p.G + (row - tok_in_tile * p.G);
+  r.pos = x.pos0 + tok_off;
+  return r;
+}
+
 // ---------------------------------------------------------------------------
 // producer (one thread)
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ bool produce_kv(const CUtensorMap* map, uint8_t* smem, Bars* bars,
+                                           uint32_t& kv_iter, int32_t kvh, int32_t page) {
+  const uint32_t stage = kv_iter % kStages;
+  if (kv_iter >= kStages && !wait_bar(&bars->kv_empty[stage], ((kv_iter / kStages) & 1) ^ 1, bars))
+    return false;
+  uint8_t* dst = smem + kSmemRing + stage * kTileBytes;
+  mbar_arrive_expect_tx(&bars->kv_full[stage], kTileBytes);
+  tma_load_4d(dst, map, &bars->kv_full[stage], 0, kvh, 0, page);
+  tma_load_4d(dst + kHalfBytes, map, &bars->kv_full[stage], 64, kvh, 0, page);
+  kv_iter++;
+  return true;
+}
+
+__device__ __forceinline__ bool produce_q(const FwdParams& p, const CUtensorMap* map_q,
+                                          uint8_t* smem, Bars* bars, uint32_t& q_iter,
+                                          const Unit& x, int s) {
+  if (q_iter > 0 && !wait_bar(&bars->q_empty[s], (q_iter - 1) & 1, bars)) return false;
+  const uint32_t box_bytes = 128u * (uint32_t)p.G * (uint32_t)p.tile_tokens;
+  const int32_t tok = x.tok_begin + (2 * x.tp + s) * p.tile_tokens;
+  uint8_t* dst = smem + kSmemQ + s * kTileBytes;
+  mbar_arrive_expect_tx(&bars->q_full[s], 2u * box_bytes);
+  tma_load_3d(dst, map_q, &bars->q_full[s], 0, x.kvh * p.G, tok);
+  tma_load_3d(dst + kHalfBytes, map_q, &bars->q_full[s], 64, x.kvh * p.G, tok);
+  q_iter++;
+  return true;
+}
+
 __device__ void run_producer(const FwdParams& p, const CUtensorMap* map_q, const CUtensorMap* map_k,
                              const CUtensorMap* map_v, uint8_t* smem, Bars* bars, int32_t n_units,
                              int64_t off_unit, int64_t off_item, int64_t off_list) {
-  uint32_t kv_iter = 0, q_iter = 0;
+  uint32_t kv_iter = 0, q_iter0 = 0, q_iter1 = 0;
   int32_t bad = 0;
   bool ok = true;
-  const uint32_t q_box_bytes = 128u * (uint32_t)p.G * (uint32_t)p.tile_tokens;
   for (int32_t u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
     const Unit x = load_unit(p.meta, off_unit, off_item, u, p.N2);
     if (x.j1 <= x.j0) continue;
-    if (q_iter > 0 && !(ok = wait_bar(&bars->q_empty, (q_iter - 1) & 1, bars))) break;
-    mbar_arrive_expect_tx(&bars->q_full, (uint32_t)x.nt * 2u * q_box_bytes);
-    for (int s = 0; s < x.nt; s++) {
-      const int32_t tok = x.tok_begin + (2 * x.tp + s) * p.tile_tokens;
-      uint8_t* dst = smem + kSmemQ + s * kTileBytes;
-      tma_load_3d(dst, map_q, &bars->q_full, 0, x.kvh * p.G, tok);
-      tma_load_3d(dst + kHalfBytes, map_q, &bars->q_full, 64, x.kvh * p.G, tok);
-    }
-    q_iter++;
     const int32_t* list = p.meta + off_list + (int64_t)x.item * p.top_k;
     const int32_t* bt = p.block_table + (int64_t)x.b * p.max_pages;
+    // order: Q0, K_0, Q1, V_0, K_1, V_1, ... (Q1 of a unit waits for the
+    // previous unit's last S1, which comes later than its last S0)
+    ok = produce_q(p, map_q, smem, bars, q_iter0, x, 0);
     for (int32_t j = x.j0; j < x.j1 && ok; j++) {
       const int32_t lb = list[j] & kEntryLbMask;
       int32_t page = lb < p.max_pages ? bt[lb] : -1;
@@ -165,18 +217,9 @@ __device__ void run_producer(const FwdParams& p, const CUtensorMap* map_q, const
         bad |= kDevBadPage;
         page = 0;
       }
-      for (int kv = 0; kv < 2; kv++) {
-        const uint32_t stage = kv_iter % kStages;
-        if (kv_iter >= kStages &&
-            !(ok = wait_bar(&bars->kv_empty[stage], ((kv_iter / kStages) & 1) ^ 1, bars)))
-          break;
-        uint8_t* dst = smem + kSmemRing + stage * kTileBytes;
-        const CUtensorMap* map = kv ? map_v : map_k;
-        mbar_arrive_expect_tx(&bars->kv_full[stage], kTileBytes);
-        tma_load_4d(dst, map, &bars->kv_full[stage], 0, x.kvh, 0, page);
-        tma_load_4d(dst + kHalfBytes, map, &bars->kv_full[stage], 64, x.kvh, 0, page);
-        kv_iter++;
-      }
+      ok = produce_kv(map_k, smem, bars, kv_iter, x.kvh, page);
+      if (ok && j == x.j0 && x.nt == 2) ok = produce_q(p, map_q, smem, bars, q_iter1, x, 1);
+      if (ok) ok = produce_kv(map_v, smem, bars, kv_iter, x.kvh, page);
     }
   }
   if (bad && p.dev_status) atomicOr(p.dev_status, bad);
@@ -188,15 +231,19 @@ __device__ void run_producer(const FwdParams& p, const CUtensorMap* map_q, const
              global_timer_ns() - t0 < kWaitLimitNs) {
       }
     }
-    if (q_iter > 0)
-      while (!mbar_try_wait(&bars->q_full, (q_iter - 1) & 1) &&
+    if (q_iter0 > 0)
+      while (!mbar_try_wait(&bars->q_full[0], (q_iter0 - 1) & 1) &&
+             global_timer_ns() - t0 < kWaitLimitNs) {
+      }
+    if (q_iter1 > 0)
+      while (!mbar_try_wait(&bars->q_full[1], (q_iter1 - 1) & 1) &&
              global_timer_ns() - t0 < kWaitLimitNs) {
       }
   }
 }
 
 // ---------------------------------------------------------------------------
-// MMA issuer (warp 1; lane 0 waits and issues, the warp zeroes stale V rows)
+// MMA issuer (one warp; lane 0 waits and issues, the warp zeroes stale V rows)
 //
 // Issue order for a two-tile unit with blocks 0..n-1 (tcgen05 MMAs of a CTA
 // execute in issue order, so an S written after the PV that reads the P
@@ -214,90 +261,108 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Bars* 
   return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
-// Low word of a descriptor holds (address >> 4) in its first 14 bits; tile
-// offsets are added there (addresses stay below 256 KiB, so no carry).
-__device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
-
-__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint64_t q_desc, uint64_t k_desc) {
-#pragma unroll
+// Descriptors are handled as 32-bit low words (start address >> 4 in bits
+// [0,14), leading byte offset >> 4 in [16,30)) plus the shared high word;
+// offsets are added to the low word (addresses stay below 256 KiB: no carry).
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_lo, uint32_t k_lo,
+                                         uint32_t hi) {
+#pragma unroll 4
   for (int kk = 0; kk < 8; kk++) {
-    const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-    mma_ss(d_tmem, desc_add(q_desc, off), desc_add(k_desc, off), kIdescQK, kk > 0 ? 1u : 0u);
+    const uint32_t off = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
+    mma_ss_lo(d_tmem, q_lo + off, k_lo + off, hi, kIdescQK, kk > 0 ? 1u : 0u);
   }
 }
 
-__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint64_t v_desc,
-                                         bool accumulate) {
-#pragma unroll
+__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_lo,
+                                         uint32_t hi, bool accumulate) {
+#pragma unroll 4
   for (int kk = 0; kk < 8; kk++)
-    mma_ts(d_tmem, p_tmem + kk * 8, desc_add(v_desc, kk * 2048), kIdescPV,
-           (accumulate || kk > 0) ? 1u : 0u);
+    mma_ts_lo(d_tmem, p_tmem + kk * 8, v_lo + ((kk * 2048) >> 4), hi, kIdescPV,
+              (accumulate || kk > 0) ? 1u : 0u);
 }
+
+// Position in the K/V ring: stage index and the parity of its current fill.
+struct RingPos {
+  uint32_t stage, phase;
+  __device__ __forceinline__ void advance() {
+    if (++stage == kStages) {
+      stage = 0;
+      phase ^= 1u;
+    }
+  }
+};
 
 __device__ void run_mma(const FwdParams& p, uint8_t* smem, Bars* bars, uint32_t tmem,
                         int32_t n_units, int64_t off_unit, int64_t off_item, int64_t off_list) {
   const uint32_t lane = lane_id();
-  uint32_t kv_iter = 0, q_iter = 0;
-  uint32_t blk0 = 0, blk1 = 0;      // blocks processed per tile slot (p_full / o_done phases)
-  uint32_t units0 = 0, units1 = 0;  // units processed per tile slot (o_free phases)
+  uint32_t q_iter0 = 0, q_iter1 = 0;
+  uint32_t blk0 = 0, blk1 = 0;      // blocks per tile slot (p_full phases)
+  uint32_t units0 = 0, units1 = 0;  // units per tile slot (o_free phases)
+  RingPos rp{0, 0};                 // next K/V tile to consume
   bool ok = true;
   const uint32_t q_addr = smem_u32(smem + kSmemQ);
   const uint32_t ring_addr = smem_u32(smem + kSmemRing);
-  const uint64_t q0_desc = smem_desc_sw128(q_addr, 16, 1024);
-  const uint64_t q1_desc = smem_desc_sw128(q_addr + kTileBytes, 16, 1024);
-  const uint64_t k_desc0 = smem_desc_sw128(ring_addr, 16, 1024);
-  const uint64_t v_desc0 = smem_desc_sw128(ring_addr, kHalfBytes, 1024);
-  const uint32_t s0 = tmem, s1 = tmem + 128, o0 = tmem + 256, o1 = tmem + 384;
+  const uint64_t d0 = smem_desc_sw128(q_addr, 16, 1024);
+  const uint32_t hi = (uint32_t)(d0 >> 32);
+  const uint32_t q0_lo = (uint32_t)d0;
+  const uint32_t q1_lo = q0_lo + (kTileBytes >> 4);
+  const uint32_t k_lo0 = (uint32_t)smem_desc_sw128(ring_addr, 16, 1024);
+  const uint32_t v_lo0 = (uint32_t)smem_desc_sw128(ring_addr, kHalfBytes, 1024);
+  constexpr uint32_t kStageLo = kTileBytes >> 4;
 
   for (int32_t u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-    const Unit x = load_unit(p.meta, off_unit, off_item, u, p.N2);
-    const int32_t n = x.j1 - x.j0;
-    const bool two = x.nt == 2;
+    const int4 rec = *reinterpret_cast<const int4*>(p.meta + off_unit + 4 * (int64_t)u);
+    const int32_t item = rec.x, j0 = rec.z & 0xffff, n = (int32_t)((uint32_t)rec.z >> 16) - j0;
+    const int4 irow = *reinterpret_cast<const int4*>(p.meta + off_item + 8 * (int64_t)item);
+    const int32_t ku = p.meta[off_item + 8 * (int64_t)item + 7];
+    const bool two = irow.z - 2 * rec.y >= 2;
     if (n > 0) {
-      if (!(ok = warp_wait(&bars->q_full, q_iter & 1, bars))) break;
-      q_iter++;
-      const int32_t* list = p.meta + off_list + (int64_t)x.item * p.top_k;
-      const uint32_t kv0 = kv_iter;
+      if (!(ok = warp_wait(&bars->q_full[0], q_iter0 & 1, bars))) break;
+      q_iter0++;
+      const int32_t* list = p.meta + off_list + (int64_t)item * p.top_k + j0;
+      uint32_t prev_vs = 0;
       for (int32_t i = 0; i < n && ok; i++) {
-        const uint32_t ki = kv0 + 2 * i, vi = ki + 1;
-        const uint32_t ks = ki % kStages, vs = vi % kStages;
         // ---- S0_i
-        if (!(ok = warp_wait(&bars->kv_full[ks], (ki / kStages) & 1, bars))) break;
+        const uint32_t ks = rp.stage;
+        if (!(ok = warp_wait(&bars->kv_full[ks], rp.phase, bars))) break;
+        rp.advance();
         if (lane == 0) {
           tc_fence_after_sync();
-          issue_qk(s0, q0_desc, desc_add(k_desc0, ks * kTileBytes));
+          issue_qk(tmem, q0_lo, k_lo0 + ks * kStageLo, hi);
           tc_commit(&bars->s_full[0]);
+          if (i == n - 1) tc_commit(&bars->q_empty[0]);
         }
         if (two) {
-          // ---- PV1_{i-1}
-          if (i > 0) {
+          if (i == 0) {
+            if (!(ok = warp_wait(&bars->q_full[1], q_iter1 & 1, bars))) break;
+            q_iter1++;
+          } else {
+            // ---- PV1_{i-1}
             if (i == 1 && units1 > 0)
               if (!(ok = warp_wait(&bars->o_free[1], (units1 - 1) & 1, bars))) break;
             if (!(ok = warp_wait(&bars->p_full[1], blk1 & 1, bars))) break;
             if (lane == 0) {
               tc_fence_after_sync();
-              const uint32_t pvs = (vi - 2) % kStages;
-              issue_pv(o1, s1, desc_add(v_desc0, pvs * kTileBytes), i - 1 > 0);
-              tc_commit(&bars->o_done[1]);
-              tc_commit(&bars->kv_empty[pvs]);
+              issue_pv(tmem + 384, tmem + 128, v_lo0 + prev_vs * kStageLo, hi, i - 1 > 0);
+              tc_commit(&bars->kv_empty[prev_vs]);
             }
             blk1++;
           }
           // ---- S1_i
           if (lane == 0) {
-            issue_qk(s1, q1_desc, desc_add(k_desc0, ks * kTileBytes));
+            issue_qk(tmem + 128, q1_lo, k_lo0 + ks * kStageLo, hi);
             tc_commit(&bars->s_full[1]);
+            if (i == n - 1) tc_commit(&bars->q_empty[1]);
           }
         }
-        if (lane == 0) {
-          tc_commit(&bars->kv_empty[ks]);
-          if (i == n - 1) tc_commit(&bars->q_empty);
-        }
+        if (lane == 0) tc_commit(&bars->kv_empty[ks]);
         // ---- V_i: zero the rows of a last page past seqused_kv
-        if (!(ok = warp_wait(&bars->kv_full[vs], (vi / kStages) & 1, bars))) break;
-        const int32_t entry = list[x.j0 + i];
+        const uint32_t vs = rp.stage;
+        if (!(ok = warp_wait(&bars->kv_full[vs], rp.phase, bars))) break;
+        rp.advance();
+        const int32_t entry = list[i];
         if (entry & kEntryPartial) {
-          const int32_t r0 = min(max(x.ku - (entry & kEntryLbMask) * kPage, 0), kPage);
+          const int32_t r0 = min(max(ku - (entry & kEntryLbMask) * kPage, 0), kPage);
           uint8_t* vt = smem + kSmemRing + vs * kTileBytes;
           const int32_t n16 = (kPage - r0) * 16;
           for (int32_t t = lane; t < n16; t += 32) {
@@ -314,11 +379,12 @@ __device__ void run_mma(const FwdParams& p, uint8_t* smem, Bars* bars, uint32_t 
         if (!(ok = warp_wait(&bars->p_full[0], blk0 & 1, bars))) break;
         if (lane == 0) {
           tc_fence_after_sync();
-          issue_pv(o0, s0, desc_add(v_desc0, vs * kTileBytes), i > 0);
-          tc_commit(&bars->o_done[0]);
+          issue_pv(tmem + 256, tmem, v_lo0 + vs * kStageLo, hi, i > 0);
+          if (i == n - 1) tc_commit(&bars->o_final[0]);
           if (!two) tc_commit(&bars->kv_empty[vs]);
         }
         blk0++;
+        prev_vs = vs;
       }
       // ---- PV1_{n-1}
       if (ok && two) {
@@ -326,14 +392,12 @@ __device__ void run_mma(const FwdParams& p, uint8_t* smem, Bars* bars, uint32_t 
         if (ok) ok = warp_wait(&bars->p_full[1], blk1 & 1, bars);
         if (ok && lane == 0) {
           tc_fence_after_sync();
-          const uint32_t pvs = (kv0 + 2 * n - 1) % kStages;
-          issue_pv(o1, s1, desc_add(v_desc0, pvs * kTileBytes), n - 1 > 0);
-          tc_commit(&bars->o_done[1]);
-          tc_commit(&bars->kv_empty[pvs]);
+          issue_pv(tmem + 384, tmem + 128, v_lo0 + prev_vs * kStageLo, hi, n - 1 > 0);
+          tc_commit(&bars->o_final[1]);
+          tc_commit(&bars->kv_empty[prev_vs]);
         }
         blk1++;
       }
-      kv_iter = kv0 + 2 * n;
     }
     units0++;
     if (two) units1++;
@@ -349,37 +413,27 @@ __device__ void run_mma(const FwdParams& p, uint8_t* smem, Bars* bars, uint32_t 
 }
 
 // ---------------------------------------------------------------------------
-// softmax + epilogue (one warpgroup per tile slot; thread = tile row)
+// softmax (one warpgroup per tile slot; thread = tile row = TMEM lane)
 // ---------------------------------------------------------------------------
 __device__ void run_softmax(const FwdParams& p, Bars* bars, uint32_t tmem, int slot,
                             int32_t n_units, int64_t off_unit, int64_t off_item, int64_t off_list) {
-  const int row = (threadIdx.x & 127);            // tile row = TMEM lane
-  const uint32_t lane_sel = (uint32_t)((threadIdx.x & 96)) << 16;  // warp's 32-lane quarter
+  const int row = threadIdx.x & 127;
+  const uint32_t lane_sel = (uint32_t)(threadIdx.x & 96) << 16;  // warp's 32-lane quarter
   const uint32_t t_s = tmem + 128 * slot + lane_sel;
   const uint32_t t_o = tmem + 256 + 128 * slot + lane_sel;
-  const int rows_in_tile = p.tile_tokens * p.G;
-  const int tok_in_tile = row / p.G;
-  const int g = row - tok_in_tile * p.G;
-  uint32_t blk_iter = 0;
-  int32_t bad = 0;
-  bool ok = true;
-  for (int32_t u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+  uint32_t blk = 0, units = 0;
+  for (int32_t u = blockIdx.x; u < n_units; u += gridDim.x) {
     const Unit x = load_unit(p.meta, off_unit, off_item, u, p.N2);
-    if (slot >= x.nt) continue;
-    const int32_t tok_off = (2 * x.tp + slot) * p.tile_tokens + tok_in_tile;
-    const bool row_store = row < rows_in_tile && tok_off < x.n_store;
-    const bool row_used = row_store && tok_off < x.n_used;
-    const int32_t tok = x.tok_begin + tok_off;
-    const int32_t h = x.kvh * p.G + g;
-    const int32_t pos = x.pos0 + tok_off;  // query position (bottom-right aligned)
-    const int32_t key_hi = min(pos, x.ku - 1);
-    const int32_t key_lo = p.win_left >= 0 ? pos - p.win_left : INT32_MIN;
-    const int32_t* list = p.meta + off_list + (int64_t)x.item * p.top_k;
-    float m = -INFINITY, l = 0.f;
     const int32_t nblk = x.j1 - x.j0;
+    if (slot >= x.nt || nblk <= 0) continue;
+    const RowInfo ri = row_info(p, x, slot, row);
+    const int32_t key_hi = min(ri.pos, x.ku - 1);
+    const int32_t key_lo = p.win_left >= 0 ? ri.pos - p.win_left : INT32_MIN;
+    const int32_t* list = p.meta + off_list + (int64_t)x.item * p.top_k + x.j0;
+    float m = -INFINITY, l = 0.f;
     for (int32_t jb = 0; jb < nblk; jb++) {
-      const int32_t entry = list[x.j0 + jb];
-      if (!(ok = wait_bar(&bars->s_full[slot], blk_iter & 1, bars))) break;
+      const int32_t entry = list[jb];
+      if (!wait_bar(&bars->s_full[slot], blk & 1, bars)) return;
       tc_fence_after_sync();
       uint32_t r[4][32];
       tmem_ld_32x32(t_s + 0, r[0]);
@@ -393,7 +447,7 @@ __device__ void run_softmax(const FwdParams& p, Bars* bars, uint32_t tmem, int s
       // visible key columns of this block for this row: [clo, chi]; the
       // element mask runs only in warps that hold a row needing it
       int32_t clo = 0, chi = kPage - 1;
-      if (!row_used) {
+      if (!ri.used) {
         clo = kPage;
         chi = -1;
       } else if (entry & kEntryMask) {
@@ -406,11 +460,14 @@ __device__ void run_softmax(const FwdParams& p, Bars* bars, uint32_t tmem, int s
         for (int c = 0; c < 128; c++)
           if (c < clo || c > chi) r[c >> 5][c & 31] = __float_as_uint(-INFINITY);
       }
-      float mx = -INFINITY;
+      // row max: eight independent partial maxima, then a tree
+      float mp[8];
 #pragma unroll
-      for (int c = 0; c < 128; c += 2)
-        mx = fmaxf(mx, fmaxf(__uint_as_float(r[c >> 5][c & 31]),
-                             __uint_as_float(r[(c + 1) >> 5][(c + 1) & 31])));
+      for (int k = 0; k < 8; k++) mp[k] = __uint_as_float(r[0][k]);
+#pragma unroll
+      for (int c = 8; c < 128; c++) mp[c & 7] = fmaxf(mp[c & 7], __uint_as_float(r[c >> 5][c & 31]));
+      const float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
+                             fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
       const float m_blk = mx * p.scale_log2;
       const float m_new = fmaxf(m, m_blk);
       // lazy rescale: keep the old reference max unless it grew by > 8 (P <= 256)
@@ -422,24 +479,21 @@ __device__ void run_softmax(const FwdParams& p, Bars* bars, uint32_t tmem, int s
         m = m_new;
       }
       const float neg_m = (m == -INFINITY) ? 0.f : -m;
-      float sum = 0.f;
+      float sp[4] = {0.f, 0.f, 0.f, 0.f};  // independent partial sums
 #pragma unroll
-      for (int half = 0; half < 2; half++) {
-        uint32_t pk[32];
+      for (int q = 0; q < 4; q++) {
+        uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 32; i++) {
-          const int c = half * 64 + 2 * i;
-          const float s0 = __uint_as_float(r[c >> 5][c & 31]);
-          const float s1 = __uint_as_float(r[(c + 1) >> 5][(c + 1) & 31]);
+        for (int i = 0; i < 16; i++) {
           // masked scores are -inf and ex2(-inf) = +0
-          const float p0 = fast_exp2(fmaf(s0, p.scale_log2, neg_m));
-          const float p1 = fast_exp2(fmaf(s1, p.scale_log2, neg_m));
-          sum += p0 + p1;
+          const float p0 = fast_exp2(fmaf(__uint_as_float(r[q][2 * i]), p.scale_log2, neg_m));
+          const float p1 = fast_exp2(fmaf(__uint_as_float(r[q][2 * i + 1]), p.scale_log2, neg_m));
+          sp[i & 3] += p0 + p1;
           pk[i] = pack_bf16x2(p0, p1);
         }
-        tmem_st_32x32(t_s + 32 * half, pk);
+        tmem_st_32x16(t_s + 16 * q, pk);
       }
-      l += sum;
+      l += (sp[0] + sp[1]) + (sp[2] + sp[3]);
       if (__any_sync(0xffffffffu, fix_o)) {
         // O holds the earlier blocks (their PV completed before this S was
         // committed); bring it to the new reference max.
@@ -456,67 +510,90 @@ __device__ void run_softmax(const FwdParams& p, Bars* bars, uint32_t tmem, int s
       tmem_wait_st();
       tc_fence_before_sync();
       mbar_arrive(&bars->p_full[slot]);
-      blk_iter++;
+      blk++;
     }
-    if (!ok) break;
-    // ---- epilogue
-    if (nblk > 0) {
-      if (!(ok = wait_bar(&bars->o_done[slot], (blk_iter - 1) & 1, bars))) break;
-      tc_fence_after_sync();
-    }
-    const bool has = nblk > 0 && row_used && l > 0.f;
-    const float inv_l = has ? 1.f / l : 0.f;
-    const float lse = has ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
-    const bool write_row = row_store && tok < p.T;
-    if (row_store && tok >= p.T) bad |= kDevBadSeqlen;
-    if (x.slot < 0) {
-      __nv_bfloat16* dst = p.out + ((int64_t)tok * p.N1 + h) * kHeadDim;
-#pragma unroll 1
-      for (int c = 0; c < 4; c++) {
-        uint32_t o[32];
-        if (nblk > 0) {
-          tmem_ld_32x32(t_o + 32 * c, o);
-          tmem_wait_ld(o);
-        }
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 16; i++)
-          pk[i] = has ? pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l,
-                                    __uint_as_float(o[2 * i + 1]) * inv_l)
-                      : 0u;
-        if (write_row) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
-#pragma unroll
-          for (int i = 0; i < 4; i++)
-            d4[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-        }
+    // hand the row statistics of this unit to the epilogue warpgroup
+    if (units > 0 && !wait_bar(&bars->stats_free[slot], (units - 1) & 1, bars)) return;
+    bars->stats[slot][row] = make_float2(m, l);
+    mbar_arrive(&bars->stats_full[slot]);
+    units++;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// epilogue (one warpgroup; thread = tile row = TMEM lane, both tile slots)
+// ---------------------------------------------------------------------------
+__device__ void run_epilogue(const FwdParams& p, Bars* bars, uint32_t tmem, int32_t n_units,
+                             int64_t off_unit, int64_t off_item) {
+  const int row = threadIdx.x & 127;
+  const uint32_t lane_sel = (uint32_t)(threadIdx.x & 96) << 16;
+  const int rows_in_tile = p.tile_tokens * p.G;
+  uint32_t units_stats[2] = {0, 0}, units_final[2] = {0, 0};
+  int32_t bad = 0;
+  bool ok = true;
+  for (int32_t u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+    const Unit x = load_unit(p.meta, off_unit, off_item, u, p.N2);
+    const int32_t nblk = x.j1 - x.j0;
+    for (int slot = 0; slot < x.nt && ok; slot++) {
+      const RowInfo ri = row_info(p, x, slot, row);
+      const uint32_t t_o = tmem + 256 + 128 * slot + lane_sel;
+      float m = -INFINITY, l = 0.f;
+      if (nblk > 0) {
+        if (!(ok = wait_bar(&bars->stats_full[slot], units_stats[slot] & 1, bars))) break;
+        const float2 st = bars->stats[slot][row];
+        m = st.x;
+        l = st.y;
+        mbar_arrive(&bars->stats_free[slot]);
+        units_stats[slot]++;
+        if (!(ok = wait_bar(&bars->o_final[slot], units_final[slot] & 1, bars))) break;
+        units_final[slot]++;
+        tc_fence_after_sync();
       }
-      if (write_row && p.return_lse) p.lse[(int64_t)tok * p.N1 + h] = lse;
-    } else {
-      const int64_t wrow = (int64_t)x.slot * p.rows_per_unit + slot * rows_in_tile + row;
-      float* dst = p.ws_o + wrow * kHeadDim;
+      const bool has = nblk > 0 && ri.used && l > 0.f;
+      const float inv_l = has ? 1.f / l : 0.f;
+      const float lse = has ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+      const bool write_row = ri.store && ri.tok < p.T;
+      if (ri.store && ri.tok >= p.T) bad |= kDevBadSeqlen;
+      if (x.slot < 0) {
+        uint4* dst = reinterpret_cast<uint4*>(p.out + ((int64_t)ri.tok * p.N1 + ri.h) * kHeadDim);
 #pragma unroll 1
-      for (int c = 0; c < 4; c++) {
-        uint32_t o[32];
-        if (nblk > 0) {
-          tmem_ld_32x32(t_o + 32 * c, o);
-          tmem_wait_ld(o);
-        }
-        if (row < rows_in_tile) {
-          float4* d4 = reinterpret_cast<float4*>(dst + 32 * c);
+        for (int c = 0; c < 8; c++) {
+          uint32_t o[16];
+          if (nblk > 0) tmem_ld_32x16_wait(t_o + 16 * c, o);
+          uint32_t pk[8];
 #pragma unroll
           for (int i = 0; i < 8; i++)
-            d4[i] = has ? make_float4(__uint_as_float(o[4 * i]) * inv_l,
-                                      __uint_as_float(o[4 * i + 1]) * inv_l,
-                                      __uint_as_float(o[4 * i + 2]) * inv_l,
-                                      __uint_as_float(o[4 * i + 3]) * inv_l)
-                        : make_float4(0.f, 0.f, 0.f, 0.f);
+            pk[i] = has ? pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l,
+                                      __uint_as_float(o[2 * i + 1]) * inv_l)
+                        : 0u;
+          if (write_row) {
+            dst[2 * c] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            dst[2 * c + 1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+          }
         }
+        if (write_row && p.return_lse) p.lse[(int64_t)ri.tok * p.N1 + ri.h] = lse;
+      } else {
+        const int64_t wrow = (int64_t)x.slot * p.rows_per_unit + slot * rows_in_tile + row;
+        float4* dst = reinterpret_cast<float4*>(p.ws_o + wrow * kHeadDim);
+#pragma unroll 1
+        for (int c = 0; c < 8; c++) {
+          uint32_t o[16];
+          if (nblk > 0) tmem_ld_32x16_wait(t_o + 16 * c, o);
+          if (row < rows_in_tile) {
+#pragma unroll
+            for (int i = 0; i < 4; i++)
+              dst[4 * c + i] = has ? make_float4(__uint_as_float(o[4 * i]) * inv_l,
+                                                 __uint_as_float(o[4 * i + 1]) * inv_l,
+                                                 __uint_as_float(o[4 * i + 2]) * inv_l,
+                                                 __uint_as_float(o[4 * i + 3]) * inv_l)
+                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+        }
+        if (row < rows_in_tile) p.ws_lse[wrow] = lse;
       }
-      if (row < rows_in_tile) p.ws_lse[wrow] = lse;
+      tc_fence_before_sync();
+      mbar_arrive(&bars->o_free[slot]);
     }
-    tc_fence_before_sync();
-    mbar_arrive(&bars->o_free[slot]);
   }
   if (bad && p.dev_status) atomicOr(p.dev_status, bad);
 }
@@ -524,42 +601,44 @@ __device__ void run_softmax(const FwdParams& p, Bars* bars, uint32_t tmem, int s
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                const __grid_constant__ CUtensorMap map_v, const FwdParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
-  Bars* bars = reinterpret_cast<Bars*>(smem + kSmemBars);
+  extern __shared__ __align__(1024) uint8_t smem[];
   const int warp = threadIdx.x >> 5;
 
-  // the work list must have been built for this problem
+  // the work list must have been built for this problem, and the swizzled
+  // tiles need a 1 KiB aligned shared-memory window
   const int32_t* meta = p.meta;
   const bool match = (uint32_t)meta[H_MAGIC] == kMagic && meta[H_VERSION] == kFormatVersion &&
                      (uint32_t)meta[H_SIGNATURE] == p.signature;
-  if (!match) {
-    if (threadIdx.x == 0 && blockIdx.x == 0 && p.dev_status) atomicOr(p.dev_status, kDevMetaMismatch);
+  if (!match || (smem_u32(smem) & 1023u) != 0) {
+    if (threadIdx.x == 0 && blockIdx.x == 0 && p.dev_status)
+      atomicOr(p.dev_status, match ? kDevTimeout : kDevMetaMismatch);
     return;
   }
   const int32_t n_units = meta[H_NUNITS];
   const int64_t off_unit = meta[H_OFF_UNIT], off_item = meta[H_OFF_ITEM], off_list = meta[H_OFF_LIST];
   if ((int32_t)blockIdx.x >= n_units) return;  // no work for this CTA (uniform)
 
+  Bars* bars = reinterpret_cast<Bars*>(smem + kSmemBars);
   if (threadIdx.x == 0) {
-    mbar_init(&bars->q_full, 1);
-    mbar_init(&bars->q_empty, 1);
+    for (int i = 0; i < 2; i++) {
+      mbar_init(&bars->q_full[i], 1);
+      mbar_init(&bars->q_empty[i], 1);
+      mbar_init(&bars->s_full[i], 1);
+      mbar_init(&bars->p_full[i], 128);
+      mbar_init(&bars->o_final[i], 1);
+      mbar_init(&bars->o_free[i], 128);
+      mbar_init(&bars->stats_full[i], 128);
+      mbar_init(&bars->stats_free[i], 128);
+    }
     for (int i = 0; i < kStages; i++) {
       mbar_init(&bars->kv_full[i], 1);
       mbar_init(&bars->kv_empty[i], 1);
-    }
-    for (int s = 0; s < 2; s++) {
-      mbar_init(&bars->s_full[s], 1);
-      mbar_init(&bars->p_full[s], 128);
-      mbar_init(&bars->o_done[s], 1);
-      mbar_init(&bars->o_free[s], 128);
     }
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
     fence_mbar_init();
   }
-  if (warp == 1) {
+  if (warp == kWarpMma) {
     tmem_alloc(&bars->tmem_base, 512);
     tmem_relinquish();
   }
@@ -568,28 +647,28 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after_sync();
   const uint32_t tmem = bars->tmem_base;
 
-  if (warp < 4) {
-    setmaxnreg_dec<kRegsControl>();
-    if (warp == 0) {
-      if (lane_id() == 0) {
-        tma_prefetch_map(&map_q);
-        tma_prefetch_map(&map_k);
-        tma_prefetch_map(&map_v);
-        run_producer(p, &map_q, &map_k, &map_v, smem, bars, n_units, off_unit, off_item,
-                     off_list);
-      }
-    } else if (warp == 1) {
-      run_mma(p, smem, bars, tmem, n_units, off_unit, off_item, off_list);
-    }
-  } else {
+  if (warp < 8) {
     setmaxnreg_inc<kRegsSoftmax>();
-    run_softmax(p, bars, tmem, (warp - 4) >> 2, n_units, off_unit, off_item, off_list);
+    run_softmax(p, bars, tmem, warp >> 2, n_units, off_unit, off_item, off_list);
+  } else if (warp < 12) {
+    setmaxnreg_dec<kRegsEpilogue>();
+    run_epilogue(p, bars, tmem, n_units, off_unit, off_item);
+  } else {
+    setmaxnreg_dec<kRegsControl>();
+    if (warp == kWarpMma) {
+      run_mma(p, smem, bars, tmem, n_units, off_unit, off_item, off_list);
+    } else if (warp == kWarpProducer && lane_id() == 0) {
+      tma_prefetch_map(&map_q);
+      tma_prefetch_map(&map_k);
+      tma_prefetch_map(&map_v);
+      run_producer(p, &map_q, &map_k, &map_v, smem, bars, n_units, off_unit, off_item, off_list);
+    }
   }
 
   tc_fence_before_sync();
   __syncthreads();
   if (threadIdx.x == 0 && bars->abort && p.dev_status) atomicOr(p.dev_status, kDevTimeout);
-  if (warp == 1) {
+  if (warp == kWarpMma) {
     tc_fence_after_sync();
     tmem_dealloc(tmem, 512);
   }
@@ -661,7 +740,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const CombineParams p) {
 
 }  // namespace
 
-size_t forward_smem_bytes() { return kSmemAlloc; }
+size_t forward_smem_bytes() { return kSmemBytes; }
 
 cudaError_t launch_forward(const CUtensorMap& map_q, const CUtensorMap& map_k,
                            const CUtensorMap& map_v, const int32_t* meta,
@@ -682,7 +761,7 @@ cudaError_t launch_forward(const CUtensorMap& map_q, const CUtensorMap& map_k,
     e = cudaFuncGetAttributes(&attr, fwd_kernel);
     if (e != cudaSuccess) return e;
     if (attr.numRegs != kLaunchRegs) return cudaErrorInvalidKernelImage;
-    e = cudaFuncSetAttribute(fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemAlloc);
+    e = cudaFuncSetAttribute(fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     configured_device = dev;
   }
@@ -707,7 +786,7 @@ cudaError_t launch_forward(const CUtensorMap& map_q, const CUtensorMap& map_k,
   p.win_left = win_left;
   p.return_lse = return_lse;
   p.scale_log2 = scale_log2;
-  fwd_kernel<<<num_ctas, kThreads, kSmemAlloc, stream>>>(map_q, map_k, map_v, p);
+  fwd_kernel<<<num_ctas, kThreads, kSmemBytes, stream>>>(map_q, map_k, map_v, p);
   e = cudaGetLastError();
   if (e != cudaSuccess || comb_cap <= 0) return e;
   CombineParams c;
