@@ -41,9 +41,9 @@ constexpr int kThreads = 512;
 // Register split: launched with kLaunchRegs per thread; the epilogue and
 // control warpgroups give registers to the two softmax warpgroups.
 constexpr int kLaunchRegs = 128;
-constexpr int kRegsSoftmax = 184;   // warpgroups 0, 1
+constexpr int kRegsSoftmax = 176;   // warpgroups 0, 1
 constexpr int kRegsEpilogue = 80;   // warpgroup 2
-constexpr int kRegsControl = 64;    // warpgroup 3 (MMA, producer)
+constexpr int kRegsControl = 80;    // warpgroup 3 (MMA, producer)
 static_assert(256 * kRegsSoftmax + 128 * kRegsEpilogue + 128 * kRegsControl <=
                   kLaunchRegs * kThreads,
               "register split exceeds the launch allocation");
@@ -199,31 +199,53 @@ __device__ __forceinline__ bool produce_q(const FwdParams& p, const CUtensorMap*
 __device__ void run_producer(const FwdParams& p, const CUtensorMap* map_q, const CUtensorMap* map_k,
                              const CUtensorMap* map_v, uint8_t* smem, Bars* bars, int32_t n_units,
                              int64_t off_unit, int64_t off_item, int64_t off_list) {
+  // The whole warp runs the loop: lanes resolve 32 list entries and their
+  // physical pages in parallel (two dependent loads per 32 blocks instead of
+  // per block); lane 0 issues the copies.
+  const uint32_t lane = lane_id();
   uint32_t kv_iter = 0, q_iter0 = 0, q_iter1 = 0;
   int32_t bad = 0;
   bool ok = true;
   for (int32_t u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
     const Unit x = load_unit(p.meta, off_unit, off_item, u, p.N2);
-    if (x.j1 <= x.j0) continue;
-    const int32_t* list = p.meta + off_list + (int64_t)x.item * p.top_k;
+    const int32_t n = x.j1 - x.j0;
+    if (n <= 0) continue;
+    const int32_t* list = p.meta + off_list + (int64_t)x.item * p.top_k + x.j0;
     const int32_t* bt = p.block_table + (int64_t)x.b * p.max_pages;
     // order: Q0, K_0, Q1, V_0, K_1, V_1, ... (Q1 of a unit waits for the
     // previous unit's last S1, which comes later than its last S0)
-    ok = produce_q(p, map_q, smem, bars, q_iter0, x, 0);
-    for (int32_t j = x.j0; j < x.j1 && ok; j++) {
-      const int32_t lb = list[j] & kEntryLbMask;
-      int32_t page = lb < p.max_pages ? bt[lb] : -1;
-      if (page < 0 || page >= p.num_pages) {
+    // pages of the first 32 entries: the loads overlap the wait for the Q slot
+    int32_t page = 0;
+    if ((int32_t)lane < n) {
+      const int32_t lb = list[lane] & kEntryLbMask;
+      page = lb < p.max_pages ? bt[lb] : -1;
+    }
+    if (lane == 0) ok = produce_q(p, map_q, smem, bars, q_iter0, x, 0);
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    for (int32_t c0 = 0; c0 < n && ok; c0 += 32) {
+      if (c0 > 0 && c0 + (int32_t)lane < n) {
+        const int32_t lb = list[c0 + lane] & kEntryLbMask;
+        page = lb < p.max_pages ? bt[lb] : -1;
+      }
+      if (c0 + (int32_t)lane < n && (page < 0 || page >= p.num_pages)) {
         bad |= kDevBadPage;
         page = 0;
       }
-      ok = produce_kv(map_k, smem, bars, kv_iter, x.kvh, page);
-      if (ok && j == x.j0 && x.nt == 2) ok = produce_q(p, map_q, smem, bars, q_iter1, x, 1);
-      if (ok) ok = produce_kv(map_v, smem, bars, kv_iter, x.kvh, page);
+      const int32_t cn = min(32, n - c0);
+      for (int32_t jj = 0; jj < cn && ok; jj++) {
+        const int32_t pg = __shfl_sync(0xffffffffu, page, jj);
+        if (lane == 0) {
+          ok = produce_kv(map_k, smem, bars, kv_iter, x.kvh, pg);
+          if (ok && c0 + jj == 0 && x.nt == 2) ok = produce_q(p, map_q, smem, bars, q_iter1, x, 1);
+          if (ok) ok = produce_kv(map_v, smem, bars, kv_iter, x.kvh, pg);
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+      }
     }
   }
-  if (bad && p.dev_status) atomicOr(p.dev_status, bad);
-  if (!ok) {
+  bad = __reduce_or_sync(0xffffffffu, bad);
+  if (lane == 0 && bad && p.dev_status) atomicOr(p.dev_status, bad);
+  if (!ok && lane == 0) {
     // drain: wait (bounded) for the copies this thread issued last
     const uint64_t t0 = global_timer_ns();
     for (uint32_t i = (kv_iter > kStages ? kv_iter - kStages : 0); i < kv_iter; i++) {
@@ -266,7 +288,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Bars* 
 // offsets are added to the low word (addresses stay below 256 KiB: no carry).
 __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_lo, uint32_t k_lo,
                                          uint32_t hi) {
-#pragma unroll 4
+#pragma unroll
   for (int kk = 0; kk < 8; kk++) {
     const uint32_t off = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
     mma_ss_lo(d_tmem, q_lo + off, k_lo + off, hi, kIdescQK, kk > 0 ? 1u : 0u);
@@ -275,7 +297,7 @@ __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_lo, uint32_
 
 __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_lo,
                                          uint32_t hi, bool accumulate) {
-#pragma unroll 4
+#pragma unroll
   for (int kk = 0; kk < 8; kk++)
     mma_ts_lo(d_tmem, p_tmem + kk * 8, v_lo + ((kk * 2048) >> 4), hi, kIdescPV,
               (accumulate || kk > 0) ? 1u : 0u);
@@ -317,11 +339,15 @@ __device__ void run_mma(const FwdParams& p, uint8_t* smem, Bars* bars, uint32_t 
     const int32_t ku = p.meta[off_item + 8 * (int64_t)item + 7];
     const bool two = irow.z - 2 * rec.y >= 2;
     if (n > 0) {
+      // list entries of this unit, 32 at a time, one per lane (no global
+      // load on the issue path); the load overlaps the wait for Q
+      const int32_t* list = p.meta + off_list + (int64_t)item * p.top_k + j0;
+      int32_t entries = (int32_t)lane < n ? list[lane] : 0;
       if (!(ok = warp_wait(&bars->q_full[0], q_iter0 & 1, bars))) break;
       q_iter0++;
-      const int32_t* list = p.meta + off_list + (int64_t)item * p.top_k + j0;
       uint32_t prev_vs = 0;
       for (int32_t i = 0; i < n && ok; i++) {
+        if (i > 0 && (i & 31) == 0) entries = i + (int32_t)lane < n ? list[i + lane] : 0;
         // ---- S0_i
         const uint32_t ks = rp.stage;
         if (!(ok = warp_wait(&bars->kv_full[ks], rp.phase, bars))) break;
@@ -360,7 +386,7 @@ __device__ void run_mma(const FwdParams& p, uint8_t* smem, Bars* bars, uint32_t 
         const uint32_t vs = rp.stage;
         if (!(ok = warp_wait(&bars->kv_full[vs], rp.phase, bars))) break;
         rp.advance();
-        const int32_t entry = list[i];
+        const int32_t entry = __shfl_sync(0xffffffffu, entries, i & 31);
         if (entry & kEntryPartial) {
           const int32_t r0 = min(max(ku - (entry & kEntryLbMask) * kPage, 0), kPage);
           uint8_t* vt = smem + kSmemRing + vs * kTileBytes;
@@ -657,10 +683,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     setmaxnreg_dec<kRegsControl>();
     if (warp == kWarpMma) {
       run_mma(p, smem, bars, tmem, n_units, off_unit, off_item, off_list);
-    } else if (warp == kWarpProducer && lane_id() == 0) {
-      tma_prefetch_map(&map_q);
-      tma_prefetch_map(&map_k);
-      tma_prefetch_map(&map_v);
+    } else if (warp == kWarpProducer) {
+      if (lane_id() == 0) {
+        tma_prefetch_map(&map_q);
+        tma_prefetch_map(&map_k);
+        tma_prefetch_map(&map_v);
+      }
       run_producer(p, &map_q, &map_k, &map_v, smem, bars, n_units, off_unit, off_item, off_list);
     }
   }
