@@ -169,29 +169,36 @@ __device__ __forceinline__ RowInfo row_info(const FwdParams& p, const Unit& x, i
 // ---------------------------------------------------------------------------
 // producer (one thread)
 // ---------------------------------------------------------------------------
+// Called by the whole producer warp: every lane waits and counts, lane 0
+// issues the copies.
 __device__ __forceinline__ bool produce_kv(const CUtensorMap* map, uint8_t* smem, Bars* bars,
-                                           uint32_t& kv_iter, int32_t kvh, int32_t page) {
+                                           uint32_t& kv_iter, int32_t kvh, int32_t page,
+                                           uint32_t lane) {
   const uint32_t stage = kv_iter % kStages;
   if (kv_iter >= kStages && !wait_bar(&bars->kv_empty[stage], ((kv_iter / kStages) & 1) ^ 1, bars))
     return false;
-  uint8_t* dst = smem + kSmemRing + stage * kTileBytes;
-  mbar_arrive_expect_tx(&bars->kv_full[stage], kTileBytes);
-  tma_load_4d(dst, map, &bars->kv_full[stage], 0, kvh, 0, page);
-  tma_load_4d(dst + kHalfBytes, map, &bars->kv_full[stage], 64, kvh, 0, page);
+  if (lane == 0) {
+    uint8_t* dst = smem + kSmemRing + stage * kTileBytes;
+    mbar_arrive_expect_tx(&bars->kv_full[stage], kTileBytes);
+    tma_load_4d(dst, map, &bars->kv_full[stage], 0, kvh, 0, page);
+    tma_load_4d(dst + kHalfBytes, map, &bars->kv_full[stage], 64, kvh, 0, page);
+  }
   kv_iter++;
   return true;
 }
 
 __device__ __forceinline__ bool produce_q(const FwdParams& p, const CUtensorMap* map_q,
                                           uint8_t* smem, Bars* bars, uint32_t& q_iter,
-                                          const Unit& x, int s) {
+                                          const Unit& x, int s, uint32_t lane) {
   if (q_iter > 0 && !wait_bar(&bars->q_empty[s], (q_iter - 1) & 1, bars)) return false;
-  const uint32_t box_bytes = 128u * (uint32_t)p.G * (uint32_t)p.tile_tokens;
-  const int32_t tok = x.tok_begin + (2 * x.tp + s) * p.tile_tokens;
-  uint8_t* dst = smem + kSmemQ + s * kTileBytes;
-  mbar_arrive_expect_tx(&bars->q_full[s], 2u * box_bytes);
-  tma_load_3d(dst, map_q, &bars->q_full[s], 0, x.kvh * p.G, tok);
-  tma_load_3d(dst + kHalfBytes, map_q, &bars->q_full[s], 64, x.kvh * p.G, tok);
+  if (lane == 0) {
+    const uint32_t box_bytes = 128u * (uint32_t)p.G * (uint32_t)p.tile_tokens;
+    const int32_t tok = x.tok_begin + (2 * x.tp + s) * p.tile_tokens;
+    uint8_t* dst = smem + kSmemQ + s * kTileBytes;
+    mbar_arrive_expect_tx(&bars->q_full[s], 2u * box_bytes);
+    tma_load_3d(dst, map_q, &bars->q_full[s], 0, x.kvh * p.G, tok);
+    tma_load_3d(dst + kHalfBytes, map_q, &bars->q_full[s], 64, x.kvh * p.G, tok);
+  }
   q_iter++;
   return true;
 }
@@ -220,8 +227,7 @@ __device__ void run_producer(const FwdParams& p, const CUtensorMap* map_q, const
       const int32_t lb = list[lane] & kEntryLbMask;
       page = lb < p.max_pages ? bt[lb] : -1;
     }
-    if (lane == 0) ok = produce_q(p, map_q, smem, bars, q_iter0, x, 0);
-    ok = __shfl_sync(0xffffffffu, ok, 0);
+    ok = produce_q(p, map_q, smem, bars, q_iter0, x, 0, lane);
     for (int32_t c0 = 0; c0 < n && ok; c0 += 32) {
       if (c0 > 0 && c0 + (int32_t)lane < n) {
         const int32_t lb = list[c0 + lane] & kEntryLbMask;
@@ -234,12 +240,9 @@ __device__ void run_producer(const FwdParams& p, const CUtensorMap* map_q, const
       const int32_t cn = min(32, n - c0);
       for (int32_t jj = 0; jj < cn && ok; jj++) {
         const int32_t pg = __shfl_sync(0xffffffffu, page, jj);
-        if (lane == 0) {
-          ok = produce_kv(map_k, smem, bars, kv_iter, x.kvh, pg);
-          if (ok && c0 + jj == 0 && x.nt == 2) ok = produce_q(p, map_q, smem, bars, q_iter1, x, 1);
-          if (ok) ok = produce_kv(map_v, smem, bars, kv_iter, x.kvh, pg);
-        }
-        ok = __shfl_sync(0xffffffffu, ok, 0);
+        ok = produce_kv(map_k, smem, bars, kv_iter, x.kvh, pg, lane);
+        if (ok && c0 + jj == 0 && x.nt == 2) ok = produce_q(p, map_q, smem, bars, q_iter1, x, 1, lane);
+        if (ok) ok = produce_kv(map_v, smem, bars, kv_iter, x.kvh, pg, lane);
       }
     }
   }
@@ -277,10 +280,13 @@ __device__ void run_producer(const FwdParams& p, const CUtensorMap* map_q, const
 // while softmax 1 works on S1_i it runs PV0_i and S0_{i+1}.  K_i is released
 // after S1_i, V_i after PV1_i, which keeps the ring in fill order.
 // ---------------------------------------------------------------------------
+// Warp-wide wait: every lane polls the barrier.  One lane polling while the
+// rest wait at a shuffle costs ~300 cycles per wait in a warp that issues
+// tcgen05 MMAs (the pipe drains meanwhile); all lanes polling costs ~20.  The
+// lanes execute each try_wait, abort read and timer read together, so they
+// agree on the result.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Bars* bars) {
-  int ok = 1;
-  if (lane_id() == 0) ok = wait_bar(bar, parity, bars) ? 1 : 0;
-  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+  return wait_bar(bar, parity, bars);
 }
 
 // Descriptors are handled as 32-bit low words (start address >> 4 in bits
