@@ -497,9 +497,11 @@ __device__ void run_softmax(const FwdParams& p, Bars* bars, uint32_t tmem, int s
 #pragma unroll
       for (int k = 0; k < 8; k++) mp[k] = __uint_as_float(r[0][k]);
 #pragma unroll
-      for (int c = 8; c < 128; c++) mp[c & 7] = fmaxf(mp[c & 7], __uint_as_float(r[c >> 5][c & 31]));
-      const float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
-                             fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
+      for (int c = 8; c < 128; c += 2)
+        mp[(c >> 1) & 7] = max3f(mp[(c >> 1) & 7], __uint_as_float(r[c >> 5][c & 31]),
+                                 __uint_as_float(r[c >> 5][(c + 1) & 31]));
+      const float mx = max3f(max3f(mp[0], mp[1], mp[2]), max3f(mp[3], mp[4], mp[5]),
+                             fmaxf(mp[6], mp[7]));
       const float m_blk = mx * p.scale_log2;
       const float m_new = fmaxf(m, m_blk);
       // lazy rescale: keep the old reference max unless it grew by > 8 (P <= 256)
@@ -511,21 +513,30 @@ __device__ void run_softmax(const FwdParams& p, Bars* bars, uint32_t tmem, int s
         m = m_new;
       }
       const float neg_m = (m == -INFINITY) ? 0.f : -m;
-      float sp[4] = {0.f, 0.f, 0.f, 0.f};  // independent partial sums
+      // scores pairwise: x = s * scale_log2 - m as one f32x2 FMA, P = 2^x,
+      // the row sum in two packed partial sums (four independent lanes)
+      const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2), nm2 = f2_pack(neg_m, neg_m);
+      uint64_t sp2[2] = {0ull, 0ull};
 #pragma unroll
       for (int q = 0; q < 4; q++) {
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; i++) {
           // masked scores are -inf and ex2(-inf) = +0
-          const float p0 = fast_exp2(fmaf(__uint_as_float(r[q][2 * i]), p.scale_log2, neg_m));
-          const float p1 = fast_exp2(fmaf(__uint_as_float(r[q][2 * i + 1]), p.scale_log2, neg_m));
-          sp[i & 3] += p0 + p1;
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(r[q][2 * i]), __uint_as_float(r[q][2 * i + 1])),
+                           sc2, nm2),
+                    x0, x1);
+          const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+          sp2[i & 1] = f2_add(sp2[i & 1], f2_pack(p0, p1));
           pk[i] = pack_bf16x2(p0, p1);
         }
         tmem_st_32x16(t_s + 16 * q, pk);
       }
-      l += (sp[0] + sp[1]) + (sp[2] + sp[3]);
+      float s0, s1, s2, s3;
+      f2_unpack(sp2[0], s0, s1);
+      f2_unpack(sp2[1], s2, s3);
+      l += (s0 + s1) + (s2 + s3);
       if (__any_sync(0xffffffffu, fix_o)) {
         // O holds the earlier blocks (their PV completed before this S was
         // committed); bring it to the new reference max.
