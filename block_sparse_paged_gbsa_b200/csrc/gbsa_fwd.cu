@@ -19,9 +19,10 @@
 //                 pages into a 5-stage ring of 32 KiB buffers
 // TMEM (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each; P (bf16,
 // packed in pairs) overwrites the first 64 columns of its S.
-// Units come from the metadata work list, longest first; CTA c takes units
-// c, c + gridDim.x, ...  Every wait is bounded: after ~1 s the kernel sets
-// GBSA_DEV_TIMEOUT, drains its own copies and MMAs, frees TMEM and returns.
+// Units come from the metadata work list, longest first; the CTAs take them
+// wave by wave, in reverse CTA order on odd waves (unit_of).  Every wait is
+// bounded: after ~1 s the kernel sets GBSA_DEV_TIMEOUT, drains its own copies
+// and MMAs, frees TMEM and returns.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -90,6 +91,15 @@ struct Bars {
 };
 constexpr int kSmemBytes = kSmemBars + (int)sizeof(Bars);
 static_assert(kSmemBytes <= 232448, "shared memory budget");
+
+// The k-th unit of this CTA.  Units are sorted longest first; wave k covers
+// units [k * gridDim.x, (k + 1) * gridDim.x) and hands them to the CTAs in
+// reverse order on odd waves, which evens out the per-CTA sums of a sorted
+// list far better than plain round robin.  Increasing in k.
+__device__ __forceinline__ int32_t unit_of(int32_t k) {
+  const int32_t c = (k & 1) ? (int32_t)(gridDim.x - 1 - blockIdx.x) : (int32_t)blockIdx.x;
+  return k * (int32_t)gridDim.x + c;
+}
 
 struct Unit {
   int32_t item, tp, j0, j1, slot;
@@ -213,7 +223,7 @@ __device__ void run_producer(const FwdParams& p, const CUtensorMap* map_q, const
   uint32_t kv_iter = 0, q_iter0 = 0, q_iter1 = 0;
   int32_t bad = 0;
   bool ok = true;
-  for (int32_t u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+  for (int32_t wave = 0, u = unit_of(0); u < n_units && ok; u = unit_of(++wave)) {
     const Unit x = load_unit(p.meta, off_unit, off_item, u, p.N2);
     const int32_t n = x.j1 - x.j0;
     if (n <= 0) continue;
@@ -338,7 +348,7 @@ __device__ void run_mma(const FwdParams& p, uint8_t* smem, Bars* bars, uint32_t 
   const uint32_t v_lo0 = (uint32_t)smem_desc_sw128(ring_addr, kHalfBytes, 1024);
   constexpr uint32_t kStageLo = kTileBytes >> 4;
 
-  for (int32_t u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+  for (int32_t wave = 0, u = unit_of(0); u < n_units && ok; u = unit_of(++wave)) {
     const int4 rec = *reinterpret_cast<const int4*>(p.meta + off_unit + 4 * (int64_t)u);
     const int32_t item = rec.x, j0 = rec.z & 0xffff, n = (int32_t)((uint32_t)rec.z >> 16) - j0;
     const int4 irow = *reinterpret_cast<const int4*>(p.meta + off_item + 8 * (int64_t)item);
@@ -454,7 +464,7 @@ __device__ void run_softmax(const FwdParams& p, Bars* bars, uint32_t tmem, int s
   const uint32_t t_s = tmem + 128 * slot + lane_sel;
   const uint32_t t_o = tmem + 256 + 128 * slot + lane_sel;
   uint32_t blk = 0, units = 0;
-  for (int32_t u = blockIdx.x; u < n_units; u += gridDim.x) {
+  for (int32_t wave = 0, u = unit_of(0); u < n_units; u = unit_of(++wave)) {
     const Unit x = load_unit(p.meta, off_unit, off_item, u, p.N2);
     const int32_t nblk = x.j1 - x.j0;
     if (slot >= x.nt || nblk <= 0) continue;
@@ -574,7 +584,7 @@ __device__ void run_epilogue(const FwdParams& p, Bars* bars, uint32_t tmem, int3
   uint32_t units_stats[2] = {0, 0}, units_final[2] = {0, 0};
   int32_t bad = 0;
   bool ok = true;
-  for (int32_t u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+  for (int32_t wave = 0, u = unit_of(0); u < n_units && ok; u = unit_of(++wave)) {
     const Unit x = load_unit(p.meta, off_unit, off_item, u, p.N2);
     const int32_t nblk = x.j1 - x.j0;
     for (int slot = 0; slot < x.nt && ok; slot++) {
