@@ -27,7 +27,8 @@ cudaError_t launch_forward(const CUtensorMap& map_q, const CUtensorMap& map_k,
                            int32_t N2, int32_t T, int32_t top_k, int32_t max_pages,
                            int32_t num_pages, int32_t tile_tokens, int32_t rows_per_unit,
                            int32_t win_left, int32_t return_lse, float scale_log2,
-                           int32_t num_ctas, int64_t comb_cap, cudaStream_t stream);
+                           int32_t num_ctas, int64_t comb_cap, bool one_tile_blocks,
+                           cudaStream_t stream);
 }  // namespace gbsa
 
 using namespace gbsa;
@@ -298,7 +299,7 @@ gbsa_status gbsa_forward(const gbsa_problem* problem, const gbsa_tensors* t, con
       problem_signature(problem, ctas), problem->N1, problem->N2, problem->T, problem->top_k,
       problem->max_pages_per_seq, problem->num_pages, g.tile_tokens, g.rows_per_unit,
       problem->win_left, problem->return_lse, (float)(scale * 1.4426950408889634), ctas,
-      g.comb_cap, static_cast<cudaStream_t>(stream));
+      g.comb_cap, g.tiles_max == 1, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) {
     cudaGetLastError();
     return GBSA_ERR_CUDA;

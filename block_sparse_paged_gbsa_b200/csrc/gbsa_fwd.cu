@@ -42,10 +42,18 @@ constexpr int kThreads = 512;
 // Register split: launched with kLaunchRegs per thread; the epilogue and
 // control warpgroups give registers to the two softmax warpgroups.
 constexpr int kLaunchRegs = 128;
-constexpr int kRegsSoftmax = 176;   // warpgroups 0, 1
-constexpr int kRegsEpilogue = 80;   // warpgroup 2
-constexpr int kRegsControl = 80;    // warpgroup 3 (MMA, producer)
-static_assert(256 * kRegsSoftmax + 128 * kRegsEpilogue + 128 * kRegsControl <=
+// The instantiation with units in halves (below) moves 8 registers from each
+// softmax thread to the MMA and producer warps, whose loop then carries both
+// unit layouts.
+template <bool kHalves>
+constexpr int regs_softmax() { return kHalves ? 168 : 176; }  // warpgroups 0, 1
+constexpr int kRegsEpilogue = 80;                              // warpgroup 2
+template <bool kHalves>
+constexpr int regs_control() { return kHalves ? 96 : 80; }    // warpgroup 3 (MMA, producer)
+static_assert(256 * regs_softmax<false>() + 128 * kRegsEpilogue + 128 * regs_control<false>() <=
+                  kLaunchRegs * kThreads,
+              "register split exceeds the launch allocation");
+static_assert(256 * regs_softmax<true>() + 128 * kRegsEpilogue + 128 * regs_control<true>() <=
                   kLaunchRegs * kThreads,
               "register split exceeds the launch allocation");
 constexpr int kWarpMma = 12;
@@ -57,6 +65,20 @@ constexpr int kSmemQ = 0;
 constexpr int kSmemRing = 2 * kTileBytes;
 constexpr int kSmemBars = kSmemRing + kStages * kTileBytes;
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
+// A unit whose item has a single tile (decode: one token x G heads) and at
+// least this many blocks runs in halves: both tile slots work on its even /
+// odd blocks, so the S -> softmax -> PV chain of one slot overlaps the other.
+// Only the kernel instantiated with kHalves (chosen by the host when every Q
+// block fits one tile) carries this code: in the other one its extra branch
+// on the MMA warp costs the two-tile units a few percent.
+// Items with more tiles keep their last odd tile on one slot: that unit reads
+// the same K/V as the item's two-tile unit on another SM, and in step with it
+// one of the two finds the pages in L2 (in halves it runs ahead and both miss).
+#ifndef GBSA_HALVES_MIN_BLOCKS
+#define GBSA_HALVES_MIN_BLOCKS 4
+#endif
+constexpr int32_t kHalvesMinBlocks = GBSA_HALVES_MIN_BLOCKS;
+static_assert(kHalvesMinBlocks >= 2, "a unit in halves needs a block per slot");
 constexpr float kRescaleThreshold = 8.0f;  // log2 of the largest allowed P (256)
 constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, false, false);
 constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, false, true);
@@ -105,8 +127,11 @@ struct Unit {
   int32_t item, tp, j0, j1, slot;
   int32_t b, n_tiles, tok_begin, n_store, n_used, pos0, ku;
   int32_t kvh, nt;  // KV head, tiles in this unit (1 or 2)
+  bool halves;      // one tile, >= 2 blocks: the two tile slots take its even
+                    // and odd blocks (two partial softmaxes, merged at the end)
 };
 
+template <bool kHalves>
 __device__ __forceinline__ Unit load_unit(const int32_t* meta, int64_t off_unit, int64_t off_item,
                                           int32_t u, int32_t N2) {
   Unit x;
@@ -127,6 +152,7 @@ __device__ __forceinline__ Unit load_unit(const int32_t* meta, int64_t off_unit,
   x.ku = c.w;
   x.kvh = x.item % N2;
   x.nt = min(2, x.n_tiles - 2 * x.tp);
+  x.halves = kHalves && x.n_tiles == 1 && x.j1 - x.j0 >= kHalvesMinBlocks;
   return x;
 }
 
@@ -213,6 +239,7 @@ __device__ __forceinline__ bool produce_q(const FwdParams& p, const CUtensorMap*
   return true;
 }
 
+template <bool kHalves>
 __device__ void run_producer(const FwdParams& p, const CUtensorMap* map_q, const CUtensorMap* map_k,
                              const CUtensorMap* map_v, uint8_t* smem, Bars* bars, int32_t n_units,
                              int64_t off_unit, int64_t off_item, int64_t off_list) {
@@ -224,13 +251,14 @@ __device__ void run_producer(const FwdParams& p, const CUtensorMap* map_q, const
   int32_t bad = 0;
   bool ok = true;
   for (int32_t wave = 0, u = unit_of(0); u < n_units && ok; u = unit_of(++wave)) {
-    const Unit x = load_unit(p.meta, off_unit, off_item, u, p.N2);
+    const Unit x = load_unit<kHalves>(p.meta, off_unit, off_item, u, p.N2);
     const int32_t n = x.j1 - x.j0;
     if (n <= 0) continue;
     const int32_t* list = p.meta + off_list + (int64_t)x.item * p.top_k + x.j0;
     const int32_t* bt = p.block_table + (int64_t)x.b * p.max_pages;
     // order: Q0, K_0, Q1, V_0, K_1, V_1, ... (Q1 of a unit waits for the
-    // previous unit's last S1, which comes later than its last S0)
+    // previous unit's last S1, which comes later than its last S0); a unit
+    // in halves: Q0, then per block pair K_j, K_j+1, V_j, V_j+1
     // pages of the first 32 entries: the loads overlap the wait for the Q slot
     int32_t page = 0;
     if ((int32_t)lane < n) {
@@ -248,6 +276,19 @@ __device__ void run_producer(const FwdParams& p, const CUtensorMap* map_q, const
         page = 0;
       }
       const int32_t cn = min(32, n - c0);
+      if (x.halves) {
+        // blocks c0 + jj (even) and c0 + jj + 1 share a 32-entry chunk
+        for (int32_t jj = 0; jj < cn && ok; jj += 2) {
+          const bool has1 = jj + 1 < cn;
+          const int32_t pg0 = __shfl_sync(0xffffffffu, page, jj);
+          const int32_t pg1 = __shfl_sync(0xffffffffu, page, (jj + 1) & 31);
+          ok = produce_kv(map_k, smem, bars, kv_iter, x.kvh, pg0, lane);
+          if (ok && has1) ok = produce_kv(map_k, smem, bars, kv_iter, x.kvh, pg1, lane);
+          if (ok) ok = produce_kv(map_v, smem, bars, kv_iter, x.kvh, pg0, lane);
+          if (ok && has1) ok = produce_kv(map_v, smem, bars, kv_iter, x.kvh, pg1, lane);
+        }
+        continue;
+      }
       for (int32_t jj = 0; jj < cn && ok; jj++) {
         const int32_t pg = __shfl_sync(0xffffffffu, page, jj);
         ok = produce_kv(map_k, smem, bars, kv_iter, x.kvh, pg, lane);
@@ -328,10 +369,38 @@ struct RingPos {
       phase ^= 1u;
     }
   }
+  // the position k fills later (k < kStages)
+  __device__ __forceinline__ RingPos ahead(uint32_t k) const {
+    RingPos r{stage + k, phase};
+    if (r.stage >= kStages) {
+      r.stage -= kStages;
+      r.phase ^= 1u;
+    }
+    return r;
+  }
 };
 
+// Zero the rows of a V tile that lie past seqused_kv on a last page (their
+// pool contents are arbitrary and P there is 0, but 0 * NaN is NaN).  Whole
+// warp; `entry` is the block's list entry.
+__device__ __forceinline__ void zero_v_tail(uint8_t* smem, uint32_t vs, int32_t entry, int32_t ku,
+                                            uint32_t lane) {
+  if (!(entry & kEntryPartial)) return;
+  const int32_t r0 = min(max(ku - (entry & kEntryLbMask) * kPage, 0), kPage);
+  uint8_t* vt = smem + kSmemRing + vs * kTileBytes;
+  const int32_t n16 = (kPage - r0) * 16;
+  for (int32_t t = lane; t < n16; t += 32) {
+    const int32_t row = r0 + (t >> 4), chunk = t & 15;
+    *reinterpret_cast<uint4*>(vt + (chunk >> 3) * kHalfBytes + row * 128 + (chunk & 7) * 16) =
+        make_uint4(0, 0, 0, 0);
+  }
+  fence_proxy_async_smem();
+  __syncwarp();
+}
+
+template <bool kHalves>
 __device__ void run_mma(const FwdParams& p, uint8_t* smem, Bars* bars, uint32_t tmem,
-                        int32_t n_units, int64_t off_unit, int64_t off_item, int64_t off_list) {
+                        int32_t n_units, int32_t off_unit, int32_t off_item, int32_t off_list) {
   const uint32_t lane = lane_id();
   uint32_t q_iter0 = 0, q_iter1 = 0;
   uint32_t blk0 = 0, blk1 = 0;      // blocks per tile slot (p_full phases)
@@ -354,7 +423,93 @@ __device__ void run_mma(const FwdParams& p, uint8_t* smem, Bars* bars, uint32_t 
     const int4 irow = *reinterpret_cast<const int4*>(p.meta + off_item + 8 * (int64_t)item);
     const int32_t ku = p.meta[off_item + 8 * (int64_t)item + 7];
     const bool two = irow.z - 2 * rec.y >= 2;
-    if (n > 0) {
+    const bool halves = kHalves && irow.z == 1 && n >= kHalvesMinBlocks;
+    if (halves) {
+      // One tile, its blocks split even (slot 0) / odd (slot 1); both S read
+      // Q0.  Ring order per block pair j, j+1: K_j, K_j+1, V_j, V_j+1, each
+      // released right after the MMA that reads it.
+      //     S0_0, S1_0, PV0_0, then for i >= 1: S0_i, PV1_{i-1}, S1_i, PV0_i,
+      //     and PV1 of the last odd block when n is even.
+      const int32_t* list = p.meta + off_list + (int64_t)item * p.top_k + j0;
+      int32_t entries = (int32_t)lane < n ? list[lane] : 0;
+      if (!(ok = warp_wait(&bars->q_full[0], q_iter0 & 1, bars))) break;
+      q_iter0++;
+      const int32_t n0 = (n + 1) >> 1, n1 = n >> 1;
+      uint32_t pv1 = 0;  // ring stage of V of the pending odd block
+      for (int32_t i = 0; i < n0 && ok; i++) {
+        const int32_t j = 2 * i;
+        const bool has1 = j + 1 < n;
+        if (i > 0 && (j & 31) == 0) entries = j + (int32_t)lane < n ? list[j + lane] : 0;
+        // ---- S0_i = Q K_j
+        if (!(ok = warp_wait(&bars->kv_full[rp.stage], rp.phase, bars))) break;
+        if (lane == 0) {
+          tc_fence_after_sync();
+          issue_qk(tmem, q0_lo, k_lo0 + rp.stage * kStageLo, hi);
+          tc_commit(&bars->s_full[0]);
+          tc_commit(&bars->kv_empty[rp.stage]);
+          if (j == n - 1) tc_commit(&bars->q_empty[0]);
+        }
+        // ---- PV1_{i-1} = P1 V_{j-1}
+        if (i > 0) {
+          if (i == 1 && units1 > 0)
+            if (!(ok = warp_wait(&bars->o_free[1], (units1 - 1) & 1, bars))) break;
+          if (!(ok = warp_wait(&bars->p_full[1], blk1 & 1, bars))) break;
+          if (lane == 0) {
+            tc_fence_after_sync();
+            issue_pv(tmem + 384, tmem + 128, v_lo0 + pv1 * kStageLo, hi, i - 1 > 0);
+            if (i == n1) tc_commit(&bars->o_final[1]);
+            tc_commit(&bars->kv_empty[pv1]);
+          }
+          blk1++;
+        }
+        // ---- S1_i = Q K_{j+1}
+        if (has1) {
+          const RingPos rk1 = rp.ahead(1);
+          if (!(ok = warp_wait(&bars->kv_full[rk1.stage], rk1.phase, bars))) break;
+          if (lane == 0) {
+            tc_fence_after_sync();
+            issue_qk(tmem + 128, q0_lo, k_lo0 + rk1.stage * kStageLo, hi);
+            tc_commit(&bars->s_full[1]);
+            tc_commit(&bars->kv_empty[rk1.stage]);
+            if (j + 1 == n - 1) tc_commit(&bars->q_empty[0]);
+          }
+        }
+        // ---- V_j, then PV0_i = P0 V_j
+        const RingPos rv0 = rp.ahead(has1 ? 2 : 1);
+        if (!(ok = warp_wait(&bars->kv_full[rv0.stage], rv0.phase, bars))) break;
+        zero_v_tail(smem, rv0.stage, __shfl_sync(0xffffffffu, entries, j & 31), ku, lane);
+        if (i == 0 && units0 > 0)
+          if (!(ok = warp_wait(&bars->o_free[0], (units0 - 1) & 1, bars))) break;
+        if (!(ok = warp_wait(&bars->p_full[0], blk0 & 1, bars))) break;
+        if (lane == 0) {
+          tc_fence_after_sync();
+          issue_pv(tmem + 256, tmem, v_lo0 + rv0.stage * kStageLo, hi, i > 0);
+          if (i == n0 - 1) tc_commit(&bars->o_final[0]);
+          tc_commit(&bars->kv_empty[rv0.stage]);
+        }
+        blk0++;
+        // ---- V_{j+1} (read by PV1_i)
+        if (has1) {
+          const RingPos rv1 = rp.ahead(3);
+          if (!(ok = warp_wait(&bars->kv_full[rv1.stage], rv1.phase, bars))) break;
+          zero_v_tail(smem, rv1.stage, __shfl_sync(0xffffffffu, entries, (j + 1) & 31), ku, lane);
+          pv1 = rv1.stage;
+        }
+        rp = rp.ahead(has1 ? 4 : 2);
+      }
+      // ---- PV1 of the last odd block when n is even
+      if (ok && n1 == n0) {
+        if (n1 == 1 && units1 > 0) ok = warp_wait(&bars->o_free[1], (units1 - 1) & 1, bars);
+        if (ok) ok = warp_wait(&bars->p_full[1], blk1 & 1, bars);
+        if (ok && lane == 0) {
+          tc_fence_after_sync();
+          issue_pv(tmem + 384, tmem + 128, v_lo0 + pv1 * kStageLo, hi, n1 - 1 > 0);
+          tc_commit(&bars->o_final[1]);
+          tc_commit(&bars->kv_empty[pv1]);
+        }
+        blk1++;
+      }
+    } else if (n > 0) {
       // list entries of this unit, 32 at a time, one per lane (no global
       // load on the issue path); the load overlaps the wait for Q
       const int32_t* list = p.meta + off_list + (int64_t)item * p.top_k + j0;
@@ -402,19 +557,7 @@ __device__ void run_mma(const FwdParams& p, uint8_t* smem, Bars* bars, uint32_t 
         const uint32_t vs = rp.stage;
         if (!(ok = warp_wait(&bars->kv_full[vs], rp.phase, bars))) break;
         rp.advance();
-        const int32_t entry = __shfl_sync(0xffffffffu, entries, i & 31);
-        if (entry & kEntryPartial) {
-          const int32_t r0 = min(max(ku - (entry & kEntryLbMask) * kPage, 0), kPage);
-          uint8_t* vt = smem + kSmemRing + vs * kTileBytes;
-          const int32_t n16 = (kPage - r0) * 16;
-          for (int32_t t = lane; t < n16; t += 32) {
-            const int32_t row = r0 + (t >> 4), chunk = t & 15;
-            *reinterpret_cast<uint4*>(vt + (chunk >> 3) * kHalfBytes + row * 128 + (chunk & 7) * 16) =
-                make_uint4(0, 0, 0, 0);
-          }
-          fence_proxy_async_smem();
-          __syncwarp();
-        }
+        zero_v_tail(smem, vs, __shfl_sync(0xffffffffu, entries, i & 31), ku, lane);
         // ---- PV0_i
         if (i == 0 && units0 > 0)
           if (!(ok = warp_wait(&bars->o_free[0], (units0 - 1) & 1, bars))) break;
@@ -442,7 +585,7 @@ __device__ void run_mma(const FwdParams& p, uint8_t* smem, Bars* bars, uint32_t 
       }
     }
     units0++;
-    if (two) units1++;
+    if (two || halves) units1++;
   }
   // all MMAs issued by this thread complete before TMEM is released
   if (lane == 0) {
@@ -457,6 +600,7 @@ __device__ void run_mma(const FwdParams& p, uint8_t* smem, Bars* bars, uint32_t 
 // ---------------------------------------------------------------------------
 // softmax (one warpgroup per tile slot; thread = tile row = TMEM lane)
 // ---------------------------------------------------------------------------
+template <bool kHalves>
 __device__ void run_softmax(const FwdParams& p, Bars* bars, uint32_t tmem, int slot,
                             int32_t n_units, int64_t off_unit, int64_t off_item, int64_t off_list) {
   const int row = threadIdx.x & 127;
@@ -465,15 +609,18 @@ __device__ void run_softmax(const FwdParams& p, Bars* bars, uint32_t tmem, int s
   const uint32_t t_o = tmem + 256 + 128 * slot + lane_sel;
   uint32_t blk = 0, units = 0;
   for (int32_t wave = 0, u = unit_of(0); u < n_units; u = unit_of(++wave)) {
-    const Unit x = load_unit(p.meta, off_unit, off_item, u, p.N2);
+    const Unit x = load_unit<kHalves>(p.meta, off_unit, off_item, u, p.N2);
     const int32_t nblk = x.j1 - x.j0;
-    if (slot >= x.nt || nblk <= 0) continue;
-    const RowInfo ri = row_info(p, x, slot, row);
+    if ((slot >= x.nt && !x.halves) || nblk <= 0) continue;
+    // a unit in halves: both slots hold the rows of its one tile, slot s
+    // takes blocks s, s + 2, ...
+    const RowInfo ri = row_info(p, x, x.halves ? 0 : slot, row);
+    const int32_t jb0 = x.halves ? slot : 0, jstep = x.halves ? 2 : 1;
     const int32_t key_hi = min(ri.pos, x.ku - 1);
     const int32_t key_lo = p.win_left >= 0 ? ri.pos - p.win_left : INT32_MIN;
     const int32_t* list = p.meta + off_list + (int64_t)x.item * p.top_k + x.j0;
     float m = -INFINITY, l = 0.f;
-    for (int32_t jb = 0; jb < nblk; jb++) {
+    for (int32_t jb = jb0; jb < nblk; jb += jstep) {
       const int32_t entry = list[jb];
       if (!wait_bar(&bars->s_full[slot], blk & 1, bars)) return;
       tc_fence_after_sync();
@@ -576,6 +723,7 @@ __device__ void run_softmax(const FwdParams& p, Bars* bars, uint32_t tmem, int s
 // ---------------------------------------------------------------------------
 // epilogue (one warpgroup; thread = tile row = TMEM lane, both tile slots)
 // ---------------------------------------------------------------------------
+template <bool kHalves>
 __device__ void run_epilogue(const FwdParams& p, Bars* bars, uint32_t tmem, int32_t n_units,
                              int64_t off_unit, int64_t off_item) {
   const int row = threadIdx.x & 127;
@@ -585,8 +733,78 @@ __device__ void run_epilogue(const FwdParams& p, Bars* bars, uint32_t tmem, int3
   int32_t bad = 0;
   bool ok = true;
   for (int32_t wave = 0, u = unit_of(0); u < n_units && ok; u = unit_of(++wave)) {
-    const Unit x = load_unit(p.meta, off_unit, off_item, u, p.N2);
+    const Unit x = load_unit<kHalves>(p.meta, off_unit, off_item, u, p.N2);
     const int32_t nblk = x.j1 - x.j0;
+    if (x.halves) {
+      // two partial softmaxes over the even and odd blocks of one tile:
+      // O = (O0 2^(m0-M) + O1 2^(m1-M)) / (l0 2^(m0-M) + l1 2^(m1-M)), M = max
+      const RowInfo ri = row_info(p, x, 0, row);
+      float2 st[2];
+      for (int s = 0; s < 2 && ok; s++) {
+        if (!(ok = wait_bar(&bars->stats_full[s], units_stats[s] & 1, bars))) break;
+        st[s] = bars->stats[s][row];
+        mbar_arrive(&bars->stats_free[s]);
+        units_stats[s]++;
+      }
+      for (int s = 0; s < 2 && ok; s++) {
+        if (!(ok = wait_bar(&bars->o_final[s], units_final[s] & 1, bars))) break;
+        units_final[s]++;
+      }
+      if (!ok) break;
+      tc_fence_after_sync();
+      const float mm = fmaxf(st[0].x, st[1].x);
+      const float w0 = st[0].y > 0.f ? fast_exp2(st[0].x - mm) : 0.f;
+      const float w1 = st[1].y > 0.f ? fast_exp2(st[1].x - mm) : 0.f;
+      const float l = st[0].y * w0 + st[1].y * w1;
+      const bool has = ri.used && l > 0.f;
+      const float inv_l = has ? 1.f / l : 0.f;
+      const float a0 = w0 * inv_l, a1 = w1 * inv_l;
+      const float lse = has ? (mm + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+      const bool write_row = ri.store && ri.tok < p.T;
+      if (ri.store && ri.tok >= p.T) bad |= kDevBadSeqlen;
+      const uint32_t t_o0 = tmem + 256 + lane_sel, t_o1 = tmem + 384 + lane_sel;
+      if (x.slot < 0) {
+        uint4* dst = reinterpret_cast<uint4*>(p.out + ((int64_t)ri.tok * p.N1 + ri.h) * kHeadDim);
+#pragma unroll 1
+        for (int c = 0; c < 16; c++) {
+          uint32_t o0[8], o1[8];
+          tmem_ld_2x32x8_wait(t_o0 + 8 * c, t_o1 + 8 * c, o0, o1);
+          uint32_t pk[4];
+#pragma unroll
+          for (int i = 0; i < 4; i++)
+            pk[i] = has ? pack_bf16x2(
+                              __uint_as_float(o0[2 * i]) * a0 + __uint_as_float(o1[2 * i]) * a1,
+                              __uint_as_float(o0[2 * i + 1]) * a0 + __uint_as_float(o1[2 * i + 1]) * a1)
+                        : 0u;
+          if (write_row) dst[c] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        }
+        if (write_row && p.return_lse) p.lse[(int64_t)ri.tok * p.N1 + ri.h] = lse;
+      } else {
+        const int64_t wrow = (int64_t)x.slot * p.rows_per_unit + row;
+        float4* dst = reinterpret_cast<float4*>(p.ws_o + wrow * kHeadDim);
+#pragma unroll 1
+        for (int c = 0; c < 16; c++) {
+          uint32_t o0[8], o1[8];
+          tmem_ld_2x32x8_wait(t_o0 + 8 * c, t_o1 + 8 * c, o0, o1);
+          if (row < rows_in_tile) {
+#pragma unroll
+            for (int i = 0; i < 2; i++) {
+              float v[4];
+#pragma unroll
+              for (int e = 0; e < 4; e++)
+                v[e] = has ? __uint_as_float(o0[4 * i + e]) * a0 + __uint_as_float(o1[4 * i + e]) * a1
+                           : 0.f;
+              dst[2 * c + i] = make_float4(v[0], v[1], v[2], v[3]);
+            }
+          }
+        }
+        if (row < rows_in_tile) p.ws_lse[wrow] = lse;
+      }
+      tc_fence_before_sync();
+      mbar_arrive(&bars->o_free[0]);
+      mbar_arrive(&bars->o_free[1]);
+      continue;
+    }
     for (int slot = 0; slot < x.nt && ok; slot++) {
       const RowInfo ri = row_info(p, x, slot, row);
       const uint32_t t_o = tmem + 256 + 128 * slot + lane_sel;
@@ -651,6 +869,7 @@ __device__ void run_epilogue(const FwdParams& p, Bars* bars, uint32_t tmem, int3
   if (bad && p.dev_status) atomicOr(p.dev_status, bad);
 }
 
+template <bool kHalves>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                const __grid_constant__ CUtensorMap map_v, const FwdParams p) {
@@ -701,22 +920,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = bars->tmem_base;
 
   if (warp < 8) {
-    setmaxnreg_inc<kRegsSoftmax>();
-    run_softmax(p, bars, tmem, warp >> 2, n_units, off_unit, off_item, off_list);
+    setmaxnreg_inc<regs_softmax<kHalves>()>();
+    run_softmax<kHalves>(p, bars, tmem, warp >> 2, n_units, off_unit, off_item, off_list);
   } else if (warp < 12) {
     setmaxnreg_dec<kRegsEpilogue>();
-    run_epilogue(p, bars, tmem, n_units, off_unit, off_item);
+    run_epilogue<kHalves>(p, bars, tmem, n_units, off_unit, off_item);
   } else {
-    setmaxnreg_dec<kRegsControl>();
+    setmaxnreg_dec<regs_control<kHalves>()>();
     if (warp == kWarpMma) {
-      run_mma(p, smem, bars, tmem, n_units, off_unit, off_item, off_list);
+      run_mma<kHalves>(p, smem, bars, tmem, n_units, (int32_t)off_unit, (int32_t)off_item, (int32_t)off_list);
     } else if (warp == kWarpProducer) {
       if (lane_id() == 0) {
         tma_prefetch_map(&map_q);
         tma_prefetch_map(&map_k);
         tma_prefetch_map(&map_v);
       }
-      run_producer(p, &map_q, &map_k, &map_v, smem, bars, n_units, off_unit, off_item, off_list);
+      run_producer<kHalves>(p, &map_q, &map_k, &map_v, smem, bars, n_units, off_unit, off_item, off_list);
     }
   }
 
@@ -804,7 +1023,8 @@ cudaError_t launch_forward(const CUtensorMap& map_q, const CUtensorMap& map_k,
                            int32_t N2, int32_t T, int32_t top_k, int32_t max_pages,
                            int32_t num_pages, int32_t tile_tokens, int32_t rows_per_unit,
                            int32_t win_left, int32_t return_lse, float scale_log2,
-                           int32_t num_ctas, int64_t comb_cap, cudaStream_t stream) {
+                           int32_t num_ctas, int64_t comb_cap, bool one_tile_blocks,
+                           cudaStream_t stream) {
   static int configured_device = -1;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -812,12 +1032,16 @@ cudaError_t launch_forward(const CUtensorMap& map_q, const CUtensorMap& map_k,
   if (configured_device != dev) {
     // The register re-split is only safe if the kernel launches with exactly
     // the registers the split was computed for.
-    cudaFuncAttributes attr;
-    e = cudaFuncGetAttributes(&attr, fwd_kernel);
-    if (e != cudaSuccess) return e;
-    if (attr.numRegs != kLaunchRegs) return cudaErrorInvalidKernelImage;
-    e = cudaFuncSetAttribute(fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e != cudaSuccess) return e;
+    for (int h = 0; h < 2; h++) {
+      const void* fn = h ? reinterpret_cast<const void*>(fwd_kernel<true>)
+                         : reinterpret_cast<const void*>(fwd_kernel<false>);
+      cudaFuncAttributes attr;
+      e = cudaFuncGetAttributes(&attr, fn);
+      if (e != cudaSuccess) return e;
+      if (attr.numRegs != kLaunchRegs) return cudaErrorInvalidKernelImage;
+      e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+      if (e != cudaSuccess) return e;
+    }
     configured_device = dev;
   }
   FwdParams p;
@@ -841,7 +1065,11 @@ cudaError_t launch_forward(const CUtensorMap& map_q, const CUtensorMap& map_k,
   p.win_left = win_left;
   p.return_lse = return_lse;
   p.scale_log2 = scale_log2;
-  fwd_kernel<<<num_ctas, kThreads, kSmemBytes, stream>>>(map_q, map_k, map_v, p);
+  // every Q block in one tile (decode-like): the instantiation with units in halves
+  if (one_tile_blocks)
+    fwd_kernel<true><<<num_ctas, kThreads, kSmemBytes, stream>>>(map_q, map_k, map_v, p);
+  else
+    fwd_kernel<false><<<num_ctas, kThreads, kSmemBytes, stream>>>(map_q, map_k, map_v, p);
   e = cudaGetLastError();
   if (e != cudaSuccess || comb_cap <= 0) return e;
   CombineParams c;

@@ -252,6 +252,23 @@ __device__ __forceinline__ void tmem_ld_32x16_wait(uint32_t taddr, uint32_t (&r)
                  "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])::"memory");
 }
 
+// Two 8-column loads (from two accumulators) completed by one wait.
+__device__ __forceinline__ void tmem_ld_2x32x8_wait(uint32_t ta, uint32_t tb, uint32_t (&a)[8],
+                                                    uint32_t (&b)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3]), "=r"(a[4]), "=r"(a[5]),
+                 "=r"(a[6]), "=r"(a[7])
+               : "r"(ta));
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(b[0]), "=r"(b[1]), "=r"(b[2]), "=r"(b[3]), "=r"(b[4]), "=r"(b[5]),
+                 "=r"(b[6]), "=r"(b[7])
+               : "r"(tb));
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(a[0]), "+r"(a[1]), "+r"(a[2]), "+r"(a[3]), "+r"(a[4]), "+r"(a[5]),
+                 "+r"(a[6]), "+r"(a[7]), "+r"(b[0]), "+r"(b[1]), "+r"(b[2]), "+r"(b[3]),
+                 "+r"(b[4]), "+r"(b[5]), "+r"(b[6]), "+r"(b[7])::"memory");
+}
+
 // Keeps registers loaded by an earlier tmem_ld_32x32 behind a wait that was
 // issued through another tmem_wait_ld call.
 __device__ __forceinline__ void reg_fence(uint32_t (&r)[32]) {

@@ -32,6 +32,13 @@ SMALL = {
                                   win_left=200, win_right=0, page_stride_factor=1.25),
     "g16_bx200": lambda: generate(name="g16", seed=79, q_storage=[450], N1=16, N2=1,
                                   block_x=200, top_k=4, selection="random_causal"),
+    # one tile per Q block (16 tokens x G=8 heads): units of >= 4 blocks run with
+    # the two tile slots on the even / odd blocks, here with causal, window and
+    # partial-page masks
+    "g8_bx16_window": lambda: generate(name="g8w", seed=80, q_storage=[1500, 900],
+                                       q_used=[1480, 900], kv_used=[1500, 1000], N1=8, N2=1,
+                                       block_x=16, top_k=12, selection="random_causal",
+                                       win_left=700, win_right=0),
 }
 
 
@@ -98,7 +105,7 @@ def test_forward_matches_oracle(name):
     _compare(w, q, kf, vf, out, lse, rows)
 
 
-@pytest.mark.parametrize("name", ["tiny", "decode_s16", "g5_window"])
+@pytest.mark.parametrize("name", ["tiny", "decode_s16", "g5_window", "g8_bx16_window"])
 def test_split_kv_and_cta_counts(name):
     """Split-KV pieces and the combine: any CTA count / forced split length
     stays within tolerance of the oracle, and every repeat is bit-identical."""
