@@ -65,7 +65,17 @@ def parse_args():
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--scale-down", type=int, default=1,
+                    help="shrink the workload's sequence lengths by this factor (same "
+                         "structure); for profiler captures that must stay small")
     return ap.parse_args()
+
+
+def describe(args) -> str:
+    d = DESCRIPTIONS[args.workload]
+    if args.scale_down != 1:
+        d += f" -- sequence lengths scaled down {args.scale_down}x (profiling case)"
+    return d
 
 
 def load_peaks():
@@ -233,7 +243,7 @@ def run_reference(args, world, rank):
         return
     from block_sparse_paged_gbsa_b200.workloads import make_values, workload
 
-    w = workload(args.workload)
+    w = workload(args.workload, scale_down=args.scale_down)
     q, kf, vf = make_values(w, "cpu")
     per_step = max(0.5, min(5.0, 150.0 / max(1, args.steps + args.warmup)))
     vals = []
@@ -250,7 +260,7 @@ def run_reference(args, world, rank):
         "ms_per_step": round(1e3 * float(np.mean([v[1] for v in vals])), 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": DESCRIPTIONS[args.workload], "sample": sample},
+        "config": {"workload": describe(args), "sample": sample},
         "cpu_baseline": {"value": round(tf, 6), "unit": UNIT, "cores": threads,
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(tf, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
@@ -283,8 +293,8 @@ def main():
                                 device_id=dev)
 
     # each rank: its own seeded batch of the same workload (weak scaling)
-    base = workload(args.workload)
-    w = workload(args.workload, seed=rank_seed(base.seed, rank))
+    base = workload(args.workload, scale_down=args.scale_down)
+    w = workload(args.workload, seed=rank_seed(base.seed, rank), scale_down=args.scale_down)
     acc = work(w)
     q, kf, vf = make_values(w, dev)
     to = lambda a, dt: torch.as_tensor(np.ascontiguousarray(a), dtype=dt, device=dev)
@@ -401,7 +411,7 @@ def main():
         achieved = nbytes / (fwd_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": round(achieved, 3), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4)}
-    roof["traffic"] = profiled_traffic(args.workload)
+    roof["traffic"] = profiled_traffic(args.workload) if args.scale_down == 1 else None
     roof["kernel"] = "gbsa forward (attention + split-KV combine launch)"
     roof["peak_source"] = peaks["source"] + " (burst)"
 
@@ -418,7 +428,7 @@ def main():
             "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": round(step_ms, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": {"workload": DESCRIPTIONS[args.workload],
+            "config": {"workload": describe(args),
                        "parallelism": f"dp{world} (independent batches, no collective)",
                        "l2": "flushed between timed steps (256 MiB write)",
                        "num_ctas": int(meta_host[7])},
