@@ -255,8 +255,9 @@ def workload(name: str, seed: Optional[int] = None, scale_down: int = 1) -> Work
 WORKLOADS = ("tiny", "dense", "long", "decode", "ragged")
 
 
-def make_values(w: Workload, device="cpu", nan_fill=True):
-    """Draws q [T,N1,D] and the K/V pools (bf16) on ``device``.
+def make_values(w: Workload, device="cpu", nan_fill=True, dtype=None):
+    """Draws q [T,N1,D] and the K/V pools on ``device``: N(0,1) rounded to
+    ``dtype`` (torch.bfloat16, the default, or torch.float16).
 
     Returns (q, k_flat, v_flat): the pools are flat buffers of
     num_pages*kv_page_stride elements; ``pool_view`` gives the
@@ -264,14 +265,15 @@ def make_values(w: Workload, device="cpu", nan_fill=True):
     """
     import torch
 
+    dtype = torch.bfloat16 if dtype is None else dtype
     g = torch.Generator(device=device)
     g.manual_seed(int(w.seed))
     q = torch.randn((w.T, w.N1, w.D), generator=g, device=device, dtype=torch.float32)
-    q = q.to(torch.bfloat16)
+    q = q.to(dtype)
     pools = []
     for _ in range(2):
         flat = torch.randn((w.pool_elems,), generator=g, device=device, dtype=torch.float32)
-        flat = flat.to(torch.bfloat16)
+        flat = flat.to(dtype)
         if nan_fill:
             _fill_unreadable(w, flat)
         pools.append(flat)
@@ -304,7 +306,8 @@ def pool_view(w: Workload, flat):
 
 
 def bf16_bits(t) -> np.ndarray:
-    """uint16 numpy copy of the bit patterns of a bf16 torch tensor."""
+    """uint16 numpy copy of the bit patterns of a 16-bit (bf16 or fp16) torch
+    tensor."""
     import torch
 
     return t.detach().contiguous().view(torch.int16).cpu().numpy().view(np.uint16)

@@ -55,9 +55,12 @@ def load_library(path: str):
     lib = ctypes.CDLL(path)
     f = lib.gbsa_oracle_attention_rows
     i32, i64, dbl, ptr = ctypes.c_int32, ctypes.c_int64, ctypes.c_double, ctypes.c_void_p
-    f.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, i32, i32, i64, dbl, i32, i32,
+    f.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, i32, i32, i64, dbl, i32, i32, i32,
                   ptr, ptr, ptr, ptr, ptr, ptr, ptr, ptr, ptr, ptr, i64, ptr, ptr, i32]
     f.restype = ctypes.c_int
+    w = lib.gbsa_oracle_widen
+    w.argtypes = [i32, ptr, i64, ptr]
+    w.restype = ctypes.c_int
     return lib
 
 
@@ -81,12 +84,25 @@ def default_threads() -> int:
     return max(1, len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count())
 
 
+DTYPES = {"bf16": 0, "fp16": 1}
+
+
+def widen(bits, dtype="bf16", lib=None):
+    """Exact float64 values of 16-bit patterns of ``dtype`` ("bf16" / "fp16")."""
+    b = _as(bits, np.uint16).reshape(-1)
+    out = np.empty(b.size, np.float64)
+    if (lib or _load()).gbsa_oracle_widen(DTYPES[dtype], _ptr(b), b.size, _ptr(out)) != 0:
+        raise ValueError(dtype)
+    return out.reshape(np.shape(bits))
+
+
 def attention_rows(*, q_bits, k_bits, v_bits, kv_page_stride, num_pages, sparse_idx, sparse_count,
                    cu_seqlens_q, seqused_q, seqused_kv, block_table, block_x, scale,
-                   win_left=-1, win_right=-1, rows, n_threads=None, lib=None):
+                   win_left=-1, win_right=-1, rows, dtype="bf16", n_threads=None, lib=None):
     """Reference out/lse for selected (token, head) rows.
 
-    q_bits:  uint16 [T, N1, D] -- bf16 bit patterns of the queries.
+    q_bits:  uint16 [T, N1, D] -- bit patterns of the queries, bf16 or fp16
+             (``dtype``); k_bits and v_bits use the same type.
     k_bits, v_bits: flat uint16 arrays of the page pool; page ``p`` row ``r``
              head ``h`` starts at ``p*kv_page_stride + (r*N2 + h)*D``.
     rows:    int64 [n, 2] -- (global token index, query head).
@@ -114,7 +130,7 @@ def attention_rows(*, q_bits, k_bits, v_bits, kv_page_stride, num_pages, sparse_
     lse = np.full((n,), -np.inf, np.float64)
     rc = (lib or _load()).gbsa_oracle_attention_rows(
         B, T, N1, N2, D, block_x, tqb, top_k, bt.shape[1], num_pages, kv_page_stride, float(scale),
-        win_left, win_right, _ptr(q_bits), _ptr(k_bits), _ptr(v_bits), _ptr(sparse_idx),
+        win_left, win_right, DTYPES[dtype], _ptr(q_bits), _ptr(k_bits), _ptr(v_bits), _ptr(sparse_idx),
         _ptr(sparse_count), _ptr(cu), _ptr(squ), _ptr(sku), _ptr(bt), _ptr(rows), n,
         _ptr(out), _ptr(lse), n_threads or default_threads())
     if rc != 0:

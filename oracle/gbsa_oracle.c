@@ -39,7 +39,8 @@
  * entries ignored, empty rows -> 0 / -inf, natural-log lse) are listed in
  * the design notes.
  *
- * Inputs are raw bf16 bit patterns (uint16); each is widened exactly to fp64.
+ * Inputs are raw 16-bit patterns (uint16) of bf16 (dtype 0) or IEEE 754
+ * binary16 (dtype 1) values; each is widened exactly to fp64.
  */
 #include <math.h>
 #include <pthread.h>
@@ -54,6 +55,7 @@ typedef struct {
   int64_t kv_page_stride;
   double scale;
   int32_t win_left, win_right;
+  double (*widen)(uint16_t); /* bf16 or fp16 bits -> exact fp64 */
   const uint16_t *q, *k, *v;
   const int32_t *sparse_idx, *sparse_count;
   const int64_t* cu_seqlens_q;
@@ -65,11 +67,34 @@ typedef struct {
   int failed;            /* set to a nonzero code by a worker on bad input */
 } oracle_ctx;
 
+/* bf16 is the upper half of an IEEE 754 binary32. */
 static double widen_bf16(uint16_t bits) {
   uint32_t u = ((uint32_t)bits) << 16;
   float f;
   memcpy(&f, &u, sizeof f);
   return (double)f;
+}
+
+/* IEEE 754 binary16: sign, 5 exponent bits (bias 15), 10 fraction bits.
+ * Exponent 0 holds zero and the subnormals f * 2^-24; 31 holds inf / NaN. */
+static double widen_fp16(uint16_t bits) {
+  const int sign = bits >> 15, e = (bits >> 10) & 0x1f, f = bits & 0x3ff;
+  double mag;
+  if (e == 0)
+    mag = ldexp((double)f, -24);
+  else if (e == 31)
+    mag = f ? NAN : INFINITY;
+  else
+    mag = ldexp((double)(1024 + f), e - 25); /* (1 + f / 1024) * 2^(e - 15) */
+  return sign ? -mag : mag;
+}
+
+/* The exact fp64 values of n 16-bit patterns (dtype 0 bf16, 1 fp16); lets
+ * the tests pin the decoding on its own.  Returns nonzero for a bad dtype. */
+int gbsa_oracle_widen(int32_t dtype, const uint16_t* bits, int64_t n, double* out) {
+  if (dtype != 0 && dtype != 1) return 1;
+  for (int64_t i = 0; i < n; i++) out[i] = dtype ? widen_fp16(bits[i]) : widen_bf16(bits[i]);
+  return 0;
 }
 
 /* Largest b with cu_seqlens_q[b] <= tg (sequences may be empty). */
@@ -136,7 +161,7 @@ static int one_row(const oracle_ctx* c, int64_t tg, int32_t h, double* out, doub
     const uint16_t* krow =
         c->k + key_page[i] * c->kv_page_stride + ((int64_t)key_row[i] * c->N2 + kvh) * D;
     double dot = 0.0;
-    for (int32_t d = 0; d < D; d++) dot += widen_bf16(qrow[d]) * widen_bf16(krow[d]);
+    for (int32_t d = 0; d < D; d++) dot += c->widen(qrow[d]) * c->widen(krow[d]);
     score[i] = c->scale * dot;
   }
 
@@ -149,7 +174,7 @@ static int one_row(const oracle_ctx* c, int64_t tg, int32_t h, double* out, doub
     const double w = exp(score[i] - m) / l;
     const uint16_t* vrow =
         c->v + key_page[i] * c->kv_page_stride + ((int64_t)key_row[i] * c->N2 + kvh) * D;
-    for (int32_t d = 0; d < D; d++) out[d] += w * widen_bf16(vrow[d]);
+    for (int32_t d = 0; d < D; d++) out[d] += w * c->widen(vrow[d]);
   }
   *lse = m + log(l);
   return 0;
@@ -186,21 +211,23 @@ static void* run_job(void* arg) {
  * Reference attention for n_rows (token, head) pairs given in `rows`
  * ([n_rows][2] int64: global token index, query head).  Writes out
  * [n_rows][D] and lse [n_rows] in fp64.  kv_page_stride is in elements.
- * seqused_q may be NULL (every storage token used).  Returns 0 on success,
- * nonzero if an argument or a device-style value is outside its range.
+ * seqused_q may be NULL (every storage token used).  dtype: 0 = bf16,
+ * 1 = fp16 element bits in q, k, v.  Returns 0 on success, nonzero if an
+ * argument or a device-style value is outside its range.
  */
 int gbsa_oracle_attention_rows(int32_t B, int32_t T, int32_t N1, int32_t N2, int32_t D,
                                int32_t block_x, int32_t total_q_blocks, int32_t top_k,
                                int32_t max_pages_per_seq, int32_t num_pages,
                                int64_t kv_page_stride, double scale, int32_t win_left,
-                               int32_t win_right, const uint16_t* q, const uint16_t* k,
+                               int32_t win_right, int32_t dtype, const uint16_t* q, const uint16_t* k,
                                const uint16_t* v, const int32_t* sparse_idx,
                                const int32_t* sparse_count, const int64_t* cu_seqlens_q,
                                const int32_t* seqused_q, const int32_t* seqused_kv,
                                const int32_t* block_table, const int64_t* rows, int64_t n_rows,
                                double* out, double* lse, int32_t n_threads) {
   if (B < 1 || T < 1 || N2 < 1 || N1 < N2 || N1 % N2 || D < 1 || block_x < 1 || top_k < 1 ||
-      total_q_blocks < 1 || max_pages_per_seq < 1 || num_pages < 1 || n_rows < 0)
+      total_q_blocks < 1 || max_pages_per_seq < 1 || num_pages < 1 || n_rows < 0 ||
+      (dtype != 0 && dtype != 1))
     return 10;
   oracle_ctx c;
   memset(&c, 0, sizeof c);
@@ -209,6 +236,7 @@ int gbsa_oracle_attention_rows(int32_t B, int32_t T, int32_t N1, int32_t N2, int
   c.max_pages_per_seq = max_pages_per_seq; c.num_pages = num_pages;
   c.kv_page_stride = kv_page_stride; c.scale = scale;
   c.win_left = win_left; c.win_right = win_right;
+  c.widen = dtype ? widen_fp16 : widen_bf16;
   c.q = q; c.k = k; c.v = v; c.sparse_idx = sparse_idx; c.sparse_count = sparse_count;
   c.cu_seqlens_q = cu_seqlens_q; c.seqused_q = seqused_q; c.seqused_kv = seqused_kv;
   c.block_table = block_table; c.rows = rows; c.n_rows = n_rows; c.out = out; c.lse = lse;

@@ -10,13 +10,22 @@ import oracle
 from block_sparse_paged_gbsa_b200.workloads import PAGE, Workload, bf16_bits
 
 
+def elem_dtype(t) -> str:
+    """The oracle's name of a torch tensor's 16-bit element type."""
+    import torch
+
+    return {torch.bfloat16: "bf16", torch.float16: "fp16"}[t.dtype]
+
+
 def oracle_rows(w: Workload, q, kf, vf, rows, n_threads=None, lib=None):
+    assert q.dtype == kf.dtype == vf.dtype
     return oracle.attention_rows(
         q_bits=bf16_bits(q), k_bits=bf16_bits(kf), v_bits=bf16_bits(vf),
         kv_page_stride=w.kv_page_stride, num_pages=w.num_pages, sparse_idx=w.sparse_idx,
         sparse_count=w.sparse_count, cu_seqlens_q=w.cu_seqlens_q, seqused_q=w.seqused_q,
         seqused_kv=w.kv_used, block_table=w.block_table, block_x=w.block_x, scale=w.scale,
-        win_left=w.win_left, win_right=w.win_right, rows=rows, n_threads=n_threads, lib=lib)
+        win_left=w.win_left, win_right=w.win_right, rows=rows, dtype=elem_dtype(q),
+        n_threads=n_threads, lib=lib)
 
 
 def oracle_all(w: Workload, q, kf, vf, n_threads=None, lib=None):
@@ -27,11 +36,17 @@ def oracle_all(w: Workload, q, kf, vf, n_threads=None, lib=None):
     return out.reshape(T, N1, w.D), lse.reshape(T, N1)
 
 
-def to_f64(bits: np.ndarray) -> np.ndarray:
+def to_f64(bits: np.ndarray, dtype: str = "bf16") -> np.ndarray:
+    """Exact float64 values of 16-bit patterns, decoded with numpy (a decoder
+    independent of the oracle's C code): bf16 is the upper half of a
+    binary32, fp16 is numpy's IEEE binary16."""
+    bits = np.asarray(bits, np.uint16)
+    if dtype == "fp16":
+        return bits.view(np.float16).astype(np.float64)
     return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
-def logical_kv(w: Workload, pool_bits: np.ndarray, b: int) -> np.ndarray:
+def logical_kv(w: Workload, pool_bits: np.ndarray, b: int, dtype: str = "bf16") -> np.ndarray:
     """[ku, N2, D] fp64 keys (or values) of sequence b in logical order."""
     ku = int(w.kv_used[b])
     rows = []
@@ -42,7 +57,7 @@ def logical_kv(w: Workload, pool_bits: np.ndarray, b: int) -> np.ndarray:
         rows.append(blk)
     if not rows:
         return np.zeros((0, w.N2, w.D))
-    return to_f64(np.concatenate(rows, 0)[:ku])
+    return to_f64(np.concatenate(rows, 0)[:ku], dtype)
 
 
 def brute_force(w: Workload, q, kf, vf):
@@ -50,8 +65,9 @@ def brute_force(w: Workload, q, kf, vf):
     multiplicity of every logical key position is found by walking the block
     list entry by entry, the masks are applied as a dense boolean vector, and
     a dense fp64 softmax with those multiplicities as weights gives out/lse."""
+    dt = elem_dtype(q)
     qb_bits, kb, vb = bf16_bits(q), bf16_bits(kf), bf16_bits(vf)
-    qd = to_f64(qb_bits)
+    qd = to_f64(qb_bits, dt)
     out = np.zeros((w.T, w.N1, w.D))
     lse = np.full((w.T, w.N1), -np.inf)
     G = w.N1 // w.N2
@@ -60,8 +76,8 @@ def brute_force(w: Workload, q, kf, vf):
         qs = int(w.cu_seqlens_q[b + 1] - w.cu_seqlens_q[b])
         qu = int(w.q_used[b]) if w.has_seqused_q else qs
         ku = int(w.kv_used[b])
-        K = logical_kv(w, kb, b)
-        V = logical_kv(w, vb, b)
+        K = logical_kv(w, kb, b, dt)
+        V = logical_kv(w, vb, b, dt)
         keys = np.arange(ku)
         for t in range(qu):
             tg = int(w.cu_seqlens_q[b]) + t
