@@ -28,7 +28,7 @@ cudaError_t launch_forward(const CUtensorMap& map_q, const CUtensorMap& map_k,
                            int32_t num_pages, int32_t tile_tokens, int32_t rows_per_unit,
                            int32_t win_left, int32_t return_lse, float scale_log2,
                            int32_t num_ctas, int64_t comb_cap, bool one_tile_blocks,
-                           cudaStream_t stream);
+                           bool fp16, cudaStream_t stream);
 }  // namespace gbsa
 
 using namespace gbsa;
@@ -57,6 +57,9 @@ gbsa_status validate(const gbsa_problem* p, bool metadata_mode) {
   if (p->return_lse != 0 && p->return_lse != 1) return GBSA_ERR_INVALID_ARG;
   if (p->has_seqused_q != 0 && p->has_seqused_q != 1) return GBSA_ERR_INVALID_ARG;
   if (p->num_ctas < 0 || p->max_blocks_per_split < 0) return GBSA_ERR_INVALID_ARG;
+  if (p->dtype != GBSA_DTYPE_BF16 && p->dtype != GBSA_DTYPE_FP16) return GBSA_ERR_INVALID_ARG;
+  if (p->softmax_precision == 1) return GBSA_ERR_UNSUPPORTED;
+  if (p->softmax_precision != 0) return GBSA_ERR_INVALID_ARG;
   if (!(p->scale >= 0.0) || isinf(p->scale)) return GBSA_ERR_INVALID_ARG;
   if ((int64_t)p->N2 * p->total_q_blocks > 0x7fffffffLL / (p->top_k + 8)) return GBSA_ERR_SHAPE;
   if (!metadata_mode) {
@@ -161,11 +164,13 @@ EncodeTiledFn encode_fn() {
 }
 
 bool encode(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims,
-            const cuuint64_t* strides_bytes, const cuuint32_t* box) {
+            const cuuint64_t* strides_bytes, const cuuint32_t* box, int32_t dtype) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint32_t es[4] = {1, 1, 1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims,
+  const CUtensorMapDataType t =
+      dtype == GBSA_DTYPE_FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  return fn(map, t, rank, const_cast<void*>(base), dims,
             strides_bytes, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -279,7 +284,7 @@ gbsa_status gbsa_forward(const gbsa_problem* problem, const gbsa_tensors* t, con
     const cuuint64_t dims[3] = {D, (cuuint64_t)problem->N1, (cuuint64_t)problem->T};
     const cuuint64_t strides[2] = {D * 2, (cuuint64_t)problem->N1 * D * 2};
     const cuuint32_t box[3] = {64, (cuuint32_t)g.G, (cuuint32_t)g.tile_tokens};
-    if (!encode(&map_q, t->q, 3, dims, strides, box)) return GBSA_ERR_CUDA;
+    if (!encode(&map_q, t->q, 3, dims, strides, box, problem->dtype)) return GBSA_ERR_CUDA;
   }
   {
     const cuuint64_t dims[4] = {D, (cuuint64_t)problem->N2, (cuuint64_t)kPage,
@@ -287,8 +292,8 @@ gbsa_status gbsa_forward(const gbsa_problem* problem, const gbsa_tensors* t, con
     const cuuint64_t strides[3] = {D * 2, (cuuint64_t)problem->N2 * D * 2,
                                    (cuuint64_t)problem->kv_page_stride * 2};
     const cuuint32_t box[4] = {64, 1, (cuuint32_t)kPage, 1};
-    if (!encode(&map_k, t->k, 4, dims, strides, box)) return GBSA_ERR_CUDA;
-    if (!encode(&map_v, t->v, 4, dims, strides, box)) return GBSA_ERR_CUDA;
+    if (!encode(&map_k, t->k, 4, dims, strides, box, problem->dtype)) return GBSA_ERR_CUDA;
+    if (!encode(&map_v, t->v, 4, dims, strides, box, problem->dtype)) return GBSA_ERR_CUDA;
   }
   const double scale = problem->scale > 0.0 ? problem->scale : 1.0 / sqrt((double)problem->D);
   float* ws_o = static_cast<float*>(workspace);
@@ -299,7 +304,8 @@ gbsa_status gbsa_forward(const gbsa_problem* problem, const gbsa_tensors* t, con
       problem_signature(problem, ctas), problem->N1, problem->N2, problem->T, problem->top_k,
       problem->max_pages_per_seq, problem->num_pages, g.tile_tokens, g.rows_per_unit,
       problem->win_left, problem->return_lse, (float)(scale * 1.4426950408889634), ctas,
-      g.comb_cap, g.tiles_max == 1, static_cast<cudaStream_t>(stream));
+      g.comb_cap, g.tiles_max == 1, problem->dtype == GBSA_DTYPE_FP16,
+      static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) {
     cudaGetLastError();
     return GBSA_ERR_CUDA;

@@ -80,13 +80,21 @@ constexpr uint64_t kWaitLimitNs = 1000000000ull;
 constexpr int32_t kHalvesMinBlocks = GBSA_HALVES_MIN_BLOCKS;
 static_assert(kHalvesMinBlocks >= 2, "a unit in halves needs a block per slot");
 constexpr float kRescaleThreshold = 8.0f;  // log2 of the largest allowed P (256)
-constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, false, false);
-constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, false, true);
+// Instruction descriptors: S = Q K^T (K-major A and B), O += P V (V MN-major);
+// bf16 or fp16 operands (the element type of Q, K, V and P), fp32 accumulator.
+template <bool kF16>
+constexpr uint32_t idesc_qk() {
+  return kF16 ? idesc_f16_f32(128, 128, false, false) : idesc_bf16_f32(128, 128, false, false);
+}
+template <bool kF16>
+constexpr uint32_t idesc_pv() {
+  return kF16 ? idesc_f16_f32(128, 128, false, true) : idesc_bf16_f32(128, 128, false, true);
+}
 
 struct FwdParams {
   const int32_t* meta;
   const int32_t* block_table;
-  __nv_bfloat16* out;
+  uint16_t* out;  // bf16 or fp16 elements
   float* lse;
   float* ws_o;    // [slot_cap][rows_per_unit][128] fp32 partial outputs
   float* ws_lse;  // [slot_cap][rows_per_unit] fp32 partial lse
@@ -343,20 +351,22 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Bars* 
 // Descriptors are handled as 32-bit low words (start address >> 4 in bits
 // [0,14), leading byte offset >> 4 in [16,30)) plus the shared high word;
 // offsets are added to the low word (addresses stay below 256 KiB: no carry).
+template <bool kF16>
 __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_lo, uint32_t k_lo,
                                          uint32_t hi) {
 #pragma unroll
   for (int kk = 0; kk < 8; kk++) {
     const uint32_t off = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
-    mma_ss_lo(d_tmem, q_lo + off, k_lo + off, hi, kIdescQK, kk > 0 ? 1u : 0u);
+    mma_ss_lo(d_tmem, q_lo + off, k_lo + off, hi, idesc_qk<kF16>(), kk > 0 ? 1u : 0u);
   }
 }
 
+template <bool kF16>
 __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_lo,
                                          uint32_t hi, bool accumulate) {
 #pragma unroll
   for (int kk = 0; kk < 8; kk++)
-    mma_ts_lo(d_tmem, p_tmem + kk * 8, v_lo + ((kk * 2048) >> 4), hi, kIdescPV,
+    mma_ts_lo(d_tmem, p_tmem + kk * 8, v_lo + ((kk * 2048) >> 4), hi, idesc_pv<kF16>(),
               (accumulate || kk > 0) ? 1u : 0u);
 }
 
@@ -398,7 +408,7 @@ __device__ __forceinline__ void zero_v_tail(uint8_t* smem, uint32_t vs, int32_t 
   __syncwarp();
 }
 
-template <bool kHalves>
+template <bool kHalves, bool kF16>
 __device__ void run_mma(const FwdParams& p, uint8_t* smem, Bars* bars, uint32_t tmem,
                         int32_t n_units, int32_t off_unit, int32_t off_item, int32_t off_list) {
   const uint32_t lane = lane_id();
@@ -444,7 +454,7 @@ __device__ void run_mma(const FwdParams& p, uint8_t* smem, Bars* bars, uint32_t 
         if (!(ok = warp_wait(&bars->kv_full[rp.stage], rp.phase, bars))) break;
         if (lane == 0) {
           tc_fence_after_sync();
-          issue_qk(tmem, q0_lo, k_lo0 + rp.stage * kStageLo, hi);
+          issue_qk<kF16>(tmem, q0_lo, k_lo0 + rp.stage * kStageLo, hi);
           tc_commit(&bars->s_full[0]);
           tc_commit(&bars->kv_empty[rp.stage]);
           if (j == n - 1) tc_commit(&bars->q_empty[0]);
@@ -456,7 +466,7 @@ __device__ void run_mma(const FwdParams& p, uint8_t* smem, Bars* bars, uint32_t 
           if (!(ok = warp_wait(&bars->p_full[1], blk1 & 1, bars))) break;
           if (lane == 0) {
             tc_fence_after_sync();
-            issue_pv(tmem + 384, tmem + 128, v_lo0 + pv1 * kStageLo, hi, i - 1 > 0);
+            issue_pv<kF16>(tmem + 384, tmem + 128, v_lo0 + pv1 * kStageLo, hi, i - 1 > 0);
             if (i == n1) tc_commit(&bars->o_final[1]);
             tc_commit(&bars->kv_empty[pv1]);
           }
@@ -468,7 +478,7 @@ __device__ void run_mma(const FwdParams& p, uint8_t* smem, Bars* bars, uint32_t 
           if (!(ok = warp_wait(&bars->kv_full[rk1.stage], rk1.phase, bars))) break;
           if (lane == 0) {
             tc_fence_after_sync();
-            issue_qk(tmem + 128, q0_lo, k_lo0 + rk1.stage * kStageLo, hi);
+            issue_qk<kF16>(tmem + 128, q0_lo, k_lo0 + rk1.stage * kStageLo, hi);
             tc_commit(&bars->s_full[1]);
             tc_commit(&bars->kv_empty[rk1.stage]);
             if (j + 1 == n - 1) tc_commit(&bars->q_empty[0]);
@@ -483,7 +493,7 @@ __device__ void run_mma(const FwdParams& p, uint8_t* smem, Bars* bars, uint32_t 
         if (!(ok = warp_wait(&bars->p_full[0], blk0 & 1, bars))) break;
         if (lane == 0) {
           tc_fence_after_sync();
-          issue_pv(tmem + 256, tmem, v_lo0 + rv0.stage * kStageLo, hi, i > 0);
+          issue_pv<kF16>(tmem + 256, tmem, v_lo0 + rv0.stage * kStageLo, hi, i > 0);
           if (i == n0 - 1) tc_commit(&bars->o_final[0]);
           tc_commit(&bars->kv_empty[rv0.stage]);
         }
@@ -503,7 +513,7 @@ __device__ void run_mma(const FwdParams& p, uint8_t* smem, Bars* bars, uint32_t 
         if (ok) ok = warp_wait(&bars->p_full[1], blk1 & 1, bars);
         if (ok && lane == 0) {
           tc_fence_after_sync();
-          issue_pv(tmem + 384, tmem + 128, v_lo0 + pv1 * kStageLo, hi, n1 - 1 > 0);
+          issue_pv<kF16>(tmem + 384, tmem + 128, v_lo0 + pv1 * kStageLo, hi, n1 - 1 > 0);
           tc_commit(&bars->o_final[1]);
           tc_commit(&bars->kv_empty[pv1]);
         }
@@ -525,7 +535,7 @@ __device__ void run_mma(const FwdParams& p, uint8_t* smem, Bars* bars, uint32_t 
         rp.advance();
         if (lane == 0) {
           tc_fence_after_sync();
-          issue_qk(tmem, q0_lo, k_lo0 + ks * kStageLo, hi);
+          issue_qk<kF16>(tmem, q0_lo, k_lo0 + ks * kStageLo, hi);
           tc_commit(&bars->s_full[0]);
           if (i == n - 1) tc_commit(&bars->q_empty[0]);
         }
@@ -540,14 +550,14 @@ __device__ void run_mma(const FwdParams& p, uint8_t* smem, Bars* bars, uint32_t 
             if (!(ok = warp_wait(&bars->p_full[1], blk1 & 1, bars))) break;
             if (lane == 0) {
               tc_fence_after_sync();
-              issue_pv(tmem + 384, tmem + 128, v_lo0 + prev_vs * kStageLo, hi, i - 1 > 0);
+              issue_pv<kF16>(tmem + 384, tmem + 128, v_lo0 + prev_vs * kStageLo, hi, i - 1 > 0);
               tc_commit(&bars->kv_empty[prev_vs]);
             }
             blk1++;
           }
           // ---- S1_i
           if (lane == 0) {
-            issue_qk(tmem + 128, q1_lo, k_lo0 + ks * kStageLo, hi);
+            issue_qk<kF16>(tmem + 128, q1_lo, k_lo0 + ks * kStageLo, hi);
             tc_commit(&bars->s_full[1]);
             if (i == n - 1) tc_commit(&bars->q_empty[1]);
           }
@@ -564,7 +574,7 @@ __device__ void run_mma(const FwdParams& p, uint8_t* smem, Bars* bars, uint32_t 
         if (!(ok = warp_wait(&bars->p_full[0], blk0 & 1, bars))) break;
         if (lane == 0) {
           tc_fence_after_sync();
-          issue_pv(tmem + 256, tmem, v_lo0 + vs * kStageLo, hi, i > 0);
+          issue_pv<kF16>(tmem + 256, tmem, v_lo0 + vs * kStageLo, hi, i > 0);
           if (i == n - 1) tc_commit(&bars->o_final[0]);
           if (!two) tc_commit(&bars->kv_empty[vs]);
         }
@@ -577,7 +587,7 @@ __device__ void run_mma(const FwdParams& p, uint8_t* smem, Bars* bars, uint32_t 
         if (ok) ok = warp_wait(&bars->p_full[1], blk1 & 1, bars);
         if (ok && lane == 0) {
           tc_fence_after_sync();
-          issue_pv(tmem + 384, tmem + 128, v_lo0 + prev_vs * kStageLo, hi, n - 1 > 0);
+          issue_pv<kF16>(tmem + 384, tmem + 128, v_lo0 + prev_vs * kStageLo, hi, n - 1 > 0);
           tc_commit(&bars->o_final[1]);
           tc_commit(&bars->kv_empty[prev_vs]);
         }
@@ -600,7 +610,7 @@ __device__ void run_mma(const FwdParams& p, uint8_t* smem, Bars* bars, uint32_t 
 // ---------------------------------------------------------------------------
 // softmax (one warpgroup per tile slot; thread = tile row = TMEM lane)
 // ---------------------------------------------------------------------------
-template <bool kHalves>
+template <bool kHalves, bool kF16>
 __device__ void run_softmax(const FwdParams& p, Bars* bars, uint32_t tmem, int slot,
                             int32_t n_units, int64_t off_unit, int64_t off_item, int64_t off_list) {
   const int row = threadIdx.x & 127;
@@ -686,7 +696,7 @@ __device__ void run_softmax(const FwdParams& p, Bars* bars, uint32_t tmem, int s
                     x0, x1);
           const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
           sp2[i & 1] = f2_add(sp2[i & 1], f2_pack(p0, p1));
-          pk[i] = pack_bf16x2(p0, p1);
+          pk[i] = pack_x2<kF16>(p0, p1);
         }
         tmem_st_32x16(t_s + 16 * q, pk);
       }
@@ -723,7 +733,7 @@ __device__ void run_softmax(const FwdParams& p, Bars* bars, uint32_t tmem, int s
 // ---------------------------------------------------------------------------
 // epilogue (one warpgroup; thread = tile row = TMEM lane, both tile slots)
 // ---------------------------------------------------------------------------
-template <bool kHalves>
+template <bool kHalves, bool kF16>
 __device__ void run_epilogue(const FwdParams& p, Bars* bars, uint32_t tmem, int32_t n_units,
                              int64_t off_unit, int64_t off_item) {
   const int row = threadIdx.x & 127;
@@ -772,7 +782,7 @@ __device__ void run_epilogue(const FwdParams& p, Bars* bars, uint32_t tmem, int3
           uint32_t pk[4];
 #pragma unroll
           for (int i = 0; i < 4; i++)
-            pk[i] = has ? pack_bf16x2(
+            pk[i] = has ? pack_x2<kF16>(
                               __uint_as_float(o0[2 * i]) * a0 + __uint_as_float(o1[2 * i]) * a1,
                               __uint_as_float(o0[2 * i + 1]) * a0 + __uint_as_float(o1[2 * i + 1]) * a1)
                         : 0u;
@@ -834,7 +844,7 @@ __device__ void run_epilogue(const FwdParams& p, Bars* bars, uint32_t tmem, int3
           uint32_t pk[8];
 #pragma unroll
           for (int i = 0; i < 8; i++)
-            pk[i] = has ? pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l,
+            pk[i] = has ? pack_x2<kF16>(__uint_as_float(o[2 * i]) * inv_l,
                                       __uint_as_float(o[2 * i + 1]) * inv_l)
                         : 0u;
           if (write_row) {
@@ -869,7 +879,7 @@ __device__ void run_epilogue(const FwdParams& p, Bars* bars, uint32_t tmem, int3
   if (bad && p.dev_status) atomicOr(p.dev_status, bad);
 }
 
-template <bool kHalves>
+template <bool kHalves, bool kF16>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                const __grid_constant__ CUtensorMap map_v, const FwdParams p) {
@@ -921,14 +931,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < 8) {
     setmaxnreg_inc<regs_softmax<kHalves>()>();
-    run_softmax<kHalves>(p, bars, tmem, warp >> 2, n_units, off_unit, off_item, off_list);
+    run_softmax<kHalves, kF16>(p, bars, tmem, warp >> 2, n_units, off_unit, off_item, off_list);
   } else if (warp < 12) {
     setmaxnreg_dec<kRegsEpilogue>();
-    run_epilogue<kHalves>(p, bars, tmem, n_units, off_unit, off_item);
+    run_epilogue<kHalves, kF16>(p, bars, tmem, n_units, off_unit, off_item);
   } else {
     setmaxnreg_dec<regs_control<kHalves>()>();
     if (warp == kWarpMma) {
-      run_mma<kHalves>(p, smem, bars, tmem, n_units, (int32_t)off_unit, (int32_t)off_item, (int32_t)off_list);
+      run_mma<kHalves, kF16>(p, smem, bars, tmem, n_units, (int32_t)off_unit, (int32_t)off_item, (int32_t)off_list);
     } else if (warp == kWarpProducer) {
       if (lane_id() == 0) {
         tma_prefetch_map(&map_q);
@@ -955,11 +965,11 @@ struct CombineParams {
   const int32_t* meta;
   const float* ws_o;
   const float* ws_lse;
-  __nv_bfloat16* out;
+  uint16_t* out;  // bf16 or fp16 elements
   float* lse;
   int32_t* dev_status;
   uint32_t signature;
-  int32_t N1, N2, G, T, tile_tokens, rows_per_unit, return_lse;
+  int32_t N1, N2, G, T, tile_tokens, rows_per_unit, return_lse, fp16;
 };
 
 __global__ void __launch_bounds__(256) combine_kernel(const CombineParams p) {
@@ -1001,11 +1011,9 @@ __global__ void __launch_bounds__(256) combine_kernel(const CombineParams p) {
       }
     }
     const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
-    __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
-    __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
     uint2 pk;
-    pk.x = *reinterpret_cast<uint32_t*>(&lo);
-    pk.y = *reinterpret_cast<uint32_t*>(&hi);
+    pk.x = p.fp16 ? pack_f16x2(acc.x * inv, acc.y * inv) : pack_bf16x2(acc.x * inv, acc.y * inv);
+    pk.y = p.fp16 ? pack_f16x2(acc.z * inv, acc.w * inv) : pack_bf16x2(acc.z * inv, acc.w * inv);
     reinterpret_cast<uint2*>(p.out + ((int64_t)tok * p.N1 + h) * kHeadDim)[lane] = pk;
     if (lane == 0 && p.return_lse)
       p.lse[(int64_t)tok * p.N1 + h] = wsum > 0.f ? mx + logf(wsum) : -INFINITY;
@@ -1024,7 +1032,7 @@ cudaError_t launch_forward(const CUtensorMap& map_q, const CUtensorMap& map_k,
                            int32_t num_pages, int32_t tile_tokens, int32_t rows_per_unit,
                            int32_t win_left, int32_t return_lse, float scale_log2,
                            int32_t num_ctas, int64_t comb_cap, bool one_tile_blocks,
-                           cudaStream_t stream) {
+                           bool fp16, cudaStream_t stream) {
   static int configured_device = -1;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -1032,9 +1040,11 @@ cudaError_t launch_forward(const CUtensorMap& map_q, const CUtensorMap& map_k,
   if (configured_device != dev) {
     // The register re-split is only safe if the kernel launches with exactly
     // the registers the split was computed for.
-    for (int h = 0; h < 2; h++) {
-      const void* fn = h ? reinterpret_cast<const void*>(fwd_kernel<true>)
-                         : reinterpret_cast<const void*>(fwd_kernel<false>);
+    const void* fns[4] = {reinterpret_cast<const void*>(fwd_kernel<false, false>),
+                          reinterpret_cast<const void*>(fwd_kernel<true, false>),
+                          reinterpret_cast<const void*>(fwd_kernel<false, true>),
+                          reinterpret_cast<const void*>(fwd_kernel<true, true>)};
+    for (const void* fn : fns) {
       cudaFuncAttributes attr;
       e = cudaFuncGetAttributes(&attr, fn);
       if (e != cudaSuccess) return e;
@@ -1047,7 +1057,7 @@ cudaError_t launch_forward(const CUtensorMap& map_q, const CUtensorMap& map_k,
   FwdParams p;
   p.meta = meta;
   p.block_table = block_table;
-  p.out = static_cast<__nv_bfloat16*>(out);
+  p.out = static_cast<uint16_t*>(out);
   p.lse = lse;
   p.ws_o = ws_o;
   p.ws_lse = ws_lse;
@@ -1065,11 +1075,20 @@ cudaError_t launch_forward(const CUtensorMap& map_q, const CUtensorMap& map_k,
   p.win_left = win_left;
   p.return_lse = return_lse;
   p.scale_log2 = scale_log2;
-  // every Q block in one tile (decode-like): the instantiation with units in halves
-  if (one_tile_blocks)
-    fwd_kernel<true><<<num_ctas, kThreads, kSmemBytes, stream>>>(map_q, map_k, map_v, p);
-  else
-    fwd_kernel<false><<<num_ctas, kThreads, kSmemBytes, stream>>>(map_q, map_k, map_v, p);
+  // every Q block in one tile (decode-like): the instantiation with units in
+  // halves; the element type picks the MMA operand type and output packing
+  const dim3 grid(num_ctas), block(kThreads);
+  if (one_tile_blocks) {
+    if (fp16)
+      fwd_kernel<true, true><<<grid, block, kSmemBytes, stream>>>(map_q, map_k, map_v, p);
+    else
+      fwd_kernel<true, false><<<grid, block, kSmemBytes, stream>>>(map_q, map_k, map_v, p);
+  } else {
+    if (fp16)
+      fwd_kernel<false, true><<<grid, block, kSmemBytes, stream>>>(map_q, map_k, map_v, p);
+    else
+      fwd_kernel<false, false><<<grid, block, kSmemBytes, stream>>>(map_q, map_k, map_v, p);
+  }
   e = cudaGetLastError();
   if (e != cudaSuccess || comb_cap <= 0) return e;
   CombineParams c;
@@ -1087,6 +1106,7 @@ cudaError_t launch_forward(const CUtensorMap& map_q, const CUtensorMap& map_k,
   c.tile_tokens = tile_tokens;
   c.rows_per_unit = rows_per_unit;
   c.return_lse = return_lse;
+  c.fp16 = fp16 ? 1 : 0;
   combine_kernel<<<(unsigned)comb_cap, 256, 0, stream>>>(c);
   return cudaGetLastError();
 }

@@ -55,7 +55,8 @@ class _Problem(ctypes.Structure):
                 ("win_left", ctypes.c_int32), ("win_right", ctypes.c_int32),
                 ("is_packed_gqa", ctypes.c_int32), ("return_lse", ctypes.c_int32),
                 ("has_seqused_q", ctypes.c_int32), ("num_ctas", ctypes.c_int32),
-                ("max_blocks_per_split", ctypes.c_int32)]
+                ("max_blocks_per_split", ctypes.c_int32), ("dtype", ctypes.c_int32),
+                ("softmax_precision", ctypes.c_int32)]
 
 
 class _Tensors(ctypes.Structure):
@@ -88,12 +89,26 @@ class Problem:
     num_ctas: int = 0
     max_blocks_per_split: int = 0
     block_y: int = 128
+    dtype: int = 0              # 0 = bf16, 1 = fp16 (q, k, v and out)
+    softmax_precision: int = 0  # 0 = fp32 online softmax (the only one built)
 
     def as_c(self) -> _Problem:
         p = _Problem()
         for f, _ in _Problem._fields_:
             setattr(p, f, getattr(self, f))
         return p
+
+
+ABI_VERSION = 2
+DTYPE_BF16, DTYPE_FP16 = 0, 1
+
+
+def _dtype_code(t) -> int:
+    import torch
+    codes = {torch.bfloat16: DTYPE_BF16, torch.float16: DTYPE_FP16}
+    if t.dtype not in codes:
+        raise ValueError(f"expected bf16 or fp16, got {t.dtype}")
+    return codes[t.dtype]
 
 
 def library_path() -> str:
@@ -122,7 +137,7 @@ def _load():
         lib.gbsa_metadata.restype = ctypes.c_int
         lib.gbsa_forward.argtypes = [P, Tn, vp, vp, sz, vp, vp]
         lib.gbsa_forward.restype = ctypes.c_int
-        if lib.gbsa_abi_version() != 1:
+        if lib.gbsa_abi_version() != ABI_VERSION:
             raise RuntimeError("libgbsa ABI version mismatch")
         _lib = lib
         return lib
@@ -239,7 +254,7 @@ def make_problem(q, k, sparse_block_idx, block_shape, block_table, cu_seqlens_q,
                    mask_mode=mask_mode, win_left=win_left, win_right=win_right,
                    is_packed_gqa=int(bool(is_packed_gqa)), return_lse=int(bool(return_softmax_lse)),
                    has_seqused_q=int(bool(has_seqused_q)), num_ctas=num_ctas,
-                   max_blocks_per_split=max_blocks_per_split)
+                   max_blocks_per_split=max_blocks_per_split, dtype=_dtype_code(q))
 
 
 def forward(q, k, v, sparse_block_idx, sparse_block_count, block_shape: Sequence[int], *,
@@ -248,16 +263,19 @@ def forward(q, k, v, sparse_block_idx, sparse_block_count, block_shape: Sequence
             win_right: int = -1, is_packed_gqa: bool = True, return_softmax_lse: bool = False,
             num_ctas: int = 0, max_blocks_per_split: int = 0, out=None, lse=None, workspace=None,
             dev_status=None):
-    """Block-sparse paged GQA attention.  Returns (out [T,N1,D] bf16,
-    lse [T,N1,1] fp32 -- an empty tensor unless return_softmax_lse)."""
+    """Block-sparse paged GQA attention.  q, k and v share one element type,
+    bf16 or fp16.  Returns (out [T,N1,D] in that type, lse [T,N1,1] fp32 --
+    an empty tensor unless return_softmax_lse)."""
     import torch
-    q = _need(q, "q", torch.bfloat16, 3)
+    if q is None or q.dtype not in (torch.bfloat16, torch.float16):
+        raise ValueError("q: expected a bf16 or fp16 tensor")
+    q = _need(q, "q", q.dtype, 3)
     dev = q.device
     if k is None or v is None or k.dim() != 4 or v.dim() != 4:
         raise ValueError("k, v: expected [num_pages, 128, N2, D] tensors")
     for name, t in (("k", k), ("v", v)):
-        if t.dtype != torch.bfloat16 or t.device != dev:
-            raise ValueError(f"{name}: expected bf16 on {dev}")
+        if t.dtype != q.dtype or t.device != dev:
+            raise ValueError(f"{name}: expected {q.dtype} (the type of q) on {dev}")
         _, page, n2, d = t.shape
         if t.stride()[1:] != (n2 * d, d, 1):
             raise ValueError(f"{name}: only dim0 (the page axis) may be strided")
@@ -279,6 +297,10 @@ def forward(q, k, v, sparse_block_idx, sparse_block_count, block_shape: Sequence
     with torch.cuda.device(dev):
         if out is None:
             out = torch.empty_like(q)
+        else:
+            out = _need(out, "out", q.dtype, 3, dev)
+            if out.shape != q.shape:
+                raise ValueError(f"out: expected shape {tuple(q.shape)}")
         if return_softmax_lse:
             if lse is None:
                 lse = torch.empty((T, N1, 1), dtype=torch.float32, device=dev)

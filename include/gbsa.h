@@ -54,7 +54,7 @@
 extern "C" {
 #endif
 
-#define GBSA_ABI_VERSION 1
+#define GBSA_ABI_VERSION 2
 
 /* Symbols of the C ABI are exported; everything else in libgbsa is hidden. */
 #if defined(__GNUC__)
@@ -112,12 +112,20 @@ typedef struct gbsa_problem {
   int32_t has_seqused_q;      /* 1: seqused_q is given; 0: every Q storage token is used      */
   int32_t num_ctas;           /* persistent CTAs of the forward; 0 = SM count of the device   */
   int32_t max_blocks_per_split; /* 0 = automatic split-KV length; > 0 forces a smaller one     */
+  int32_t dtype;              /* element type of q, k, v and out: GBSA_DTYPE_BF16 or _FP16    */
+  int32_t softmax_precision;  /* softmaxPrecision: 0 = fp32 online softmax (the one built);
+                                 1 (fp16 softmax) returns GBSA_ERR_UNSUPPORTED               */
 } gbsa_problem;
+
+/* Element types (GBSA article, "Constraints: data types": bf16 and fp16 for
+ * Q, K, V and the output; lse is fp32 either way).  Accumulation is fp32. */
+#define GBSA_DTYPE_BF16 0
+#define GBSA_DTYPE_FP16 1
 
 /* Device pointers of one call (caller-owned).  Unused optional pointers are NULL. */
 typedef struct gbsa_tensors {
-  const void* q;               /* bf16 [T, N1, D]                                 */
-  const void* k;               /* bf16 [num_pages, 128, N2, D], page stride above */
+  const void* q;               /* dtype [T, N1, D]                                */
+  const void* k;               /* dtype [num_pages, 128, N2, D], page stride above*/
   const void* v;               /* same layout and stride as k                     */
   const int32_t* sparse_idx;   /* [N2, total_q_blocks, top_k]                     */
   const int32_t* sparse_count; /* [N2, total_q_blocks]                            */
@@ -125,7 +133,7 @@ typedef struct gbsa_tensors {
   const int32_t* seqused_q;    /* [B] or NULL (has_seqused_q = 0)                 */
   const int32_t* seqused_kv;   /* [B]                                             */
   const int32_t* block_table;  /* [B, max_pages_per_seq]                          */
-  void* out;                   /* bf16 [T, N1, D]                                 */
+  void* out;                   /* dtype [T, N1, D]                                */
   float* lse;                  /* fp32 [T, N1] or NULL (return_lse = 0)           */
 } gbsa_tensors;
 

@@ -36,7 +36,7 @@ def test_exports_every_declared_symbol(lib):
             "gbsa_workspace_size"} <= set(names)
     for n in names:
         assert hasattr(lib, n), n
-    assert lib.gbsa_abi_version() == 1
+    assert lib.gbsa_abi_version() == 2
     for code in range(0, 9):
         assert lib.gbsa_status_string(code).decode().startswith("GBSA_")
 
@@ -77,6 +77,9 @@ CASES = [
     (dict(block_x=0), "GBSA_ERR_SHAPE"),
     (dict(win_left=-2), "GBSA_ERR_INVALID_ARG"),
     (dict(scale=-1.0), "GBSA_ERR_INVALID_ARG"),
+    (dict(dtype=2), "GBSA_ERR_INVALID_ARG"),                # neither bf16 nor fp16
+    (dict(softmax_precision=1), "GBSA_ERR_UNSUPPORTED"),    # fp16 online softmax: not built
+    (dict(softmax_precision=7), "GBSA_ERR_INVALID_ARG"),
 ]
 
 
