@@ -305,6 +305,33 @@ def pool_view(w: Workload, flat):
                            (w.kv_page_stride, w.N2 * w.D, w.D, 1))
 
 
+def tnd_kv(w: Workload, kf, vf, pad_rows=None, seed=0):
+    """The same logical keys and values in the non-paged TND layout: k, v of
+    shape [T_kv, N2, D] with sequence b in rows [cu_kv[b], cu_kv[b+1]); its
+    first seqused_kv[b] rows are the positions 0.. of the paged pool, the rest
+    (``pad_rows`` per sequence, default U[0,40]) are NaN.  Returns
+    (k, v, cu_kv int64 [B+1]) on the pool's device."""
+    import torch
+
+    rng = np.random.Generator(np.random.PCG64(seed + 4242))
+    pads = (rng.integers(0, 41, size=w.B) if pad_rows is None
+            else np.broadcast_to(np.asarray(pad_rows), (w.B,)))
+    kp, vp = pool_view(w, kf), pool_view(w, vf)
+    ks, vs, lens = [], [], []
+    for b in range(w.B):
+        ku = int(w.kv_used[b])
+        pages = [int(w.block_table[b, lb]) for lb in range(-(-ku // PAGE))]
+        for src, dst in ((kp, ks), (vp, vs)):
+            rows = (torch.cat([src[pg] for pg in pages], 0)[:ku] if pages
+                    else src.new_zeros((0, w.N2, w.D)))
+            pad = src.new_full((int(pads[b]), w.N2, w.D), float("nan"))
+            dst.append(torch.cat([rows, pad], 0))
+        lens.append(ku + int(pads[b]))
+    cu = np.zeros(w.B + 1, np.int64)
+    cu[1:] = np.cumsum(lens)
+    return torch.cat(ks, 0).contiguous(), torch.cat(vs, 0).contiguous(), cu
+
+
 def bf16_bits(t) -> np.ndarray:
     """uint16 numpy copy of the bit patterns of a 16-bit (bf16 or fp16) torch
     tensor."""

@@ -56,7 +56,7 @@ def load_library(path: str):
     f = lib.gbsa_oracle_attention_rows
     i32, i64, dbl, ptr = ctypes.c_int32, ctypes.c_int64, ctypes.c_double, ctypes.c_void_p
     f.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, i32, i32, i64, dbl, i32, i32, i32,
-                  ptr, ptr, ptr, ptr, ptr, ptr, ptr, ptr, ptr, ptr, i64, ptr, ptr, i32]
+                  ptr, ptr, ptr, ptr, ptr, ptr, ptr, ptr, ptr, ptr, ptr, i64, ptr, ptr, i32]
     f.restype = ctypes.c_int
     w = lib.gbsa_oracle_widen
     w.argtypes = [i32, ptr, i64, ptr]
@@ -98,13 +98,17 @@ def widen(bits, dtype="bf16", lib=None):
 
 def attention_rows(*, q_bits, k_bits, v_bits, kv_page_stride, num_pages, sparse_idx, sparse_count,
                    cu_seqlens_q, seqused_q, seqused_kv, block_table, block_x, scale,
-                   win_left=-1, win_right=-1, rows, dtype="bf16", n_threads=None, lib=None):
+                   win_left=-1, win_right=-1, rows, dtype="bf16", cu_seqlens_kv=None,
+                   n_threads=None, lib=None):
     """Reference out/lse for selected (token, head) rows.
 
     q_bits:  uint16 [T, N1, D] -- bit patterns of the queries, bf16 or fp16
              (``dtype``); k_bits and v_bits use the same type.
     k_bits, v_bits: flat uint16 arrays of the page pool; page ``p`` row ``r``
-             head ``h`` starts at ``p*kv_page_stride + (r*N2 + h)*D``.
+             head ``h`` starts at ``p*kv_page_stride + (r*N2 + h)*D``.  With
+             ``cu_seqlens_kv`` they are TND instead: position ``p`` of
+             sequence ``b``, head ``h`` starts at ``((cu_seqlens_kv[b]+p)*N2 + h)*D``
+             (block_table, num_pages, kv_page_stride unused).
     rows:    int64 [n, 2] -- (global token index, query head).
     Returns (out [n, D] float64, lse [n] float64).  Rows past seqused_q, or
     with no visible key, give out = 0 and lse = -inf.
@@ -119,9 +123,15 @@ def attention_rows(*, q_bits, k_bits, v_bits, kv_page_stride, num_pages, sparse_
     cu = _as(cu_seqlens_q, np.int64)
     squ = _as(seqused_q, np.int32)
     sku = _as(seqused_kv, np.int32)
-    bt = _as(block_table, np.int32)
+    cukv = _as(cu_seqlens_kv, np.int64)
     B = cu.shape[0] - 1
-    need = (num_pages - 1) * kv_page_stride + 128 * N2 * D
+    if cukv is None:
+        bt = _as(block_table, np.int32)
+        max_pages = bt.shape[1]
+        need = (num_pages - 1) * kv_page_stride + 128 * N2 * D
+    else:
+        bt, max_pages, num_pages, kv_page_stride = None, 0, 0, 0
+        need = int(cukv[-1]) * N2 * D
     if k_bits.size < need or v_bits.size < need:
         raise ValueError("page pool arrays are shorter than num_pages pages")
     rows = _as(rows, np.int64).reshape(-1, 2)
@@ -129,9 +139,9 @@ def attention_rows(*, q_bits, k_bits, v_bits, kv_page_stride, num_pages, sparse_
     out = np.zeros((n, D), np.float64)
     lse = np.full((n,), -np.inf, np.float64)
     rc = (lib or _load()).gbsa_oracle_attention_rows(
-        B, T, N1, N2, D, block_x, tqb, top_k, bt.shape[1], num_pages, kv_page_stride, float(scale),
+        B, T, N1, N2, D, block_x, tqb, top_k, max_pages, num_pages, kv_page_stride, float(scale),
         win_left, win_right, DTYPES[dtype], _ptr(q_bits), _ptr(k_bits), _ptr(v_bits), _ptr(sparse_idx),
-        _ptr(sparse_count), _ptr(cu), _ptr(squ), _ptr(sku), _ptr(bt), _ptr(rows), n,
+        _ptr(sparse_count), _ptr(cu), _ptr(squ), _ptr(sku), _ptr(bt), _ptr(cukv), _ptr(rows), n,
         _ptr(out), _ptr(lse), n_threads or default_threads())
     if rc != 0:
         raise ValueError(f"oracle rejected the inputs (code {rc})")

@@ -19,7 +19,8 @@
  *            r in [0,128), that satisfy p < ku, p <= pos,
  *            (win_left  < 0 or p >= pos - win_left),
  *            (win_right < 0 or p <= pos + win_right);
- *            position p is stored in physical page block_table[b][lb], row r.
+ *            position p is stored in physical page block_table[b][lb], row r
+ *            (paged pool), or in row cu_seqlens_kv[b] + p of k and v (TND).
  *   s_p    = scale * sum_d q[tg][h][d] * k[page][r][kvh][d]
  *   out    = sum_p exp(s_p - m) v_p / sum_p exp(s_p - m),  m = max_p s_p
  *   lse    = m + ln(sum_p exp(s_p - m))
@@ -60,6 +61,7 @@ typedef struct {
   const int32_t *sparse_idx, *sparse_count;
   const int64_t* cu_seqlens_q;
   const int32_t *seqused_q, *seqused_kv, *block_table;
+  const int64_t* cu_seqlens_kv; /* TND K/V: [B+1] row offsets; NULL for the paged pool */
   const int64_t* rows; /* pairs (tg, h) */
   int64_t n_rows;
   double *out, *lse;
@@ -141,16 +143,25 @@ static int one_row(const oracle_ctx* c, int64_t tg, int32_t h, double* out, doub
   for (int64_t j = 0; j < n; j++) {
     const int64_t lb = list[j];
     if (lb < 0 || lb >= blocks_in_seq) continue; /* out-of-range entries add nothing */
-    const int64_t page = c->block_table[(int64_t)b * c->max_pages_per_seq + lb];
-    if (page < 0 || page >= c->num_pages) return 3;
+    int64_t page = -1;
+    if (!c->cu_seqlens_kv) {
+      page = c->block_table[(int64_t)b * c->max_pages_per_seq + lb];
+      if (page < 0 || page >= c->num_pages) return 3;
+    }
     for (int32_t r = 0; r < ORACLE_PAGE; r++) {
       const int64_t p = lb * ORACLE_PAGE + r;
       if (p >= ku) continue;
       if (p > pos) continue;
       if (c->win_left >= 0 && p < pos - c->win_left) continue;
       if (c->win_right >= 0 && p > pos + c->win_right) continue;
-      key_page[nk] = page;
-      key_row[nk] = r;
+      if (c->cu_seqlens_kv) {
+        /* TND: the token row of position p; the "page" stride is one row */
+        key_page[nk] = c->cu_seqlens_kv[b] + p;
+        key_row[nk] = 0;
+      } else {
+        key_page[nk] = page;
+        key_row[nk] = r;
+      }
       nk++;
     }
   }
@@ -212,8 +223,12 @@ static void* run_job(void* arg) {
  * ([n_rows][2] int64: global token index, query head).  Writes out
  * [n_rows][D] and lse [n_rows] in fp64.  kv_page_stride is in elements.
  * seqused_q may be NULL (every storage token used).  dtype: 0 = bf16,
- * 1 = fp16 element bits in q, k, v.  Returns 0 on success, nonzero if an
- * argument or a device-style value is outside its range.
+ * 1 = fp16 element bits in q, k, v.  cu_seqlens_kv == NULL: k and v are the
+ * paged pool read through block_table; otherwise they are TND [T_kv][N2][D]
+ * with sequence b in rows [cu_seqlens_kv[b], cu_seqlens_kv[b+1]) (block_table,
+ * num_pages, max_pages_per_seq and kv_page_stride are then unused).  Returns 0
+ * on success, nonzero if an argument or a device-style value is outside its
+ * range.
  */
 int gbsa_oracle_attention_rows(int32_t B, int32_t T, int32_t N1, int32_t N2, int32_t D,
                                int32_t block_x, int32_t total_q_blocks, int32_t top_k,
@@ -223,12 +238,20 @@ int gbsa_oracle_attention_rows(int32_t B, int32_t T, int32_t N1, int32_t N2, int
                                const uint16_t* v, const int32_t* sparse_idx,
                                const int32_t* sparse_count, const int64_t* cu_seqlens_q,
                                const int32_t* seqused_q, const int32_t* seqused_kv,
-                               const int32_t* block_table, const int64_t* rows, int64_t n_rows,
+                               const int32_t* block_table, const int64_t* cu_seqlens_kv,
+                               const int64_t* rows, int64_t n_rows,
                                double* out, double* lse, int32_t n_threads) {
   if (B < 1 || T < 1 || N2 < 1 || N1 < N2 || N1 % N2 || D < 1 || block_x < 1 || top_k < 1 ||
-      total_q_blocks < 1 || max_pages_per_seq < 1 || num_pages < 1 || n_rows < 0 ||
-      (dtype != 0 && dtype != 1))
+      total_q_blocks < 1 || n_rows < 0 || (dtype != 0 && dtype != 1))
     return 10;
+  if (!cu_seqlens_kv && (max_pages_per_seq < 1 || num_pages < 1)) return 10;
+  if (cu_seqlens_kv) {
+    /* TND rows: every sequence's used keys lie inside its own rows */
+    if (cu_seqlens_kv[0] != 0) return 14;
+    for (int32_t b = 0; b < B; b++)
+      if (seqused_kv[b] < 0 || seqused_kv[b] > cu_seqlens_kv[b + 1] - cu_seqlens_kv[b]) return 14;
+    kv_page_stride = (int64_t)N2 * D;
+  }
   oracle_ctx c;
   memset(&c, 0, sizeof c);
   c.B = B; c.T = T; c.N1 = N1; c.N2 = N2; c.D = D; c.block_x = block_x;
@@ -239,7 +262,7 @@ int gbsa_oracle_attention_rows(int32_t B, int32_t T, int32_t N1, int32_t N2, int
   c.widen = dtype ? widen_fp16 : widen_bf16;
   c.q = q; c.k = k; c.v = v; c.sparse_idx = sparse_idx; c.sparse_count = sparse_count;
   c.cu_seqlens_q = cu_seqlens_q; c.seqused_q = seqused_q; c.seqused_kv = seqused_kv;
-  c.block_table = block_table; c.rows = rows; c.n_rows = n_rows; c.out = out; c.lse = lse;
+  c.block_table = block_table; c.cu_seqlens_kv = cu_seqlens_kv; c.rows = rows; c.n_rows = n_rows; c.out = out; c.lse = lse;
 
   /* Q blocks are counted over storage lengths ("Constraints: block split"). */
   c.q_block_base = (int64_t*)malloc(sizeof(int64_t) * (size_t)B);

@@ -36,6 +36,21 @@ def oracle_all(w: Workload, q, kf, vf, n_threads=None, lib=None):
     return out.reshape(T, N1, w.D), lse.reshape(T, N1)
 
 
+def oracle_all_tnd(w: Workload, q, k_tnd, v_tnd, cu_kv, n_threads=None):
+    """Oracle over every row with K/V in the TND layout (see workloads.tnd_kv)."""
+    T, N1 = w.T, w.N1
+    tt, hh = np.meshgrid(np.arange(T), np.arange(N1), indexing="ij")
+    rows = np.stack([tt.reshape(-1), hh.reshape(-1)], axis=1)
+    out, lse = oracle.attention_rows(
+        q_bits=bf16_bits(q), k_bits=bf16_bits(k_tnd), v_bits=bf16_bits(v_tnd),
+        kv_page_stride=0, num_pages=0, sparse_idx=w.sparse_idx, sparse_count=w.sparse_count,
+        cu_seqlens_q=w.cu_seqlens_q, seqused_q=w.seqused_q, seqused_kv=w.kv_used,
+        block_table=None, block_x=w.block_x, scale=w.scale, win_left=w.win_left,
+        win_right=w.win_right, rows=rows, dtype=elem_dtype(q), cu_seqlens_kv=cu_kv,
+        n_threads=n_threads)
+    return out.reshape(T, N1, w.D), lse.reshape(T, N1)
+
+
 def to_f64(bits: np.ndarray, dtype: str = "bf16") -> np.ndarray:
     """Exact float64 values of 16-bit patterns, decoded with numpy (a decoder
     independent of the oracle's C code): bf16 is the upper half of a

@@ -22,8 +22,8 @@ MUTANTS = {
     "head_modulo": ("const int32_t kvh = h / G;", "const int32_t kvh = h % c->N2;"),
     "dropped_scale": ("score[i] = c->scale * dot;", "score[i] = dot;"),
     "window_off_by_one": ("p < pos - c->win_left", "p <= pos - c->win_left"),
-    "no_block_table": ("const int64_t page = c->block_table[(int64_t)b * c->max_pages_per_seq + lb];",
-                       "const int64_t page = lb;"),
+    "no_block_table": ("page = c->block_table[(int64_t)b * c->max_pages_per_seq + lb];",
+                       "page = lb;"),
     "lse_without_max": ("*lse = m + log(l);", "*lse = log(l);"),
     "qblock_without_base": ("const int64_t qb = c->q_block_base[b] + t / c->block_x;",
                             "const int64_t qb = t / c->block_x;"),

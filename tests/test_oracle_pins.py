@@ -311,3 +311,22 @@ def test_oracle_rejects_bad_page():
     w.sparse_count[0, 0] = max(int(w.sparse_count[0, 0]), 1)
     with pytest.raises(ValueError):
         oracle_all(w, q, kf, vf)
+
+
+@pytest.mark.parametrize("name", ["tiny", "window"])
+def test_tnd_layout_equals_paged_pool(name):
+    # the non-paged TND layout (k, v [T_kv, N2, D] with cu_seqlens_kv) holds the
+    # same logical keys: the oracle must give bit-identical rows; NaN padding
+    # between sequences must never be read
+    from block_sparse_paged_gbsa_b200.workloads import tnd_kv
+    from tests.helpers import oracle_all_tnd
+    w = (workload("tiny") if name == "tiny" else
+         generate(name="tw", seed=9, q_storage=[300, 90], q_used=[290, 90], kv_used=[500, 130],
+                  N1=4, N2=2, block_x=64, top_k=4, selection="random_causal", win_left=150,
+                  win_right=0, page_stride_factor=1.25))
+    q, kf, vf = make_values(w, "cpu")
+    kt, vt, cu = tnd_kv(w, kf, vf)
+    po, pl = oracle_all(w, q, kf, vf)
+    to, tl = oracle_all_tnd(w, q, kt, vt, cu)
+    assert np.array_equal(po, to) and np.array_equal(pl, tl)
+    assert np.isfinite(to).all()
