@@ -22,7 +22,8 @@ cudaError_t launch_metadata(const MetaParams& p, cudaStream_t stream);
 size_t forward_smem_bytes();
 cudaError_t launch_forward(const CUtensorMap& map_q, const CUtensorMap& map_k,
                            const CUtensorMap& map_v, const int32_t* meta,
-                           const int32_t* block_table, void* out, float* lse, float* ws_o,
+                           const int32_t* block_table, const int64_t* cu_seqlens_kv, void* out,
+                           float* lse, float* ws_o,
                            float* ws_lse, int32_t* dev_status, uint32_t signature, int32_t N1,
                            int32_t N2, int32_t T, int32_t top_k, int32_t max_pages,
                            int32_t num_pages, int32_t tile_tokens, int32_t rows_per_unit,
@@ -52,7 +53,10 @@ gbsa_status validate(const gbsa_problem* p, bool metadata_mode) {
   if (p->N1 / p->N2 > 128) return GBSA_ERR_UNSUPPORTED;
   if (p->top_k > kMaxTopK) return GBSA_ERR_UNSUPPORTED;
   if (p->mask_mode != 1) return GBSA_ERR_UNSUPPORTED;
-  if (p->is_packed_gqa != 1) return GBSA_ERR_UNSUPPORTED;
+  // is_packed_gqa = 0 (one head per tile in the article's scheduling) is
+  // accepted and run with the packed tiles: every (token, head) row's
+  // softmax is computed on its own, so the packing changes no result
+  if (p->is_packed_gqa != 0 && p->is_packed_gqa != 1) return GBSA_ERR_INVALID_ARG;
   if (p->win_left < -1 || p->win_right < -1) return GBSA_ERR_INVALID_ARG;
   if (p->return_lse != 0 && p->return_lse != 1) return GBSA_ERR_INVALID_ARG;
   if (p->has_seqused_q != 0 && p->has_seqused_q != 1) return GBSA_ERR_INVALID_ARG;
@@ -62,7 +66,10 @@ gbsa_status validate(const gbsa_problem* p, bool metadata_mode) {
   if (p->softmax_precision != 0) return GBSA_ERR_INVALID_ARG;
   if (!(p->scale >= 0.0) || isinf(p->scale)) return GBSA_ERR_INVALID_ARG;
   if ((int64_t)p->N2 * p->total_q_blocks > 0x7fffffffLL / (p->top_k + 8)) return GBSA_ERR_SHAPE;
-  if (!metadata_mode) {
+  if (p->kv_layout != GBSA_KV_PAGED && p->kv_layout != GBSA_KV_TND) return GBSA_ERR_INVALID_ARG;
+  if (!metadata_mode && p->kv_layout == GBSA_KV_TND) {
+    if (p->T_kv < 1) return GBSA_ERR_SHAPE;
+  } else if (!metadata_mode) {
     if (p->num_pages < 1 || p->max_pages_per_seq < 1) return GBSA_ERR_SHAPE;
     const int64_t page_elems = (int64_t)kPage * p->N2 * p->D;
     if (p->kv_page_stride < page_elems || p->kv_page_stride % ((int64_t)p->N2 * p->D) != 0)
@@ -264,8 +271,9 @@ gbsa_status gbsa_forward(const gbsa_problem* problem, const gbsa_tensors* t, con
                          void* workspace, size_t ws_bytes, int32_t* dev_status, void* stream) {
   gbsa_status st = validate(problem, false);
   if (st != GBSA_OK) return st;
+  const bool tnd = problem->kv_layout == GBSA_KV_TND;
   if (!t || !meta || !t->q || !t->k || !t->v || !t->sparse_idx || !t->sparse_count ||
-      !t->cu_seqlens_q || !t->seqused_kv || !t->block_table || !t->out ||
+      !t->cu_seqlens_q || !t->seqused_kv || !t->out || (tnd ? !t->cu_seqlens_kv : !t->block_table) ||
       (problem->return_lse && !t->lse) || (problem->has_seqused_q && !t->seqused_q))
     return GBSA_ERR_INVALID_ARG;
   if (!aligned16(t->q) || !aligned16(t->k) || !aligned16(t->v) || !aligned16(t->out) ||
@@ -286,7 +294,14 @@ gbsa_status gbsa_forward(const gbsa_problem* problem, const gbsa_tensors* t, con
     const cuuint32_t box[3] = {64, (cuuint32_t)g.G, (cuuint32_t)g.tile_tokens};
     if (!encode(&map_q, t->q, 3, dims, strides, box, problem->dtype)) return GBSA_ERR_CUDA;
   }
-  {
+  if (tnd) {
+    // rows of [T_kv, N2, D]; a box is 128 rows of one head (rows past T_kv read as 0)
+    const cuuint64_t dims[3] = {D, (cuuint64_t)problem->N2, (cuuint64_t)problem->T_kv};
+    const cuuint64_t strides[2] = {D * 2, (cuuint64_t)problem->N2 * D * 2};
+    const cuuint32_t box[3] = {64, 1, (cuuint32_t)kPage};
+    if (!encode(&map_k, t->k, 3, dims, strides, box, problem->dtype)) return GBSA_ERR_CUDA;
+    if (!encode(&map_v, t->v, 3, dims, strides, box, problem->dtype)) return GBSA_ERR_CUDA;
+  } else {
     const cuuint64_t dims[4] = {D, (cuuint64_t)problem->N2, (cuuint64_t)kPage,
                                 (cuuint64_t)problem->num_pages};
     const cuuint64_t strides[3] = {D * 2, (cuuint64_t)problem->N2 * D * 2,
@@ -299,7 +314,8 @@ gbsa_status gbsa_forward(const gbsa_problem* problem, const gbsa_tensors* t, con
   float* ws_o = static_cast<float*>(workspace);
   float* ws_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + wl.lse_off);
   const cudaError_t e = launch_forward(
-      map_q, map_k, map_v, static_cast<const int32_t*>(meta), t->block_table, t->out,
+      map_q, map_k, map_v, static_cast<const int32_t*>(meta), tnd ? nullptr : t->block_table,
+      tnd ? t->cu_seqlens_kv : nullptr, t->out,
       problem->return_lse ? t->lse : nullptr, ws_o, ws_lse, dev_status,
       problem_signature(problem, ctas), problem->N1, problem->N2, problem->T, problem->top_k,
       problem->max_pages_per_seq, problem->num_pages, g.tile_tokens, g.rows_per_unit,

@@ -93,7 +93,8 @@ constexpr uint32_t idesc_pv() {
 
 struct FwdParams {
   const int32_t* meta;
-  const int32_t* block_table;
+  const int32_t* block_table;  // paged K/V
+  const int64_t* cu_kv;        // TND K/V: first row of each sequence (block_table unused)
   uint16_t* out;  // bf16 or fp16 elements
   float* lse;
   float* ws_o;    // [slot_cap][rows_per_unit][128] fp32 partial outputs
@@ -214,18 +215,24 @@ __device__ __forceinline__ RowInfo row_info(const FwdParams& p, const Unit& x, i
 // producer (one thread)
 // ---------------------------------------------------------------------------
 // Called by the whole producer warp: every lane waits and counts, lane 0
-// issues the copies.
+// issues the copies.  `where` is the physical page (paged pool: 4-D map) or,
+// with `tnd`, the first row of the block in k / v [T_kv, N2, D] (3-D map).
 __device__ __forceinline__ bool produce_kv(const CUtensorMap* map, uint8_t* smem, Bars* bars,
-                                           uint32_t& kv_iter, int32_t kvh, int32_t page,
-                                           uint32_t lane) {
+                                           uint32_t& kv_iter, int32_t kvh, int32_t where,
+                                           bool tnd, uint32_t lane) {
   const uint32_t stage = kv_iter % kStages;
   if (kv_iter >= kStages && !wait_bar(&bars->kv_empty[stage], ((kv_iter / kStages) & 1) ^ 1, bars))
     return false;
   if (lane == 0) {
     uint8_t* dst = smem + kSmemRing + stage * kTileBytes;
     mbar_arrive_expect_tx(&bars->kv_full[stage], kTileBytes);
-    tma_load_4d(dst, map, &bars->kv_full[stage], 0, kvh, 0, page);
-    tma_load_4d(dst + kHalfBytes, map, &bars->kv_full[stage], 64, kvh, 0, page);
+    if (tnd) {
+      tma_load_3d(dst, map, &bars->kv_full[stage], 0, kvh, where);
+      tma_load_3d(dst + kHalfBytes, map, &bars->kv_full[stage], 64, kvh, where);
+    } else {
+      tma_load_4d(dst, map, &bars->kv_full[stage], 0, kvh, 0, where);
+      tma_load_4d(dst + kHalfBytes, map, &bars->kv_full[stage], 64, kvh, 0, where);
+    }
   }
   kv_iter++;
   return true;
@@ -263,23 +270,27 @@ __device__ void run_producer(const FwdParams& p, const CUtensorMap* map_q, const
     const int32_t n = x.j1 - x.j0;
     if (n <= 0) continue;
     const int32_t* list = p.meta + off_list + (int64_t)x.item * p.top_k + x.j0;
-    const int32_t* bt = p.block_table + (int64_t)x.b * p.max_pages;
+    const bool tnd = p.cu_kv != nullptr;
+    const int32_t* bt = tnd ? nullptr : p.block_table + (int64_t)x.b * p.max_pages;
+    const int64_t row0 = tnd ? p.cu_kv[x.b] : 0;  // TND: first row of the sequence
     // order: Q0, K_0, Q1, V_0, K_1, V_1, ... (Q1 of a unit waits for the
     // previous unit's last S1, which comes later than its last S0); a unit
     // in halves: Q0, then per block pair K_j, K_j+1, V_j, V_j+1
     // pages of the first 32 entries: the loads overlap the wait for the Q slot
+    // per lane: the page of an entry (paged), or its first row (TND); live
+    // entries lie inside the sequence, so a TND row stays inside k / v
     int32_t page = 0;
     if ((int32_t)lane < n) {
       const int32_t lb = list[lane] & kEntryLbMask;
-      page = lb < p.max_pages ? bt[lb] : -1;
+      page = tnd ? (int32_t)(row0 + (int64_t)lb * kPage) : (lb < p.max_pages ? bt[lb] : -1);
     }
     ok = produce_q(p, map_q, smem, bars, q_iter0, x, 0, lane);
     for (int32_t c0 = 0; c0 < n && ok; c0 += 32) {
       if (c0 > 0 && c0 + (int32_t)lane < n) {
         const int32_t lb = list[c0 + lane] & kEntryLbMask;
-        page = lb < p.max_pages ? bt[lb] : -1;
+        page = tnd ? (int32_t)(row0 + (int64_t)lb * kPage) : (lb < p.max_pages ? bt[lb] : -1);
       }
-      if (c0 + (int32_t)lane < n && (page < 0 || page >= p.num_pages)) {
+      if (!tnd && c0 + (int32_t)lane < n && (page < 0 || page >= p.num_pages)) {
         bad |= kDevBadPage;
         page = 0;
       }
@@ -290,18 +301,18 @@ __device__ void run_producer(const FwdParams& p, const CUtensorMap* map_q, const
           const bool has1 = jj + 1 < cn;
           const int32_t pg0 = __shfl_sync(0xffffffffu, page, jj);
           const int32_t pg1 = __shfl_sync(0xffffffffu, page, (jj + 1) & 31);
-          ok = produce_kv(map_k, smem, bars, kv_iter, x.kvh, pg0, lane);
-          if (ok && has1) ok = produce_kv(map_k, smem, bars, kv_iter, x.kvh, pg1, lane);
-          if (ok) ok = produce_kv(map_v, smem, bars, kv_iter, x.kvh, pg0, lane);
-          if (ok && has1) ok = produce_kv(map_v, smem, bars, kv_iter, x.kvh, pg1, lane);
+          ok = produce_kv(map_k, smem, bars, kv_iter, x.kvh, pg0, tnd, lane);
+          if (ok && has1) ok = produce_kv(map_k, smem, bars, kv_iter, x.kvh, pg1, tnd, lane);
+          if (ok) ok = produce_kv(map_v, smem, bars, kv_iter, x.kvh, pg0, tnd, lane);
+          if (ok && has1) ok = produce_kv(map_v, smem, bars, kv_iter, x.kvh, pg1, tnd, lane);
         }
         continue;
       }
       for (int32_t jj = 0; jj < cn && ok; jj++) {
         const int32_t pg = __shfl_sync(0xffffffffu, page, jj);
-        ok = produce_kv(map_k, smem, bars, kv_iter, x.kvh, pg, lane);
+        ok = produce_kv(map_k, smem, bars, kv_iter, x.kvh, pg, tnd, lane);
         if (ok && c0 + jj == 0 && x.nt == 2) ok = produce_q(p, map_q, smem, bars, q_iter1, x, 1, lane);
-        if (ok) ok = produce_kv(map_v, smem, bars, kv_iter, x.kvh, pg, lane);
+        if (ok) ok = produce_kv(map_v, smem, bars, kv_iter, x.kvh, pg, tnd, lane);
       }
     }
   }
@@ -1026,7 +1037,8 @@ size_t forward_smem_bytes() { return kSmemBytes; }
 
 cudaError_t launch_forward(const CUtensorMap& map_q, const CUtensorMap& map_k,
                            const CUtensorMap& map_v, const int32_t* meta,
-                           const int32_t* block_table, void* out, float* lse, float* ws_o,
+                           const int32_t* block_table, const int64_t* cu_seqlens_kv, void* out,
+                           float* lse, float* ws_o,
                            float* ws_lse, int32_t* dev_status, uint32_t signature, int32_t N1,
                            int32_t N2, int32_t T, int32_t top_k, int32_t max_pages,
                            int32_t num_pages, int32_t tile_tokens, int32_t rows_per_unit,
@@ -1057,6 +1069,7 @@ cudaError_t launch_forward(const CUtensorMap& map_q, const CUtensorMap& map_k,
   FwdParams p;
   p.meta = meta;
   p.block_table = block_table;
+  p.cu_kv = cu_seqlens_kv;
   p.out = static_cast<uint16_t*>(out);
   p.lse = lse;
   p.ws_o = ws_o;

@@ -56,13 +56,14 @@ class _Problem(ctypes.Structure):
                 ("is_packed_gqa", ctypes.c_int32), ("return_lse", ctypes.c_int32),
                 ("has_seqused_q", ctypes.c_int32), ("num_ctas", ctypes.c_int32),
                 ("max_blocks_per_split", ctypes.c_int32), ("dtype", ctypes.c_int32),
-                ("softmax_precision", ctypes.c_int32)]
+                ("softmax_precision", ctypes.c_int32), ("kv_layout", ctypes.c_int32),
+                ("T_kv", ctypes.c_int32)]
 
 
 class _Tensors(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
                 ("q", "k", "v", "sparse_idx", "sparse_count", "cu_seqlens_q", "seqused_q",
-                 "seqused_kv", "block_table", "out", "lse")]
+                 "seqused_kv", "block_table", "out", "lse", "cu_seqlens_kv")]
 
 
 @dataclasses.dataclass
@@ -91,6 +92,8 @@ class Problem:
     block_y: int = 128
     dtype: int = 0              # 0 = bf16, 1 = fp16 (q, k, v and out)
     softmax_precision: int = 0  # 0 = fp32 online softmax (the only one built)
+    kv_layout: int = 0          # 0 = paged pool + block_table, 1 = TND + cu_seqlens_kv
+    T_kv: int = 0               # TND: rows of k and v
 
     def as_c(self) -> _Problem:
         p = _Problem()
@@ -99,7 +102,7 @@ class Problem:
         return p
 
 
-ABI_VERSION = 2
+ABI_VERSION = 3
 DTYPE_BF16, DTYPE_FP16 = 0, 1
 
 
@@ -243,14 +246,20 @@ def make_problem(q, k, sparse_block_idx, block_shape, block_table, cu_seqlens_q,
                  softmax_scale=0.0, mask_mode=1, win_left=-1, win_right=-1, is_packed_gqa=True,
                  return_softmax_lse=False, has_seqused_q=False, num_ctas=0,
                  max_blocks_per_split=0) -> Problem:
-    """The gbsa_problem a forward call with these tensors describes."""
+    """The gbsa_problem a forward call with these tensors describes.  A 4-d k
+    is the page pool (block_table given); a 3-d k is TND [T_kv, N2, D]."""
     T, N1, D = q.shape
-    num_pages, page, N2, Dk = k.shape
     N2i, tqb, top_k = sparse_block_idx.shape
     bx, by = _block_shape(block_shape)
+    if k.dim() == 3:
+        T_kv, N2, Dk = k.shape
+        paged = dict(kv_layout=1, T_kv=T_kv, max_pages_per_seq=0, num_pages=0, kv_page_stride=0)
+    else:
+        num_pages, page, N2, Dk = k.shape
+        paged = dict(kv_layout=0, T_kv=0, max_pages_per_seq=block_table.shape[1],
+                     num_pages=num_pages, kv_page_stride=k.stride(0))
     return Problem(B=cu_seqlens_q.shape[0] - 1, T=T, N1=N1, N2=N2, D=D, block_x=bx, block_y=by,
-                   total_q_blocks=tqb, top_k=top_k, max_pages_per_seq=block_table.shape[1],
-                   num_pages=num_pages, kv_page_stride=k.stride(0), scale=float(softmax_scale),
+                   total_q_blocks=tqb, top_k=top_k, **paged, scale=float(softmax_scale),
                    mask_mode=mask_mode, win_left=win_left, win_right=win_right,
                    is_packed_gqa=int(bool(is_packed_gqa)), return_lse=int(bool(return_softmax_lse)),
                    has_seqused_q=int(bool(has_seqused_q)), num_ctas=num_ctas,
@@ -258,24 +267,36 @@ def make_problem(q, k, sparse_block_idx, block_shape, block_table, cu_seqlens_q,
 
 
 def forward(q, k, v, sparse_block_idx, sparse_block_count, block_shape: Sequence[int], *,
-            metadata, cu_seqlens_q, seqused_kv, block_table, seqused_q=None,
+            metadata, cu_seqlens_q, seqused_kv, block_table=None, seqused_q=None,
+            cu_seqlens_kv=None,
             softmax_scale: float = 0.0, mask_mode: int = 1, win_left: int = -1,
             win_right: int = -1, is_packed_gqa: bool = True, return_softmax_lse: bool = False,
             num_ctas: int = 0, max_blocks_per_split: int = 0, out=None, lse=None, workspace=None,
             dev_status=None):
     """Block-sparse paged GQA attention.  q, k and v share one element type,
-    bf16 or fp16.  Returns (out [T,N1,D] in that type, lse [T,N1,1] fp32 --
+    bf16 or fp16.  K/V come as the page pool [num_pages, 128, N2, D] with
+    ``block_table`` (PA_BBND), or, when ``cu_seqlens_kv`` is given, as TND
+    [T_kv, N2, D] with sequence b in rows cu_seqlens_kv[b]..cu_seqlens_kv[b+1]
+    (no block table).  Returns (out [T,N1,D] in q's type, lse [T,N1,1] fp32 --
     an empty tensor unless return_softmax_lse)."""
     import torch
     if q is None or q.dtype not in (torch.bfloat16, torch.float16):
         raise ValueError("q: expected a bf16 or fp16 tensor")
     q = _need(q, "q", q.dtype, 3)
     dev = q.device
-    if k is None or v is None or k.dim() != 4 or v.dim() != 4:
+    tnd = cu_seqlens_kv is not None
+    if tnd:
+        if k is None or v is None or k.dim() != 3 or v.dim() != 3:
+            raise ValueError("k, v: expected [T_kv, N2, D] tensors (cu_seqlens_kv given)")
+    elif k is None or v is None or k.dim() != 4 or v.dim() != 4:
         raise ValueError("k, v: expected [num_pages, 128, N2, D] tensors")
     for name, t in (("k", k), ("v", v)):
         if t.dtype != q.dtype or t.device != dev:
             raise ValueError(f"{name}: expected {q.dtype} (the type of q) on {dev}")
+        if tnd:
+            if not t.is_contiguous():
+                raise ValueError(f"{name}: TND k / v must be contiguous")
+            continue
         _, page, n2, d = t.shape
         if t.stride()[1:] != (n2 * d, d, 1):
             raise ValueError(f"{name}: only dim0 (the page axis) may be strided")
@@ -285,7 +306,8 @@ def forward(q, k, v, sparse_block_idx, sparse_block_count, block_shape: Sequence
     cnt = _need(sparse_block_count, "sparse_block_count", torch.int32, 2, dev)
     cu = _need(cu_seqlens_q, "cu_seqlens_q", torch.int64, 1, dev)
     sku = _need(seqused_kv, "seqused_kv", torch.int32, 1, dev)
-    bt = _need(block_table, "block_table", torch.int32, 2, dev)
+    bt = None if tnd else _need(block_table, "block_table", torch.int32, 2, dev)
+    cukv = _need(cu_seqlens_kv, "cu_seqlens_kv", torch.int64, 1, dev) if tnd else None
     squ = None if seqused_q is None else _need(seqused_q, "seqused_q", torch.int32, 1, dev)
     meta = _need(metadata, "metadata", torch.int32, 1, dev)
     prob = make_problem(q, k, idx, block_shape, bt, cu, softmax_scale=softmax_scale,
@@ -312,7 +334,7 @@ def forward(q, k, v, sparse_block_idx, sparse_block_count, block_shape: Sequence
         ten = _Tensors(q=_ptr(q), k=_ptr(k), v=_ptr(v), sparse_idx=_ptr(idx),
                        sparse_count=_ptr(cnt), cu_seqlens_q=_ptr(cu), seqused_q=_ptr(squ),
                        seqused_kv=_ptr(sku), block_table=_ptr(bt), out=_ptr(out),
-                       lse=_ptr(lse) if return_softmax_lse else None)
+                       lse=_ptr(lse) if return_softmax_lse else None, cu_seqlens_kv=_ptr(cukv))
         _check(_load().gbsa_forward(ctypes.byref(prob.as_c()), ctypes.byref(ten),
                                     meta.data_ptr(), workspace.data_ptr(),
                                     workspace.numel() * workspace.element_size(),

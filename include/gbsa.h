@@ -54,7 +54,7 @@
 extern "C" {
 #endif
 
-#define GBSA_ABI_VERSION 2
+#define GBSA_ABI_VERSION 3
 
 /* Symbols of the C ABI are exported; everything else in libgbsa is hidden. */
 #if defined(__GNUC__)
@@ -107,7 +107,9 @@ typedef struct gbsa_problem {
   int32_t mask_mode;          /* 1 = built-in causal (the only mode the article supports)    */
   int32_t win_left;           /* -1 = unbounded; else keys >= pos - win_left are kept         */
   int32_t win_right;          /* -1 = unbounded; else keys <= pos + win_right are kept        */
-  int32_t is_packed_gqa;      /* 1: the G heads of a group share each K/V tile (required)    */
+  int32_t is_packed_gqa;      /* 1: the G heads of a group share each K/V tile; 0 (a head per
+                                 tile) is accepted and gives the same rows: the library always
+                                 packs, and no row's arithmetic depends on the packing        */
   int32_t return_lse;         /* 1: write lse                                                 */
   int32_t has_seqused_q;      /* 1: seqused_q is given; 0: every Q storage token is used      */
   int32_t num_ctas;           /* persistent CTAs of the forward; 0 = SM count of the device   */
@@ -115,7 +117,19 @@ typedef struct gbsa_problem {
   int32_t dtype;              /* element type of q, k, v and out: GBSA_DTYPE_BF16 or _FP16    */
   int32_t softmax_precision;  /* softmaxPrecision: 0 = fp32 online softmax (the one built);
                                  1 (fp16 softmax) returns GBSA_ERR_UNSUPPORTED               */
+  int32_t kv_layout;          /* GBSA_KV_PAGED (k, v: the page pool, block_table) or
+                                 GBSA_KV_TND (k, v: [T_kv, N2, D], cu_seqlens_kv)             */
+  int32_t T_kv;               /* GBSA_KV_TND: rows of k and v (= cu_seqlens_kv[B]); else 0   */
 } gbsa_problem;
+
+/* K/V layouts (GBSA article, "Constraints: layouts": PA_BBND page pool, or
+ * TND with cuSeqLengthsKv).  TND: sequence b's keys are rows
+ * [cu_seqlens_kv[b], cu_seqlens_kv[b+1]) of k and v, contiguous, and a
+ * "block" lb of its list is rows cu_seqlens_kv[b] + 128*lb ...; block_table,
+ * num_pages, max_pages_per_seq and kv_page_stride are unused.  seqused_kv is
+ * required in both layouts and must not exceed the sequence's TND rows. */
+#define GBSA_KV_PAGED 0
+#define GBSA_KV_TND 1
 
 /* Element types (GBSA article, "Constraints: data types": bf16 and fp16 for
  * Q, K, V and the output; lse is fp32 either way).  Accumulation is fp32. */
@@ -135,6 +149,7 @@ typedef struct gbsa_tensors {
   const int32_t* block_table;  /* [B, max_pages_per_seq]                          */
   void* out;                   /* dtype [T, N1, D]                                */
   float* lse;                  /* fp32 [T, N1] or NULL (return_lse = 0)           */
+  const int64_t* cu_seqlens_kv; /* [B+1] for GBSA_KV_TND, else NULL               */
 } gbsa_tensors;
 
 /* Version of this header the library was built from (GBSA_ABI_VERSION). */

@@ -36,7 +36,7 @@ def test_exports_every_declared_symbol(lib):
             "gbsa_workspace_size"} <= set(names)
     for n in names:
         assert hasattr(lib, n), n
-    assert lib.gbsa_abi_version() == 2
+    assert lib.gbsa_abi_version() == 3
     for code in range(0, 9):
         assert lib.gbsa_status_string(code).decode().startswith("GBSA_")
 
@@ -71,7 +71,7 @@ CASES = [
     (dict(N1=258, N2=2), "GBSA_ERR_UNSUPPORTED"),
     (dict(top_k=257), "GBSA_ERR_UNSUPPORTED"),
     (dict(mask_mode=0), "GBSA_ERR_UNSUPPORTED"),
-    (dict(is_packed_gqa=0), "GBSA_ERR_UNSUPPORTED"),
+    (dict(is_packed_gqa=2), "GBSA_ERR_INVALID_ARG"),
     (dict(B=0), "GBSA_ERR_SHAPE"),
     (dict(top_k=0), "GBSA_ERR_SHAPE"),
     (dict(block_x=0), "GBSA_ERR_SHAPE"),
@@ -80,6 +80,7 @@ CASES = [
     (dict(dtype=2), "GBSA_ERR_INVALID_ARG"),                # neither bf16 nor fp16
     (dict(softmax_precision=1), "GBSA_ERR_UNSUPPORTED"),    # fp16 online softmax: not built
     (dict(softmax_precision=7), "GBSA_ERR_INVALID_ARG"),
+    (dict(kv_layout=2), "GBSA_ERR_INVALID_ARG"),            # neither paged nor TND
 ]
 
 
@@ -96,6 +97,7 @@ FWD_CASES = [
     (dict(kv_page_stride=128 * 2 * 128 + 128), "GBSA_ERR_SHAPE"),      # not a multiple of N2*D
     (dict(num_pages=0), "GBSA_ERR_SHAPE"),
     (dict(T=0), "GBSA_ERR_SHAPE"),
+    (dict(kv_layout=1, T_kv=0), "GBSA_ERR_SHAPE"),          # TND without rows
 ]
 
 

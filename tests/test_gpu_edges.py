@@ -10,7 +10,7 @@ import numpy as np
 import pytest
 import torch
 
-from block_sparse_paged_gbsa_b200.workloads import generate, workload
+from block_sparse_paged_gbsa_b200.workloads import generate, make_values, workload
 from tests.gpu_helpers import run_gpu
 from tests.helpers import assert_lse_close, assert_out_close, oracle_all
 
@@ -81,3 +81,26 @@ def test_group_of_128_one_token_per_tile():
                  selection="random_causal")
     q, kf, vf, meta, out, lse = run_gpu(w)
     _compare_all(w, q, kf, vf, out, lse)
+
+
+def test_unpacked_gqa_gives_the_same_rows():
+    # is_packed_gqa = 0 (the article's per-head scheduling) is computed with
+    # the packed tiles; every row's arithmetic is independent of the packing
+    import block_sparse_paged_gbsa_b200 as gbsa
+    from block_sparse_paged_gbsa_b200.workloads import pool_view
+    from tests.gpu_helpers import device_tensors, run_metadata
+    w = workload("tiny")
+    q, kf, vf = make_values(w, "cuda")
+    t = device_tensors(w)
+    outs = []
+    for packed in (True, False):
+        meta = gbsa.metadata(t["idx"], t["cnt"], w.N1, w.N2, w.D, [w.block_x, 128],
+                             cu_seqlens_q=t["cu"], seqused_q=t["squ"], seqused_kv=t["sku"],
+                             num_tokens=w.T, is_packed_gqa=packed)
+        outs.append(gbsa.forward(q, pool_view(w, kf), pool_view(w, vf), t["idx"], t["cnt"],
+                                 [w.block_x, 128], metadata=meta, cu_seqlens_q=t["cu"],
+                                 seqused_q=t["squ"], seqused_kv=t["sku"], block_table=t["bt"],
+                                 softmax_scale=w.scale, is_packed_gqa=packed,
+                                 return_softmax_lse=True))
+    torch.cuda.synchronize()
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
