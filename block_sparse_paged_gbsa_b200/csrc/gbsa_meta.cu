@@ -241,10 +241,10 @@ struct PieceShape {
   int32_t cA, cB;  // long / short pieces per tile pair
 };
 
-__device__ __forceinline__ PieceShape piece_shape(const int32_t* item_row, int32_t L) {
+__device__ __forceinline__ PieceShape piece_shape(int32_t U, int32_t n, int32_t L) {
   PieceShape s;
-  s.U = (item_row[2] + 1) / 2;
-  s.n = item_row[1];
+  s.U = U;
+  s.n = n;
   s.k = s.n <= L ? 1 : (s.n + L - 1) / L;
   s.a = s.n / s.k;
   s.cA = s.n - s.k * s.a;
@@ -252,8 +252,60 @@ __device__ __forceinline__ PieceShape piece_shape(const int32_t* item_row, int32
   return s;
 }
 
+// Block-wide exclusive scans of NV int64 values per thread in one pass (one
+// set of barriers).  `scratch` holds 32 * NV int64.  res[v] gets the
+// exclusive prefix of v[v], total[v] the block sum.
+template <int NV>
+__device__ void block_exclusive_scan_n(const int64_t (&v)[NV], int64_t* scratch, int64_t (&res)[NV],
+                                       int64_t (&total)[NV]) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  int64_t incl[NV];
+#pragma unroll
+  for (int c = 0; c < NV; c++) incl[c] = v[c];
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+#pragma unroll
+    for (int c = 0; c < NV; c++) {
+      const int64_t n = __shfl_up_sync(0xffffffffu, incl[c], o);
+      if (lane >= o) incl[c] += n;
+    }
+  }
+  __syncthreads();
+  if (lane == 31) {
+#pragma unroll
+    for (int c = 0; c < NV; c++) scratch[32 * c + warp] = incl[c];
+  }
+  __syncthreads();
+  if (warp < NV) {
+    int64_t w = lane < nwarps ? scratch[32 * warp + lane] : 0;
+    int64_t wi = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int64_t n = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += n;
+    }
+    // lanes >= nwarps add 0, so lane 31's inclusive sum is the total; write
+    // it after every lane has read its own slot
+    __syncwarp();
+    if (lane < nwarps) scratch[32 * warp + lane] = wi - w;
+    if (lane == 31) scratch[32 * NV + warp] = wi;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int c = 0; c < NV; c++) {
+    res[c] = scratch[32 * c + warp] + incl[c] - v[c];
+    total[c] = scratch[32 * NV + c];
+  }
+  __syncthreads();
+}
+
+// Item fields (tile pairs, live blocks) of the first kPlanCache chunks of
+// blockDim items stay in registers across the three passes; further items
+// are re-read from the item table.
+constexpr int kPlanCache = 4;
+
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const MetaParams p) {
-  __shared__ int64_t scratch[32];
+  __shared__ int64_t scratch[32 * 4];
   __shared__ int32_t hist[kNumKeys];
   __shared__ int32_t bucket_start[kNumKeys];
   __shared__ int32_t key_run[kNumKeys];
@@ -266,6 +318,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const MetaParams p) 
   const int32_t* items = meta + g.off_item;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t n_items = g.n_items;
+  const int64_t chunks = (n_items + blockDim.x - 1) / blockDim.x;
 
   for (int i = tid; i < kNumKeys; i += blockDim.x) {
     hist[i] = 0;
@@ -273,6 +326,38 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const MetaParams p) 
   }
   for (int i = tid; i < kPlanWarps * kNumKeys; i += blockDim.x) (&warp_key[0][0])[i] = 0;
   if (tid == 0) abort_sh = (meta[H_STATUS] & kDevBadSeqlen) ? 1 : 0;
+
+  // the item fields of this thread's items (chunk k: item k * blockDim + tid)
+  int32_t cU[kPlanCache], cn[kPlanCache];
+#pragma unroll
+  for (int k = 0; k < kPlanCache; k++) {
+    const int64_t i = (int64_t)k * blockDim.x + tid;
+    cU[k] = 0;
+    cn[k] = 0;
+    if (i < n_items) {
+      // item rows are 8 words on a 16-byte boundary: (.., n, n_tiles, ..)
+      const int4 r = *reinterpret_cast<const int4*>(items + 8 * i);
+      cn[k] = r.y;
+      cU[k] = (r.z + 1) / 2;
+    }
+  }
+  auto fields = [&](int64_t k, int32_t& U, int32_t& n) {
+    U = 0;
+    n = 0;
+#pragma unroll
+    for (int c = 0; c < kPlanCache; c++)
+      if (c == k) {
+        U = cU[c];
+        n = cn[c];
+      }
+    if (k >= kPlanCache) {
+      const int64_t i = k * blockDim.x + tid;
+      if (i < n_items) {
+        n = items[8 * i + 1];
+        U = (items[8 * i + 2] + 1) / 2;
+      }
+    }
+  };
   __syncthreads();
   if (abort_sh) {
     if (tid == 0) {
@@ -288,33 +373,41 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const MetaParams p) 
 
   // pass 1: total cost
   int64_t cost = 0;
-  for (int64_t i = tid; i < n_items; i += blockDim.x) {
-    const int32_t* r = items + 8 * i;
-    cost += (int64_t)((r[2] + 1) / 2) * r[1];
+  for (int64_t k = 0; k < chunks; k++) {
+    int32_t U, n;
+    fields(k, U, n);
+    cost += (int64_t)U * n;
   }
-  int64_t total_cost;
-  block_exclusive_scan(cost, scratch, &total_cost);
+  {
+    const int64_t v[1] = {cost};
+    int64_t r[1], t[1];
+    block_exclusive_scan_n<1>(v, scratch, r, t);
+    cost = t[0];
+  }
   if (tid == 0) {
     int64_t L;
     if (p.forced_split > 0) {
       L = p.forced_split;
     } else {
-      L = cdiv64(total_cost, 4LL * p.num_ctas);
+      L = cdiv64(cost, 4LL * p.num_ctas);
       if (L < kMinSplitLen) L = kMinSplitLen;
     }
     if (L > 0x7fffffffLL) L = 0x7fffffffLL;
     split_len_sh = (int32_t)L;
     meta[H_SPLIT_LEN] = (int32_t)L;
-    meta[H_COST_LO] = (int32_t)(uint32_t)(total_cost & 0xffffffffLL);
-    meta[H_COST_HI] = (int32_t)(uint32_t)((uint64_t)total_cost >> 32);
+    meta[H_COST_LO] = (int32_t)(uint32_t)(cost & 0xffffffffLL);
+    meta[H_COST_HI] = (int32_t)(uint32_t)((uint64_t)cost >> 32);
   }
   __syncthreads();
   const int32_t L = split_len_sh;
 
   // pass 2: histogram of piece lengths (weighted), totals
   int64_t pieces = 0, slots = 0, combs = 0;
-  for (int64_t i = tid; i < n_items; i += blockDim.x) {
-    const PieceShape s = piece_shape(items + 8 * i, L);
+  for (int64_t k = 0; k < chunks; k++) {
+    int32_t U, n;
+    fields(k, U, n);
+    if (k * blockDim.x + tid >= n_items) continue;
+    const PieceShape s = piece_shape(U, n, L);
     if (s.cA) atomicAdd(&hist[s.a + 1], s.U * s.cA);
     if (s.cB) atomicAdd(&hist[s.a], s.U * s.cB);
     pieces += (int64_t)s.U * s.k;
@@ -324,9 +417,23 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const MetaParams p) 
     }
   }
   int64_t n_units, n_slots, n_comb;
-  block_exclusive_scan(pieces, scratch, &n_units);
-  block_exclusive_scan(slots, scratch, &n_slots);
-  block_exclusive_scan(combs, scratch, &n_comb);
+  {
+    const int64_t v[3] = {pieces, slots, combs};
+    int64_t r[3], t[3];
+    block_exclusive_scan_n<3>(v, scratch, r, t);  // its barriers also publish hist
+    n_units = t[0];
+    n_slots = t[1];
+    n_comb = t[2];
+  }
+  // bucket starts, longest first: an exclusive scan over the keys in
+  // descending order (thread j holds key kNumKeys - 1 - j)
+  {
+    const int key = kNumKeys - 1 - tid;
+    const int64_t v[1] = {tid < kNumKeys ? (int64_t)hist[key] : 0};
+    int64_t r[1], t[1];
+    block_exclusive_scan_n<1>(v, scratch, r, t);
+    if (tid < kNumKeys) bucket_start[key] = (int32_t)r[0];
+  }
   if (tid == 0) {
     const bool over = n_units > g.unit_cap || n_slots > g.slot_cap || n_comb > g.comb_cap;
     abort_sh = over ? 1 : 0;
@@ -334,12 +441,6 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const MetaParams p) 
     meta[H_NSLOTS] = over ? 0 : (int32_t)n_slots;
     meta[H_NCOMB] = over ? 0 : (int32_t)n_comb;
     if (over) raise_status(p, kDevCapacity);
-    // bucket starts, longest first
-    int32_t acc = 0;
-    for (int key = kNumKeys - 1; key >= 0; key--) {
-      bucket_start[key] = acc;
-      acc += hist[key];
-    }
   }
   __syncthreads();
   if (abort_sh) return;
@@ -348,11 +449,15 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const MetaParams p) 
   int32_t* units = meta + g.off_unit;
   int32_t* comb = meta + g.off_comb;
   int64_t slot_run = 0, comb_run = 0;
-  for (int64_t base = 0; base < n_items; base += blockDim.x) {
-    const int64_t i = base + tid;
+  for (int64_t k = 0; k < chunks; k++) {
+    const int64_t i = k * blockDim.x + tid;
     PieceShape s{0, 0, 1, 0, 0, 0};
     const bool valid = i < n_items;
-    if (valid) s = piece_shape(items + 8 * i, L);
+    if (valid) {
+      int32_t U, n;
+      fields(k, U, n);
+      s = piece_shape(U, n, L);
+    }
     const int32_t kA = (valid && s.cA) ? s.a + 1 : -1;
     const int32_t wA = (valid && s.cA) ? s.U * s.cA : 0;
     const int32_t kB = (valid && s.cB) ? s.a : -1;
@@ -373,11 +478,16 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const MetaParams p) 
     if (kB >= 0) atomicAdd(&warp_key[warp][kB], wB);
     const int64_t my_slots = (valid && s.k > 1) ? (int64_t)s.U * s.k : 0;
     const int64_t my_combs = (valid && s.k > 1) ? s.U : 0;
-    int64_t tot_slots, tot_combs;
-    const int64_t slot_base = slot_run + block_exclusive_scan(my_slots, scratch, &tot_slots);
-    const int64_t comb_base = comb_run + block_exclusive_scan(my_combs, scratch, &tot_combs);
-    slot_run += tot_slots;
-    comb_run += tot_combs;
+    int64_t slot_base, comb_base;
+    {
+      const int64_t v[2] = {my_slots, my_combs};
+      int64_t r[2], t[2];
+      block_exclusive_scan_n<2>(v, scratch, r, t);  // its barriers also publish warp_key
+      slot_base = slot_run + r[0];
+      comb_base = comb_run + r[1];
+      slot_run += t[0];
+      comb_run += t[1];
+    }
     // per key: exclusive prefix over warps, plus the run of earlier chunks
     for (int key = tid; key < kNumKeys; key += blockDim.x) {
       int32_t acc = key_run[key];
