@@ -36,6 +36,29 @@ def oracle_all(w: Workload, q, kf, vf, n_threads=None, lib=None):
     return out.reshape(T, N1, w.D), lse.reshape(T, N1)
 
 
+def oracle_rows_fp8(w: Workload, q8, kf8, vf8, scales, rows, n_threads=None):
+    """Oracle rows for E4M3 inputs with per-tensor dequantization scales
+    (q_scale, k_scale, v_scale): every E4M3 value is exact in fp16, so the
+    values go to the oracle's fp16 decode unchanged; the scores carry
+    scale * q_scale * k_scale and the output v_scale.  Returns (out, lse,
+    out_abs) with out_abs = sum_p w_p |v_scale * v_p| (the error scale of a
+    rounding of the weights)."""
+    import torch
+
+    qs, ks, vs = scales
+    rows = np.asarray(rows, np.int64).reshape(-1, 2)
+    out_abs = np.zeros((rows.shape[0], w.D), np.float64)
+    out, lse = oracle.attention_rows(
+        q_bits=bf16_bits(q8.to(torch.float16)), k_bits=bf16_bits(kf8.to(torch.float16)),
+        v_bits=bf16_bits(vf8.to(torch.float16)), kv_page_stride=w.kv_page_stride,
+        num_pages=w.num_pages, sparse_idx=w.sparse_idx, sparse_count=w.sparse_count,
+        cu_seqlens_q=w.cu_seqlens_q, seqused_q=w.seqused_q, seqused_kv=w.kv_used,
+        block_table=w.block_table, block_x=w.block_x, scale=w.scale * qs * ks,
+        win_left=w.win_left, win_right=w.win_right, rows=rows, dtype="fp16", out_abs=out_abs,
+        n_threads=n_threads)
+    return out * vs, lse, out_abs * abs(vs)
+
+
 def oracle_all_tnd(w: Workload, q, k_tnd, v_tnd, cu_kv, n_threads=None):
     """Oracle over every row with K/V in the TND layout (see workloads.tnd_kv)."""
     T, N1 = w.T, w.N1
