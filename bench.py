@@ -65,6 +65,9 @@ def parse_args():
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--dtype", default="bf16", choices=["bf16", "fp16", "e4m3"],
+                    help="element type of q, k and v (e4m3: the quantised mode with "
+                         "per-tensor dequantization scales, bf16 out)")
     ap.add_argument("--scale-down", type=int, default=1,
                     help="shrink the workload's sequence lengths by this factor (same "
                          "structure); for profiler captures that must stay small")
@@ -75,6 +78,8 @@ def describe(args) -> str:
     d = DESCRIPTIONS[args.workload]
     if args.scale_down != 1:
         d += f" -- sequence lengths scaled down {args.scale_down}x (profiling case)"
+    if args.dtype != "bf16":
+        d += f" -- q, k, v in {args.dtype}"
     return d
 
 
@@ -202,13 +207,22 @@ def cpu_cores() -> int:
     return len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
 
 
-def oracle_sample(w, q, kf, vf, target_s: float, seed: int = 0):
+def oracle_sample(w, q, kf, vf, target_s: float, seed: int = 0, scales=(1.0, 1.0, 1.0)):
     """Times the oracle on a bounded random sample of rows sized to about
-    target_s seconds.  Returns (TFLOPS, seconds, rows, description)."""
+    target_s seconds.  E4M3 values go to the oracle as fp16 (exact) with the
+    dequantization scales folded in.  Returns (TFLOPS, seconds, rows,
+    description)."""
+    import torch
     import oracle
     from block_sparse_paged_gbsa_b200.accounting import row_flops
     from block_sparse_paged_gbsa_b200.workloads import bf16_bits
 
+    if q.dtype == torch.float8_e4m3fn:
+        q, kf, vf = (t.to(torch.float16) for t in (q, kf, vf))
+        scale = w.scale * scales[0] * scales[1]
+    else:
+        scale = w.scale
+    odt = "fp16" if q.dtype == torch.float16 else "bf16"
     qb, kb, vb = bf16_bits(q), bf16_bits(kf), bf16_bits(vf)
     rng = np.random.default_rng(seed)
     threads = cpu_cores()
@@ -220,9 +234,9 @@ def oracle_sample(w, q, kf, vf, target_s: float, seed: int = 0):
                               num_pages=w.num_pages, sparse_idx=w.sparse_idx,
                               sparse_count=w.sparse_count, cu_seqlens_q=w.cu_seqlens_q,
                               seqused_q=w.seqused_q, seqused_kv=w.kv_used,
-                              block_table=w.block_table, block_x=w.block_x, scale=w.scale,
+                              block_table=w.block_table, block_x=w.block_x, scale=scale,
                               win_left=w.win_left, win_right=w.win_right, rows=rows,
-                              n_threads=threads)
+                              dtype=odt, n_threads=threads)
         return time.perf_counter() - t0, rows
 
     n = 4 * threads
@@ -295,8 +309,11 @@ def main():
     # each rank: its own seeded batch of the same workload (weak scaling)
     base = workload(args.workload, scale_down=args.scale_down)
     w = workload(args.workload, seed=rank_seed(base.seed, rank), scale_down=args.scale_down)
-    acc = work(w)
-    q, kf, vf = make_values(w, dev)
+    tdt = {"bf16": torch.bfloat16, "fp16": torch.float16, "e4m3": torch.float8_e4m3fn}[args.dtype]
+    fp8 = args.dtype == "e4m3"
+    scales = (1.0, 1.0, 1.0)  # E4M3 dequantization scales (the speed does not depend on them)
+    acc = work(w, in_bytes=1 if fp8 else 2)
+    q, kf, vf = make_values(w, dev, dtype=tdt)
     to = lambda a, dt: torch.as_tensor(np.ascontiguousarray(a), dtype=dt, device=dev)
     idx, cnt = to(w.sparse_idx, torch.int32), to(w.sparse_count, torch.int32)
     cu, sku, bt = to(w.cu_seqlens_q, torch.int64), to(w.kv_used, torch.int32), to(w.block_table, torch.int32)
@@ -305,10 +322,11 @@ def main():
     block_shape = [w.block_x, 128]
     prob = gbsa.gbsa.make_problem(q, k, idx, block_shape, bt, cu, softmax_scale=w.scale,
                                   win_left=w.win_left, win_right=w.win_right,
-                                  return_softmax_lse=w.return_lse, has_seqused_q=squ is not None)
+                                  return_softmax_lse=w.return_lse, has_seqused_q=squ is not None,
+                                  dequant_scales=scales)
     meta_buf = torch.empty(gbsa.metadata_size(prob) // 4, dtype=torch.int32, device=dev)
     ws = torch.empty(max(gbsa.workspace_size(prob), 16), dtype=torch.uint8, device=dev)
-    out = torch.empty_like(q)
+    out = torch.empty(q.shape, dtype=torch.bfloat16 if fp8 else tdt, device=dev)
     lse = torch.empty((w.T, w.N1, 1), dtype=torch.float32, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
@@ -326,7 +344,9 @@ def main():
                      seqused_q=su, seqused_kv=kv, block_table=tb, softmax_scale=w.scale,
                      win_left=w.win_left, win_right=w.win_right,
                      return_softmax_lse=w.return_lse, out=out if oo is None else oo,
-                     lse=lse if ll is None else ll, workspace=ws, dev_status=status)
+                     lse=lse if ll is None else ll, workspace=ws, dev_status=status,
+                     q_dequant_scale=scales[0], k_dequant_scale=scales[1],
+                     v_dequant_scale=scales[2])
         if ev is not None:
             ev[2].record()
 
@@ -431,26 +451,31 @@ def main():
                             "steps overlap on three streams"}
 
     peaks = load_peaks()
+    # the tensor peak of the operand type: fp16 runs at the bf16 rate, E4M3 at
+    # twice it (the nominal dense ratio, 4.5 / 2.25 PFLOP/s)
+    t_peak = peaks["bf16_tflops"] * (2.0 if fp8 else 1.0)
     flops, nbytes = acc["flops_block"], acc["bytes"]
     value = job_value(total_flops, step_ms)
-    t_roof = max(flops / (peaks["bf16_tflops"] * 1e12), nbytes / (peaks["hbm_gbs"] * 1e9))
-    bound = "tensor" if flops / (peaks["bf16_tflops"] * 1e12) >= nbytes / (peaks["hbm_gbs"] * 1e9) else "hbm"
+    t_roof = max(flops / (t_peak * 1e12), nbytes / (peaks["hbm_gbs"] * 1e9))
+    bound = "tensor" if flops / (t_peak * 1e12) >= nbytes / (peaks["hbm_gbs"] * 1e9) else "hbm"
     if bound == "tensor":
         achieved = flops / (fwd_ms * 1e-3) / 1e12
-        roof = {"bound": "tensor", "achieved": round(achieved, 3), "peak": peaks["bf16_tflops"],
-                "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4)}
+        roof = {"bound": "tensor", "achieved": round(achieved, 3), "peak": round(t_peak, 3),
+                "unit": "TFLOP/s", "frac": round(achieved / t_peak, 4)}
     else:
         achieved = nbytes / (fwd_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": round(achieved, 3), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4)}
-    roof["traffic"] = profiled_traffic(args.workload) if args.scale_down == 1 else None
+    roof["traffic"] = (profiled_traffic(args.workload)
+                       if args.scale_down == 1 and args.dtype == "bf16" else None)
     roof["kernel"] = "gbsa forward (attention + split-KV combine launch)"
-    roof["peak_source"] = peaks["source"] + " (burst)"
+    roof["peak_source"] = peaks["source"] + " (burst)" + (
+        "; E4M3 tensor peak = measured bf16 x 2 (nominal ratio)" if fp8 and bound == "tensor" else "")
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         qc, kc, vc = q.cpu(), kf.cpu(), vf.cpu()
-        tf, dt, n, threads = oracle_sample(w, qc, kc, vc, args.cpu_seconds)
+        tf, dt, n, threads = oracle_sample(w, qc, kc, vc, args.cpu_seconds, scales=scales)
         cpu = {"value": round(tf, 8), "unit": UNIT, "cores": threads, "kind": "oracle",
                "sample": f"{n} random (token, head) rows of the same workload, {dt:.1f} s"}
 
@@ -458,8 +483,8 @@ def main():
         line = {
             "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": round(step_ms, 4),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": args.dtype, "data": "synthetic",
             "config": {"workload": describe(args),
                        "parallelism": f"dp{world} (independent batches, no collective)",
                        "l2": "flushed between timed steps (256 MiB write)",

@@ -9,9 +9,11 @@ Definitions (what the benchmark reports):
   4 * used_rows * G * keys_in_block * D  (QK^T and PV, 2 FLOPs per MAC);
 * element-exact FLOPs: 4 * D * the number of visible (query row, head, key)
   triples, i.e. without the masked parts of partial blocks;
-* algorithmic bytes: Q and O (bf16, used rows), LSE (fp32) if requested,
-  64 KiB of K+V per live (Q block, KV head, block) -- what the method moves
-  without cache reuse -- plus the index, count and block-table words.
+* algorithmic bytes: Q and O (used rows; 2 bytes per element, Q 1 byte for
+  E4M3 inputs), LSE (fp32) if requested, 2 x 128 x D elements of K+V per live
+  (Q block, KV head, block) -- 64 KiB for 16-bit types, 32 KiB for E4M3: what
+  the method moves without cache reuse -- plus the index, count and
+  block-table words.
 """
 from __future__ import annotations
 
@@ -35,7 +37,9 @@ def _items(w: Workload):
     return b_of_qb, n_used, pos0, ku[b_of_qb]
 
 
-def work(w: Workload, exact: bool = True) -> dict:
+def work(w: Workload, exact: bool = True, in_bytes: int = 2) -> dict:
+    """in_bytes: bytes per element of q, k and v (2, or 1 for E4M3); out is
+    always 2 bytes per element."""
     b_of_qb, n_used, pos0, ku = _items(w)
     n = np.clip(w.sparse_count.astype(np.int64), 0, w.top_k)           # [N2, TQB]
     j = np.arange(w.top_k)[None, None, :]
@@ -55,9 +59,9 @@ def work(w: Workload, exact: bool = True) -> dict:
     flops_block = float((4 * n_used[None, :, None] * G * keys * D).sum())
     n_live = int(live.sum())
     res = dict(flops_block=flops_block, live_blocks=n_live, selected_blocks=int(sel.sum()),
-               kv_bytes=float(n_live) * 2 * PAGE * D * 2)
+               kv_bytes=float(n_live) * 2 * PAGE * D * in_bytes)
     used_rows = int(n_used.sum())
-    res["q_bytes"] = float(used_rows * w.N1 * D * 2)
+    res["q_bytes"] = float(used_rows * w.N1 * D * in_bytes)
     res["o_bytes"] = float(used_rows * w.N1 * D * 2)
     res["lse_bytes"] = float(used_rows * w.N1 * 4) if w.return_lse else 0.0
     res["index_bytes"] = float(w.sparse_idx.nbytes + w.sparse_count.nbytes + w.block_table.nbytes)

@@ -29,7 +29,7 @@ cudaError_t launch_forward(const CUtensorMap& map_q, const CUtensorMap& map_k,
                            int32_t num_pages, int32_t tile_tokens, int32_t rows_per_unit,
                            int32_t win_left, int32_t return_lse, float scale_log2,
                            int32_t num_ctas, int64_t comb_cap, bool one_tile_blocks,
-                           bool fp16, cudaStream_t stream);
+                           int32_t dtype, float out_scale, cudaStream_t stream);
 }  // namespace gbsa
 
 using namespace gbsa;
@@ -61,7 +61,18 @@ gbsa_status validate(const gbsa_problem* p, bool metadata_mode) {
   if (p->return_lse != 0 && p->return_lse != 1) return GBSA_ERR_INVALID_ARG;
   if (p->has_seqused_q != 0 && p->has_seqused_q != 1) return GBSA_ERR_INVALID_ARG;
   if (p->num_ctas < 0 || p->max_blocks_per_split < 0) return GBSA_ERR_INVALID_ARG;
-  if (p->dtype != GBSA_DTYPE_BF16 && p->dtype != GBSA_DTYPE_FP16) return GBSA_ERR_INVALID_ARG;
+  if (p->dtype != GBSA_DTYPE_BF16 && p->dtype != GBSA_DTYPE_FP16 &&
+      p->dtype != GBSA_DTYPE_FP8_E4M3)
+    return GBSA_ERR_INVALID_ARG;
+  if (p->dtype == GBSA_DTYPE_FP8_E4M3) {
+    for (double s : {p->q_scale, p->k_scale, p->v_scale})
+      if (!(s > 0.0) || isinf(s)) return GBSA_ERR_INVALID_ARG;
+    // the folded score scale and v_scale must stay finite, normal fp32
+    const double sc = p->scale > 0.0 ? p->scale : 1.0 / sqrt((double)p->D);
+    const double folded = sc * p->q_scale * p->k_scale;
+    if (folded > 1e30 || folded < 1e-30 || p->v_scale > 1e30 || p->v_scale < 1e-30)
+      return GBSA_ERR_INVALID_ARG;
+  }
   if (p->softmax_precision == 1) return GBSA_ERR_UNSUPPORTED;
   if (p->softmax_precision != 0) return GBSA_ERR_INVALID_ARG;
   if (!(p->scale >= 0.0) || isinf(p->scale)) return GBSA_ERR_INVALID_ARG;
@@ -170,13 +181,22 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+// Bytes per element of q, k and v.
+cuuint64_t elem_bytes(int32_t dtype) { return dtype == GBSA_DTYPE_FP8_E4M3 ? 1 : 2; }
+
+// A box row is 128 B: 64 elements of a 16-bit type or 128 E4M3 codes (the
+// 128-byte swizzle span).
+cuuint32_t box_inner(int32_t dtype) { return (cuuint32_t)(128 / elem_bytes(dtype)); }
+
 bool encode(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims,
             const cuuint64_t* strides_bytes, const cuuint32_t* box, int32_t dtype) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint32_t es[4] = {1, 1, 1, 1};
-  const CUtensorMapDataType t =
-      dtype == GBSA_DTYPE_FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  // E4M3 codes travel as plain bytes
+  const CUtensorMapDataType t = dtype == GBSA_DTYPE_FP16       ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                : dtype == GBSA_DTYPE_FP8_E4M3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                                               : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   return fn(map, t, rank, const_cast<void*>(base), dims,
             strides_bytes, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
@@ -286,31 +306,34 @@ gbsa_status gbsa_forward(const gbsa_problem* problem, const gbsa_tensors* t, con
   if (ws_bytes < wl.total || (wl.total > 0 && (!workspace || !aligned16(workspace))))
     return GBSA_ERR_WORKSPACE_TOO_SMALL;
 
-  const cuuint64_t D = kHeadDim;
+  const cuuint64_t D = kHeadDim, es = elem_bytes(problem->dtype);
+  const cuuint32_t bx = box_inner(problem->dtype);
   CUtensorMap map_q, map_k, map_v;
   {
     const cuuint64_t dims[3] = {D, (cuuint64_t)problem->N1, (cuuint64_t)problem->T};
-    const cuuint64_t strides[2] = {D * 2, (cuuint64_t)problem->N1 * D * 2};
-    const cuuint32_t box[3] = {64, (cuuint32_t)g.G, (cuuint32_t)g.tile_tokens};
+    const cuuint64_t strides[2] = {D * es, (cuuint64_t)problem->N1 * D * es};
+    const cuuint32_t box[3] = {bx, (cuuint32_t)g.G, (cuuint32_t)g.tile_tokens};
     if (!encode(&map_q, t->q, 3, dims, strides, box, problem->dtype)) return GBSA_ERR_CUDA;
   }
   if (tnd) {
     // rows of [T_kv, N2, D]; a box is 128 rows of one head (rows past T_kv read as 0)
     const cuuint64_t dims[3] = {D, (cuuint64_t)problem->N2, (cuuint64_t)problem->T_kv};
-    const cuuint64_t strides[2] = {D * 2, (cuuint64_t)problem->N2 * D * 2};
-    const cuuint32_t box[3] = {64, 1, (cuuint32_t)kPage};
+    const cuuint64_t strides[2] = {D * es, (cuuint64_t)problem->N2 * D * es};
+    const cuuint32_t box[3] = {bx, 1, (cuuint32_t)kPage};
     if (!encode(&map_k, t->k, 3, dims, strides, box, problem->dtype)) return GBSA_ERR_CUDA;
     if (!encode(&map_v, t->v, 3, dims, strides, box, problem->dtype)) return GBSA_ERR_CUDA;
   } else {
     const cuuint64_t dims[4] = {D, (cuuint64_t)problem->N2, (cuuint64_t)kPage,
                                 (cuuint64_t)problem->num_pages};
-    const cuuint64_t strides[3] = {D * 2, (cuuint64_t)problem->N2 * D * 2,
-                                   (cuuint64_t)problem->kv_page_stride * 2};
-    const cuuint32_t box[4] = {64, 1, (cuuint32_t)kPage, 1};
+    const cuuint64_t strides[3] = {D * es, (cuuint64_t)problem->N2 * D * es,
+                                   (cuuint64_t)problem->kv_page_stride * es};
+    const cuuint32_t box[4] = {bx, 1, (cuuint32_t)kPage, 1};
     if (!encode(&map_k, t->k, 4, dims, strides, box, problem->dtype)) return GBSA_ERR_CUDA;
     if (!encode(&map_v, t->v, 4, dims, strides, box, problem->dtype)) return GBSA_ERR_CUDA;
   }
-  const double scale = problem->scale > 0.0 ? problem->scale : 1.0 / sqrt((double)problem->D);
+  const bool fp8 = problem->dtype == GBSA_DTYPE_FP8_E4M3;
+  double scale = problem->scale > 0.0 ? problem->scale : 1.0 / sqrt((double)problem->D);
+  if (fp8) scale *= problem->q_scale * problem->k_scale;  // dequantization folds into the scores
   float* ws_o = static_cast<float*>(workspace);
   float* ws_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + wl.lse_off);
   const cudaError_t e = launch_forward(
@@ -320,7 +343,7 @@ gbsa_status gbsa_forward(const gbsa_problem* problem, const gbsa_tensors* t, con
       problem_signature(problem, ctas), problem->N1, problem->N2, problem->T, problem->top_k,
       problem->max_pages_per_seq, problem->num_pages, g.tile_tokens, g.rows_per_unit,
       problem->win_left, problem->return_lse, (float)(scale * 1.4426950408889634), ctas,
-      g.comb_cap, g.tiles_max == 1, problem->dtype == GBSA_DTYPE_FP16,
+      g.comb_cap, g.tiles_max == 1, problem->dtype, fp8 ? (float)problem->v_scale : 1.f,
       static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) {
     cudaGetLastError();

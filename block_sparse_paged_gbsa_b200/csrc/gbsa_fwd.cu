@@ -79,23 +79,46 @@ constexpr uint64_t kWaitLimitNs = 1000000000ull;
 #endif
 constexpr int32_t kHalvesMinBlocks = GBSA_HALVES_MIN_BLOCKS;
 static_assert(kHalvesMinBlocks >= 2, "a unit in halves needs a block per slot");
-constexpr float kRescaleThreshold = 8.0f;  // log2 of the largest allowed P (256)
-// Instruction descriptors: S = Q K^T (K-major A and B), O += P V (V MN-major);
-// bf16 or fp16 operands (the element type of Q, K, V and P), fp32 accumulator.
-template <bool kF16>
+// Element types of Q, K, V (and P): 0 = bf16, 1 = fp16, 2 = E4M3.  A D = 128
+// row is two 64-element halves of 128 B for the 16-bit types and one 128 B
+// half for E4M3; E4M3 MMAs (kind::f8f6f4) take K = 32 per instruction, so a
+// block needs 4 instead of 8 per product.  The output is fp16 for fp16
+// inputs and bf16 otherwise.
+constexpr int kDtBf16 = 0, kDtFp16 = 1, kDtE4m3 = 2;
+template <int kDt>
+constexpr int d_halves() { return kDt == kDtE4m3 ? 1 : 2; }
+// The K/V ring: kStages stages of a 16-bit block (32 KiB), or twice as many
+// E4M3 blocks (16 KiB) in the same bytes, so that as many bytes stay in
+// flight per SM (decode is bound by that, not by the arithmetic).
+constexpr int kMaxStages = 2 * kStages;
+template <int kDt>
+constexpr int ring_stages() { return kStages * 2 / d_halves<kDt>(); }
+template <int kDt>
+constexpr int stage_bytes() { return kHalfBytes * d_halves<kDt>(); }
+// Instruction descriptors: S = Q K^T (K-major A and B), O += P V (V MN-major),
+// fp32 accumulator.  E4M3 and fp16 share the format code 0.
+template <int kDt>
 constexpr uint32_t idesc_qk() {
-  return kF16 ? idesc_f16_f32(128, 128, false, false) : idesc_bf16_f32(128, 128, false, false);
+  return kDt == kDtBf16 ? idesc_bf16_f32(128, 128, false, false)
+                        : idesc_f16_f32(128, 128, false, false);
 }
-template <bool kF16>
+template <int kDt>
 constexpr uint32_t idesc_pv() {
-  return kF16 ? idesc_f16_f32(128, 128, false, true) : idesc_bf16_f32(128, 128, false, true);
+  return kDt == kDtBf16 ? idesc_bf16_f32(128, 128, false, true)
+                        : idesc_f16_f32(128, 128, false, true);
 }
+// Lazy-rescale threshold (log2 units).  16-bit P: the reference max may lag
+// the row max by up to 8 (P <= 256).  E4M3 P is formed as 2^8 * p so that the
+// small weights stay above its 2^-9 floor; the reference may then lag by 0.5
+// at most (P <= 362 < 448, the largest E4M3 value).
+template <int kDt>
+constexpr float rescale_threshold() { return kDt == kDtE4m3 ? 0.5f : 8.0f; }
 
 struct FwdParams {
   const int32_t* meta;
   const int32_t* block_table;  // paged K/V
   const int64_t* cu_kv;        // TND K/V: first row of each sequence (block_table unused)
-  uint16_t* out;  // bf16 or fp16 elements
+  uint16_t* out;  // fp16 for fp16 inputs, else bf16
   float* lse;
   float* ws_o;    // [slot_cap][rows_per_unit][128] fp32 partial outputs
   float* ws_lse;  // [slot_cap][rows_per_unit] fp32 partial lse
@@ -103,12 +126,13 @@ struct FwdParams {
   uint32_t signature;
   int32_t N1, N2, G, T, top_k, max_pages, num_pages, tile_tokens, rows_per_unit;
   int32_t win_left, return_lse;
-  float scale_log2;
+  float scale_log2;  // softmax scale (E4M3: times q_scale * k_scale) x log2(e)
+  float out_scale;   // E4M3: v_scale
 };
 
 struct Bars {
   uint64_t q_full[2], q_empty[2];
-  uint64_t kv_full[kStages], kv_empty[kStages];
+  uint64_t kv_full[kMaxStages], kv_empty[kMaxStages];
   uint64_t s_full[2];      // S of a block ready (MMA commit)
   uint64_t p_full[2];      // P of a block in TMEM, O rescaled (128 softmax threads)
   uint64_t o_final[2];     // last PV of a unit complete (MMA commit)
@@ -217,27 +241,32 @@ __device__ __forceinline__ RowInfo row_info(const FwdParams& p, const Unit& x, i
 // Called by the whole producer warp: every lane waits and counts, lane 0
 // issues the copies.  `where` is the physical page (paged pool: 4-D map) or,
 // with `tnd`, the first row of the block in k / v [T_kv, N2, D] (3-D map).
+// A block is d_halves<kDt>() boxes of 128 rows x 128 B (64 elements of a
+// 16-bit type, or 128 E4M3 elements).
+template <int kDt>
 __device__ __forceinline__ bool produce_kv(const CUtensorMap* map, uint8_t* smem, Bars* bars,
                                            uint32_t& kv_iter, int32_t kvh, int32_t where,
                                            bool tnd, uint32_t lane) {
-  const uint32_t stage = kv_iter % kStages;
-  if (kv_iter >= kStages && !wait_bar(&bars->kv_empty[stage], ((kv_iter / kStages) & 1) ^ 1, bars))
+  constexpr uint32_t kN = ring_stages<kDt>();
+  const uint32_t stage = kv_iter % kN;
+  if (kv_iter >= kN && !wait_bar(&bars->kv_empty[stage], ((kv_iter / kN) & 1) ^ 1, bars))
     return false;
   if (lane == 0) {
-    uint8_t* dst = smem + kSmemRing + stage * kTileBytes;
-    mbar_arrive_expect_tx(&bars->kv_full[stage], kTileBytes);
-    if (tnd) {
-      tma_load_3d(dst, map, &bars->kv_full[stage], 0, kvh, where);
-      tma_load_3d(dst + kHalfBytes, map, &bars->kv_full[stage], 64, kvh, where);
-    } else {
-      tma_load_4d(dst, map, &bars->kv_full[stage], 0, kvh, 0, where);
-      tma_load_4d(dst + kHalfBytes, map, &bars->kv_full[stage], 64, kvh, 0, where);
+    uint8_t* dst = smem + kSmemRing + stage * stage_bytes<kDt>();
+    mbar_arrive_expect_tx(&bars->kv_full[stage], d_halves<kDt>() * kHalfBytes);
+#pragma unroll
+    for (int h = 0; h < d_halves<kDt>(); h++) {
+      if (tnd)
+        tma_load_3d(dst + h * kHalfBytes, map, &bars->kv_full[stage], 64 * h, kvh, where);
+      else
+        tma_load_4d(dst + h * kHalfBytes, map, &bars->kv_full[stage], 64 * h, kvh, 0, where);
     }
   }
   kv_iter++;
   return true;
 }
 
+template <int kDt>
 __device__ __forceinline__ bool produce_q(const FwdParams& p, const CUtensorMap* map_q,
                                           uint8_t* smem, Bars* bars, uint32_t& q_iter,
                                           const Unit& x, int s, uint32_t lane) {
@@ -246,15 +275,16 @@ __device__ __forceinline__ bool produce_q(const FwdParams& p, const CUtensorMap*
     const uint32_t box_bytes = 128u * (uint32_t)p.G * (uint32_t)p.tile_tokens;
     const int32_t tok = x.tok_begin + (2 * x.tp + s) * p.tile_tokens;
     uint8_t* dst = smem + kSmemQ + s * kTileBytes;
-    mbar_arrive_expect_tx(&bars->q_full[s], 2u * box_bytes);
-    tma_load_3d(dst, map_q, &bars->q_full[s], 0, x.kvh * p.G, tok);
-    tma_load_3d(dst + kHalfBytes, map_q, &bars->q_full[s], 64, x.kvh * p.G, tok);
+    mbar_arrive_expect_tx(&bars->q_full[s], (uint32_t)d_halves<kDt>() * box_bytes);
+#pragma unroll
+    for (int h = 0; h < d_halves<kDt>(); h++)
+      tma_load_3d(dst + h * kHalfBytes, map_q, &bars->q_full[s], 64 * h, x.kvh * p.G, tok);
   }
   q_iter++;
   return true;
 }
 
-template <bool kHalves>
+template <bool kHalves, int kDt>
 __device__ void run_producer(const FwdParams& p, const CUtensorMap* map_q, const CUtensorMap* map_k,
                              const CUtensorMap* map_v, uint8_t* smem, Bars* bars, int32_t n_units,
                              int64_t off_unit, int64_t off_item, int64_t off_list) {
@@ -284,7 +314,7 @@ __device__ void run_producer(const FwdParams& p, const CUtensorMap* map_q, const
       const int32_t lb = list[lane] & kEntryLbMask;
       page = tnd ? (int32_t)(row0 + (int64_t)lb * kPage) : (lb < p.max_pages ? bt[lb] : -1);
     }
-    ok = produce_q(p, map_q, smem, bars, q_iter0, x, 0, lane);
+    ok = produce_q<kDt>(p, map_q, smem, bars, q_iter0, x, 0, lane);
     for (int32_t c0 = 0; c0 < n && ok; c0 += 32) {
       if (c0 > 0 && c0 + (int32_t)lane < n) {
         const int32_t lb = list[c0 + lane] & kEntryLbMask;
@@ -301,18 +331,18 @@ __device__ void run_producer(const FwdParams& p, const CUtensorMap* map_q, const
           const bool has1 = jj + 1 < cn;
           const int32_t pg0 = __shfl_sync(0xffffffffu, page, jj);
           const int32_t pg1 = __shfl_sync(0xffffffffu, page, (jj + 1) & 31);
-          ok = produce_kv(map_k, smem, bars, kv_iter, x.kvh, pg0, tnd, lane);
-          if (ok && has1) ok = produce_kv(map_k, smem, bars, kv_iter, x.kvh, pg1, tnd, lane);
-          if (ok) ok = produce_kv(map_v, smem, bars, kv_iter, x.kvh, pg0, tnd, lane);
-          if (ok && has1) ok = produce_kv(map_v, smem, bars, kv_iter, x.kvh, pg1, tnd, lane);
+          ok = produce_kv<kDt>(map_k, smem, bars, kv_iter, x.kvh, pg0, tnd, lane);
+          if (ok && has1) ok = produce_kv<kDt>(map_k, smem, bars, kv_iter, x.kvh, pg1, tnd, lane);
+          if (ok) ok = produce_kv<kDt>(map_v, smem, bars, kv_iter, x.kvh, pg0, tnd, lane);
+          if (ok && has1) ok = produce_kv<kDt>(map_v, smem, bars, kv_iter, x.kvh, pg1, tnd, lane);
         }
         continue;
       }
       for (int32_t jj = 0; jj < cn && ok; jj++) {
         const int32_t pg = __shfl_sync(0xffffffffu, page, jj);
-        ok = produce_kv(map_k, smem, bars, kv_iter, x.kvh, pg, tnd, lane);
-        if (ok && c0 + jj == 0 && x.nt == 2) ok = produce_q(p, map_q, smem, bars, q_iter1, x, 1, lane);
-        if (ok) ok = produce_kv(map_v, smem, bars, kv_iter, x.kvh, pg, tnd, lane);
+        ok = produce_kv<kDt>(map_k, smem, bars, kv_iter, x.kvh, pg, tnd, lane);
+        if (ok && c0 + jj == 0 && x.nt == 2) ok = produce_q<kDt>(p, map_q, smem, bars, q_iter1, x, 1, lane);
+        if (ok) ok = produce_kv<kDt>(map_v, smem, bars, kv_iter, x.kvh, pg, tnd, lane);
       }
     }
   }
@@ -321,8 +351,9 @@ __device__ void run_producer(const FwdParams& p, const CUtensorMap* map_q, const
   if (!ok && lane == 0) {
     // drain: wait (bounded) for the copies this thread issued last
     const uint64_t t0 = global_timer_ns();
-    for (uint32_t i = (kv_iter > kStages ? kv_iter - kStages : 0); i < kv_iter; i++) {
-      while (!mbar_try_wait(&bars->kv_full[i % kStages], (i / kStages) & 1) &&
+    constexpr uint32_t kN = ring_stages<kDt>();
+    for (uint32_t i = (kv_iter > kN ? kv_iter - kN : 0); i < kv_iter; i++) {
+      while (!mbar_try_wait(&bars->kv_full[i % kN], (i / kN) & 1) &&
              global_timer_ns() - t0 < kWaitLimitNs) {
       }
     }
@@ -362,39 +393,60 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Bars* 
 // Descriptors are handled as 32-bit low words (start address >> 4 in bits
 // [0,14), leading byte offset >> 4 in [16,30)) plus the shared high word;
 // offsets are added to the low word (addresses stay below 256 KiB: no carry).
-template <bool kF16>
+template <int kDt>
 __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_lo, uint32_t k_lo,
                                          uint32_t hi) {
+  if constexpr (kDt == kDtE4m3) {
 #pragma unroll
-  for (int kk = 0; kk < 8; kk++) {
-    const uint32_t off = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
-    mma_ss_lo(d_tmem, q_lo + off, k_lo + off, hi, idesc_qk<kF16>(), kk > 0 ? 1u : 0u);
+    for (int kk = 0; kk < 4; kk++) {  // 32 E4M3 elements (32 B) per step, one 128 B half
+      const uint32_t off = (kk * 32) >> 4;
+      mma_ss_lo_f8(d_tmem, q_lo + off, k_lo + off, hi, idesc_qk<kDt>(), kk > 0 ? 1u : 0u);
+    }
+  } else {
+#pragma unroll
+    for (int kk = 0; kk < 8; kk++) {
+      const uint32_t off = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
+      mma_ss_lo(d_tmem, q_lo + off, k_lo + off, hi, idesc_qk<kDt>(), kk > 0 ? 1u : 0u);
+    }
   }
 }
 
-template <bool kF16>
+template <int kDt>
 __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_lo,
                                          uint32_t hi, bool accumulate) {
+  if constexpr (kDt == kDtE4m3) {
+    // P: 4 E4M3 per TMEM column, 32 keys (8 columns) per step; V: 32 keys of
+    // 128 B per step
 #pragma unroll
-  for (int kk = 0; kk < 8; kk++)
-    mma_ts_lo(d_tmem, p_tmem + kk * 8, v_lo + ((kk * 2048) >> 4), hi, idesc_pv<kF16>(),
-              (accumulate || kk > 0) ? 1u : 0u);
+    for (int kk = 0; kk < 4; kk++)
+      mma_ts_lo_f8(d_tmem, p_tmem + kk * 8, v_lo + ((kk * 4096) >> 4), hi, idesc_pv<kDt>(),
+                   (accumulate || kk > 0) ? 1u : 0u);
+  } else {
+    // P: 2 elements per column, 16 keys (8 columns) per step; V: 16 keys of
+    // two 128 B halves per step
+#pragma unroll
+    for (int kk = 0; kk < 8; kk++)
+      mma_ts_lo(d_tmem, p_tmem + kk * 8, v_lo + ((kk * 2048) >> 4), hi, idesc_pv<kDt>(),
+                (accumulate || kk > 0) ? 1u : 0u);
+  }
 }
 
-// Position in the K/V ring: stage index and the parity of its current fill.
+// Position in a K/V ring of kN stages: stage index and the parity of its
+// current fill.
+template <uint32_t kN>
 struct RingPos {
   uint32_t stage, phase;
   __device__ __forceinline__ void advance() {
-    if (++stage == kStages) {
+    if (++stage == kN) {
       stage = 0;
       phase ^= 1u;
     }
   }
-  // the position k fills later (k < kStages)
+  // the position k fills later (k < kN)
   __device__ __forceinline__ RingPos ahead(uint32_t k) const {
     RingPos r{stage + k, phase};
-    if (r.stage >= kStages) {
-      r.stage -= kStages;
+    if (r.stage >= kN) {
+      r.stage -= kN;
       r.phase ^= 1u;
     }
     return r;
@@ -404,14 +456,16 @@ struct RingPos {
 // Zero the rows of a V tile that lie past seqused_kv on a last page (their
 // pool contents are arbitrary and P there is 0, but 0 * NaN is NaN).  Whole
 // warp; `entry` is the block's list entry.
+template <int kDt>
 __device__ __forceinline__ void zero_v_tail(uint8_t* smem, uint32_t vs, int32_t entry, int32_t ku,
                                             uint32_t lane) {
   if (!(entry & kEntryPartial)) return;
   const int32_t r0 = min(max(ku - (entry & kEntryLbMask) * kPage, 0), kPage);
-  uint8_t* vt = smem + kSmemRing + vs * kTileBytes;
-  const int32_t n16 = (kPage - r0) * 16;
+  uint8_t* vt = smem + kSmemRing + vs * stage_bytes<kDt>();
+  constexpr int32_t kChunks = 8 * d_halves<kDt>();  // 16-byte chunks of a row
+  const int32_t n16 = (kPage - r0) * kChunks;
   for (int32_t t = lane; t < n16; t += 32) {
-    const int32_t row = r0 + (t >> 4), chunk = t & 15;
+    const int32_t row = r0 + t / kChunks, chunk = t % kChunks;
     *reinterpret_cast<uint4*>(vt + (chunk >> 3) * kHalfBytes + row * 128 + (chunk & 7) * 16) =
         make_uint4(0, 0, 0, 0);
   }
@@ -419,14 +473,15 @@ __device__ __forceinline__ void zero_v_tail(uint8_t* smem, uint32_t vs, int32_t 
   __syncwarp();
 }
 
-template <bool kHalves, bool kF16>
+template <bool kHalves, int kDt>
 __device__ void run_mma(const FwdParams& p, uint8_t* smem, Bars* bars, uint32_t tmem,
                         int32_t n_units, int32_t off_unit, int32_t off_item, int32_t off_list) {
   const uint32_t lane = lane_id();
   uint32_t q_iter0 = 0, q_iter1 = 0;
   uint32_t blk0 = 0, blk1 = 0;      // blocks per tile slot (p_full phases)
   uint32_t units0 = 0, units1 = 0;  // units per tile slot (o_free phases)
-  RingPos rp{0, 0};                 // next K/V tile to consume
+  using Ring = RingPos<ring_stages<kDt>()>;
+  Ring rp{0, 0};                    // next K/V tile to consume
   bool ok = true;
   const uint32_t q_addr = smem_u32(smem + kSmemQ);
   const uint32_t ring_addr = smem_u32(smem + kSmemRing);
@@ -436,7 +491,7 @@ __device__ void run_mma(const FwdParams& p, uint8_t* smem, Bars* bars, uint32_t 
   const uint32_t q1_lo = q0_lo + (kTileBytes >> 4);
   const uint32_t k_lo0 = (uint32_t)smem_desc_sw128(ring_addr, 16, 1024);
   const uint32_t v_lo0 = (uint32_t)smem_desc_sw128(ring_addr, kHalfBytes, 1024);
-  constexpr uint32_t kStageLo = kTileBytes >> 4;
+  constexpr uint32_t kStageLo = stage_bytes<kDt>() >> 4;
 
   for (int32_t wave = 0, u = unit_of(0); u < n_units && ok; u = unit_of(++wave)) {
     const int4 rec = *reinterpret_cast<const int4*>(p.meta + off_unit + 4 * (int64_t)u);
@@ -465,7 +520,7 @@ __device__ void run_mma(const FwdParams& p, uint8_t* smem, Bars* bars, uint32_t 
         if (!(ok = warp_wait(&bars->kv_full[rp.stage], rp.phase, bars))) break;
         if (lane == 0) {
           tc_fence_after_sync();
-          issue_qk<kF16>(tmem, q0_lo, k_lo0 + rp.stage * kStageLo, hi);
+          issue_qk<kDt>(tmem, q0_lo, k_lo0 + rp.stage * kStageLo, hi);
           tc_commit(&bars->s_full[0]);
           tc_commit(&bars->kv_empty[rp.stage]);
           if (j == n - 1) tc_commit(&bars->q_empty[0]);
@@ -477,7 +532,7 @@ __device__ void run_mma(const FwdParams& p, uint8_t* smem, Bars* bars, uint32_t 
           if (!(ok = warp_wait(&bars->p_full[1], blk1 & 1, bars))) break;
           if (lane == 0) {
             tc_fence_after_sync();
-            issue_pv<kF16>(tmem + 384, tmem + 128, v_lo0 + pv1 * kStageLo, hi, i - 1 > 0);
+            issue_pv<kDt>(tmem + 384, tmem + 128, v_lo0 + pv1 * kStageLo, hi, i - 1 > 0);
             if (i == n1) tc_commit(&bars->o_final[1]);
             tc_commit(&bars->kv_empty[pv1]);
           }
@@ -485,35 +540,35 @@ __device__ void run_mma(const FwdParams& p, uint8_t* smem, Bars* bars, uint32_t 
         }
         // ---- S1_i = Q K_{j+1}
         if (has1) {
-          const RingPos rk1 = rp.ahead(1);
+          const Ring rk1 = rp.ahead(1);
           if (!(ok = warp_wait(&bars->kv_full[rk1.stage], rk1.phase, bars))) break;
           if (lane == 0) {
             tc_fence_after_sync();
-            issue_qk<kF16>(tmem + 128, q0_lo, k_lo0 + rk1.stage * kStageLo, hi);
+            issue_qk<kDt>(tmem + 128, q0_lo, k_lo0 + rk1.stage * kStageLo, hi);
             tc_commit(&bars->s_full[1]);
             tc_commit(&bars->kv_empty[rk1.stage]);
             if (j + 1 == n - 1) tc_commit(&bars->q_empty[0]);
           }
         }
         // ---- V_j, then PV0_i = P0 V_j
-        const RingPos rv0 = rp.ahead(has1 ? 2 : 1);
+        const Ring rv0 = rp.ahead(has1 ? 2 : 1);
         if (!(ok = warp_wait(&bars->kv_full[rv0.stage], rv0.phase, bars))) break;
-        zero_v_tail(smem, rv0.stage, __shfl_sync(0xffffffffu, entries, j & 31), ku, lane);
+        zero_v_tail<kDt>(smem, rv0.stage, __shfl_sync(0xffffffffu, entries, j & 31), ku, lane);
         if (i == 0 && units0 > 0)
           if (!(ok = warp_wait(&bars->o_free[0], (units0 - 1) & 1, bars))) break;
         if (!(ok = warp_wait(&bars->p_full[0], blk0 & 1, bars))) break;
         if (lane == 0) {
           tc_fence_after_sync();
-          issue_pv<kF16>(tmem + 256, tmem, v_lo0 + rv0.stage * kStageLo, hi, i > 0);
+          issue_pv<kDt>(tmem + 256, tmem, v_lo0 + rv0.stage * kStageLo, hi, i > 0);
           if (i == n0 - 1) tc_commit(&bars->o_final[0]);
           tc_commit(&bars->kv_empty[rv0.stage]);
         }
         blk0++;
         // ---- V_{j+1} (read by PV1_i)
         if (has1) {
-          const RingPos rv1 = rp.ahead(3);
+          const Ring rv1 = rp.ahead(3);
           if (!(ok = warp_wait(&bars->kv_full[rv1.stage], rv1.phase, bars))) break;
-          zero_v_tail(smem, rv1.stage, __shfl_sync(0xffffffffu, entries, (j + 1) & 31), ku, lane);
+          zero_v_tail<kDt>(smem, rv1.stage, __shfl_sync(0xffffffffu, entries, (j + 1) & 31), ku, lane);
           pv1 = rv1.stage;
         }
         rp = rp.ahead(has1 ? 4 : 2);
@@ -524,7 +579,7 @@ __device__ void run_mma(const FwdParams& p, uint8_t* smem, Bars* bars, uint32_t 
         if (ok) ok = warp_wait(&bars->p_full[1], blk1 & 1, bars);
         if (ok && lane == 0) {
           tc_fence_after_sync();
-          issue_pv<kF16>(tmem + 384, tmem + 128, v_lo0 + pv1 * kStageLo, hi, n1 - 1 > 0);
+          issue_pv<kDt>(tmem + 384, tmem + 128, v_lo0 + pv1 * kStageLo, hi, n1 - 1 > 0);
           tc_commit(&bars->o_final[1]);
           tc_commit(&bars->kv_empty[pv1]);
         }
@@ -546,7 +601,7 @@ __device__ void run_mma(const FwdParams& p, uint8_t* smem, Bars* bars, uint32_t 
         rp.advance();
         if (lane == 0) {
           tc_fence_after_sync();
-          issue_qk<kF16>(tmem, q0_lo, k_lo0 + ks * kStageLo, hi);
+          issue_qk<kDt>(tmem, q0_lo, k_lo0 + ks * kStageLo, hi);
           tc_commit(&bars->s_full[0]);
           if (i == n - 1) tc_commit(&bars->q_empty[0]);
         }
@@ -561,14 +616,14 @@ __device__ void run_mma(const FwdParams& p, uint8_t* smem, Bars* bars, uint32_t 
             if (!(ok = warp_wait(&bars->p_full[1], blk1 & 1, bars))) break;
             if (lane == 0) {
               tc_fence_after_sync();
-              issue_pv<kF16>(tmem + 384, tmem + 128, v_lo0 + prev_vs * kStageLo, hi, i - 1 > 0);
+              issue_pv<kDt>(tmem + 384, tmem + 128, v_lo0 + prev_vs * kStageLo, hi, i - 1 > 0);
               tc_commit(&bars->kv_empty[prev_vs]);
             }
             blk1++;
           }
           // ---- S1_i
           if (lane == 0) {
-            issue_qk<kF16>(tmem + 128, q1_lo, k_lo0 + ks * kStageLo, hi);
+            issue_qk<kDt>(tmem + 128, q1_lo, k_lo0 + ks * kStageLo, hi);
             tc_commit(&bars->s_full[1]);
             if (i == n - 1) tc_commit(&bars->q_empty[1]);
           }
@@ -578,14 +633,14 @@ __device__ void run_mma(const FwdParams& p, uint8_t* smem, Bars* bars, uint32_t 
         const uint32_t vs = rp.stage;
         if (!(ok = warp_wait(&bars->kv_full[vs], rp.phase, bars))) break;
         rp.advance();
-        zero_v_tail(smem, vs, __shfl_sync(0xffffffffu, entries, i & 31), ku, lane);
+        zero_v_tail<kDt>(smem, vs, __shfl_sync(0xffffffffu, entries, i & 31), ku, lane);
         // ---- PV0_i
         if (i == 0 && units0 > 0)
           if (!(ok = warp_wait(&bars->o_free[0], (units0 - 1) & 1, bars))) break;
         if (!(ok = warp_wait(&bars->p_full[0], blk0 & 1, bars))) break;
         if (lane == 0) {
           tc_fence_after_sync();
-          issue_pv<kF16>(tmem + 256, tmem, v_lo0 + vs * kStageLo, hi, i > 0);
+          issue_pv<kDt>(tmem + 256, tmem, v_lo0 + vs * kStageLo, hi, i > 0);
           if (i == n - 1) tc_commit(&bars->o_final[0]);
           if (!two) tc_commit(&bars->kv_empty[vs]);
         }
@@ -598,7 +653,7 @@ __device__ void run_mma(const FwdParams& p, uint8_t* smem, Bars* bars, uint32_t 
         if (ok) ok = warp_wait(&bars->p_full[1], blk1 & 1, bars);
         if (ok && lane == 0) {
           tc_fence_after_sync();
-          issue_pv<kF16>(tmem + 384, tmem + 128, v_lo0 + prev_vs * kStageLo, hi, n - 1 > 0);
+          issue_pv<kDt>(tmem + 384, tmem + 128, v_lo0 + prev_vs * kStageLo, hi, n - 1 > 0);
           tc_commit(&bars->o_final[1]);
           tc_commit(&bars->kv_empty[prev_vs]);
         }
@@ -621,7 +676,7 @@ __device__ void run_mma(const FwdParams& p, uint8_t* smem, Bars* bars, uint32_t 
 // ---------------------------------------------------------------------------
 // softmax (one warpgroup per tile slot; thread = tile row = TMEM lane)
 // ---------------------------------------------------------------------------
-template <bool kHalves, bool kF16>
+template <bool kHalves, int kDt>
 __device__ void run_softmax(const FwdParams& p, Bars* bars, uint32_t tmem, int slot,
                             int32_t n_units, int64_t off_unit, int64_t off_item, int64_t off_list) {
   const int row = threadIdx.x & 127;
@@ -682,22 +737,25 @@ __device__ void run_softmax(const FwdParams& p, Bars* bars, uint32_t tmem, int s
                              fmaxf(mp[6], mp[7]));
       const float m_blk = mx * p.scale_log2;
       const float m_new = fmaxf(m, m_blk);
-      // lazy rescale: keep the old reference max unless it grew by > 8 (P <= 256)
-      const bool rescale = m_new != -INFINITY && (m == -INFINITY || m_new > m + kRescaleThreshold);
+      // lazy rescale: keep the old reference max unless it grew past the threshold
+      const bool rescale =
+          m_new != -INFINITY && (m == -INFINITY || m_new > m + rescale_threshold<kDt>());
       const bool fix_o = rescale && m != -INFINITY;
       const float factor = fix_o ? fast_exp2(m - m_new) : 1.f;
       if (rescale) {
         l *= factor;
         m = m_new;
       }
-      const float neg_m = (m == -INFINITY) ? 0.f : -m;
+      // E4M3 P carries a factor 2^8 (the row sum l too; the statistics
+      // handed on below take it out of m)
+      const float neg_m = ((m == -INFINITY) ? 0.f : -m) + (kDt == kDtE4m3 ? 8.f : 0.f);
       // scores pairwise: x = s * scale_log2 - m as one f32x2 FMA, P = 2^x,
       // the row sum in two packed partial sums (four independent lanes)
       const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2), nm2 = f2_pack(neg_m, neg_m);
       uint64_t sp2[2] = {0ull, 0ull};
 #pragma unroll
       for (int q = 0; q < 4; q++) {
-        uint32_t pk[16];
+        float pf[32];
 #pragma unroll
         for (int i = 0; i < 16; i++) {
           // masked scores are -inf and ex2(-inf) = +0
@@ -705,11 +763,23 @@ __device__ void run_softmax(const FwdParams& p, Bars* bars, uint32_t tmem, int s
           f2_unpack(f2_fma(f2_pack(__uint_as_float(r[q][2 * i]), __uint_as_float(r[q][2 * i + 1])),
                            sc2, nm2),
                     x0, x1);
-          const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
-          sp2[i & 1] = f2_add(sp2[i & 1], f2_pack(p0, p1));
-          pk[i] = pack_x2<kF16>(p0, p1);
+          pf[2 * i] = fast_exp2(x0);
+          pf[2 * i + 1] = fast_exp2(x1);
+          sp2[i & 1] = f2_add(sp2[i & 1], f2_pack(pf[2 * i], pf[2 * i + 1]));
         }
-        tmem_st_32x16(t_s + 16 * q, pk);
+        if constexpr (kDt == kDtE4m3) {
+          // four E4M3 weights per TMEM column: 32 keys in 8 columns
+          uint32_t pk[8];
+#pragma unroll
+          for (int i = 0; i < 8; i++)
+            pk[i] = pack_e4m3x4(pf[4 * i], pf[4 * i + 1], pf[4 * i + 2], pf[4 * i + 3]);
+          tmem_st_32x8(t_s + 8 * q, pk);
+        } else {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; i++) pk[i] = pack_x2<kDt == kDtFp16>(pf[2 * i], pf[2 * i + 1]);
+          tmem_st_32x16(t_s + 16 * q, pk);
+        }
       }
       float s0, s1, s2, s3;
       f2_unpack(sp2[0], s0, s1);
@@ -735,7 +805,8 @@ __device__ void run_softmax(const FwdParams& p, Bars* bars, uint32_t tmem, int s
     }
     // hand the row statistics of this unit to the epilogue warpgroup
     if (units > 0 && !wait_bar(&bars->stats_free[slot], (units - 1) & 1, bars)) return;
-    bars->stats[slot][row] = make_float2(m, l);
+    // (E4M3: P and l carry 2^8, so the reference max handed on is m - 8)
+    bars->stats[slot][row] = make_float2(kDt == kDtE4m3 && m != -INFINITY ? m - 8.f : m, l);
     mbar_arrive(&bars->stats_full[slot]);
     units++;
   }
@@ -744,7 +815,14 @@ __device__ void run_softmax(const FwdParams& p, Bars* bars, uint32_t tmem, int s
 // ---------------------------------------------------------------------------
 // epilogue (one warpgroup; thread = tile row = TMEM lane, both tile slots)
 // ---------------------------------------------------------------------------
-template <bool kHalves, bool kF16>
+// E4M3 V carries a per-tensor dequantization scale, applied with 1 / l (the
+// split-KV partials too: the merge is linear in them).
+template <int kDt>
+__device__ __forceinline__ float out_numerator(const FwdParams& p) {
+  return kDt == kDtE4m3 ? p.out_scale : 1.f;
+}
+
+template <bool kHalves, int kDt>
 __device__ void run_epilogue(const FwdParams& p, Bars* bars, uint32_t tmem, int32_t n_units,
                              int64_t off_unit, int64_t off_item) {
   const int row = threadIdx.x & 127;
@@ -778,7 +856,7 @@ __device__ void run_epilogue(const FwdParams& p, Bars* bars, uint32_t tmem, int3
       const float w1 = st[1].y > 0.f ? fast_exp2(st[1].x - mm) : 0.f;
       const float l = st[0].y * w0 + st[1].y * w1;
       const bool has = ri.used && l > 0.f;
-      const float inv_l = has ? 1.f / l : 0.f;
+      const float inv_l = has ? out_numerator<kDt>(p) / l : 0.f;
       const float a0 = w0 * inv_l, a1 = w1 * inv_l;
       const float lse = has ? (mm + __log2f(l)) * 0.69314718055994531f : -INFINITY;
       const bool write_row = ri.store && ri.tok < p.T;
@@ -793,7 +871,7 @@ __device__ void run_epilogue(const FwdParams& p, Bars* bars, uint32_t tmem, int3
           uint32_t pk[4];
 #pragma unroll
           for (int i = 0; i < 4; i++)
-            pk[i] = has ? pack_x2<kF16>(
+            pk[i] = has ? pack_x2<kDt == kDtFp16>(
                               __uint_as_float(o0[2 * i]) * a0 + __uint_as_float(o1[2 * i]) * a1,
                               __uint_as_float(o0[2 * i + 1]) * a0 + __uint_as_float(o1[2 * i + 1]) * a1)
                         : 0u;
@@ -842,7 +920,7 @@ __device__ void run_epilogue(const FwdParams& p, Bars* bars, uint32_t tmem, int3
         tc_fence_after_sync();
       }
       const bool has = nblk > 0 && ri.used && l > 0.f;
-      const float inv_l = has ? 1.f / l : 0.f;
+      const float inv_l = has ? out_numerator<kDt>(p) / l : 0.f;
       const float lse = has ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
       const bool write_row = ri.store && ri.tok < p.T;
       if (ri.store && ri.tok >= p.T) bad |= kDevBadSeqlen;
@@ -855,7 +933,7 @@ __device__ void run_epilogue(const FwdParams& p, Bars* bars, uint32_t tmem, int3
           uint32_t pk[8];
 #pragma unroll
           for (int i = 0; i < 8; i++)
-            pk[i] = has ? pack_x2<kF16>(__uint_as_float(o[2 * i]) * inv_l,
+            pk[i] = has ? pack_x2<kDt == kDtFp16>(__uint_as_float(o[2 * i]) * inv_l,
                                       __uint_as_float(o[2 * i + 1]) * inv_l)
                         : 0u;
           if (write_row) {
@@ -890,7 +968,7 @@ __device__ void run_epilogue(const FwdParams& p, Bars* bars, uint32_t tmem, int3
   if (bad && p.dev_status) atomicOr(p.dev_status, bad);
 }
 
-template <bool kHalves, bool kF16>
+template <bool kHalves, int kDt>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                const __grid_constant__ CUtensorMap map_v, const FwdParams p) {
@@ -923,7 +1001,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->stats_full[i], 128);
       mbar_init(&bars->stats_free[i], 128);
     }
-    for (int i = 0; i < kStages; i++) {
+    for (int i = 0; i < kMaxStages; i++) {
       mbar_init(&bars->kv_full[i], 1);
       mbar_init(&bars->kv_empty[i], 1);
     }
@@ -942,21 +1020,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < 8) {
     setmaxnreg_inc<regs_softmax<kHalves>()>();
-    run_softmax<kHalves, kF16>(p, bars, tmem, warp >> 2, n_units, off_unit, off_item, off_list);
+    run_softmax<kHalves, kDt>(p, bars, tmem, warp >> 2, n_units, off_unit, off_item, off_list);
   } else if (warp < 12) {
     setmaxnreg_dec<kRegsEpilogue>();
-    run_epilogue<kHalves, kF16>(p, bars, tmem, n_units, off_unit, off_item);
+    run_epilogue<kHalves, kDt>(p, bars, tmem, n_units, off_unit, off_item);
   } else {
     setmaxnreg_dec<regs_control<kHalves>()>();
     if (warp == kWarpMma) {
-      run_mma<kHalves, kF16>(p, smem, bars, tmem, n_units, (int32_t)off_unit, (int32_t)off_item, (int32_t)off_list);
+      run_mma<kHalves, kDt>(p, smem, bars, tmem, n_units, (int32_t)off_unit, (int32_t)off_item, (int32_t)off_list);
     } else if (warp == kWarpProducer) {
       if (lane_id() == 0) {
         tma_prefetch_map(&map_q);
         tma_prefetch_map(&map_k);
         tma_prefetch_map(&map_v);
       }
-      run_producer<kHalves>(p, &map_q, &map_k, &map_v, smem, bars, n_units, off_unit, off_item, off_list);
+      run_producer<kHalves, kDt>(p, &map_q, &map_k, &map_v, smem, bars, n_units, off_unit, off_item, off_list);
     }
   }
 
@@ -976,7 +1054,7 @@ struct CombineParams {
   const int32_t* meta;
   const float* ws_o;
   const float* ws_lse;
-  uint16_t* out;  // bf16 or fp16 elements
+  uint16_t* out;  // fp16 for fp16 inputs, else bf16
   float* lse;
   int32_t* dev_status;
   uint32_t signature;
@@ -1044,7 +1122,14 @@ cudaError_t launch_forward(const CUtensorMap& map_q, const CUtensorMap& map_k,
                            int32_t num_pages, int32_t tile_tokens, int32_t rows_per_unit,
                            int32_t win_left, int32_t return_lse, float scale_log2,
                            int32_t num_ctas, int64_t comb_cap, bool one_tile_blocks,
-                           bool fp16, cudaStream_t stream) {
+                           int32_t dtype, float out_scale, cudaStream_t stream) {
+  using Kernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const FwdParams);
+  // [element type][one_tile_blocks]
+  static const Kernel kernels[3][2] = {
+      {fwd_kernel<false, kDtBf16>, fwd_kernel<true, kDtBf16>},
+      {fwd_kernel<false, kDtFp16>, fwd_kernel<true, kDtFp16>},
+      {fwd_kernel<false, kDtE4m3>, fwd_kernel<true, kDtE4m3>}};
+  if (dtype < 0 || dtype > 2) return cudaErrorInvalidValue;
   static int configured_device = -1;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -1052,11 +1137,8 @@ cudaError_t launch_forward(const CUtensorMap& map_q, const CUtensorMap& map_k,
   if (configured_device != dev) {
     // The register re-split is only safe if the kernel launches with exactly
     // the registers the split was computed for.
-    const void* fns[4] = {reinterpret_cast<const void*>(fwd_kernel<false, false>),
-                          reinterpret_cast<const void*>(fwd_kernel<true, false>),
-                          reinterpret_cast<const void*>(fwd_kernel<false, true>),
-                          reinterpret_cast<const void*>(fwd_kernel<true, true>)};
-    for (const void* fn : fns) {
+    for (int i = 0; i < 6; i++) {
+      const void* fn = reinterpret_cast<const void*>(kernels[i / 2][i % 2]);
       cudaFuncAttributes attr;
       e = cudaFuncGetAttributes(&attr, fn);
       if (e != cudaSuccess) return e;
@@ -1088,20 +1170,11 @@ cudaError_t launch_forward(const CUtensorMap& map_q, const CUtensorMap& map_k,
   p.win_left = win_left;
   p.return_lse = return_lse;
   p.scale_log2 = scale_log2;
+  p.out_scale = out_scale;
   // every Q block in one tile (decode-like): the instantiation with units in
-  // halves; the element type picks the MMA operand type and output packing
-  const dim3 grid(num_ctas), block(kThreads);
-  if (one_tile_blocks) {
-    if (fp16)
-      fwd_kernel<true, true><<<grid, block, kSmemBytes, stream>>>(map_q, map_k, map_v, p);
-    else
-      fwd_kernel<true, false><<<grid, block, kSmemBytes, stream>>>(map_q, map_k, map_v, p);
-  } else {
-    if (fp16)
-      fwd_kernel<false, true><<<grid, block, kSmemBytes, stream>>>(map_q, map_k, map_v, p);
-    else
-      fwd_kernel<false, false><<<grid, block, kSmemBytes, stream>>>(map_q, map_k, map_v, p);
-  }
+  // halves; the element type picks the MMA kind, P's format and the output type
+  kernels[dtype][one_tile_blocks ? 1 : 0]<<<num_ctas, kThreads, kSmemBytes, stream>>>(
+      map_q, map_k, map_v, p);
   e = cudaGetLastError();
   if (e != cudaSuccess || comb_cap <= 0) return e;
   CombineParams c;
@@ -1119,7 +1192,7 @@ cudaError_t launch_forward(const CUtensorMap& map_q, const CUtensorMap& map_k,
   c.tile_tokens = tile_tokens;
   c.rows_per_unit = rows_per_unit;
   c.return_lse = return_lse;
-  c.fp16 = fp16 ? 1 : 0;
+  c.fp16 = dtype == kDtFp16 ? 1 : 0;
   combine_kernel<<<(unsigned)comb_cap, 256, 0, stream>>>(c);
   return cudaGetLastError();
 }

@@ -57,7 +57,8 @@ class _Problem(ctypes.Structure):
                 ("has_seqused_q", ctypes.c_int32), ("num_ctas", ctypes.c_int32),
                 ("max_blocks_per_split", ctypes.c_int32), ("dtype", ctypes.c_int32),
                 ("softmax_precision", ctypes.c_int32), ("kv_layout", ctypes.c_int32),
-                ("T_kv", ctypes.c_int32)]
+                ("T_kv", ctypes.c_int32), ("q_scale", ctypes.c_double),
+                ("k_scale", ctypes.c_double), ("v_scale", ctypes.c_double)]
 
 
 class _Tensors(ctypes.Structure):
@@ -90,10 +91,13 @@ class Problem:
     num_ctas: int = 0
     max_blocks_per_split: int = 0
     block_y: int = 128
-    dtype: int = 0              # 0 = bf16, 1 = fp16 (q, k, v and out)
+    dtype: int = 0              # 0 = bf16, 1 = fp16, 2 = E4M3 (q, k, v; out bf16 for E4M3)
     softmax_precision: int = 0  # 0 = fp32 online softmax (the only one built)
     kv_layout: int = 0          # 0 = paged pool + block_table, 1 = TND + cu_seqlens_kv
     T_kv: int = 0               # TND: rows of k and v
+    q_scale: float = 1.0        # E4M3: per-tensor dequantization scales
+    k_scale: float = 1.0
+    v_scale: float = 1.0
 
     def as_c(self) -> _Problem:
         p = _Problem()
@@ -102,16 +106,23 @@ class Problem:
         return p
 
 
-ABI_VERSION = 3
-DTYPE_BF16, DTYPE_FP16 = 0, 1
+ABI_VERSION = 4
+DTYPE_BF16, DTYPE_FP16, DTYPE_FP8_E4M3 = 0, 1, 2
 
 
 def _dtype_code(t) -> int:
     import torch
-    codes = {torch.bfloat16: DTYPE_BF16, torch.float16: DTYPE_FP16}
+    codes = {torch.bfloat16: DTYPE_BF16, torch.float16: DTYPE_FP16,
+             torch.float8_e4m3fn: DTYPE_FP8_E4M3}
     if t.dtype not in codes:
-        raise ValueError(f"expected bf16 or fp16, got {t.dtype}")
+        raise ValueError(f"expected bf16, fp16 or float8_e4m3fn, got {t.dtype}")
     return codes[t.dtype]
+
+
+def _out_dtype(t):
+    """Element type of out: q's type, except bf16 for E4M3 inputs."""
+    import torch
+    return torch.bfloat16 if t.dtype == torch.float8_e4m3fn else t.dtype
 
 
 def library_path() -> str:
@@ -245,7 +256,7 @@ def metadata(sparse_block_idx, sparse_block_count, num_heads_q: int, num_heads_k
 def make_problem(q, k, sparse_block_idx, block_shape, block_table, cu_seqlens_q, *,
                  softmax_scale=0.0, mask_mode=1, win_left=-1, win_right=-1, is_packed_gqa=True,
                  return_softmax_lse=False, has_seqused_q=False, num_ctas=0,
-                 max_blocks_per_split=0) -> Problem:
+                 max_blocks_per_split=0, dequant_scales=(1.0, 1.0, 1.0)) -> Problem:
     """The gbsa_problem a forward call with these tensors describes.  A 4-d k
     is the page pool (block_table given); a 3-d k is TND [T_kv, N2, D]."""
     T, N1, D = q.shape
@@ -263,7 +274,9 @@ def make_problem(q, k, sparse_block_idx, block_shape, block_table, cu_seqlens_q,
                    mask_mode=mask_mode, win_left=win_left, win_right=win_right,
                    is_packed_gqa=int(bool(is_packed_gqa)), return_lse=int(bool(return_softmax_lse)),
                    has_seqused_q=int(bool(has_seqused_q)), num_ctas=num_ctas,
-                   max_blocks_per_split=max_blocks_per_split, dtype=_dtype_code(q))
+                   max_blocks_per_split=max_blocks_per_split, dtype=_dtype_code(q),
+                   q_scale=float(dequant_scales[0]), k_scale=float(dequant_scales[1]),
+                   v_scale=float(dequant_scales[2]))
 
 
 def forward(q, k, v, sparse_block_idx, sparse_block_count, block_shape: Sequence[int], *,
@@ -272,17 +285,22 @@ def forward(q, k, v, sparse_block_idx, sparse_block_count, block_shape: Sequence
             softmax_scale: float = 0.0, mask_mode: int = 1, win_left: int = -1,
             win_right: int = -1, is_packed_gqa: bool = True, return_softmax_lse: bool = False,
             num_ctas: int = 0, max_blocks_per_split: int = 0, out=None, lse=None, workspace=None,
-            dev_status=None):
+            dev_status=None, q_dequant_scale=None, k_dequant_scale=None, v_dequant_scale=None):
     """Block-sparse paged GQA attention.  q, k and v share one element type,
-    bf16 or fp16.  K/V come as the page pool [num_pages, 128, N2, D] with
-    ``block_table`` (PA_BBND), or, when ``cu_seqlens_kv`` is given, as TND
-    [T_kv, N2, D] with sequence b in rows cu_seqlens_kv[b]..cu_seqlens_kv[b+1]
-    (no block table).  Returns (out [T,N1,D] in q's type, lse [T,N1,1] fp32 --
-    an empty tensor unless return_softmax_lse)."""
+    bf16, fp16 or float8_e4m3fn.  K/V come as the page pool [num_pages, 128,
+    N2, D] with ``block_table`` (PA_BBND), or, when ``cu_seqlens_kv`` is given,
+    as TND [T_kv, N2, D] with sequence b in rows cu_seqlens_kv[b]..
+    cu_seqlens_kv[b+1] (no block table).  E4M3 inputs (the quantised mode
+    with static per-tensor scales) take ``q/k/v_dequant_scale`` as positive
+    host floats (default 1.0; ignored for the 16-bit types) and give a bf16
+    out.  Returns (out [T,N1,D] in q's type -- bf16 for E4M3 --, lse [T,N1,1]
+    fp32, an empty tensor unless return_softmax_lse)."""
     import torch
-    if q is None or q.dtype not in (torch.bfloat16, torch.float16):
-        raise ValueError("q: expected a bf16 or fp16 tensor")
+    if q is None or q.dtype not in (torch.bfloat16, torch.float16, torch.float8_e4m3fn):
+        raise ValueError("q: expected a bf16, fp16 or float8_e4m3fn tensor")
     q = _need(q, "q", q.dtype, 3)
+    scales = tuple(1.0 if s is None else float(s)
+                   for s in (q_dequant_scale, k_dequant_scale, v_dequant_scale))
     dev = q.device
     tnd = cu_seqlens_kv is not None
     if tnd:
@@ -314,13 +332,13 @@ def forward(q, k, v, sparse_block_idx, sparse_block_count, block_shape: Sequence
                         mask_mode=mask_mode, win_left=win_left, win_right=win_right,
                         is_packed_gqa=is_packed_gqa, return_softmax_lse=return_softmax_lse,
                         has_seqused_q=squ is not None, num_ctas=num_ctas,
-                        max_blocks_per_split=max_blocks_per_split)
+                        max_blocks_per_split=max_blocks_per_split, dequant_scales=scales)
     T, N1, D = q.shape
     with torch.cuda.device(dev):
         if out is None:
-            out = torch.empty_like(q)
+            out = torch.empty(q.shape, dtype=_out_dtype(q), device=dev)
         else:
-            out = _need(out, "out", q.dtype, 3, dev)
+            out = _need(out, "out", _out_dtype(q), 3, dev)
             if out.shape != q.shape:
                 raise ValueError(f"out: expected shape {tuple(q.shape)}")
         if return_softmax_lse:

@@ -257,7 +257,8 @@ WORKLOADS = ("tiny", "dense", "long", "decode", "ragged")
 
 def make_values(w: Workload, device="cpu", nan_fill=True, dtype=None):
     """Draws q [T,N1,D] and the K/V pools on ``device``: N(0,1) rounded to
-    ``dtype`` (torch.bfloat16, the default, or torch.float16).
+    ``dtype`` (torch.bfloat16, the default, torch.float16 or
+    torch.float8_e4m3fn; unreadable pool slots are NaN in each).
 
     Returns (q, k_flat, v_flat): the pools are flat buffers of
     num_pages*kv_page_stride elements; ``pool_view`` gives the
@@ -273,10 +274,9 @@ def make_values(w: Workload, device="cpu", nan_fill=True, dtype=None):
     pools = []
     for _ in range(2):
         flat = torch.randn((w.pool_elems,), generator=g, device=device, dtype=torch.float32)
-        flat = flat.to(dtype)
         if nan_fill:
             _fill_unreadable(w, flat)
-        pools.append(flat)
+        pools.append(flat.to(dtype))
     return q, pools[0], pools[1]
 
 

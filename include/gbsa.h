@@ -54,7 +54,7 @@
 extern "C" {
 #endif
 
-#define GBSA_ABI_VERSION 3
+#define GBSA_ABI_VERSION 4
 
 /* Symbols of the C ABI are exported; everything else in libgbsa is hidden. */
 #if defined(__GNUC__)
@@ -114,12 +114,15 @@ typedef struct gbsa_problem {
   int32_t has_seqused_q;      /* 1: seqused_q is given; 0: every Q storage token is used      */
   int32_t num_ctas;           /* persistent CTAs of the forward; 0 = SM count of the device   */
   int32_t max_blocks_per_split; /* 0 = automatic split-KV length; > 0 forces a smaller one     */
-  int32_t dtype;              /* element type of q, k, v and out: GBSA_DTYPE_BF16 or _FP16    */
+  int32_t dtype;              /* element type of q, k, v: GBSA_DTYPE_BF16, _FP16, _FP8_E4M3   */
   int32_t softmax_precision;  /* softmaxPrecision: 0 = fp32 online softmax (the one built);
                                  1 (fp16 softmax) returns GBSA_ERR_UNSUPPORTED               */
   int32_t kv_layout;          /* GBSA_KV_PAGED (k, v: the page pool, block_table) or
                                  GBSA_KV_TND (k, v: [T_kv, N2, D], cu_seqlens_kv)             */
   int32_t T_kv;               /* GBSA_KV_TND: rows of k and v (= cu_seqlens_kv[B]); else 0   */
+  double q_scale;             /* GBSA_DTYPE_FP8_E4M3: per-tensor dequantization scales, each */
+  double k_scale;             /*   finite and > 0 (q = q_scale * code, ...); the other dtypes */
+  double v_scale;             /*   ignore them                                                 */
 } gbsa_problem;
 
 /* K/V layouts (GBSA article, "Constraints: layouts": PA_BBND page pool, or
@@ -132,13 +135,20 @@ typedef struct gbsa_problem {
 #define GBSA_KV_TND 1
 
 /* Element types (GBSA article, "Constraints: data types": bf16 and fp16 for
- * Q, K, V and the output; lse is fp32 either way).  Accumulation is fp32. */
+ * Q, K, V and the output; lse is fp32 either way).  Accumulation is fp32.
+ * GBSA_DTYPE_FP8_E4M3 (the article's quantised-input arguments, with one
+ * dequantization scale per tensor): q, k, v hold E4M3 codes (1 byte, no
+ * infinity, S.1111.111 = NaN), scores are (q_scale*q).(k_scale*k)*scale, the
+ * softmax weights are rounded to E4M3 (times 2^8) for the P.V product, and
+ * out is bf16 holding softmax(.) (v_scale*v).  Expected error per element:
+ * about 2^-4 of sum_p w_p |v_scale*v_p| (the weights' E4M3 rounding). */
 #define GBSA_DTYPE_BF16 0
 #define GBSA_DTYPE_FP16 1
+#define GBSA_DTYPE_FP8_E4M3 2
 
 /* Device pointers of one call (caller-owned).  Unused optional pointers are NULL. */
 typedef struct gbsa_tensors {
-  const void* q;               /* dtype [T, N1, D]                                */
+  const void* q;               /* dtype [T, N1, D] (E4M3: 1 byte per element)     */
   const void* k;               /* dtype [num_pages, 128, N2, D], page stride above*/
   const void* v;               /* same layout and stride as k                     */
   const int32_t* sparse_idx;   /* [N2, total_q_blocks, top_k]                     */
@@ -147,7 +157,7 @@ typedef struct gbsa_tensors {
   const int32_t* seqused_q;    /* [B] or NULL (has_seqused_q = 0)                 */
   const int32_t* seqused_kv;   /* [B]                                             */
   const int32_t* block_table;  /* [B, max_pages_per_seq]                          */
-  void* out;                   /* dtype [T, N1, D]                                */
+  void* out;                   /* [T, N1, D]: fp16 for FP16, else bf16            */
   float* lse;                  /* fp32 [T, N1] or NULL (return_lse = 0)           */
   const int64_t* cu_seqlens_kv; /* [B+1] for GBSA_KV_TND, else NULL               */
 } gbsa_tensors;

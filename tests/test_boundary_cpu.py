@@ -36,7 +36,7 @@ def test_exports_every_declared_symbol(lib):
             "gbsa_workspace_size"} <= set(names)
     for n in names:
         assert hasattr(lib, n), n
-    assert lib.gbsa_abi_version() == 3
+    assert lib.gbsa_abi_version() == 4
     for code in range(0, 9):
         assert lib.gbsa_status_string(code).decode().startswith("GBSA_")
 
@@ -77,7 +77,12 @@ CASES = [
     (dict(block_x=0), "GBSA_ERR_SHAPE"),
     (dict(win_left=-2), "GBSA_ERR_INVALID_ARG"),
     (dict(scale=-1.0), "GBSA_ERR_INVALID_ARG"),
-    (dict(dtype=2), "GBSA_ERR_INVALID_ARG"),                # neither bf16 nor fp16
+    (dict(dtype=3), "GBSA_ERR_INVALID_ARG"),                # not bf16, fp16 or E4M3
+    (dict(dtype=2, q_scale=0.0), "GBSA_ERR_INVALID_ARG"),   # E4M3 scales must be > 0
+    (dict(dtype=2, k_scale=-1.0), "GBSA_ERR_INVALID_ARG"),
+    (dict(dtype=2, v_scale=float("inf")), "GBSA_ERR_INVALID_ARG"),
+    (dict(dtype=2, v_scale=float("nan")), "GBSA_ERR_INVALID_ARG"),
+    (dict(dtype=2, q_scale=1e-20, k_scale=1e-20), "GBSA_ERR_INVALID_ARG"),  # folded scale underflows
     (dict(softmax_precision=1), "GBSA_ERR_UNSUPPORTED"),    # fp16 online softmax: not built
     (dict(softmax_precision=7), "GBSA_ERR_INVALID_ARG"),
     (dict(kv_layout=2), "GBSA_ERR_INVALID_ARG"),            # neither paged nor TND
@@ -151,3 +156,12 @@ def test_metadata_pointer_rules(lib):
     rc = lib.gbsa_metadata(ctypes.byref(p.as_c()), ctypes.byref(_fake_tensors()), 16, 8, None,
                            None)
     assert rc == 6                                                        # METADATA_TOO_SMALL
+
+
+def test_fp8_scales_are_ignored_for_16_bit_types(lib):
+    # the dequantization scales belong to the E4M3 mode only
+    for dt in (0, 1):
+        p, _ = _problem(dtype=dt, q_scale=0.0, k_scale=float("nan"))
+        assert gbsa.metadata_size(p) > 0
+    p, _ = _problem(dtype=2, q_scale=0.5, k_scale=2.0, v_scale=3.0)
+    assert gbsa.metadata_size(p) > 0
