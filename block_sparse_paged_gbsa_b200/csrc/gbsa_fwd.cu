@@ -674,8 +674,184 @@ __device__ void run_mma(const FwdParams& p, uint8_t* smem, Bars* bars, uint32_t 
 }
 
 // ---------------------------------------------------------------------------
+// softmax of a narrow tile (at most kNarrowRows live rows: decode with
+// G <= 8).  The live rows sit in TMEM lanes 0..7, all read by the first warp
+// of the warpgroup, which in the row-per-thread layout would spend 32 lanes
+// of exp2 per live row.  Instead that warp moves the 8 rows of S through
+// shared memory (the second Q slot, unused when every Q block is one tile)
+// so that each lane takes 32 keys of one row: lane = 4 * row + segment.  Row
+// maxima and sums reduce over the 4 lanes of a row; P goes back through
+// shared memory to the row's own lane for the TMEM store.  Lanes 8..127 of
+// S, P and O are padding rows that no output reads (their P is zero).  The
+// other three warps of the warpgroup only keep the barrier counts.
+// ---------------------------------------------------------------------------
+constexpr int kNarrowRows = 8;
+constexpr int kNarrowSStride = 148;  // floats per S row (spreads banks for both access patterns)
+constexpr int kNarrowSSeg = 36;      // floats between the 32-key segments of a row
+constexpr int kNarrowPStride = 68;   // words per P row
+constexpr int kNarrowSBytes = kNarrowRows * kNarrowSStride * 4;
+constexpr int kNarrowPBytes = kNarrowRows * kNarrowPStride * 4;
+static_assert(2 * kNarrowSBytes <= kHalfBytes && 2 * kNarrowPBytes <= kHalfBytes,
+              "the narrow scratch fits the second Q slot");
+static_assert(3 * kNarrowSSeg + 32 <= kNarrowSStride, "the segments fit a row");
+
+// One block of a narrow tile, run by the warpgroup's first warp.  m and l
+// are this lane's row statistics (m the same in the row's 4 lanes, l the
+// lane's partial sum).  ri, key_lo and key_hi describe row lane / 4.
+template <int kDt>
+__device__ __forceinline__ void softmax_narrow_block(const FwdParams& p, uint32_t t_s, uint32_t t_o,
+                                                     float* scr_s, uint32_t* scr_p, int32_t entry,
+                                                     const RowInfo& ri, int32_t key_lo,
+                                                     int32_t key_hi, float& m, float& l,
+                                                     uint32_t lane) {
+  const int nrow = (int)(lane >> 2), seg = (int)(lane & 3);
+#pragma unroll
+  for (int h = 0; h < 2; h++) {  // 64 columns at a time
+    uint32_t r[2][32];
+    tmem_ld_32x32(t_s + 64 * h, r[0]);
+    tmem_ld_32x32(t_s + 64 * h + 32, r[1]);
+    tmem_wait_ld(r[0]);
+    reg_fence(r[1]);
+    if (lane < (uint32_t)kNarrowRows) {
+      float* dst = scr_s + lane * kNarrowSStride + 2 * h * kNarrowSSeg;
+#pragma unroll
+      for (int q = 0; q < 2; q++)
+#pragma unroll
+        for (int i = 0; i < 8; i++)
+          *reinterpret_cast<uint4*>(dst + q * kNarrowSSeg + 4 * i) =
+              make_uint4(r[q][4 * i], r[q][4 * i + 1], r[q][4 * i + 2], r[q][4 * i + 3]);
+    }
+  }
+  __syncwarp();
+  float sv[32];
+  {
+    const float* src = scr_s + nrow * kNarrowSStride + seg * kNarrowSSeg;
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+      const float4 v = *reinterpret_cast<const float4*>(src + 4 * i);
+      sv[4 * i] = v.x;
+      sv[4 * i + 1] = v.y;
+      sv[4 * i + 2] = v.z;
+      sv[4 * i + 3] = v.w;
+    }
+  }
+  // visible keys of this block for the row: [clo, chi] (as in the wide path)
+  int32_t clo = 0, chi = kPage - 1;
+  if (!ri.used) {
+    clo = kPage;
+    chi = -1;
+  } else if (entry & kEntryMask) {
+    const int32_t base = (entry & kEntryLbMask) * kPage;
+    clo = key_lo == INT32_MIN ? 0 : max(key_lo - base, 0);
+    chi = min(key_hi - base, kPage - 1);
+  }
+  const int32_t k0 = seg * 32;
+  if (__any_sync(0xffffffffu, clo > k0 || chi < k0 + 31)) {
+#pragma unroll
+    for (int c = 0; c < 32; c++)
+      if (k0 + c < clo || k0 + c > chi) sv[c] = -INFINITY;
+  }
+  float mp[4];
+#pragma unroll
+  for (int k = 0; k < 4; k++) mp[k] = sv[k];
+#pragma unroll
+  for (int c = 4; c < 32; c += 2) mp[(c >> 1) & 3] = max3f(mp[(c >> 1) & 3], sv[c], sv[c + 1]);
+  float mx = fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3]));
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+  const float m_blk = mx * p.scale_log2;
+  const float m_new = fmaxf(m, m_blk);
+  const bool rescale =
+      m_new != -INFINITY && (m == -INFINITY || m_new > m + rescale_threshold<kDt>());
+  const bool fix_o = rescale && m != -INFINITY;
+  const float factor = fix_o ? fast_exp2(m - m_new) : 1.f;
+  if (rescale) {
+    l *= factor;
+    m = m_new;
+  }
+  const float neg_m = ((m == -INFINITY) ? 0.f : -m) + (kDt == kDtE4m3 ? 8.f : 0.f);
+  float pf[32];
+  float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+  for (int c = 0; c < 32; c += 2) {
+    pf[c] = fast_exp2(fmaf(sv[c], p.scale_log2, neg_m));
+    pf[c + 1] = fast_exp2(fmaf(sv[c + 1], p.scale_log2, neg_m));
+    s0 += pf[c];
+    s1 += pf[c + 1];
+  }
+  l += s0 + s1;
+  // the lane's 32 keys of P into the row's P line
+  constexpr int kPw = kDt == kDtE4m3 ? 8 : 16;  // words per 32 keys
+  {
+    uint32_t pk[kPw];
+    if constexpr (kDt == kDtE4m3) {
+#pragma unroll
+      for (int i = 0; i < 8; i++)
+        pk[i] = pack_e4m3x4(pf[4 * i], pf[4 * i + 1], pf[4 * i + 2], pf[4 * i + 3]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; i++) pk[i] = pack_x2<kDt == kDtFp16>(pf[2 * i], pf[2 * i + 1]);
+    }
+    uint32_t* dst = scr_p + nrow * kNarrowPStride + seg * kPw;
+#pragma unroll
+    for (int i = 0; i < kPw / 4; i++)
+      *reinterpret_cast<uint4*>(dst + 4 * i) =
+          make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+  }
+  __syncwarp();
+  // lane r < 8 stores row r's P (4 * kPw words) into its TMEM lane; the
+  // padding lanes store zeros
+  {
+    const bool own = lane < (uint32_t)kNarrowRows;
+    const uint32_t* src = scr_p + (lane & (kNarrowRows - 1)) * kNarrowPStride;
+#pragma unroll
+    for (int q = 0; q < 4; q++) {
+      uint32_t w[kPw];
+#pragma unroll
+      for (int i = 0; i < kPw / 4; i++) {
+        const uint4 v = own ? *reinterpret_cast<const uint4*>(src + q * kPw + 4 * i)
+                            : make_uint4(0u, 0u, 0u, 0u);
+        w[4 * i] = v.x;
+        w[4 * i + 1] = v.y;
+        w[4 * i + 2] = v.z;
+        w[4 * i + 3] = v.w;
+      }
+      if constexpr (kDt == kDtE4m3)
+        tmem_st_32x8(t_s + 8 * q, w);
+      else
+        tmem_st_32x16(t_s + 16 * q, w);
+    }
+  }
+  // O of the live rows to the new reference max (row r's factor is held by
+  // lanes 4r..4r+3)
+  const int src_lane = (int)(lane & (kNarrowRows - 1)) * 4;
+  const float f_own = __shfl_sync(0xffffffffu, factor, src_lane);
+  const bool fix_own =
+      __shfl_sync(0xffffffffu, fix_o ? 1 : 0, src_lane) != 0 && lane < (uint32_t)kNarrowRows;
+  if (__any_sync(0xffffffffu, fix_own)) {
+    const float f = fix_own ? f_own : 1.f;
+#pragma unroll 1
+    for (int c = 0; c < 4; c++) {
+      uint32_t o[32];
+      tmem_ld_32x32(t_o + 32 * c, o);
+      tmem_wait_ld(o);
+#pragma unroll
+      for (int i = 0; i < 32; i++) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
+      tmem_st_32x32(t_o + 32 * c, o);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // softmax (one warpgroup per tile slot; thread = tile row = TMEM lane)
 // ---------------------------------------------------------------------------
+// The kernel's dynamic shared memory (every extern __shared__ array starts at
+// the same address): offsets from it are constants, with no register.
+__device__ __forceinline__ uint8_t* dyn_smem() {
+  extern __shared__ __align__(1024) uint8_t dsm[];
+  return dsm;
+}
+
 template <bool kHalves, int kDt>
 __device__ void run_softmax(const FwdParams& p, Bars* bars, uint32_t tmem, int slot,
                             int32_t n_units, int64_t off_unit, int64_t off_item, int64_t off_list) {
@@ -683,125 +859,161 @@ __device__ void run_softmax(const FwdParams& p, Bars* bars, uint32_t tmem, int s
   const uint32_t lane_sel = (uint32_t)(threadIdx.x & 96) << 16;  // warp's 32-lane quarter
   const uint32_t t_s = tmem + 128 * slot + lane_sel;
   const uint32_t t_o = tmem + 256 + 128 * slot + lane_sel;
+  // narrow tiles (the one-tile instantiation only: the second Q slot is free)
+  const bool narrow = kHalves && p.tile_tokens * p.G <= kNarrowRows;
   uint32_t blk = 0, units = 0;
   for (int32_t wave = 0, u = unit_of(0); u < n_units; u = unit_of(++wave)) {
     const Unit x = load_unit<kHalves>(p.meta, off_unit, off_item, u, p.N2);
     const int32_t nblk = x.j1 - x.j0;
     if ((slot >= x.nt && !x.halves) || nblk <= 0) continue;
     // a unit in halves: both slots hold the rows of its one tile, slot s
-    // takes blocks s, s + 2, ...
-    const RowInfo ri = row_info(p, x, x.halves ? 0 : slot, row);
+    // takes blocks s, s + 2, ...  (narrow: this lane works on row lane / 4)
+    const bool narrow_lead = narrow && (threadIdx.x & 96) == 0;
+    const RowInfo ri = row_info(p, x, x.halves ? 0 : slot, narrow_lead ? (row >> 2) : row);
     const int32_t jb0 = x.halves ? slot : 0, jstep = x.halves ? 2 : 1;
     const int32_t key_hi = min(ri.pos, x.ku - 1);
     const int32_t key_lo = p.win_left >= 0 ? ri.pos - p.win_left : INT32_MIN;
     const int32_t* list = p.meta + off_list + (int64_t)x.item * p.top_k + x.j0;
     float m = -INFINITY, l = 0.f;
-    for (int32_t jb = jb0; jb < nblk; jb += jstep) {
-      const int32_t entry = list[jb];
-      if (!wait_bar(&bars->s_full[slot], blk & 1, bars)) return;
-      tc_fence_after_sync();
-      uint32_t r[4][32];
-      tmem_ld_32x32(t_s + 0, r[0]);
-      tmem_ld_32x32(t_s + 32, r[1]);
-      tmem_ld_32x32(t_s + 64, r[2]);
-      tmem_ld_32x32(t_s + 96, r[3]);
-      tmem_wait_ld(r[0]);
-      reg_fence(r[1]);
-      reg_fence(r[2]);
-      reg_fence(r[3]);
-      // visible key columns of this block for this row: [clo, chi]; the
-      // element mask runs only in warps that hold a row needing it
-      int32_t clo = 0, chi = kPage - 1;
-      if (!ri.used) {
-        clo = kPage;
-        chi = -1;
-      } else if (entry & kEntryMask) {
-        const int32_t base = (entry & kEntryLbMask) * kPage;
-        clo = key_lo == INT32_MIN ? 0 : max(key_lo - base, 0);
-        chi = min(key_hi - base, kPage - 1);
-      }
-      if (__any_sync(0xffffffffu, clo > 0 || chi < kPage - 1)) {
-#pragma unroll
-        for (int c = 0; c < 128; c++)
-          if (c < clo || c > chi) r[c >> 5][c & 31] = __float_as_uint(-INFINITY);
-      }
-      // row max: eight independent partial maxima, then a tree
-      float mp[8];
-#pragma unroll
-      for (int k = 0; k < 8; k++) mp[k] = __uint_as_float(r[0][k]);
-#pragma unroll
-      for (int c = 8; c < 128; c += 2)
-        mp[(c >> 1) & 7] = max3f(mp[(c >> 1) & 7], __uint_as_float(r[c >> 5][c & 31]),
-                                 __uint_as_float(r[c >> 5][(c + 1) & 31]));
-      const float mx = max3f(max3f(mp[0], mp[1], mp[2]), max3f(mp[3], mp[4], mp[5]),
-                             fmaxf(mp[6], mp[7]));
-      const float m_blk = mx * p.scale_log2;
-      const float m_new = fmaxf(m, m_blk);
-      // lazy rescale: keep the old reference max unless it grew past the threshold
-      const bool rescale =
-          m_new != -INFINITY && (m == -INFINITY || m_new > m + rescale_threshold<kDt>());
-      const bool fix_o = rescale && m != -INFINITY;
-      const float factor = fix_o ? fast_exp2(m - m_new) : 1.f;
-      if (rescale) {
-        l *= factor;
-        m = m_new;
-      }
-      // E4M3 P carries a factor 2^8 (the row sum l too; the statistics
-      // handed on below take it out of m)
-      const float neg_m = ((m == -INFINITY) ? 0.f : -m) + (kDt == kDtE4m3 ? 8.f : 0.f);
-      // scores pairwise: x = s * scale_log2 - m as one f32x2 FMA, P = 2^x,
-      // the row sum in two packed partial sums (four independent lanes)
-      const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2), nm2 = f2_pack(neg_m, neg_m);
-      uint64_t sp2[2] = {0ull, 0ull};
-#pragma unroll
-      for (int q = 0; q < 4; q++) {
-        float pf[32];
-#pragma unroll
-        for (int i = 0; i < 16; i++) {
-          // masked scores are -inf and ex2(-inf) = +0
-          float x0, x1;
-          f2_unpack(f2_fma(f2_pack(__uint_as_float(r[q][2 * i]), __uint_as_float(r[q][2 * i + 1])),
-                           sc2, nm2),
-                    x0, x1);
-          pf[2 * i] = fast_exp2(x0);
-          pf[2 * i + 1] = fast_exp2(x1);
-          sp2[i & 1] = f2_add(sp2[i & 1], f2_pack(pf[2 * i], pf[2 * i + 1]));
+    if (kHalves && narrow) {
+      for (int32_t jb = jb0; jb < nblk; jb += jstep) {
+        const int32_t entry = list[jb];
+        if (!wait_bar(&bars->s_full[slot], blk & 1, bars)) return;
+        if (narrow_lead) {
+          tc_fence_after_sync();
+          float* scr_s =
+              reinterpret_cast<float*>(dyn_smem() + kSmemQ + kTileBytes + slot * kNarrowSBytes);
+          uint32_t* scr_p = reinterpret_cast<uint32_t*>(dyn_smem() + kSmemQ + kTileBytes +
+                                                        kHalfBytes + slot * kNarrowPBytes);
+          softmax_narrow_block<kDt>(p, t_s, t_o, scr_s, scr_p, entry, ri, key_lo, key_hi, m, l,
+                                    lane_id());
+          tmem_wait_st();
+          tc_fence_before_sync();
         }
-        if constexpr (kDt == kDtE4m3) {
-          // four E4M3 weights per TMEM column: 32 keys in 8 columns
-          uint32_t pk[8];
-#pragma unroll
-          for (int i = 0; i < 8; i++)
-            pk[i] = pack_e4m3x4(pf[4 * i], pf[4 * i + 1], pf[4 * i + 2], pf[4 * i + 3]);
-          tmem_st_32x8(t_s + 8 * q, pk);
-        } else {
-          uint32_t pk[16];
-#pragma unroll
-          for (int i = 0; i < 16; i++) pk[i] = pack_x2<kDt == kDtFp16>(pf[2 * i], pf[2 * i + 1]);
-          tmem_st_32x16(t_s + 16 * q, pk);
-        }
+        mbar_arrive(&bars->p_full[slot]);
+        blk++;
       }
-      float s0, s1, s2, s3;
-      f2_unpack(sp2[0], s0, s1);
-      f2_unpack(sp2[1], s2, s3);
-      l += (s0 + s1) + (s2 + s3);
-      if (__any_sync(0xffffffffu, fix_o)) {
-        // O holds the earlier blocks (their PV completed before this S was
-        // committed); bring it to the new reference max.
-#pragma unroll 1
-        for (int c = 0; c < 4; c++) {
-          uint32_t o[32];
-          tmem_ld_32x32(t_o + 32 * c, o);
-          tmem_wait_ld(o);
-#pragma unroll
-          for (int i = 0; i < 32; i++) o[i] = __float_as_uint(__uint_as_float(o[i]) * factor);
-          tmem_st_32x32(t_o + 32 * c, o);
+    } else {
+      for (int32_t jb = jb0; jb < nblk; jb += jstep) {
+        const int32_t entry = list[jb];
+        if (!wait_bar(&bars->s_full[slot], blk & 1, bars)) return;
+        tc_fence_after_sync();
+        uint32_t r[4][32];
+        tmem_ld_32x32(t_s + 0, r[0]);
+        tmem_ld_32x32(t_s + 32, r[1]);
+        tmem_ld_32x32(t_s + 64, r[2]);
+        tmem_ld_32x32(t_s + 96, r[3]);
+        tmem_wait_ld(r[0]);
+        reg_fence(r[1]);
+        reg_fence(r[2]);
+        reg_fence(r[3]);
+        // visible key columns of this block for this row: [clo, chi]; the
+        // element mask runs only in warps that hold a row needing it
+        int32_t clo = 0, chi = kPage - 1;
+        if (!ri.used) {
+          clo = kPage;
+          chi = -1;
+        } else if (entry & kEntryMask) {
+          const int32_t base = (entry & kEntryLbMask) * kPage;
+          clo = key_lo == INT32_MIN ? 0 : max(key_lo - base, 0);
+          chi = min(key_hi - base, kPage - 1);
         }
+        if (__any_sync(0xffffffffu, clo > 0 || chi < kPage - 1)) {
+  #pragma unroll
+          for (int c = 0; c < 128; c++)
+            if (c < clo || c > chi) r[c >> 5][c & 31] = __float_as_uint(-INFINITY);
+        }
+        // row max: eight independent partial maxima, then a tree
+        float mp[8];
+  #pragma unroll
+        for (int k = 0; k < 8; k++) mp[k] = __uint_as_float(r[0][k]);
+  #pragma unroll
+        for (int c = 8; c < 128; c += 2)
+          mp[(c >> 1) & 7] = max3f(mp[(c >> 1) & 7], __uint_as_float(r[c >> 5][c & 31]),
+                                   __uint_as_float(r[c >> 5][(c + 1) & 31]));
+        const float mx = max3f(max3f(mp[0], mp[1], mp[2]), max3f(mp[3], mp[4], mp[5]),
+                               fmaxf(mp[6], mp[7]));
+        const float m_blk = mx * p.scale_log2;
+        const float m_new = fmaxf(m, m_blk);
+        // lazy rescale: keep the old reference max unless it grew past the threshold
+        const bool rescale =
+            m_new != -INFINITY && (m == -INFINITY || m_new > m + rescale_threshold<kDt>());
+        const bool fix_o = rescale && m != -INFINITY;
+        const float factor = fix_o ? fast_exp2(m - m_new) : 1.f;
+        if (rescale) {
+          l *= factor;
+          m = m_new;
+        }
+        // E4M3 P carries a factor 2^8 (the row sum l too; the statistics
+        // handed on below take it out of m)
+        const float neg_m = ((m == -INFINITY) ? 0.f : -m) + (kDt == kDtE4m3 ? 8.f : 0.f);
+        // scores pairwise: x = s * scale_log2 - m as one f32x2 FMA, P = 2^x,
+        // the row sum in two packed partial sums (four independent lanes)
+        const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2), nm2 = f2_pack(neg_m, neg_m);
+        uint64_t sp2[2] = {0ull, 0ull};
+  #pragma unroll
+        for (int q = 0; q < 4; q++) {
+          float pf[32];
+  #pragma unroll
+          for (int i = 0; i < 16; i++) {
+            // masked scores are -inf and ex2(-inf) = +0
+            float x0, x1;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(r[q][2 * i]), __uint_as_float(r[q][2 * i + 1])),
+                             sc2, nm2),
+                      x0, x1);
+            pf[2 * i] = fast_exp2(x0);
+            pf[2 * i + 1] = fast_exp2(x1);
+            sp2[i & 1] = f2_add(sp2[i & 1], f2_pack(pf[2 * i], pf[2 * i + 1]));
+          }
+          if constexpr (kDt == kDtE4m3) {
+            // four E4M3 weights per TMEM column: 32 keys in 8 columns
+            uint32_t pk[8];
+  #pragma unroll
+            for (int i = 0; i < 8; i++)
+              pk[i] = pack_e4m3x4(pf[4 * i], pf[4 * i + 1], pf[4 * i + 2], pf[4 * i + 3]);
+            tmem_st_32x8(t_s + 8 * q, pk);
+          } else {
+            uint32_t pk[16];
+  #pragma unroll
+            for (int i = 0; i < 16; i++) pk[i] = pack_x2<kDt == kDtFp16>(pf[2 * i], pf[2 * i + 1]);
+            tmem_st_32x16(t_s + 16 * q, pk);
+          }
+        }
+        float s0, s1, s2, s3;
+        f2_unpack(sp2[0], s0, s1);
+        f2_unpack(sp2[1], s2, s3);
+        l += (s0 + s1) + (s2 + s3);
+        if (__any_sync(0xffffffffu, fix_o)) {
+          // O holds the earlier blocks (their PV completed before this S was
+          // committed); bring it to the new reference max.
+  #pragma unroll 1
+          for (int c = 0; c < 4; c++) {
+            uint32_t o[32];
+            tmem_ld_32x32(t_o + 32 * c, o);
+            tmem_wait_ld(o);
+  #pragma unroll
+            for (int i = 0; i < 32; i++) o[i] = __float_as_uint(__uint_as_float(o[i]) * factor);
+            tmem_st_32x32(t_o + 32 * c, o);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before_sync();
+        mbar_arrive(&bars->p_full[slot]);
+        blk++;
       }
-      tmem_wait_st();
-      tc_fence_before_sync();
-      mbar_arrive(&bars->p_full[slot]);
-      blk++;
+    }
+    if (kHalves && narrow) {
+      // row sums over the 4 lanes of a row, then lane r takes row r's
+      // statistics (rows past the live ones, and the other warps: none)
+      l += __shfl_xor_sync(0xffffffffu, l, 1);
+      l += __shfl_xor_sync(0xffffffffu, l, 2);
+      const uint32_t lane = lane_id();
+      const int src_lane = (int)(lane & (kNarrowRows - 1)) * 4;
+      const float m_r = __shfl_sync(0xffffffffu, m, src_lane);
+      const float l_r = __shfl_sync(0xffffffffu, l, src_lane);
+      const bool live = (threadIdx.x & 96) == 0 && lane < (uint32_t)kNarrowRows;
+      m = live ? m_r : -INFINITY;
+      l = live ? l_r : 0.f;
     }
     // hand the row statistics of this unit to the epilogue warpgroup
     if (units > 0 && !wait_bar(&bars->stats_free[slot], (units - 1) & 1, bars)) return;
