@@ -1186,6 +1186,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                const __grid_constant__ CUtensorMap map_v, const FwdParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const int warp = threadIdx.x >> 5;
+  allow_dependents();
+  grid_dependency_wait();  // the work list (and, before it, q, k and v)
 
   // the work list must have been built for this problem, and the swizzled
   // tiles need a 1 KiB aligned shared-memory window
@@ -1274,6 +1276,7 @@ struct CombineParams {
 };
 
 __global__ void __launch_bounds__(256) combine_kernel(const CombineParams p) {
+  grid_dependency_wait();  // the forward's partials
   const int32_t* meta = p.meta;
   if ((uint32_t)meta[H_MAGIC] != kMagic || (uint32_t)meta[H_SIGNATURE] != p.signature) return;
   const int32_t n_comb = meta[H_NCOMB];
@@ -1385,9 +1388,8 @@ cudaError_t launch_forward(const CUtensorMap& map_q, const CUtensorMap& map_k,
   p.out_scale = out_scale;
   // every Q block in one tile (decode-like): the instantiation with units in
   // halves; the element type picks the MMA kind, P's format and the output type
-  kernels[dtype][one_tile_blocks ? 1 : 0]<<<num_ctas, kThreads, kSmemBytes, stream>>>(
-      map_q, map_k, map_v, p);
-  e = cudaGetLastError();
+  e = launch_dependent(kernels[dtype][one_tile_blocks ? 1 : 0], dim3(num_ctas), dim3(kThreads),
+                       kSmemBytes, stream, map_q, map_k, map_v, p);
   if (e != cudaSuccess || comb_cap <= 0) return e;
   CombineParams c;
   c.meta = meta;
@@ -1405,8 +1407,7 @@ cudaError_t launch_forward(const CUtensorMap& map_q, const CUtensorMap& map_k,
   c.rows_per_unit = rows_per_unit;
   c.return_lse = return_lse;
   c.fp16 = dtype == kDtFp16 ? 1 : 0;
-  combine_kernel<<<(unsigned)comb_cap, 256, 0, stream>>>(c);
-  return cudaGetLastError();
+  return launch_dependent(combine_kernel, dim3((unsigned)comb_cap), dim3(256), 0, stream, c);
 }
 
 }  // namespace gbsa

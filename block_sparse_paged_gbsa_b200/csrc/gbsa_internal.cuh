@@ -25,6 +25,9 @@
 #pragma once
 
 #include <stdint.h>
+#ifdef __CUDACC__
+#include <cuda_runtime.h>
+#endif
 
 namespace gbsa {
 
@@ -77,5 +80,36 @@ struct MetaParams {
   int32_t* meta;
   int32_t* dev_status;
 };
+
+#ifdef __CUDACC__
+// Programmatic dependent launch.  Every kernel after the first of a call is
+// launched with programmatic stream serialization: it may start while the
+// kernel before it in the stream is still running, and waits in
+// grid_dependency_wait() -- before it touches global memory -- until that
+// kernel has completed and its writes are visible.  allow_dependents() lets
+// the next kernel start early (it still waits for this one to complete).
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void allow_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... Params, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem,
+                             cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+}
+#endif
 
 }  // namespace gbsa

@@ -79,6 +79,7 @@ __global__ void __launch_bounds__(kSeqThreads) seq_kernel(const MetaParams p) {
   __shared__ int32_t bad_sh;
   const Geometry& g = p.geo;
   int32_t* meta = p.meta;
+  allow_dependents();
   if (threadIdx.x == 0) bad_sh = 0;
   if (threadIdx.x < kHeaderWords) meta[threadIdx.x] = 0;
   __syncthreads();
@@ -151,6 +152,8 @@ __global__ void __launch_bounds__(kSeqThreads) seq_kernel(const MetaParams p) {
 constexpr int kItemWarps = 8;
 
 __global__ void __launch_bounds__(kItemWarps * 32) item_kernel(const MetaParams p) {
+  allow_dependents();
+  grid_dependency_wait();  // the sequence table
   const Geometry& g = p.geo;
   const int lane = threadIdx.x & 31;
   const int64_t item = (int64_t)blockIdx.x * kItemWarps + (threadIdx.x >> 5);
@@ -313,6 +316,8 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const MetaParams p) 
   __shared__ int32_t split_len_sh;
   __shared__ int32_t abort_sh;
 
+  allow_dependents();
+  grid_dependency_wait();  // the item table and live lists
   const Geometry& g = p.geo;
   int32_t* meta = p.meta;
   const int32_t* items = meta + g.off_item;
@@ -540,11 +545,9 @@ cudaError_t launch_metadata(const MetaParams& p, cudaStream_t stream) {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int64_t blocks = (p.geo.n_items + kItemWarps - 1) / kItemWarps;
-  item_kernel<<<(unsigned)blocks, kItemWarps * 32, 0, stream>>>(p);
-  e = cudaGetLastError();
+  e = launch_dependent(item_kernel, dim3((unsigned)blocks), dim3(kItemWarps * 32), 0, stream, p);
   if (e != cudaSuccess) return e;
-  plan_kernel<<<1, kPlanThreads, 0, stream>>>(p);
-  return cudaGetLastError();
+  return launch_dependent(plan_kernel, dim3(1), dim3(kPlanThreads), 0, stream, p);
 }
 
 }  // namespace gbsa
