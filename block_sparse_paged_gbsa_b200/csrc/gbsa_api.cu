@@ -197,9 +197,14 @@ bool encode(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims
   const CUtensorMapDataType t = dtype == GBSA_DTYPE_FP16       ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
                                 : dtype == GBSA_DTYPE_FP8_E4M3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
                                                                : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  return fn(map, t, rank, const_cast<void*>(base), dims,
-            strides_bytes, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  // L2 fills of the box rows' own size: a 16-bit head row is 256 B, an E4M3
+  // one 128 B (a 256 B fill would bring in the next head's row as well)
+  const CUtensorMapL2promotion promo = dtype == GBSA_DTYPE_FP8_E4M3
+                                           ? CU_TENSOR_MAP_L2_PROMOTION_L2_128B
+                                           : CU_TENSOR_MAP_L2_PROMOTION_L2_256B;
+  return fn(map, t, rank, const_cast<void*>(base), dims, strides_bytes, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, promo,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
