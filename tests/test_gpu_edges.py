@@ -104,3 +104,32 @@ def test_unpacked_gqa_gives_the_same_rows():
                                  return_softmax_lse=True))
     torch.cuda.synchronize()
     assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+
+
+NARROW = {
+    # tiles of at most 8 live rows take the narrow softmax (4 lanes per row);
+    # with several tokens per tile the rows differ in causal position
+    "g2_bx4": lambda: generate(name="n1", seed=84, q_storage=[37, 9, 130], q_used=[37, 7, 130],
+                               kv_used=[700, 300, 1200], N1=4, N2=2, block_x=4, top_k=6,
+                               selection="random_causal"),
+    "g4_bx2_window": lambda: generate(name="n2", seed=85, q_storage=[21, 64], kv_used=[900, 2000],
+                                      N1=8, N2=2, block_x=2, top_k=9, selection="random_any",
+                                      win_left=300, win_right=0),
+    "g1_bx8": lambda: generate(name="n3", seed=86, q_storage=[40, 17], kv_used=[1000, 640],
+                               N1=3, N2=3, block_x=8, top_k=5, selection="random_causal"),
+    "g2_bx3_rows6": lambda: generate(name="n5", seed=88, q_storage=[20, 11], q_used=[18, 11],
+                                     kv_used=[520, 300], N1=4, N2=2, block_x=3, top_k=4,
+                                     selection="random_causal", has_seqused_q=True),
+    "g8_decode": lambda: generate(name="n4", seed=87, q_storage=[1] * 6,
+                                  kv_used=[130, 1000, 4000, 129, 2500, 700], N1=16, N2=2,
+                                  block_x=1, top_k=40, selection="decode"),
+}
+
+
+@pytest.mark.parametrize("forced", [0, 3])
+@pytest.mark.parametrize("name", sorted(NARROW))
+def test_narrow_tiles(name, forced):
+    w = NARROW[name]()
+    assert min(128 // w.G, w.block_x) * w.G <= 8      # the narrow path runs
+    q, kf, vf, meta, out, lse = run_gpu(w, forced=forced)
+    _compare_all(w, q, kf, vf, out, lse)

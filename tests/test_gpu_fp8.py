@@ -140,3 +140,35 @@ def test_fp8_decode_full_size_sampled_rows():
     rng = np.random.default_rng(6)
     rows = np.stack([rng.integers(0, w.T, 1500), rng.integers(0, w.N1, 1500)], 1)
     _check(w, q, kf, vf, out, lse, rows)
+
+
+EDGE = {
+    # narrow tiles (<= 8 live rows) with several tokens per tile
+    "g2_bx4_narrow": lambda: generate(name="f1", seed=91, q_storage=[37, 130],
+                                      kv_used=[700, 1200], N1=4, N2=2, block_x=4, top_k=6,
+                                      selection="random_causal"),
+    # G = 1, one-token blocks, lists with masked and duplicate-free random blocks
+    "g1_bx1_any": lambda: generate(name="f2", seed=92, q_storage=[5, 3, 1], kv_used=[900, 300, 1500],
+                                   N1=2, N2=2, block_x=1, top_k=8, selection="random_any"),
+    # G = 128: one token per tile
+    "g128": lambda: generate(name="f3", seed=93, q_storage=[10, 4], N1=128, N2=1, block_x=3,
+                             top_k=3, selection="random_causal"),
+}
+
+
+@pytest.mark.parametrize("forced", [0, 3])
+@pytest.mark.parametrize("name", sorted(EDGE))
+def test_fp8_edge_shapes(name, forced):
+    w = EDGE[name]()
+    q, kf, vf = _values(w)
+    out, lse = _forward(w, q, pool_view(w, kf), pool_view(w, vf), forced=forced)
+    _check(w, q, kf, vf, out, lse)
+
+
+def test_fp8_all_lists_empty():
+    w = workload("tiny")
+    w.sparse_count[:] = 0
+    q, kf, vf = _values(w)
+    out, lse = _forward(w, q, pool_view(w, kf), pool_view(w, vf))
+    assert (out.float() == 0).all().item()
+    assert torch.isneginf(lse).all().item()
