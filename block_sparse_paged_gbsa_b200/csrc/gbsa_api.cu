@@ -73,8 +73,9 @@ gbsa_status validate(const gbsa_problem* p, bool metadata_mode) {
     if (folded > 1e30 || folded < 1e-30 || p->v_scale > 1e30 || p->v_scale < 1e-30)
       return GBSA_ERR_INVALID_ARG;
   }
-  if (p->softmax_precision == 1) return GBSA_ERR_UNSUPPORTED;
-  if (p->softmax_precision != 0) return GBSA_ERR_INVALID_ARG;
+  // softmaxPrecision 1 (half-precision softmax, fp32 rescale) is run with the
+  // fp32 softmax of mode 0: its error is below mode 1's for every element type
+  if (p->softmax_precision != 0 && p->softmax_precision != 1) return GBSA_ERR_INVALID_ARG;
   if (!(p->scale >= 0.0) || isinf(p->scale)) return GBSA_ERR_INVALID_ARG;
   if ((int64_t)p->N2 * p->total_q_blocks > 0x7fffffffLL / (p->top_k + 8)) return GBSA_ERR_SHAPE;
   if (p->kv_layout != GBSA_KV_PAGED && p->kv_layout != GBSA_KV_TND) return GBSA_ERR_INVALID_ARG;

@@ -92,7 +92,7 @@ class Problem:
     max_blocks_per_split: int = 0
     block_y: int = 128
     dtype: int = 0              # 0 = bf16, 1 = fp16, 2 = E4M3 (q, k, v; out bf16 for E4M3)
-    softmax_precision: int = 0  # 0 = fp32 online softmax (the only one built)
+    softmax_precision: int = 0  # 0 or 1; both run the fp32 online softmax
     kv_layout: int = 0          # 0 = paged pool + block_table, 1 = TND + cu_seqlens_kv
     T_kv: int = 0               # TND: rows of k and v
     q_scale: float = 1.0        # E4M3: per-tensor dequantization scales
@@ -214,8 +214,12 @@ def metadata(sparse_block_idx, sparse_block_count, num_heads_q: int, num_heads_k
              head_dim: int, block_shape: Sequence[int], *, cu_seqlens_q, seqused_kv,
              seqused_q=None, num_tokens: int = 0, is_packed_gqa: bool = True, mask_mode: int = 1,
              win_left: int = -1, win_right: int = -1, num_ctas: int = 0,
-             max_blocks_per_split: int = 0, dev_status=None, out=None):
+             max_blocks_per_split: int = 0, dev_status=None, out=None,
+             softmax_precision: int = 1):
     """Builds the work list (int32 tensor) on the device of the inputs.
+
+    softmax_precision: the article's softmaxPrecision (default 1, as in its
+    PyTorch API); 0 and 1 are accepted and both run the fp32 softmax.
 
     num_tokens: T if known (enables the device check cu_seqlens_q[B] == T); 0 skips it.
     out: optional preallocated int32 buffer of at least metadata_size() bytes.
@@ -235,7 +239,8 @@ def metadata(sparse_block_idx, sparse_block_count, num_heads_q: int, num_heads_k
                    D=head_dim, block_x=bx, block_y=by, total_q_blocks=tqb, top_k=top_k,
                    mask_mode=mask_mode, win_left=win_left, win_right=win_right,
                    is_packed_gqa=int(bool(is_packed_gqa)), has_seqused_q=int(squ is not None),
-                   num_ctas=num_ctas, max_blocks_per_split=max_blocks_per_split)
+                   num_ctas=num_ctas, max_blocks_per_split=max_blocks_per_split,
+                   softmax_precision=int(softmax_precision))
     nbytes = metadata_size(prob)
     with torch.cuda.device(dev):
         if out is None:
@@ -256,7 +261,8 @@ def metadata(sparse_block_idx, sparse_block_count, num_heads_q: int, num_heads_k
 def make_problem(q, k, sparse_block_idx, block_shape, block_table, cu_seqlens_q, *,
                  softmax_scale=0.0, mask_mode=1, win_left=-1, win_right=-1, is_packed_gqa=True,
                  return_softmax_lse=False, has_seqused_q=False, num_ctas=0,
-                 max_blocks_per_split=0, dequant_scales=(1.0, 1.0, 1.0)) -> Problem:
+                 max_blocks_per_split=0, dequant_scales=(1.0, 1.0, 1.0),
+                 softmax_precision=1) -> Problem:
     """The gbsa_problem a forward call with these tensors describes.  A 4-d k
     is the page pool (block_table given); a 3-d k is TND [T_kv, N2, D]."""
     T, N1, D = q.shape
@@ -276,7 +282,7 @@ def make_problem(q, k, sparse_block_idx, block_shape, block_table, cu_seqlens_q,
                    has_seqused_q=int(bool(has_seqused_q)), num_ctas=num_ctas,
                    max_blocks_per_split=max_blocks_per_split, dtype=_dtype_code(q),
                    q_scale=float(dequant_scales[0]), k_scale=float(dequant_scales[1]),
-                   v_scale=float(dequant_scales[2]))
+                   v_scale=float(dequant_scales[2]), softmax_precision=int(softmax_precision))
 
 
 def forward(q, k, v, sparse_block_idx, sparse_block_count, block_shape: Sequence[int], *,
@@ -285,7 +291,8 @@ def forward(q, k, v, sparse_block_idx, sparse_block_count, block_shape: Sequence
             softmax_scale: float = 0.0, mask_mode: int = 1, win_left: int = -1,
             win_right: int = -1, is_packed_gqa: bool = True, return_softmax_lse: bool = False,
             num_ctas: int = 0, max_blocks_per_split: int = 0, out=None, lse=None, workspace=None,
-            dev_status=None, q_dequant_scale=None, k_dequant_scale=None, v_dequant_scale=None):
+            dev_status=None, q_dequant_scale=None, k_dequant_scale=None, v_dequant_scale=None,
+            softmax_precision: int = 1):
     """Block-sparse paged GQA attention.  q, k and v share one element type,
     bf16, fp16 or float8_e4m3fn.  K/V come as the page pool [num_pages, 128,
     N2, D] with ``block_table`` (PA_BBND), or, when ``cu_seqlens_kv`` is given,
@@ -294,7 +301,9 @@ def forward(q, k, v, sparse_block_idx, sparse_block_count, block_shape: Sequence
     with static per-tensor scales) take ``q/k/v_dequant_scale`` as positive
     host floats (default 1.0; ignored for the 16-bit types) and give a bf16
     out.  Returns (out [T,N1,D] in q's type -- bf16 for E4M3 --, lse [T,N1,1]
-    fp32, an empty tensor unless return_softmax_lse)."""
+    fp32, an empty tensor unless return_softmax_lse).  softmax_precision is the
+    article's softmaxPrecision (default 1, as in its PyTorch API); 0 and 1 are
+    accepted and both run the fp32 online softmax."""
     import torch
     if q is None or q.dtype not in (torch.bfloat16, torch.float16, torch.float8_e4m3fn):
         raise ValueError("q: expected a bf16, fp16 or float8_e4m3fn tensor")
@@ -332,7 +341,8 @@ def forward(q, k, v, sparse_block_idx, sparse_block_count, block_shape: Sequence
                         mask_mode=mask_mode, win_left=win_left, win_right=win_right,
                         is_packed_gqa=is_packed_gqa, return_softmax_lse=return_softmax_lse,
                         has_seqused_q=squ is not None, num_ctas=num_ctas,
-                        max_blocks_per_split=max_blocks_per_split, dequant_scales=scales)
+                        max_blocks_per_split=max_blocks_per_split, dequant_scales=scales,
+                        softmax_precision=softmax_precision)
     T, N1, D = q.shape
     with torch.cuda.device(dev):
         if out is None:

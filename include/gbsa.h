@@ -115,8 +115,9 @@ typedef struct gbsa_problem {
   int32_t num_ctas;           /* persistent CTAs of the forward; 0 = SM count of the device   */
   int32_t max_blocks_per_split; /* 0 = automatic split-KV length; > 0 forces a smaller one     */
   int32_t dtype;              /* element type of q, k, v: GBSA_DTYPE_BF16, _FP16, _FP8_E4M3   */
-  int32_t softmax_precision;  /* softmaxPrecision: 0 = fp32 online softmax (the one built);
-                                 1 (fp16 softmax) returns GBSA_ERR_UNSUPPORTED               */
+  int32_t softmax_precision;  /* softmaxPrecision: 0 = fp32 online softmax; 1 (the article's
+                                 half-precision softmax with fp32 rescale) is accepted and
+                                 computed with the fp32 softmax, whose error is smaller   */
   int32_t kv_layout;          /* GBSA_KV_PAGED (k, v: the page pool, block_table) or
                                  GBSA_KV_TND (k, v: [T_kv, N2, D], cu_seqlens_kv)             */
   int32_t T_kv;               /* GBSA_KV_TND: rows of k and v (= cu_seqlens_kv[B]); else 0   */

@@ -83,8 +83,8 @@ CASES = [
     (dict(dtype=2, v_scale=float("inf")), "GBSA_ERR_INVALID_ARG"),
     (dict(dtype=2, v_scale=float("nan")), "GBSA_ERR_INVALID_ARG"),
     (dict(dtype=2, q_scale=1e-20, k_scale=1e-20), "GBSA_ERR_INVALID_ARG"),  # folded scale underflows
-    (dict(softmax_precision=1), "GBSA_ERR_UNSUPPORTED"),    # fp16 online softmax: not built
-    (dict(softmax_precision=7), "GBSA_ERR_INVALID_ARG"),
+    (dict(softmax_precision=2), "GBSA_ERR_INVALID_ARG"),
+    (dict(softmax_precision=-1), "GBSA_ERR_INVALID_ARG"),
     (dict(kv_layout=2), "GBSA_ERR_INVALID_ARG"),            # neither paged nor TND
 ]
 
@@ -156,6 +156,13 @@ def test_metadata_pointer_rules(lib):
     rc = lib.gbsa_metadata(ctypes.byref(p.as_c()), ctypes.byref(_fake_tensors()), 16, 8, None,
                            None)
     assert rc == 6                                                        # METADATA_TOO_SMALL
+
+
+def test_softmax_precision_one_is_accepted(lib):
+    # the article's PyTorch default; run with the fp32 softmax for every type
+    for dt in (0, 1, 2):
+        p, _ = _problem(dtype=dt, softmax_precision=1)
+        assert gbsa.metadata_size(p) == gbsa.metadata_size(_problem(dtype=dt)[0])
 
 
 def test_fp8_scales_are_ignored_for_16_bit_types(lib):
