@@ -12,13 +12,16 @@
 // Design (one persistent CTA per SM, 512 threads, four warpgroups):
 //   warps 0..3    softmax of tile 0 (TMEM lanes = tile rows)
 //   warps 4..7    softmax of tile 1
-//   warps 8..11   epilogue: O / l -> out (bf16) and lse, or split partials
+//   warps 8..11   epilogue: O / l -> out (bf16, or fp16 for fp16 inputs)
+//                 and lse, or split partials
 //   warp 12       MMA issuer: S = Q K^T (SS MMA), O += P V (TS MMA, P read
 //                 from TMEM); zeroes V rows of a last page past seqused_kv
 //   warp 13       TMA producer: Q tiles and, per live block, the K and V
-//                 pages into a 5-stage ring of 32 KiB buffers
-// TMEM (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each; P (bf16,
-// packed in pairs) overwrites the first 64 columns of its S.
+//                 pages into a ring of 5 x 32 KiB (10 x 16 KiB for E4M3)
+// TMEM (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each; P overwrites
+// the first columns of its S (two 16-bit or four E4M3 weights per column).
+// Element types (kDt): bf16, fp16 (kind::f16 MMAs) and E4M3 (kind::f8f6f4,
+// per-tensor dequantization scales folded into the score scale and 1 / l).
 // Units come from the metadata work list, longest first; the CTAs take them
 // wave by wave, in reverse CTA order on odd waves (unit_of).  Every wait is
 // bounded: after ~1 s the kernel sets GBSA_DEV_TIMEOUT, drains its own copies
@@ -59,7 +62,7 @@ static_assert(256 * regs_softmax<true>() + 128 * kRegsEpilogue + 128 * regs_cont
 constexpr int kWarpMma = 12;
 constexpr int kWarpProducer = 13;
 constexpr int kStages = 5;
-constexpr int kTileBytes = 32768;  // 128 rows x 128 bf16 (two 64-column SW128 boxes)
+constexpr int kTileBytes = 32768;  // 128 rows x 128 16-bit elements (two SW128 boxes)
 constexpr int kHalfBytes = 16384;
 constexpr int kSmemQ = 0;
 constexpr int kSmemRing = 2 * kTileBytes;
@@ -208,10 +211,11 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Bars* b
 
 // Operand layouts in shared memory (128-byte swizzle, tiles 1 KiB aligned):
 //   Q and K tiles, K-major: 128 rows x 128 B per 64-column half, halves
-//   16 KiB apart; a K step of 16 bf16 advances 32 B inside the row.
+//   16 KiB apart; a K step of 16 16-bit elements advances 32 B inside the
+//   row.  E4M3: one half of 128 columns, a K step of 32 elements (32 B).
 //   V tile, MN-major (N = D): the two 64-column halves of D 16 KiB apart
 //   (leading byte offset), 8-key groups 1 KiB apart; a K step of 16 keys
-//   advances 2 KiB.
+//   advances 2 KiB (E4M3: D in one 128 B row, a K step of 32 keys 4 KiB).
 
 // Row identity of TMEM lane `row` in tile `slot` of unit x.
 struct RowInfo {

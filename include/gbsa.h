@@ -32,17 +32,24 @@
  *     the host (GBSA article, "Constraints": tiling does not check values);
  *     when `dev_status` is non-NULL the kernels OR GBSA_DEV_* bits into that
  *     device int32 instead (and skip the offending work; they never trap).
- *   - Layouts (GBSA article, "Parameters" and the aclnn example call):
- *       q            [T, N1, D]                 bf16, contiguous   (TND)
- *       k, v         [num_pages, 128, N2, D]    bf16; only dim0 may be
- *                    strided: stride0 = kv_page_stride elements  (PA_BBND)
+ *   - Every kernel after the first of a call is launched with programmatic
+ *     stream serialization: it may start while the previous kernel on the
+ *     stream is finishing, and waits for that kernel's completion before it
+ *     reads or writes global memory, so stream order holds as usual.
+ *   - Layouts (GBSA article, "Parameters" and the aclnn example call); the
+ *     element type of q, k and v is gbsa_problem.dtype (bf16, fp16 or E4M3):
+ *       q            [T, N1, D]                 contiguous   (TND)
+ *       k, v         [num_pages, 128, N2, D]    only dim0 may be strided:
+ *                    stride0 = kv_page_stride elements  (PA_BBND), or
+ *                    [T_kv, N2, D] contiguous with cu_seqlens_kv (TND)
  *       sparse_idx   [N2, total_q_blocks, top_k] int32, contiguous
  *       sparse_count [N2, total_q_blocks]        int32, contiguous
  *       cu_seqlens_q [B+1]                       int64 prefix sums of the
  *                                                Q storage lengths
  *       seqused_q    [B] int32 (optional), seqused_kv [B] int32 (required)
  *       block_table  [B, max_pages_per_seq]      int32 logical->physical page
- *       out          [T, N1, D] bf16;  lse [T, N1] fp32 (natural log)
+ *       out          [T, N1, D] fp16 for fp16 inputs, else bf16;
+ *       lse          [T, N1] fp32 (natural log)
  */
 #ifndef GBSA_H
 #define GBSA_H

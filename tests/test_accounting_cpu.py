@@ -70,3 +70,36 @@ def test_block_flops_match_work_list(case):
     tt, hh = np.meshgrid(np.arange(w.T), np.arange(w.N1), indexing="ij")
     rows = np.stack([tt.reshape(-1), hh.reshape(-1)], 1)
     assert row_flops(w, rows) == flops
+
+
+def _bench_module():
+    import importlib.util
+    import os
+    path = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "bench.py")
+    spec = importlib.util.spec_from_file_location("gbsa_bench", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def test_kernel_hash_ignores_comments_only():
+    b = _bench_module()
+    src = 'int a = 1; // note\n/* block\n comment */ asm("x // y /* z */"); char c = \'/\';\n'
+    assert b.code_tokens(src) == b.code_tokens(src.replace("note", "other").replace("block", "b"))
+    assert b.code_tokens(src) != b.code_tokens(src.replace("a = 1", "a = 2"))
+    assert b.code_tokens(src) != b.code_tokens(src.replace("x // y", "x // w"))  # inside a string
+    assert "note" not in b.code_tokens(src) and "x // y /* z */" in b.code_tokens(src)
+
+
+def test_committed_traffic_records_are_well_formed():
+    # bench.py reads a record only while its kernel_sha equals kernel_hash()
+    import glob
+    import json
+    import os
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    recs = glob.glob(os.path.join(root, "profiles", "forward_*_traffic.json"))
+    assert recs
+    for r in recs:
+        d = json.load(open(r))
+        assert len(d["kernel_sha"]) == 16 and int(d["dram_bytes_per_launch"]) > 0, r
+        assert "--clock-control none" in d["command"], r
