@@ -172,3 +172,35 @@ def test_fp8_scales_are_ignored_for_16_bit_types(lib):
         assert gbsa.metadata_size(p) > 0
     p, _ = _problem(dtype=2, q_scale=0.5, k_scale=2.0, v_scale=3.0)
     assert gbsa.metadata_size(p) > 0
+
+
+def test_binding_element_types():
+    # the Python binding maps torch dtypes to gbsa_problem.dtype and out's type
+    import torch
+    from block_sparse_paged_gbsa_b200.gbsa import _dtype_code, _out_dtype, make_problem
+    w = workload("tiny")
+    for dt, code, out in ((torch.bfloat16, 0, torch.bfloat16), (torch.float16, 1, torch.float16),
+                          (torch.float8_e4m3fn, 2, torch.bfloat16)):
+        q = torch.zeros((w.T, w.N1, w.D), dtype=dt)
+        k = torch.zeros((w.num_pages, 128, w.N2, w.D), dtype=dt)
+        assert _dtype_code(q) == code and _out_dtype(q) == out
+        idx = torch.zeros((w.N2, w.total_q_blocks, w.top_k), dtype=torch.int32)
+        bt = torch.zeros((w.B, w.max_pages_per_seq), dtype=torch.int32)
+        cu = torch.zeros((w.B + 1,), dtype=torch.int64)
+        prob = make_problem(q, k, idx, [w.block_x, 128], bt, cu, dequant_scales=(0.5, 2.0, 4.0),
+                            num_ctas=148)
+        assert prob.dtype == code and (prob.q_scale, prob.k_scale, prob.v_scale) == (0.5, 2.0, 4.0)
+        assert gbsa.metadata_size(prob) > 0
+    with pytest.raises(ValueError):
+        _dtype_code(torch.zeros(1, dtype=torch.float32))
+
+
+def test_binding_rejects_other_element_types():
+    # checked before anything touches a device
+    import torch
+    w = workload("tiny")
+    q = torch.zeros((w.T, w.N1, w.D), dtype=torch.float32)
+    z = torch.zeros(1, dtype=torch.int32)
+    with pytest.raises(ValueError, match="bf16, fp16 or float8_e4m3fn"):
+        gbsa.forward(q, q, q, z, z, [w.block_x, 128], metadata=z, cu_seqlens_q=z, seqused_kv=z,
+                     block_table=z)
