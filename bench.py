@@ -285,8 +285,11 @@ def run_reference(args, world, rank):
         return
     from block_sparse_paged_gbsa_b200.workloads import make_values, workload
 
+    import torch
+
     w = workload(args.workload, scale_down=args.scale_down)
-    q, kf, vf = make_values(w, "cpu")
+    tdt = {"bf16": torch.bfloat16, "fp16": torch.float16, "e4m3": torch.float8_e4m3fn}[args.dtype]
+    q, kf, vf = make_values(w, "cpu", dtype=tdt)  # the inputs of the GPU arm's --dtype
     per_step = max(0.5, min(5.0, 150.0 / max(1, args.steps + args.warmup)))
     vals = []
     for i in range(args.warmup + args.steps):
