@@ -250,6 +250,8 @@ def metadata(sparse_block_idx, sparse_block_count, num_heads_q: int, num_heads_k
             if meta.numel() * 4 < nbytes:
                 raise ValueError(f"out: needs {nbytes} bytes")
             nbytes = meta.numel() * 4
+        if dev_status is not None:
+            dev_status = _need(dev_status, "dev_status", torch.int32, 1, dev)
         ten = _Tensors(sparse_idx=_ptr(idx), sparse_count=_ptr(cnt), cu_seqlens_q=_ptr(cu),
                        seqused_q=_ptr(squ), seqused_kv=_ptr(sku))
         _check(_load().gbsa_metadata(ctypes.byref(prob.as_c()), ctypes.byref(ten),
@@ -354,11 +356,19 @@ def forward(q, k, v, sparse_block_idx, sparse_block_count, block_shape: Sequence
         if return_softmax_lse:
             if lse is None:
                 lse = torch.empty((T, N1, 1), dtype=torch.float32, device=dev)
+            else:
+                lse = _need(lse, "lse", torch.float32, 3, dev)
+                if tuple(lse.shape) != (T, N1, 1):
+                    raise ValueError(f"lse: expected shape {(T, N1, 1)}")
         else:
             lse = torch.empty((0,), dtype=torch.float32, device=dev)
         ws_bytes = workspace_size(prob)
         if workspace is None:
             workspace = torch.empty((max(ws_bytes, 16),), dtype=torch.uint8, device=dev)
+        else:
+            workspace = _need(workspace, "workspace", torch.uint8, 1, dev)
+        if dev_status is not None:
+            dev_status = _need(dev_status, "dev_status", torch.int32, 1, dev)
         ten = _Tensors(q=_ptr(q), k=_ptr(k), v=_ptr(v), sparse_idx=_ptr(idx),
                        sparse_count=_ptr(cnt), cu_seqlens_q=_ptr(cu), seqused_q=_ptr(squ),
                        seqused_kv=_ptr(sku), block_table=_ptr(bt), out=_ptr(out),
