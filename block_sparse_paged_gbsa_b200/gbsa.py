@@ -210,13 +210,34 @@ def _block_shape(block_shape: Sequence[int]):
     return bx, by
 
 
+QUANT_NONE, QUANT_FP8_E4M3_STATIC_CAST_P = 0, 5  # the article's quant_mode values
+
+
+def _check_layouts(layout_q, layout_kv, quant_mode):
+    """The article's layout and quantisation arguments: TND queries, PA_BBND
+    or TND keys/values, quant_mode 0 or 5 (anything else is unsupported)."""
+    if layout_q != "TND":
+        raise ValueError(f"layout_q: only 'TND' is supported, got {layout_q!r}")
+    if layout_kv is not None and layout_kv not in ("PA_BBND", "TND"):
+        raise ValueError(f"layout_kv: 'PA_BBND' or 'TND', got {layout_kv!r}")
+    if quant_mode is not None and int(quant_mode) not in (QUANT_NONE, QUANT_FP8_E4M3_STATIC_CAST_P):
+        raise ValueError(f"quant_mode: 0 or 5 are supported, got {quant_mode!r}")
+
+
 def metadata(sparse_block_idx, sparse_block_count, num_heads_q: int, num_heads_kv: int,
              head_dim: int, block_shape: Sequence[int], *, cu_seqlens_q, seqused_kv,
              seqused_q=None, num_tokens: int = 0, is_packed_gqa: bool = True, mask_mode: int = 1,
              win_left: int = -1, win_right: int = -1, num_ctas: int = 0,
              max_blocks_per_split: int = 0, dev_status=None, out=None,
-             softmax_precision: int = 1):
+             softmax_precision: int = 1, cu_seqlens_kv=None, max_seqlen_q: int = -1,
+             max_seqlen_kv: int = -1, layout_q: str = "TND", layout_kv: str = "PA_BBND",
+             quant_mode: int = 0):
     """Builds the work list (int32 tensor) on the device of the inputs.
+
+    The article's remaining metadata arguments are accepted: layout_q
+    ('TND'), layout_kv ('PA_BBND' or 'TND') and quant_mode (0 or 5) are
+    checked; cu_seqlens_kv and max_seqlen_q / max_seqlen_kv do not enter the
+    work list (it depends on seqused_kv and the Q lengths only).
 
     softmax_precision: the article's softmaxPrecision (default 1, as in its
     PyTorch API); 0 and 1 are accepted and both run the fp32 softmax.
@@ -225,6 +246,7 @@ def metadata(sparse_block_idx, sparse_block_count, num_heads_q: int, num_heads_k
     out: optional preallocated int32 buffer of at least metadata_size() bytes.
     """
     import torch
+    _check_layouts(layout_q, layout_kv, quant_mode)
     idx = _need(sparse_block_idx, "sparse_block_idx", torch.int32, 3)
     dev = idx.device
     cnt = _need(sparse_block_count, "sparse_block_count", torch.int32, 2, dev)
@@ -294,7 +316,9 @@ def forward(q, k, v, sparse_block_idx, sparse_block_count, block_shape: Sequence
             win_right: int = -1, is_packed_gqa: bool = True, return_softmax_lse: bool = False,
             num_ctas: int = 0, max_blocks_per_split: int = 0, out=None, lse=None, workspace=None,
             dev_status=None, q_dequant_scale=None, k_dequant_scale=None, v_dequant_scale=None,
-            softmax_precision: int = 1):
+            softmax_precision: int = 1, attn_mask=None, p_quant_scale=None,
+            layout_q: str = "TND", layout_kv=None, quant_mode=None, dst_type_max: float = 0.0,
+            attention_out_dtype=None):
     """Block-sparse paged GQA attention.  q, k and v share one element type,
     bf16, fp16 or float8_e4m3fn.  K/V come as the page pool [num_pages, 128,
     N2, D] with ``block_table`` (PA_BBND), or, when ``cu_seqlens_kv`` is given,
@@ -305,10 +329,31 @@ def forward(q, k, v, sparse_block_idx, sparse_block_count, block_shape: Sequence
     out.  Returns (out [T,N1,D] in q's type -- bf16 for E4M3 --, lse [T,N1,1]
     fp32, an empty tensor unless return_softmax_lse).  softmax_precision is the
     article's softmaxPrecision (default 1, as in its PyTorch API); 0 and 1 are
-    accepted and both run the fp32 online softmax."""
+    accepted and both run the fp32 online softmax.
+
+    The article's remaining arguments: attn_mask must be None (only the
+    built-in causal mask, mask_mode 1, exists); layout_q is 'TND'; layout_kv,
+    when given, must agree with the tensors ('TND' with cu_seqlens_kv,
+    'PA_BBND' with block_table); quant_mode, when given, must agree with q's
+    type (0: bf16 / fp16, 5: float8_e4m3fn); p_quant_scale must be None (the
+    weights are cast with the fixed factor 2^8); attention_out_dtype, when
+    given, must be the type of out (q's, bf16 for E4M3); dst_type_max is not
+    used."""
     import torch
     if q is None or q.dtype not in (torch.bfloat16, torch.float16, torch.float8_e4m3fn):
         raise ValueError("q: expected a bf16, fp16 or float8_e4m3fn tensor")
+    _check_layouts(layout_q, layout_kv, quant_mode)
+    if attn_mask is not None:
+        raise ValueError("attn_mask: only the built-in causal mask (mask_mode 1) is supported")
+    if p_quant_scale is not None:
+        raise ValueError("p_quant_scale: the weights are cast with a fixed factor 2^8; pass None")
+    fp8_in = q.dtype == torch.float8_e4m3fn
+    if quant_mode is not None and (int(quant_mode) == QUANT_FP8_E4M3_STATIC_CAST_P) != fp8_in:
+        raise ValueError("quant_mode: 5 goes with float8_e4m3fn inputs, 0 with bf16 / fp16")
+    if attention_out_dtype is not None and attention_out_dtype != _out_dtype(q):
+        raise ValueError(f"attention_out_dtype: this input type gives {_out_dtype(q)}")
+    if layout_kv is not None and (layout_kv == "TND") != (cu_seqlens_kv is not None):
+        raise ValueError("layout_kv: 'TND' goes with cu_seqlens_kv, 'PA_BBND' with block_table")
     q = _need(q, "q", q.dtype, 3)
     scales = tuple(1.0 if s is None else float(s)
                    for s in (q_dequant_scale, k_dequant_scale, v_dequant_scale))

@@ -204,3 +204,41 @@ def test_binding_rejects_other_element_types():
     with pytest.raises(ValueError, match="bf16, fp16 or float8_e4m3fn"):
         gbsa.forward(q, q, q, z, z, [w.block_x, 128], metadata=z, cu_seqlens_q=z, seqused_kv=z,
                      block_table=z)
+
+
+@pytest.mark.parametrize("kw,match", [
+    (dict(layout_q="BSND"), "layout_q"),
+    (dict(layout_kv="BNSD"), "layout_kv"),
+    (dict(quant_mode=1), "quant_mode"),
+    (dict(quant_mode=5), "quant_mode"),            # bf16 inputs with the E4M3 mode
+    (dict(attn_mask=1), "attn_mask"),
+    (dict(p_quant_scale=1.0), "p_quant_scale"),
+    (dict(attention_out_dtype="float16"), "attention_out_dtype"),
+    (dict(layout_kv="TND"), "layout_kv"),          # TND without cu_seqlens_kv
+])
+def test_article_arguments_are_checked_before_launch(kw, match):
+    # the remaining arguments of the article's PyTorch API: accepted where the
+    # library implements them, rejected (before any device use) otherwise
+    import torch
+    w = workload("tiny")
+    q = torch.zeros((w.T, w.N1, w.D), dtype=torch.bfloat16)
+    z = torch.zeros(1, dtype=torch.int32)
+    with pytest.raises(ValueError, match=match):
+        gbsa.forward(q, q, q, z, z, [w.block_x, 128], metadata=z, cu_seqlens_q=z, seqused_kv=z,
+                     block_table=z, **kw)
+
+
+def test_article_arguments_accepted_forms_reach_the_device_checks():
+    # consistent values pass the argument checks (and stop only at the
+    # device check on a host without CUDA tensors)
+    import torch
+    w = workload("tiny")
+    z = torch.zeros(1, dtype=torch.int32)
+    for dt, qm, od in ((torch.bfloat16, 0, torch.bfloat16), (torch.float8_e4m3fn, 5, torch.bfloat16)):
+        q = torch.zeros((w.T, w.N1, w.D), dtype=dt)
+        with pytest.raises(ValueError, match="CUDA"):
+            gbsa.forward(q, q, q, z, z, [w.block_x, 128], metadata=z, cu_seqlens_q=z,
+                         seqused_kv=z, block_table=z, layout_q="TND", layout_kv="PA_BBND",
+                         quant_mode=qm, attention_out_dtype=od, dst_type_max=0.0)
+    with pytest.raises(ValueError, match="layout"):
+        gbsa.metadata(z, z, 8, 2, 128, [64, 128], cu_seqlens_q=z, seqused_kv=z, layout_q="BSH")
