@@ -11,8 +11,9 @@ import pytest
 import torch
 
 import oracle
-from block_sparse_paged_gbsa_b200.workloads import bf16_bits, generate, make_values
-from tests.helpers import brute_force, logical_kv, oracle_all, oracle_rows
+from block_sparse_paged_gbsa_b200.workloads import (bf16_bits, generate, make_values, tnd_kv,
+                                                    workload)
+from tests.helpers import brute_force, logical_kv, oracle_all, oracle_rows, to_f64
 from tests.test_oracle_pins import GOLDEN, _fixture_workload
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "gbsa_oracle.c")
@@ -35,6 +36,13 @@ MUTANTS = {
                           "const int64_t qu = qs;"),
     "count_not_clamped": ("if (n > c->top_k) n = c->top_k;", "if (n > c->top_k + 1) n = c->top_k + 1;"),
     "causal_strict": ("if (p > pos) continue;", "if (p >= pos) continue;"),
+    # the fp16 decoder, the TND addressing and the E4M3 error scale
+    "fp16_subnormal_scale": ("mag = ldexp((double)f, -24);", "mag = ldexp((double)f, -25);"),
+    "fp16_exponent_bias": ("mag = ldexp((double)(1024 + f), e - 25);",
+                           "mag = ldexp((double)(1024 + f), e - 24);"),
+    "tnd_without_sequence_base": ("key_page[nk] = c->cu_seqlens_kv[b] + p;", "key_page[nk] = p;"),
+    "out_abs_signed": ("out_abs[d] += w * fabs(c->widen(vrow[d]));",
+                       "out_abs[d] += w * c->widen(vrow[d]);"),
 }
 
 
@@ -95,8 +103,60 @@ def _sdpa_ok(lib):
     return np.allclose(out, ref.transpose(0, 1).numpy(), atol=1e-10, rtol=0)
 
 
+def _widen_ok(lib):
+    # both decoders against numpy's on every 16-bit pattern
+    bits = np.arange(65536, dtype=np.uint16)
+    for dt in ("bf16", "fp16"):
+        with np.errstate(invalid="ignore"):  # the NaN patterns
+            got, ref = oracle.widen(bits, dt, lib=lib), to_f64(bits, dt)
+        if not ((got == ref) | (np.isnan(got) & np.isnan(ref))).all():
+            return False
+    return True
+
+
+def _rows(lib, w, q, k, v, rows, **kw):
+    args = dict(kv_page_stride=w.kv_page_stride, num_pages=w.num_pages,
+                block_table=w.block_table)
+    args.update(kw)
+    return oracle.attention_rows(
+        q_bits=bf16_bits(q), k_bits=bf16_bits(k), v_bits=bf16_bits(v), sparse_idx=w.sparse_idx,
+        sparse_count=w.sparse_count, cu_seqlens_q=w.cu_seqlens_q, seqused_q=w.seqused_q,
+        seqused_kv=w.kv_used, block_x=w.block_x, scale=w.scale, win_left=w.win_left,
+        win_right=w.win_right, rows=rows, lib=lib, **args)
+
+
+def _all_rows(w):
+    return np.stack([np.arange(w.T).repeat(w.N1), np.tile(np.arange(w.N1), w.T)], 1)
+
+
+def _tnd_ok(lib):
+    # the same logical keys in the TND layout give the paged pool's rows
+    w = generate(name="tw", seed=9, q_storage=[300, 90], q_used=[290, 90], kv_used=[500, 130],
+                 N1=4, N2=2, block_x=64, top_k=4, selection="random_causal", win_left=150,
+                 win_right=0, page_stride_factor=1.25)
+    q, kf, vf = make_values(w, "cpu")
+    kt, vt, cu = tnd_kv(w, kf, vf)
+    rows = _all_rows(w)
+    po, pl = _rows(lib, w, q, kf, vf, rows)
+    to, tl = _rows(lib, w, q, kt, vt, rows, kv_page_stride=0, num_pages=0, block_table=None,
+                   cu_seqlens_kv=cu)
+    return np.array_equal(po, to) and np.array_equal(pl, tl) and np.isfinite(to).all()
+
+
+def _out_abs_ok(lib):
+    # out_abs is the output on |V| (the weights do not see V)
+    w = workload("tiny", scale_down=4)
+    q, kf, vf = make_values(w, "cpu", nan_fill=False)
+    rows = _all_rows(w)
+    oa = np.zeros((rows.shape[0], w.D))
+    _rows(lib, w, q, kf, vf, rows, out_abs=oa)
+    ra, _ = _rows(lib, w, q, kf, vf.abs(), rows)
+    return bool(np.allclose(oa, ra, rtol=1e-14, atol=0) and (oa >= 0).all())
+
+
 def _all_pins_pass(lib):
-    return _golden_ok(lib) and _brute_ok(lib) and _sdpa_ok(lib)
+    return (_golden_ok(lib) and _brute_ok(lib) and _sdpa_ok(lib) and _widen_ok(lib) and
+            _tnd_ok(lib) and _out_abs_ok(lib))
 
 
 def test_unmodified_oracle_passes(tmp_path):
