@@ -67,6 +67,10 @@ def _expected_live(w, qb, kvh):
 def test_work_list_invariants(name):
     w = CASES[name]()
     p, m = _build(w)
+    _check_invariants(w, p, m, name)
+
+
+def _check_invariants(w, p, m, name):
     g = scheduler.geometry(p)
     assert m[0] == scheduler.MAGIC and m[1] == 1
     assert int(m[2]) & 0xFFFFFFFF == scheduler.signature(p)
@@ -112,7 +116,7 @@ def test_work_list_invariants(name):
     # split length rule and capacities
     total = sum(-(-int(item[i, 2]) // 2) * int(item[i, 1]) for i in range(n_items))
     assert (int(m[16]) | (int(m[17]) << 32)) == total
-    assert L == max(8, -(-total // (4 * 148)))
+    assert L == max(8, -(-total // (4 * int(p["num_ctas"]))))
     assert n_units <= g["unit_cap"] and n_slots <= g["slot_cap"] and n_comb <= g["comb_cap"]
     comb = m[g["off_comb"]:g["off_comb"] + 4 * n_comb].reshape(n_comb, 4)
     assert int(comb[:, 3].sum()) == n_slots if n_comb else n_slots == 0
@@ -157,3 +161,35 @@ def test_signature_distinguishes_problems():
     b = scheduler.signature(_problem(w, num_ctas=147))
     c = scheduler.signature(_problem(w, forced=4))
     assert len({a, b, c}) == 3
+
+
+def test_work_list_invariants_on_random_problems():
+    # the same independent checks on random small problems: sequence mixes
+    # with empty and one-token sequences, seqused below storage, GQA groups
+    # 1..8, Q block sizes, list kinds, windows and CTA counts
+    from hypothesis import HealthCheck, given, settings
+    from hypothesis import strategies as st
+
+    @settings(max_examples=30, deadline=None, derandomize=True,
+              suppress_health_check=[HealthCheck.too_slow])
+    @given(st.data())
+    def run(data):
+        B = data.draw(st.integers(1, 3))
+        qs = data.draw(st.lists(st.integers(1, 160), min_size=B, max_size=B))
+        qu = [data.draw(st.integers(0, s)) for s in qs]
+        ku = [data.draw(st.integers(max(1, u), u + 400)) for u in qu]
+        N2 = data.draw(st.sampled_from([1, 2]))
+        G = data.draw(st.sampled_from([1, 2, 3, 5, 8]))
+        bx = data.draw(st.sampled_from([1, 3, 16, 64, 128]))
+        top_k = data.draw(st.integers(1, 6))
+        sel = data.draw(st.sampled_from(["random_causal", "random_any", "all_causal"]))
+        win = data.draw(st.sampled_from([-1, 0, 100]))
+        ctas = data.draw(st.sampled_from([3, 37, 148]))
+        seed = data.draw(st.integers(0, 10_000))
+        w = generate(name="h", seed=seed, q_storage=qs, q_used=qu, kv_used=ku, N1=N2 * G, N2=N2,
+                     block_x=bx, top_k=top_k, selection=sel, win_left=win,
+                     win_right=0 if win >= 0 else -1, has_seqused_q=True)
+        p, m = _build(w, num_ctas=ctas)
+        _check_invariants(w, p, m, "random")
+
+    run()
