@@ -125,6 +125,42 @@ def test_brute_force_matches(case):
     np.testing.assert_allclose(lse[~inf], bl[~inf], atol=1e-12, rtol=0)
 
 
+def test_brute_force_matches_on_random_problems():
+    # the same comparison on random tiny problems: sequence mixes with
+    # unused rows, GQA groups, Q block sizes, list kinds (with duplicates and
+    # masked blocks), both window sides, fp16 values and strided pools
+    from hypothesis import HealthCheck, given, settings
+    from hypothesis import strategies as st
+
+    @settings(max_examples=25, deadline=None, derandomize=True,
+              suppress_health_check=[HealthCheck.too_slow])
+    @given(st.data())
+    def run(data):
+        B = data.draw(st.integers(1, 2))
+        qs = data.draw(st.lists(st.integers(1, 40), min_size=B, max_size=B))
+        qu = [data.draw(st.integers(0, s)) for s in qs]
+        ku = [data.draw(st.integers(max(1, u), u + 300)) for u in qu]
+        N2 = data.draw(st.sampled_from([1, 2]))
+        G = data.draw(st.sampled_from([1, 2, 3]))
+        w = generate(name="hb", seed=data.draw(st.integers(0, 10_000)), q_storage=qs, q_used=qu,
+                     kv_used=ku, N1=N2 * G, N2=N2, block_x=data.draw(st.sampled_from([1, 5, 16])),
+                     top_k=data.draw(st.integers(1, 4)),
+                     selection=data.draw(st.sampled_from(["random_causal", "random_any"])),
+                     win_left=data.draw(st.sampled_from([-1, 0, 60])),
+                     win_right=data.draw(st.sampled_from([-1, 0, 7])), has_seqused_q=True,
+                     page_stride_factor=data.draw(st.sampled_from([1.0, 1.5])))
+        dt = data.draw(st.sampled_from([torch.bfloat16, torch.float16]))
+        q, kf, vf = make_values(w, "cpu", dtype=dt)
+        out, lse = oracle_all(w, q, kf, vf)
+        bo, bl = brute_force(w, q, kf, vf)
+        np.testing.assert_allclose(out, bo, atol=1e-12, rtol=0)
+        inf = np.isneginf(bl)
+        assert np.array_equal(np.isneginf(lse), inf)
+        np.testing.assert_allclose(lse[~inf], bl[~inf], atol=1e-12, rtol=0)
+
+    run()
+
+
 def test_counts_outside_range_and_bad_entries():
     """count > top_k is clamped, count < 0 is empty, entries outside the
     sequence's blocks contribute nothing (brute force applies the same reading)."""
