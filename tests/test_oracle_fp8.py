@@ -5,7 +5,10 @@ through fp16, which holds every one of them exactly; the dequantization
 scales fold into the score scale and the output.  Pinned here: the E4M3
 decode against the format's definition on all 256 patterns, the fp16
 conversion, the scale folding, and the out_abs error scale."""
+import glob
+import json
 import math
+import os
 
 import numpy as np
 import pytest
@@ -14,6 +17,7 @@ import torch
 import oracle
 from block_sparse_paged_gbsa_b200.workloads import PAGE, make_values, workload
 from tests.helpers import oracle_rows, oracle_rows_fp8
+from tests.test_oracle_pins import GOLDEN, _fixture_workload
 
 ALL8 = torch.arange(256, dtype=torch.int32).to(torch.uint8)
 
@@ -167,3 +171,18 @@ def test_r22_bound_holds_for_the_e4m3_reading(name, scale_down):
     if name != "tiny":
         bad = _emulate_e4m3_p(w, q8, k8, v8, scales, rows, threshold=8.0)
         assert not _r22_check(w, ro, ra, bad, fin, vmax)[0]
+
+
+@pytest.mark.parametrize("path", sorted(glob.glob(os.path.join(GOLDEN, "e4m3_*.json"))))
+def test_e4m3_golden_fixture(path):
+    # hand-derived closed forms of E4M3 codes with dequantization scales
+    fx = json.load(open(path))
+    w, q, kf, vf = _fixture_workload(fx)
+    to8 = lambda t: t.float().to(torch.float8_e4m3fn)
+    assert torch.equal(to8(q).float(), q.float())          # the codes are exact in E4M3
+    rows = np.array([[e["t"], e["h"]] for e in fx["expected"]], np.int64)
+    out, lse, _ = oracle_rows_fp8(w, to8(q), to8(kf), to8(vf), tuple(fx["scales"]), rows)
+    for i, e in enumerate(fx["expected"]):
+        assert lse[i] == pytest.approx(e["lse"], abs=1e-12)
+        for d, val in e["out"].items():
+            assert out[i, int(d)] == pytest.approx(val, abs=1e-12)

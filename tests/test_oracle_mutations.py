@@ -48,7 +48,7 @@ MUTANTS = {
 
 def _golden_ok(lib):
     for path in sorted(glob.glob(os.path.join(GOLDEN, "*.json"))):
-        if path.endswith("example_call_shapes.json"):
+        if path.endswith("example_call_shapes.json") or os.path.basename(path).startswith("e4m3_"):
             continue
         fx = json.load(open(path))
         w, q, kf, vf = _fixture_workload(fx)
