@@ -367,3 +367,14 @@ def test_tnd_layout_equals_paged_pool(name):
     to, tl = oracle_all_tnd(w, q, kt, vt, cu)
     assert np.array_equal(po, to) and np.array_equal(pl, tl)
     assert np.isfinite(to).all()
+
+
+def test_thread_count_changes_nothing():
+    # rows are independent: any split of them over threads gives the same bits
+    w = workload("tiny")
+    q, kf, vf = make_values(w, "cpu")
+    rows = np.stack([np.arange(w.T).repeat(w.N1), np.tile(np.arange(w.N1), w.T)], 1)
+    o1, l1 = oracle_rows(w, q, kf, vf, rows, n_threads=1)
+    for n in (2, 7):
+        on, ln = oracle_rows(w, q, kf, vf, rows, n_threads=n)
+        assert np.array_equal(o1, on) and np.array_equal(l1, ln)
