@@ -41,6 +41,14 @@ MUTANTS = {
     "fp16_exponent_bias": ("mag = ldexp((double)(1024 + f), e - 25);",
                            "mag = ldexp((double)(1024 + f), e - 24);"),
     "tnd_without_sequence_base": ("key_page[nk] = c->cu_seqlens_kv[b] + p;", "key_page[nk] = p;"),
+    # a token at the start of a sequence given to an empty sequence that
+    # shares its start (walking back to the first sequence starting there)
+    "empty_sequence_owner": (
+        "  while (lo + 1 < c->B && c->cu_seqlens_q[lo + 1] <= tg) lo++;",
+        "  while (lo > 0 && c->cu_seqlens_q[lo - 1] == c->cu_seqlens_q[lo]) lo--;"),
+    # a Q-block base that counts every sequence as at least one block
+    "empty_sequence_counts_a_block": ("acc += (qs + block_x - 1) / block_x;",
+                                      "acc += qs > 0 ? (qs + block_x - 1) / block_x : 1;"),
     "out_abs_signed": ("out_abs[d] += w * fabs(c->widen(vrow[d]));",
                        "out_abs[d] += w * c->widen(vrow[d]);"),
 }

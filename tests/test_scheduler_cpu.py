@@ -70,11 +70,30 @@ def test_work_list_invariants(name):
     _check_invariants(w, p, m, name)
 
 
+def _expected_status(w):
+    """Status bits the inputs call for: a count outside [0, top_k] (0x04), a
+    listed entry j < clamped count outside the sequence's blocks (0x02)."""
+    bits = 0
+    qb = 0
+    for b in range(w.B):
+        nblk = -(-int(w.kv_used[b]) // PAGE)
+        for _ in range(-(-int(w.q_storage[b]) // w.block_x)):
+            for kvh in range(w.N2):
+                c = int(w.sparse_count[kvh, qb])
+                if c < 0 or c > w.top_k:
+                    bits |= 0x04
+                for j in range(min(max(c, 0), w.top_k)):
+                    if not 0 <= int(w.sparse_idx[kvh, qb, j]) < nblk:
+                        bits |= 0x02
+            qb += 1
+    return bits
+
+
 def _check_invariants(w, p, m, name):
     g = scheduler.geometry(p)
     assert m[0] == scheduler.MAGIC and m[1] == 1
     assert int(m[2]) & 0xFFFFFFFF == scheduler.signature(p)
-    assert m[15] == 0, "valid inputs raise no status bit"
+    assert m[15] == _expected_status(w), "status bits are those the inputs call for"
     n_items, top_k = g["n_items"], w.top_k
     item = m[g["off_item"]:g["off_item"] + 8 * n_items].reshape(n_items, 8)
     lists = m[g["off_list"]:g["off_list"] + top_k * n_items].reshape(n_items, top_k)
@@ -170,14 +189,18 @@ def test_work_list_invariants_on_random_problems():
     from hypothesis import HealthCheck, given, settings
     from hypothesis import strategies as st
 
-    @settings(max_examples=30, deadline=None, derandomize=True,
+    @settings(max_examples=50, deadline=None, derandomize=True,
               suppress_health_check=[HealthCheck.too_slow])
     @given(st.data())
     def run(data):
-        B = data.draw(st.integers(1, 3))
-        qs = data.draw(st.lists(st.integers(1, 160), min_size=B, max_size=B))
+        B = data.draw(st.integers(1, 4))
+        # empty storage sequences (repeated cu_seqlens_q values) and
+        # sequences with seqused_kv = 0; one sequence is non-empty
+        qs = data.draw(st.lists(st.integers(0, 160), min_size=B, max_size=B))
+        if sum(qs) == 0:
+            qs[data.draw(st.integers(0, B - 1))] = data.draw(st.integers(1, 160))
         qu = [data.draw(st.integers(0, s)) for s in qs]
-        ku = [data.draw(st.integers(max(1, u), u + 400)) for u in qu]
+        ku = [data.draw(st.sampled_from([0, u]) | st.integers(0, u + 400)) for u in qu]
         N2 = data.draw(st.sampled_from([1, 2]))
         G = data.draw(st.sampled_from([1, 2, 3, 5, 8]))
         bx = data.draw(st.sampled_from([1, 3, 16, 64, 128]))
