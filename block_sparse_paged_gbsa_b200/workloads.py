@@ -115,13 +115,21 @@ def _choose(rng, pool, k):
 def generate(*, name="custom", seed=0, q_storage, q_used=None, kv_used=None, N1, N2, block_x,
              top_k, selection="random_causal", win_left=-1, win_right=-1, return_lse=True,
              has_seqused_q=None, scale=None, page_stride_factor=1.0, extra_pages=None,
-             count_range=None, pad_fill="garbage", sorted_lists=True) -> Workload:
+             count_range=None, pad_fill="garbage", list_order="ascending") -> Workload:
     """Draws the structure of one workload (no bf16 values; see ``make_values``).
 
     selection: "random_causal" | "all_causal" | "sink_diag_random" | "decode" | "random_any".
     count_range: (lo, hi) bounds of the count draw where the selection uses one.
+    list_order: order of each selection list -- "ascending" (the named
+    workloads), "descending" (the diagonal / last block first) or "shuffled"
+    (a random permutation); "drawn" keeps the order of the draw.
     """
+    if list_order not in ("ascending", "descending", "shuffled", "drawn"):
+        raise ValueError(list_order)
     rng = np.random.Generator(np.random.PCG64(seed))
+    # shuffled lists draw from their own stream: the selections stay those of
+    # the other orders
+    order_rng = np.random.Generator(np.random.PCG64(seed + 31337))
     q_storage = np.asarray(q_storage, np.int64)
     B = int(q_storage.size)
     q_used = q_storage.astype(np.int32) if q_used is None else np.asarray(q_used, np.int32)
@@ -191,8 +199,12 @@ def generate(*, name="custom", seed=0, q_storage, q_used=None, kv_used=None, N1,
                     else:
                         raise ValueError(selection)
                 chosen = np.asarray(chosen, np.int64)
-                if sorted_lists:
+                if list_order == "ascending":
                     chosen = np.sort(chosen)
+                elif list_order == "descending":
+                    chosen = np.sort(chosen)[::-1]
+                elif list_order == "shuffled":
+                    chosen = order_rng.permutation(np.sort(chosen))
                 c = int(chosen.size)
                 cnt[h, qb] = c
                 idx[h, qb, :c] = chosen
@@ -213,24 +225,26 @@ def _lognormal_lengths(rng, n, median, sigma, lo, hi):
     return np.clip(np.round(x), lo, hi).astype(np.int64)
 
 
-def workload(name: str, seed: Optional[int] = None, scale_down: int = 1) -> Workload:
+def workload(name: str, seed: Optional[int] = None, scale_down: int = 1,
+             list_order: str = "ascending") -> Workload:
     """One of the five named workloads.  ``scale_down`` > 1 shrinks sequence
     lengths (and the decode KV range) by that factor for oracle-sized cases
-    that keep the same structure."""
+    that keep the same structure; ``list_order`` as in ``generate``."""
     s = scale_down
+    o = dict(list_order=list_order)
     if name == "tiny":
         seed = 1001 if seed is None else seed
         return generate(name=name, seed=seed, q_storage=[512 // s] * 2, N1=8, N2=2, block_x=64,
-                        top_k=4, selection="random_causal")
+                        top_k=4, selection="random_causal", **o)
     if name == "dense":
         seed = 1002 if seed is None else seed
         n = max(4096 // s, 128)
         return generate(name=name, seed=seed, q_storage=[n] * 4, N1=32, N2=8, block_x=128,
-                        top_k=max(n // 128, 1), selection="all_causal")
+                        top_k=max(n // 128, 1), selection="all_causal", **o)
     if name == "long":
         seed = 1003 if seed is None else seed
         return generate(name=name, seed=seed, q_storage=[max(131072 // s, 256)], N1=32, N2=4,
-                        block_x=128, top_k=64, selection="sink_diag_random")
+                        block_x=128, top_k=64, selection="sink_diag_random", **o)
     if name == "decode":
         seed = 1004 if seed is None else seed
         rng = np.random.Generator(np.random.PCG64(seed + 7919))
@@ -238,7 +252,7 @@ def workload(name: str, seed: Optional[int] = None, scale_down: int = 1) -> Work
         top_k = 256
         return generate(name=name, seed=seed, q_storage=[1] * 64, q_used=[1] * 64, kv_used=kv,
                         N1=64, N2=8, block_x=1, top_k=top_k, selection="decode",
-                        count_range=(max(64 // s, 1), 256), has_seqused_q=False)
+                        count_range=(max(64 // s, 1), 256), has_seqused_q=False, **o)
     if name == "ragged":
         seed = 1005 if seed is None else seed
         rng = np.random.Generator(np.random.PCG64(seed + 7919))
@@ -248,7 +262,7 @@ def workload(name: str, seed: Optional[int] = None, scale_down: int = 1) -> Work
         return generate(name=name, seed=seed, q_storage=qs, q_used=used, kv_used=used, N1=40,
                         N2=8, block_x=64, top_k=128, selection="random_causal",
                         win_left=4096 // s, win_right=0, page_stride_factor=1.25,
-                        has_seqused_q=True)
+                        has_seqused_q=True, **o)
     raise KeyError(name)
 
 
