@@ -11,6 +11,7 @@
 // module creates on every GPU that loads this library and keeps until the
 // process exits.  The caller still passes the inputs, the outputs and the
 // metadata buffer.
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -26,11 +27,49 @@ constexpr int kMaxDevices = 64;
 // Split-KV scratch shared by every call on a device.
 static __device__ __align__(256) uint8_t g_static_scratch[kScratchBytes];
 
+// The address is a property of the context that loaded the module: after
+// cudaDeviceReset the primary context (and the module in it) is created
+// anew, and a caller may make another context of the same device current.
+// So the cache of each device remembers the unique id of the context it was
+// filled in, and the set-up runs again when the current context differs.
+struct Cached {
+  unsigned long long ctx_id;
+  void* ptr;
+};
 std::mutex g_lock;
-void* g_scratch_ptr[kMaxDevices] = {};
+Cached g_cache[kMaxDevices] = {};
 
-// Device address of g_static_scratch on the current device, looked up once
-// per device (the host-side symbol is not a device address).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+template <typename Fn>
+Fn driver_fn(const char* name) {
+  void* ptr = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &ptr, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  return reinterpret_cast<Fn>(ptr);
+}
+
+// Unique id of the context current on this thread (made current by the
+// runtime call before it); 0 if it cannot be read.
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+  static CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx ||
+      get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
+// Device address of g_static_scratch in the current context.  The set-up
+// (cudaGetSymbolAddress, which also loads the module holding the array on
+// first use) runs once per device and context; later calls read the cache.
 gbsa_status scratch_address(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) {
@@ -38,16 +77,21 @@ gbsa_status scratch_address(void** out) {
     return GBSA_ERR_NO_DEVICE;
   }
   if (dev < 0 || dev >= kMaxDevices) return GBSA_ERR_NO_DEVICE;
+  // 0 when no context is current yet (the runtime makes the device's primary
+  // context current in the set-up below)
+  const unsigned long long ctx = current_context_id();
   std::lock_guard<std::mutex> guard(g_lock);
-  if (!g_scratch_ptr[dev]) {
+  Cached& c = g_cache[dev];
+  if (!c.ptr || ctx == 0 || c.ctx_id != ctx) {
     void* ptr = nullptr;
     if (cudaGetSymbolAddress(&ptr, g_static_scratch) != cudaSuccess || !ptr) {
       cudaGetLastError();
+      c = Cached{0, nullptr};
       return GBSA_ERR_CUDA;
     }
-    g_scratch_ptr[dev] = ptr;
+    c = Cached{current_context_id(), ptr};
   }
-  *out = g_scratch_ptr[dev];
+  *out = c.ptr;
   return GBSA_OK;
 }
 

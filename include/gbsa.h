@@ -222,8 +222,15 @@ GBSA_API gbsa_status gbsa_forward(const gbsa_problem* problem, const gbsa_tensor
  *     GBSA_STATIC_SCRATCH_BYTES are rejected with GBSA_ERR_WORKSPACE_TOO_SMALL
  *     before anything is launched (decode-shaped problems fit; prefill-shaped
  *     ones need gbsa_forward() with a caller-provided workspace).
- *   - The first call on a device looks up the array's device address; make
- *     that first call before any stream capture on that device.
+ *   - The array comes into being when the CUDA module holding it is loaded
+ *     in a context.  With lazy module loading (the CUDA default) that is the
+ *     first call of this entry point on a device: that call loads the module,
+ *     which reserves GBSA_STATIC_SCRATCH_BYTES of device memory, and looks up
+ *     the array's device address.  A caller with a fixed memory budget should
+ *     make one call during start-up, before the budget is fixed, and make
+ *     that first call before any stream capture on that device.  The address
+ *     is looked up again when another context of the device is current (for
+ *     instance after cudaDeviceReset), which loads the module there too.
  *   - Every call on a device shares the one array, which keeps the last
  *     call's contents (nothing in it needs to start at zero: every partial the
  *     merge reads is written earlier in the same call).  Calls whose work
