@@ -56,7 +56,7 @@ def load_library(path: str):
     f = lib.gbsa_oracle_attention_rows
     i32, i64, dbl, ptr = ctypes.c_int32, ctypes.c_int64, ctypes.c_double, ctypes.c_void_p
     f.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, i32, i32, i64, dbl, i32, i32, i32,
-                  ptr, ptr, ptr, ptr, ptr, ptr, ptr, ptr, ptr, ptr, ptr, i64, ptr, ptr, ptr, i32]
+                  ptr, ptr, ptr, ptr, ptr, ptr, ptr, ptr, ptr, ptr, ptr, i64, ptr, ptr, ptr, ptr, i32]
     f.restype = ctypes.c_int
     w = lib.gbsa_oracle_widen
     w.argtypes = [i32, ptr, i64, ptr]
@@ -99,7 +99,7 @@ def widen(bits, dtype="bf16", lib=None):
 def attention_rows(*, q_bits, k_bits, v_bits, kv_page_stride, num_pages, sparse_idx, sparse_count,
                    cu_seqlens_q, seqused_q, seqused_kv, block_table, block_x, scale,
                    win_left=-1, win_right=-1, rows, dtype="bf16", cu_seqlens_kv=None,
-                   out_abs=None, n_threads=None, lib=None):
+                   out_abs=None, gap_abs=None, n_threads=None, lib=None):
     """Reference out/lse for selected (token, head) rows.
 
     q_bits:  uint16 [T, N1, D] -- bit patterns of the queries, bf16 or fp16
@@ -111,6 +111,8 @@ def attention_rows(*, q_bits, k_bits, v_bits, kv_page_stride, num_pages, sparse_
              (block_table, num_pages, kv_page_stride unused).
     rows:    int64 [n, 2] -- (global token index, query head).
     out_abs: optional float64 [n, D] array filled with sum_p w_p |v_p[d]|.
+    gap_abs: optional float64 [n, D] array filled with sum_p w_p (m - s_p) |v_p[d]|
+             (m the row's largest score s_p, natural-log units).
     Returns (out [n, D] float64, lse [n] float64).  Rows past seqused_q, or
     with no visible key, give out = 0 and lse = -inf.
     """
@@ -139,15 +141,16 @@ def attention_rows(*, q_bits, k_bits, v_bits, kv_page_stride, num_pages, sparse_
     n = rows.shape[0]
     out = np.zeros((n, D), np.float64)
     lse = np.full((n,), -np.inf, np.float64)
-    if out_abs is not None and (out_abs.shape != (n, D) or out_abs.dtype != np.float64
-                                or not out_abs.flags.c_contiguous):
-        raise ValueError("out_abs: expected a contiguous float64 [n, D] array")
+    for name, a in (("out_abs", out_abs), ("gap_abs", gap_abs)):
+        if a is not None and (a.shape != (n, D) or a.dtype != np.float64
+                              or not a.flags.c_contiguous):
+            raise ValueError(f"{name}: expected a contiguous float64 [n, D] array")
     rc = (lib or _load()).gbsa_oracle_attention_rows(
         B, T, N1, N2, D, block_x, tqb, top_k, max_pages, num_pages, kv_page_stride, float(scale),
         win_left, win_right, DTYPES[dtype], _ptr(q_bits), _ptr(k_bits), _ptr(v_bits), _ptr(sparse_idx),
         _ptr(sparse_count), _ptr(cu), _ptr(squ), _ptr(sku), _ptr(bt), _ptr(cukv), _ptr(rows), n,
         _ptr(out), _ptr(lse), None if out_abs is None else _ptr(out_abs),
-        n_threads or default_threads())
+        None if gap_abs is None else _ptr(gap_abs), n_threads or default_threads())
     if rc != 0:
         raise ValueError(f"oracle rejected the inputs (code {rc})")
     return out, lse

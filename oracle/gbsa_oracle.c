@@ -66,6 +66,7 @@ typedef struct {
   int64_t n_rows;
   double *out, *lse;
   double* out_abs; /* optional: per row and d, sum_p w_p |v_p[d]| (rounding-error scale) */
+  double* gap_abs; /* optional: per row and d, sum_p w_p (m - s_p) |v_p[d]|, m = max_p s_p */
   int64_t* q_block_base; /* [B]: Q blocks of the sequences before b */
   int failed;            /* set to a nonzero code by a worker on bad input */
 } oracle_ctx;
@@ -114,11 +115,14 @@ static int32_t find_sequence(const oracle_ctx* c, int64_t tg) {
 
 /* Computes one (tg, h) row; scratch holds room for top_k*128 keys. */
 static int one_row(const oracle_ctx* c, int64_t tg, int32_t h, double* out, double* lse,
-                   double* out_abs, double* score, int64_t* key_page, int32_t* key_row) {
+                   double* out_abs, double* gap_abs, double* score, int64_t* key_page,
+                   int32_t* key_row) {
   const int32_t D = c->D;
   for (int32_t d = 0; d < D; d++) out[d] = 0.0;
   if (out_abs)
     for (int32_t d = 0; d < D; d++) out_abs[d] = 0.0;
+  if (gap_abs)
+    for (int32_t d = 0; d < D; d++) gap_abs[d] = 0.0;
   *lse = -INFINITY;
   if (tg < 0 || tg >= c->T || h < 0 || h >= c->N1) return 1;
 
@@ -191,6 +195,8 @@ static int one_row(const oracle_ctx* c, int64_t tg, int32_t h, double* out, doub
     for (int32_t d = 0; d < D; d++) out[d] += w * c->widen(vrow[d]);
     if (out_abs)
       for (int32_t d = 0; d < D; d++) out_abs[d] += w * fabs(c->widen(vrow[d]));
+    if (gap_abs)
+      for (int32_t d = 0; d < D; d++) gap_abs[d] += w * (m - score[i]) * fabs(c->widen(vrow[d]));
   }
   *lse = m + log(l);
   return 0;
@@ -213,8 +219,8 @@ static void* run_job(void* arg) {
   } else {
     for (int64_t i = job->begin; i < job->end; i++) {
       const int rc = one_row(c, c->rows[2 * i], (int32_t)c->rows[2 * i + 1], c->out + i * c->D,
-                             c->lse + i, c->out_abs ? c->out_abs + i * c->D : NULL, score,
-                             key_page, key_row);
+                             c->lse + i, c->out_abs ? c->out_abs + i * c->D : NULL,
+                             c->gap_abs ? c->gap_abs + i * c->D : NULL, score, key_page, key_row);
       if (rc) c->failed = rc;
     }
   }
@@ -234,7 +240,10 @@ static void* run_job(void* arg) {
  * with sequence b in rows [cu_seqlens_kv[b], cu_seqlens_kv[b+1]) (block_table,
  * num_pages, max_pages_per_seq and kv_page_stride are then unused).  out_abs
  * (optional, [n_rows][D]) gets sum_p w_p |v_p[d]|, the scale of the error a
- * rounding of the weights can cause.  Returns 0 on success, nonzero if an
+ * rounding of the weights can cause; gap_abs (optional, [n_rows][D]) gets
+ * sum_p w_p (m - s_p) |v_p[d]| with m the row's largest score, the scale of
+ * the error of weights whose exponent is rounded in proportion to its size
+ * (s_p - m, up to a constant).  Returns 0 on success, nonzero if an
  * argument or a device-style value is outside its range.
  */
 int gbsa_oracle_attention_rows(int32_t B, int32_t T, int32_t N1, int32_t N2, int32_t D,
@@ -247,7 +256,8 @@ int gbsa_oracle_attention_rows(int32_t B, int32_t T, int32_t N1, int32_t N2, int
                                const int32_t* seqused_q, const int32_t* seqused_kv,
                                const int32_t* block_table, const int64_t* cu_seqlens_kv,
                                const int64_t* rows, int64_t n_rows,
-                               double* out, double* lse, double* out_abs, int32_t n_threads) {
+                               double* out, double* lse, double* out_abs, double* gap_abs,
+                               int32_t n_threads) {
   if (B < 1 || T < 1 || N2 < 1 || N1 < N2 || N1 % N2 || D < 1 || block_x < 1 || top_k < 1 ||
       total_q_blocks < 1 || n_rows < 0 || (dtype != 0 && dtype != 1))
     return 10;
@@ -271,6 +281,7 @@ int gbsa_oracle_attention_rows(int32_t B, int32_t T, int32_t N1, int32_t N2, int
   c.cu_seqlens_q = cu_seqlens_q; c.seqused_q = seqused_q; c.seqused_kv = seqused_kv;
   c.block_table = block_table; c.cu_seqlens_kv = cu_seqlens_kv; c.rows = rows; c.n_rows = n_rows; c.out = out; c.lse = lse;
   c.out_abs = out_abs;
+  c.gap_abs = gap_abs;
 
   /* Q blocks are counted over storage lengths ("Constraints: block split"). */
   c.q_block_base = (int64_t*)malloc(sizeof(int64_t) * (size_t)B);

@@ -98,16 +98,18 @@ def logical_kv(w: Workload, pool_bits: np.ndarray, b: int, dtype: str = "bf16") 
     return to_f64(np.concatenate(rows, 0)[:ku], dtype)
 
 
-def brute_force(w: Workload, q, kf, vf):
+def brute_force(w: Workload, q, kf, vf, gap=False):
     """A second formulation of the operator: for every (token, head) the
     multiplicity of every logical key position is found by walking the block
     list entry by entry, the masks are applied as a dense boolean vector, and
-    a dense fp64 softmax with those multiplicities as weights gives out/lse."""
+    a dense fp64 softmax with those multiplicities as weights gives out/lse.
+    With gap=True also returns sum_p w_p (max s - s_p) |v_p| per element."""
     dt = elem_dtype(q)
     qb_bits, kb, vb = bf16_bits(q), bf16_bits(kf), bf16_bits(vf)
     qd = to_f64(qb_bits, dt)
     out = np.zeros((w.T, w.N1, w.D))
     lse = np.full((w.T, w.N1), -np.inf)
+    gap_abs = np.zeros((w.T, w.N1, w.D))
     G = w.N1 // w.N2
     qbase = 0
     for b in range(w.B):
@@ -142,8 +144,11 @@ def brute_force(w: Workload, q, kf, vf):
                 e = np.where(wgt > 0, wgt * np.exp(np.where(wgt > 0, s - m, 0.0)), 0.0)
                 out[tg, h] = e @ V[:, kvh, :] / e.sum()
                 lse[tg, h] = m + math.log(e.sum())
+                if gap:
+                    g = np.where(wgt > 0, m - s, 0.0)
+                    gap_abs[tg, h] = (e * g) @ np.abs(V[:, kvh, :]) / e.sum()
         qbase += -(-qs // w.block_x)
-    return out, lse
+    return (out, lse, gap_abs) if gap else (out, lse)
 
 
 def bf16_half_ulp(x: np.ndarray) -> np.ndarray:
@@ -195,3 +200,29 @@ def assert_lse_close(gpu_lse, ref_lse, tol=LSE_TOL):
     if (~inf_r).any():
         worst = float(np.abs(g[~inf_r] - r[~inf_r]).max())
         assert worst <= tol, f"lse: max abs error {worst:.4g} > {tol}"
+
+
+def keys_bound(w, rows):
+    """An upper bound of the visible keys of each row: its clamped count x 128."""
+    qbase = np.concatenate([[0], np.cumsum(-(-np.diff(w.cu_seqlens_q) // w.block_x))])
+    b = np.searchsorted(w.cu_seqlens_q, rows[:, 0], side="right") - 1
+    qb = qbase[b] + (rows[:, 0] - w.cu_seqlens_q[b]) // w.block_x
+    cnt = np.clip(w.sparse_count[rows[:, 1] // w.G, qb], 0, w.top_k)
+    return cnt.astype(np.float64) * PAGE
+
+
+def r24_bound(dtype, ref, out_abs, gap_abs, n_keys, vmax):
+    """The per-element bound of reading R24 (softmaxPrecision 1; derivation in
+    tests/test_gpu_softmax_precision.py): the f16 exponent and exponential
+    against the oracle's out_abs and gap_abs, the weights lost below the f16
+    range, the 16-bit output, fp32 accumulation; bf16 adds the rounding of P
+    to bf16, E4M3 the R22 bound of the weights' E4M3 cast."""
+    d0 = 2.0 ** -9.9 + 8.0 * math.log(2.0) * 2.0 ** -11
+    b = 2.0 * (1.0 + 2.0 ** -8) * (d0 * out_abs + 2.0 ** -11 * gap_abs)
+    b = b + 2.0 * n_keys[:, None] * 2.0 ** -24 * vmax + 2.0 ** -9 * np.abs(ref) + 1e-5 * out_abs
+    if dtype == "bf16":
+        b = b + 2.0 ** -9 * out_abs
+    if dtype == "e4m3":
+        # the weights' E4M3 cast (R22): 2^-4 relative, 2^-10 below 2^-6
+        b = b + 2.0 ** -4 * out_abs + 2.0 ** -18 * n_keys[:, None] * vmax
+    return b

@@ -49,6 +49,10 @@ MUTANTS = {
     # a Q-block base that counts every sequence as at least one block
     "empty_sequence_counts_a_block": ("acc += (qs + block_x - 1) / block_x;",
                                       "acc += qs > 0 ? (qs + block_x - 1) / block_x : 1;"),
+    "gap_abs_signed": ("gap_abs[d] += w * (m - score[i]) * fabs(c->widen(vrow[d]));",
+                       "gap_abs[d] += w * (score[i] - m) * fabs(c->widen(vrow[d]));"),
+    "gap_abs_unweighted": ("gap_abs[d] += w * (m - score[i]) * fabs(c->widen(vrow[d]));",
+                           "gap_abs[d] += (m - score[i]) * fabs(c->widen(vrow[d]));"),
     "out_abs_signed": ("out_abs[d] += w * fabs(c->widen(vrow[d]));",
                        "out_abs[d] += w * c->widen(vrow[d]);"),
 }
@@ -162,9 +166,21 @@ def _out_abs_ok(lib):
     return bool(np.allclose(oa, ra, rtol=1e-14, atol=0) and (oa >= 0).all())
 
 
+def _gap_abs_ok(lib):
+    # gap_abs against the brute force's sum_p w_p (max s - s_p) |v_p|
+    w = generate(name="ga", seed=12, q_storage=[150, 60], N1=4, N2=2, block_x=32, top_k=3,
+                 selection="random_causal", win_left=70, win_right=0)
+    q, kf, vf = make_values(w, "cpu")
+    rows = _all_rows(w)
+    ga = np.zeros((rows.shape[0], w.D))
+    _rows(lib, w, q, kf, vf, rows, gap_abs=ga)
+    _, _, bg = brute_force(w, q, kf, vf, gap=True)
+    return bool(np.allclose(ga, bg.reshape(-1, w.D), atol=1e-10, rtol=0) and (ga >= 0).all())
+
+
 def _all_pins_pass(lib):
     return (_golden_ok(lib) and _brute_ok(lib) and _sdpa_ok(lib) and _widen_ok(lib) and
-            _tnd_ok(lib) and _out_abs_ok(lib))
+            _tnd_ok(lib) and _out_abs_ok(lib) and _gap_abs_ok(lib))
 
 
 def test_unmodified_oracle_passes(tmp_path):

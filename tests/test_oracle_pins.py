@@ -415,3 +415,52 @@ def test_list_order_changes_nothing(name):
         np.testing.assert_allclose(lse[~inf], ref_l[~inf], atol=1e-12, rtol=0)
         bo, bl = brute_force(w, q, kf, vf)
         np.testing.assert_allclose(bo, ref_o, atol=1e-12, rtol=0)
+
+
+def test_gap_abs_matches_brute_force_and_closed_forms():
+    """gap_abs = sum_p w_p (m - s_p) |v_p| (the error scale of weights whose
+    exponent is rounded in proportion to its size): equal to the brute
+    force's, zero when every visible key has the same score (q = 0), and
+    w_1 * 1 * |v_1| for two keys whose scores differ by 1."""
+    w = generate(name="gp", seed=14, q_storage=[200, 90], q_used=[190, 90], kv_used=[260, 90],
+                 N1=6, N2=2, block_x=16, top_k=4, selection="random_causal", win_left=80,
+                 win_right=0)
+    q, kf, vf = make_values(w, "cpu")
+    tt, hh = np.meshgrid(np.arange(w.T), np.arange(w.N1), indexing="ij")
+    rows = np.stack([tt.reshape(-1), hh.reshape(-1)], 1)
+    ga = np.zeros((rows.shape[0], w.D))
+    oracle_rows_gap(w, q, kf, vf, rows, ga)
+    _, _, bg = brute_force(w, q, kf, vf, gap=True)
+    np.testing.assert_allclose(ga, bg.reshape(-1, w.D), atol=1e-12, rtol=0)
+    assert (ga >= 0).all() and ga.max() > 0
+    # q = 0: every score is 0
+    ga0 = np.zeros_like(ga)
+    oracle_rows_gap(w, torch.zeros_like(q), kf, vf, rows, ga0)
+    assert np.abs(ga0).max() == 0.0
+    # two keys, scores 0 and -1 (scale 1, q.k = 0 and -1), v = 3 and -5 in dim 0
+    t = generate(name="two", seed=15, q_storage=[1], q_used=[1], kv_used=[2], N1=1, N2=1,
+                 block_x=1, top_k=1, selection="random_causal", scale=1.0)
+    t.sparse_count[0, 0] = 1
+    t.sparse_idx[0, 0, 0] = 0
+    qq = torch.zeros((1, 1, 128), dtype=torch.bfloat16)
+    qq[0, 0, 0] = 1.0
+    kk = torch.zeros((t.pool_elems,), dtype=torch.bfloat16)
+    vv = torch.zeros((t.pool_elems,), dtype=torch.bfloat16)
+    page = int(t.block_table[0, 0]) * t.kv_page_stride
+    kk[page + 128 * 1 + 0] = -1.0           # key 1 (row 1): q.k = -1
+    vv[page + 0] = 3.0
+    vv[page + 128 * 1 + 0] = -5.0
+    g2 = np.zeros((1, 128))
+    oracle_rows_gap(t, qq, kk, vv, np.array([[0, 0]]), g2)
+    w1 = math.exp(-1.0) / (1.0 + math.exp(-1.0))
+    assert g2[0, 0] == pytest.approx(w1 * 1.0 * 5.0, abs=1e-14)
+    assert np.abs(g2[0, 1:]).max() == 0.0
+
+
+def oracle_rows_gap(w, q, kf, vf, rows, gap_abs):
+    return oracle.attention_rows(
+        q_bits=bf16_bits(q), k_bits=bf16_bits(kf), v_bits=bf16_bits(vf),
+        kv_page_stride=w.kv_page_stride, num_pages=w.num_pages, sparse_idx=w.sparse_idx,
+        sparse_count=w.sparse_count, cu_seqlens_q=w.cu_seqlens_q, seqused_q=w.seqused_q,
+        seqused_kv=w.kv_used, block_table=w.block_table, block_x=w.block_x, scale=w.scale,
+        win_left=w.win_left, win_right=w.win_right, rows=rows, gap_abs=gap_abs)
