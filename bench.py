@@ -1,7 +1,7 @@
 #!/usr/bin/env python
 """Benchmark: block-sparse paged GQA attention forward on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload dense]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload all]
     python bench.py --impl reference ...    # the fp64 CPU oracle arm
 
 One step = the whole hot path over one batch of synthetic input: the
@@ -11,6 +11,12 @@ through the C ABI.  Inputs are resident in HBM before timing; L2 is flushed
 on the launching stream; with N GPUs each rank runs its own seeded batch
 (independent problems, no collective on the data path, weak scaling) and the
 time is the max over ranks.  Prints one JSON line on rank 0.
+
+By default (--workload all) one run times all five workloads: the line's
+headline value, roofline, end-to-end figure and CPU baseline are those of the
+largest one, the 131072-token long-context prefill, and ``per_config``
+carries the same step, forward and roofline figures, with the clocks sampled
+during each, for the other four.  --workload NAME times one workload alone.
 
 Metric: effective TFLOPS counted over selected, unmasked (live) blocks, with
 KV-page GB/s and the roofline fraction beside it.  The fp64 oracle is timed
@@ -54,13 +60,19 @@ KERNEL_SOURCES = ["block_sparse_paged_gbsa_b200/csrc/gbsa_fwd.cu",
                   "block_sparse_paged_gbsa_b200/csrc/gbsa_internal.cuh"]
 
 
+HEADLINE = "long"
+ORDER = ["long", "tiny", "dense", "decode", "ragged"]
+
+
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["gbsa", "reference"], default="gbsa")
-    ap.add_argument("--workload", default="dense", choices=sorted(DESCRIPTIONS))
+    ap.add_argument("--workload", default="all", choices=["all"] + sorted(DESCRIPTIONS),
+                    help="all (default): the long-context workload as the headline and the "
+                         "other four in per_config; or one workload")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -68,18 +80,27 @@ def parse_args():
     ap.add_argument("--dtype", default="bf16", choices=["bf16", "fp16", "e4m3"],
                     help="element type of q, k and v (e4m3: the quantised mode with "
                          "per-tensor dequantization scales, bf16 out)")
+    ap.add_argument("--softmax-precision", type=int, default=0, choices=[0, 1],
+                    help="the article's softmaxPrecision (0: fp32 online softmax; 1: "
+                         "half-precision exponentials with fp32 rescale and row sums)")
     ap.add_argument("--scale-down", type=int, default=1,
                     help="shrink the workload's sequence lengths by this factor (same "
                          "structure); for profiler captures that must stay small")
     return ap.parse_args()
 
 
-def describe(args) -> str:
-    d = DESCRIPTIONS[args.workload]
+def headline_name(args) -> str:
+    return HEADLINE if args.workload == "all" else args.workload
+
+
+def describe(name, args) -> str:
+    d = DESCRIPTIONS[name]
     if args.scale_down != 1:
         d += f" -- sequence lengths scaled down {args.scale_down}x (profiling case)"
     if args.dtype != "bf16":
         d += f" -- q, k, v in {args.dtype}"
+    if args.softmax_precision:
+        d += " -- softmaxPrecision 1"
     return d
 
 
@@ -147,10 +168,12 @@ def profiled_traffic(workload: str):
 
 
 class ClockSampler:
-    """nvidia-smi sampling (50 ms) around the timed region."""
+    """nvidia-smi sampling (50 ms) during the run; ``window`` summarises the
+    samples of one timed region."""
     FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
     def __init__(self, index: int):
         self.index = index
@@ -166,12 +189,7 @@ class ClockSampler:
         except OSError:
             self.proc = None
 
-    def stop(self, t0: float, t1: float) -> dict:
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        time.sleep(0.12)
-        self.proc.terminate()
-        self.proc.wait()
+    def _rows(self):
         self.file.flush()
         rows = []
         with open(self.file.name) as f:
@@ -185,17 +203,33 @@ class ClockSampler:
                     rows.append((ts + frac, float(parts[2]), float(parts[3]), parts[6:10]))
                 except ValueError:
                     continue
-        os.unlink(self.file.name)
+        return rows
+
+    def window(self, t0: float, t1: float) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.12)  # the sample after the region
+        rows = self._rows()
         inside = [r for r in rows if t0 - 0.06 <= r[0] <= t1 + 0.06]
         if not inside:
             after = [r for r in rows if r[0] >= t0 - 0.06]
             inside = after[:1]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in inside for i, v in enumerate(r[3]) if v == "Active"})
+        reasons = sorted({self.NAMES[i] for r in inside for i, v in enumerate(r[3])
+                          if v == "Active"})
         sm = [r[1] for r in inside]
         return {"sm_mhz": float(np.median(sm)) if sm else None,
                 "sm_max_mhz": max((r[2] for r in inside), default=None), "reasons": reasons,
                 "samples": len(inside)}
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            self.proc.wait()
+            self.proc = None
+        try:
+            os.unlink(self.file.name)
+        except OSError:
+            pass
 
 
 def rank_seed(base_seed: int, rank: int) -> int:
@@ -280,14 +314,15 @@ def oracle_sample(w, q, kf, vf, target_s: float, seed: int = 0, scales=(1.0, 1.0
 
 def run_reference(args, world, rank):
     """The CPU oracle arm: each step is the oracle over a bounded random
-    sample of rows of the same workload, on the host cores."""
+    sample of rows of the headline workload, on the host cores."""
     if rank != 0:
         return
     from block_sparse_paged_gbsa_b200.workloads import make_values, workload
 
     import torch
 
-    w = workload(args.workload, scale_down=args.scale_down)
+    name = headline_name(args)
+    w = workload(name, scale_down=args.scale_down)
     tdt = {"bf16": torch.bfloat16, "fp16": torch.float16, "e4m3": torch.float8_e4m3fn}[args.dtype]
     q, kf, vf = make_values(w, "cpu", dtype=tdt)  # the inputs of the GPU arm's --dtype
     per_step = max(0.5, min(5.0, 150.0 / max(1, args.steps + args.warmup)))
@@ -305,7 +340,7 @@ def run_reference(args, world, rank):
         "ms_per_step": round(1e3 * float(np.mean([v[1] for v in vals])), 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": describe(args), "sample": sample},
+        "config": {"workload": describe(name, args), "sample": sample},
         "cpu_baseline": {"value": round(tf, 6), "unit": UNIT, "cores": threads,
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(tf, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
@@ -314,34 +349,43 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
-def main():
-    args = parse_args()
-    world, rank, local = dist_info()
-    if args.impl == "reference":
-        run_reference(args, world, rank)
-        return
+def roofline(acc, fwd_ms, peaks, fp8, traffic):
+    """The forward kernel's roofline object: the bound the workload's FLOPs
+    and algorithmic bytes put it at, the achieved rate over the forward's
+    device time, and its fraction of the measured peak."""
+    t_peak = peaks["bf16_tflops"] * (2.0 if fp8 else 1.0)
+    flops, nbytes = acc["flops_block"], acc["bytes"]
+    tensor = flops / (t_peak * 1e12) >= nbytes / (peaks["hbm_gbs"] * 1e9)
+    if tensor:
+        achieved = flops / (fwd_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": round(achieved, 3), "peak": round(t_peak, 3),
+                "unit": "TFLOP/s", "frac": round(achieved / t_peak, 4)}
+    else:
+        achieved = nbytes / (fwd_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 3), "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4)}
+    roof["traffic"] = traffic
+    roof["kernel"] = "gbsa forward (attention + split-KV combine launch)"
+    roof["peak_source"] = peaks["source"] + " (burst)" + (
+        "; E4M3 tensor peak = measured bf16 x 2 (nominal ratio)" if fp8 and tensor else "")
+    return roof
 
+
+def measure(name, args, dev, world, rank, sampler, dist, headline):
+    """Times one workload: warm-up, then args.steps steps with CUDA events;
+    for the headline also the end-to-end pipeline and the CPU baseline."""
     import torch
-    import torch.distributed as dist
 
     import block_sparse_paged_gbsa_b200 as gbsa
     from block_sparse_paged_gbsa_b200.accounting import work
     from block_sparse_paged_gbsa_b200.workloads import make_values, pool_view, workload
 
-    if not torch.cuda.is_available():
-        raise SystemExit("bench.py needs a CUDA device (the CPU oracle arm is --impl reference)")
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=dev)
-
     # each rank: its own seeded batch of the same workload (weak scaling)
-    base = workload(args.workload, scale_down=args.scale_down)
-    w = workload(args.workload, seed=rank_seed(base.seed, rank), scale_down=args.scale_down)
+    base = workload(name, scale_down=args.scale_down)
+    w = workload(name, seed=rank_seed(base.seed, rank), scale_down=args.scale_down)
     tdt = {"bf16": torch.bfloat16, "fp16": torch.float16, "e4m3": torch.float8_e4m3fn}[args.dtype]
     fp8 = args.dtype == "e4m3"
+    sp = args.softmax_precision
     scales = (1.0, 1.0, 1.0)  # E4M3 dequantization scales (the speed does not depend on them)
     acc = work(w, in_bytes=1 if fp8 else 2)
     q, kf, vf = make_values(w, dev, dtype=tdt)
@@ -354,7 +398,7 @@ def main():
     prob = gbsa.gbsa.make_problem(q, k, idx, block_shape, bt, cu, softmax_scale=w.scale,
                                   win_left=w.win_left, win_right=w.win_right,
                                   return_softmax_lse=w.return_lse, has_seqused_q=squ is not None,
-                                  dequant_scales=scales)
+                                  dequant_scales=scales, softmax_precision=sp)
     meta_buf = torch.empty(gbsa.metadata_size(prob) // 4, dtype=torch.int32, device=dev)
     ws = torch.empty(max(gbsa.workspace_size(prob), 16), dtype=torch.uint8, device=dev)
     out = torch.empty(q.shape, dtype=torch.bfloat16 if fp8 else tdt, device=dev)
@@ -377,12 +421,10 @@ def main():
                      return_softmax_lse=w.return_lse, out=out if oo is None else oo,
                      lse=lse if ll is None else ll, workspace=ws, dev_status=status,
                      q_dequant_scale=scales[0], k_dequant_scale=scales[1],
-                     v_dequant_scale=scales[2])
+                     v_dequant_scale=scales[2], softmax_precision=sp)
         if ev is not None:
             ev[2].record()
 
-    sampler = ClockSampler(local)
-    sampler.start()
     for _ in range(max(3, args.warmup)):
         flush.zero_()
         step()
@@ -403,7 +445,7 @@ def main():
     if world > 1:
         dist.barrier()
     t_wall1 = time.time()
-    clocks = sampler.stop(t_wall0, t_wall1)
+    clocks = sampler.window(t_wall0, t_wall1)
     step_ms = float(np.mean([e[0].elapsed_time(e[2]) for e in events]))
     meta_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in events]))
     fwd_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in events]))
@@ -420,13 +462,13 @@ def main():
     # throughput, device time from the first upload to the last download over
     # the timed steps.
     e2e = None
-    if not args.no_e2e:
-        host = {name: t.cpu().pin_memory() for name, t in
+    if headline and not args.no_e2e:
+        host = {name_: t.cpu().pin_memory() for name_, t in
                 dict(q=q, kf=kf, vf=vf, idx=idx, cnt=cnt, cu=cu, sku=sku, bt=bt).items()}
         if squ is not None:
             host["squ"] = squ.cpu().pin_memory()
         nbuf = 2
-        dev_in = [{name: torch.empty_like(t, device=dev) for name, t in host.items()}
+        dev_in = [{name_: torch.empty_like(t, device=dev) for name_, t in host.items()}
                   for _ in range(nbuf)]
         dev_out = [(torch.empty_like(out), torch.empty_like(lse)) for _ in range(nbuf)]
         host_out = [(torch.empty(out.shape, dtype=out.dtype).pin_memory(),
@@ -447,8 +489,8 @@ def main():
                         s_in.wait_event(ev_cmp[b])  # step i-2 no longer reads these inputs
                     if i == 0 and t0 is not None:
                         t0.record(s_in)
-                    for name, t in host.items():
-                        di[name].copy_(t, non_blocking=True)
+                    for name_, t in host.items():
+                        di[name_].copy_(t, non_blocking=True)
                     ev_in[b].record(s_in)
                 with torch.cuda.stream(s_cmp):
                     s_cmp.wait_event(ev_in[b])
@@ -480,56 +522,94 @@ def main():
                "ms_per_step": round(e2e_ms, 4),
                "pipelined": "two buffer sets; upload, compute and download of successive "
                             "steps overlap on three streams"}
+        del host, dev_in, dev_out, host_out
 
     peaks = load_peaks()
-    # the tensor peak of the operand type: fp16 runs at the bf16 rate, E4M3 at
-    # twice it (the nominal dense ratio, 4.5 / 2.25 PFLOP/s)
+    traffic = (profiled_traffic(name)
+               if args.scale_down == 1 and args.dtype == "bf16" and sp == 0 else None)
+    roof = roofline(acc, fwd_ms, peaks, fp8, traffic)
     t_peak = peaks["bf16_tflops"] * (2.0 if fp8 else 1.0)
     flops, nbytes = acc["flops_block"], acc["bytes"]
-    value = job_value(total_flops, step_ms)
     t_roof = max(flops / (t_peak * 1e12), nbytes / (peaks["hbm_gbs"] * 1e9))
-    bound = "tensor" if flops / (t_peak * 1e12) >= nbytes / (peaks["hbm_gbs"] * 1e9) else "hbm"
-    if bound == "tensor":
-        achieved = flops / (fwd_ms * 1e-3) / 1e12
-        roof = {"bound": "tensor", "achieved": round(achieved, 3), "peak": round(t_peak, 3),
-                "unit": "TFLOP/s", "frac": round(achieved / t_peak, 4)}
-    else:
-        achieved = nbytes / (fwd_ms * 1e-3) / 1e9
-        roof = {"bound": "hbm", "achieved": round(achieved, 3), "peak": peaks["hbm_gbs"],
-                "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4)}
-    roof["traffic"] = (profiled_traffic(args.workload)
-                       if args.scale_down == 1 and args.dtype == "bf16" else None)
-    roof["kernel"] = "gbsa forward (attention + split-KV combine launch)"
-    roof["peak_source"] = peaks["source"] + " (burst)" + (
-        "; E4M3 tensor peak = measured bf16 x 2 (nominal ratio)" if fp8 and bound == "tensor" else "")
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if headline and rank == 0 and world == 1 and not args.no_cpu_baseline:
         qc, kc, vc = q.cpu(), kf.cpu(), vf.cpu()
         tf, dt, n, threads = oracle_sample(w, qc, kc, vc, args.cpu_seconds, scales=scales)
         cpu = {"value": round(tf, 8), "unit": UNIT, "cores": threads, "kind": "oracle",
                "sample": f"{n} random (token, head) rows of the same workload, {dt:.1f} s"}
 
+    res = {
+        "workload": describe(name, args),
+        "value": round(job_value(total_flops, step_ms), 4), "unit": UNIT,
+        "ms_per_step": round(step_ms, 4), "metadata_ms": round(meta_ms, 4),
+        "forward_ms": round(fwd_ms, 4),
+        "kv_gbs": round(total_kv / (step_ms * 1e-3) / 1e9, 2),
+        "roofline": roof,
+        "roofline_step": {"time_ms": round(t_roof * 1e3, 5),
+                          "frac": round(t_roof * 1e3 / step_ms, 4),
+                          "flops": flops, "bytes": nbytes},
+        "flops_exact": acc["flops_exact"],
+        "clocks": clocks, "gpu_launches": launches_per_step * args.steps,
+        "num_ctas": int(meta_host[7]), "dev_status": dev_bits,
+    }
+    del q, kf, vf, k, v, out, lse, ws, meta_buf, flush
+    torch.cuda.empty_cache()
+    return res, e2e, cpu
+
+
+def main():
+    args = parse_args()
+    world, rank, local = dist_info()
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the CPU oracle arm is --impl reference)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    names = ORDER if args.workload == "all" else [args.workload]
+    head = headline_name(args)
+    sampler = ClockSampler(local)
+    sampler.start()
+    results = {}
+    try:
+        for name in names:
+            results[name] = measure(name, args, dev, world, rank, sampler, dist,
+                                    headline=name == head)
+    finally:
+        sampler.stop()
+
     if rank == 0:
+        res, e2e, cpu = results[head]
         line = {
-            "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world,
-            "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": round(step_ms, 4),
+            "metric": METRIC, "value": res["value"], "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": max(3, args.warmup),
+            "ms_per_step": res["ms_per_step"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": args.dtype, "data": "synthetic",
-            "config": {"workload": describe(args),
+            "config": {"workload": res["workload"],
                        "parallelism": f"dp{world} (independent batches, no collective)",
                        "l2": "flushed between timed steps (256 MiB write)",
-                       "num_ctas": int(meta_host[7])},
-            "kv_gbs": round(total_kv / (step_ms * 1e-3) / 1e9, 2),
-            "roofline_step": {"time_ms": round(t_roof * 1e3, 5),
-                              "frac": round(t_roof * 1e3 / step_ms, 4),
-                              "flops": flops, "bytes": nbytes},
-            "flops_exact": acc["flops_exact"],
-            "metadata_ms": round(meta_ms, 4), "forward_ms": round(fwd_ms, 4),
-            "roofline": roof, "clocks": clocks, "e2e": e2e, "cpu_baseline": cpu,
-            "gpu_launches": launches_per_step * args.steps,
-            "dev_status": dev_bits,
+                       "num_ctas": res["num_ctas"]},
+            "kv_gbs": res["kv_gbs"], "roofline_step": res["roofline_step"],
+            "flops_exact": res["flops_exact"],
+            "metadata_ms": res["metadata_ms"], "forward_ms": res["forward_ms"],
+            "roofline": res["roofline"], "clocks": res["clocks"], "e2e": e2e,
+            "cpu_baseline": cpu, "gpu_launches": res["gpu_launches"],
+            "dev_status": res["dev_status"],
         }
+        if len(names) > 1:
+            line["per_config"] = {n: results[n][0] for n in names if n != head}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

@@ -29,7 +29,8 @@ cudaError_t launch_forward(const CUtensorMap& map_q, const CUtensorMap& map_k,
                            int32_t num_pages, int32_t tile_tokens, int32_t rows_per_unit,
                            int32_t win_left, int32_t return_lse, float scale_log2,
                            int32_t num_ctas, int64_t comb_cap, bool one_tile_blocks,
-                           int32_t dtype, float out_scale, cudaStream_t stream);
+                           int32_t dtype, bool half_softmax, float out_scale,
+                           uint64_t wait_limit_ns, cudaStream_t stream);
 }  // namespace gbsa
 
 using namespace gbsa;
@@ -37,6 +38,9 @@ using namespace gbsa;
 namespace {
 
 int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Bound of a pipeline wait in the forward kernel unless the problem sets one.
+constexpr uint64_t kDefaultWaitLimitNs = 1000000000ull;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -73,10 +77,11 @@ gbsa_status validate(const gbsa_problem* p, bool metadata_mode) {
     if (folded > 1e30 || folded < 1e-30 || p->v_scale > 1e30 || p->v_scale < 1e-30)
       return GBSA_ERR_INVALID_ARG;
   }
-  // softmaxPrecision 1 (half-precision softmax, fp32 rescale) is run with the
-  // fp32 softmax of mode 0: its error is below mode 1's for every element type
+  // softmaxPrecision: 0 = fp32 online softmax, 1 = half-precision
+  // exponentials with the fp32 rescale and fp32 row sums
   if (p->softmax_precision != 0 && p->softmax_precision != 1) return GBSA_ERR_INVALID_ARG;
   if (!(p->scale >= 0.0) || isinf(p->scale)) return GBSA_ERR_INVALID_ARG;
+  if (p->wait_limit_ns < 0) return GBSA_ERR_INVALID_ARG;
   if ((int64_t)p->N2 * p->total_q_blocks > 0x7fffffffLL / (p->top_k + 8)) return GBSA_ERR_SHAPE;
   if (p->kv_layout != GBSA_KV_PAGED && p->kv_layout != GBSA_KV_TND) return GBSA_ERR_INVALID_ARG;
   if (!metadata_mode && p->kv_layout == GBSA_KV_TND) {
@@ -286,6 +291,7 @@ gbsa_status gbsa_metadata(const gbsa_problem* problem, const gbsa_tensors* t, vo
   p.seqused_kv = t->seqused_kv;
   p.meta = static_cast<int32_t*>(meta);
   p.dev_status = dev_status;
+  NvtxRange range("gbsa_metadata");
   if (launch_metadata(p, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
     cudaGetLastError();
     return GBSA_ERR_CUDA;
@@ -349,7 +355,9 @@ gbsa_status gbsa_forward(const gbsa_problem* problem, const gbsa_tensors* t, con
       problem_signature(problem, ctas), problem->N1, problem->N2, problem->T, problem->top_k,
       problem->max_pages_per_seq, problem->num_pages, g.tile_tokens, g.rows_per_unit,
       problem->win_left, problem->return_lse, (float)(scale * 1.4426950408889634), ctas,
-      g.comb_cap, g.tiles_max == 1, problem->dtype, fp8 ? (float)problem->v_scale : 1.f,
+      g.comb_cap, g.tiles_max == 1, problem->dtype, problem->softmax_precision == 1,
+      fp8 ? (float)problem->v_scale : 1.f,
+      problem->wait_limit_ns > 0 ? (uint64_t)problem->wait_limit_ns : kDefaultWaitLimitNs,
       static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) {
     cudaGetLastError();

@@ -24,8 +24,9 @@
 // per-tensor dequantization scales folded into the score scale and 1 / l).
 // Units come from the metadata work list, longest first; the CTAs take them
 // wave by wave, in reverse CTA order on odd waves (unit_of).  Every wait is
-// bounded: after ~1 s the kernel sets GBSA_DEV_TIMEOUT, drains its own copies
-// and MMAs, frees TMEM and returns.
+// bounded (by FwdParams::wait_limit_ns, 1 s unless the caller sets another):
+// after it the kernel sets GBSA_DEV_TIMEOUT, drains its own copies and MMAs
+// (each drain bounded by 1 s), frees TMEM and returns.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -67,6 +68,8 @@ constexpr int kHalfBytes = 16384;
 constexpr int kSmemQ = 0;
 constexpr int kSmemRing = 2 * kTileBytes;
 constexpr int kSmemBars = kSmemRing + kStages * kTileBytes;
+// Bound of the final drains (the copies and MMAs a CTA issued must land
+// before it exits); the pipeline waits use FwdParams::wait_limit_ns.
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
 // A unit whose item has a single tile (decode: one token x G heads) and at
 // least this many blocks runs in halves: both tile slots work on its even /
@@ -117,6 +120,10 @@ constexpr uint32_t idesc_pv() {
 template <int kDt>
 constexpr float rescale_threshold() { return kDt == kDtE4m3 ? 0.5f : 8.0f; }
 
+// A score held as a float, or as the raw 32-bit word a TMEM load gives.
+__device__ __forceinline__ float as_float(float x) { return x; }
+__device__ __forceinline__ float as_float(uint32_t x) { return __uint_as_float(x); }
+
 struct FwdParams {
   const int32_t* meta;
   const int32_t* block_table;  // paged K/V
@@ -131,6 +138,7 @@ struct FwdParams {
   int32_t win_left, return_lse;
   float scale_log2;  // softmax scale (E4M3: times q_scale * k_scale) x log2(e)
   float out_scale;   // E4M3: v_scale
+  uint64_t wait_limit_ns;  // bound of every pipeline wait
 };
 
 struct Bars {
@@ -143,6 +151,7 @@ struct Bars {
   uint64_t stats_full[2];  // row max / sum of a unit in `stats` (128 softmax threads)
   uint64_t stats_free[2];  // epilogue has read them (128 epilogue threads)
   uint64_t drain;
+  uint64_t wait_limit_ns;  // FwdParams::wait_limit_ns, read on the slow path of a wait
   uint32_t tmem_base;
   int32_t abort;
   float2 stats[2][128];    // (reference max in log2 units, row sum) per tile row
@@ -193,16 +202,21 @@ __device__ __forceinline__ Unit load_unit(const int32_t* meta, int64_t off_unit,
 }
 
 // Bounded wait on an mbarrier phase.  Returns false (and raises the CTA's
-// abort flag) after kWaitLimitNs, or at once if another role aborted.
+// abort flag) after the pipeline wait limit, or at once if another role
+// aborted.  Every probe suspends the thread at most kProbeHintNs, so the
+// limit holds to within about 10 us whatever the hardware's own suspend
+// window is.
+constexpr uint32_t kProbeHintNs = 1000;
+
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Bars* bars) {
-  if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_try_wait_hint(bar, parity, kProbeHintNs)) return true;
   const uint64_t t0 = global_timer_ns();
   for (;;) {
 #pragma unroll 1
-    for (int i = 0; i < 32; i++)
-      if (mbar_try_wait(bar, parity)) return true;
+    for (int i = 0; i < 8; i++)
+      if (mbar_try_wait_hint(bar, parity, kProbeHintNs)) return true;
     if (*reinterpret_cast<volatile int32_t*>(&bars->abort)) return false;
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
+    if (global_timer_ns() - t0 > bars->wait_limit_ns) {
       atomicExch(&bars->abort, 1);
       return false;
     }
@@ -689,6 +703,36 @@ __device__ void run_mma(const FwdParams& p, uint8_t* smem, Bars* bars, uint32_t 
 // S, P and O are padding rows that no output reads (their P is zero).  The
 // other three warps of the warpgroup only keep the barrier counts.
 // ---------------------------------------------------------------------------
+// softmaxPrecision 1 (GBSA article, "Softmax precision": the softmax in half
+// precision, the rescale in fp32): 32 scores s (fp32) of one row to their
+// weights P = 2^(s * scale_log2 - m).  The exponent x is formed in fp32 (one
+// f32x2 FMA per pair), rounded to an f16 pair, and one ex2.approx.f16x2 gives
+// both weights in f16 -- half the MUFU operations of the fp32 path.  The f16
+// weights are P itself for fp16 (ph), are rounded to bf16 for bf16 and cast
+// to E4M3 for E4M3 (pk); the row sum adds the f16 weights widened exactly to
+// fp32 (sp2, two lanes), so it sums the weights the P.V product uses.  The
+// running max and the O rescale stay fp32.
+template <int kDt, typename S>
+__device__ __forceinline__ void exp2_half_chunk(const S (&sv)[32], uint64_t sc2, uint64_t nm2,
+                                                uint32_t (&ph)[16],
+                                                uint32_t (&pk)[kDt == kDtE4m3 ? 8 : 16],
+                                                uint64_t& sp2) {
+#pragma unroll
+  for (int i = 0; i < 16; i++) {
+    float x0, x1;
+    f2_unpack(f2_fma(f2_pack(as_float(sv[2 * i]), as_float(sv[2 * i + 1])), sc2, nm2), x0, x1);
+    ph[i] = exp2_f16x2(pack_f16x2(x0, x1));
+    float e0, e1;
+    f16x2_to_f32(ph[i], e0, e1);
+    sp2 = f2_add(sp2, f2_pack(e0, e1));
+    if constexpr (kDt == kDtBf16) pk[i] = pack_bf16x2(e0, e1);
+    if constexpr (kDt == kDtFp16) pk[i] = ph[i];
+    if constexpr (kDt == kDtE4m3) {
+      if (i & 1) pk[i >> 1] = pack_e4m3x4_f16(ph[i - 1], ph[i]);
+    }
+  }
+}
+
 constexpr int kNarrowRows = 8;
 constexpr int kNarrowSStride = 148;  // floats per S row (spreads banks for both access patterns)
 constexpr int kNarrowSSeg = 36;      // floats between the 32-key segments of a row
@@ -702,7 +746,7 @@ static_assert(3 * kNarrowSSeg + 32 <= kNarrowSStride, "the segments fit a row");
 // One block of a narrow tile, run by the warpgroup's first warp.  m and l
 // are this lane's row statistics (m the same in the row's 4 lanes, l the
 // lane's partial sum).  ri, key_lo and key_hi describe row lane / 4.
-template <int kDt>
+template <int kDt, bool kHalfSm>
 __device__ __forceinline__ void softmax_narrow_block(const FwdParams& p, uint32_t t_s, uint32_t t_o,
                                                      float* scr_s, uint32_t* scr_p, int32_t entry,
                                                      const RowInfo& ri, int32_t key_lo,
@@ -774,27 +818,37 @@ __device__ __forceinline__ void softmax_narrow_block(const FwdParams& p, uint32_
     m = m_new;
   }
   const float neg_m = ((m == -INFINITY) ? 0.f : -m) + (kDt == kDtE4m3 ? 8.f : 0.f);
-  float pf[32];
-  float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-  for (int c = 0; c < 32; c += 2) {
-    pf[c] = fast_exp2(fmaf(sv[c], p.scale_log2, neg_m));
-    pf[c + 1] = fast_exp2(fmaf(sv[c + 1], p.scale_log2, neg_m));
-    s0 += pf[c];
-    s1 += pf[c + 1];
-  }
-  l += s0 + s1;
   // the lane's 32 keys of P into the row's P line
   constexpr int kPw = kDt == kDtE4m3 ? 8 : 16;  // words per 32 keys
   {
     uint32_t pk[kPw];
-    if constexpr (kDt == kDtE4m3) {
-#pragma unroll
-      for (int i = 0; i < 8; i++)
-        pk[i] = pack_e4m3x4(pf[4 * i], pf[4 * i + 1], pf[4 * i + 2], pf[4 * i + 3]);
+    if constexpr (kHalfSm) {
+      const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2), nm2 = f2_pack(neg_m, neg_m);
+      uint64_t sp2 = 0ull;
+      uint32_t ph[16];
+      exp2_half_chunk<kDt>(sv, sc2, nm2, ph, pk, sp2);
+      float s0, s1;
+      f2_unpack(sp2, s0, s1);
+      l += s0 + s1;
     } else {
+      float pf[32];
+      float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-      for (int i = 0; i < 16; i++) pk[i] = pack_x2<kDt == kDtFp16>(pf[2 * i], pf[2 * i + 1]);
+      for (int c = 0; c < 32; c += 2) {
+        pf[c] = fast_exp2(fmaf(sv[c], p.scale_log2, neg_m));
+        pf[c + 1] = fast_exp2(fmaf(sv[c + 1], p.scale_log2, neg_m));
+        s0 += pf[c];
+        s1 += pf[c + 1];
+      }
+      l += s0 + s1;
+      if constexpr (kDt == kDtE4m3) {
+#pragma unroll
+        for (int i = 0; i < 8; i++)
+          pk[i] = pack_e4m3x4(pf[4 * i], pf[4 * i + 1], pf[4 * i + 2], pf[4 * i + 3]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; i++) pk[i] = pack_x2<kDt == kDtFp16>(pf[2 * i], pf[2 * i + 1]);
+      }
     }
     uint32_t* dst = scr_p + nrow * kNarrowPStride + seg * kPw;
 #pragma unroll
@@ -856,7 +910,7 @@ __device__ __forceinline__ uint8_t* dyn_smem() {
   return dsm;
 }
 
-template <bool kHalves, int kDt>
+template <bool kHalves, int kDt, bool kHalfSm>
 __device__ void run_softmax(const FwdParams& p, Bars* bars, uint32_t tmem, int slot,
                             int32_t n_units, int64_t off_unit, int64_t off_item, int64_t off_list) {
   const int row = threadIdx.x & 127;
@@ -889,8 +943,8 @@ __device__ void run_softmax(const FwdParams& p, Bars* bars, uint32_t tmem, int s
               reinterpret_cast<float*>(dyn_smem() + kSmemQ + kTileBytes + slot * kNarrowSBytes);
           uint32_t* scr_p = reinterpret_cast<uint32_t*>(dyn_smem() + kSmemQ + kTileBytes +
                                                         kHalfBytes + slot * kNarrowPBytes);
-          softmax_narrow_block<kDt>(p, t_s, t_o, scr_s, scr_p, entry, ri, key_lo, key_hi, m, l,
-                                    lane_id());
+          softmax_narrow_block<kDt, kHalfSm>(p, t_s, t_o, scr_s, scr_p, entry, ri, key_lo,
+                                             key_hi, m, l, lane_id());
           tmem_wait_st();
           tc_fence_before_sync();
         }
@@ -957,30 +1011,42 @@ __device__ void run_softmax(const FwdParams& p, Bars* bars, uint32_t tmem, int s
         uint64_t sp2[2] = {0ull, 0ull};
   #pragma unroll
         for (int q = 0; q < 4; q++) {
-          float pf[32];
-  #pragma unroll
-          for (int i = 0; i < 16; i++) {
-            // masked scores are -inf and ex2(-inf) = +0
-            float x0, x1;
-            f2_unpack(f2_fma(f2_pack(__uint_as_float(r[q][2 * i]), __uint_as_float(r[q][2 * i + 1])),
-                             sc2, nm2),
-                      x0, x1);
-            pf[2 * i] = fast_exp2(x0);
-            pf[2 * i + 1] = fast_exp2(x1);
-            sp2[i & 1] = f2_add(sp2[i & 1], f2_pack(pf[2 * i], pf[2 * i + 1]));
-          }
-          if constexpr (kDt == kDtE4m3) {
-            // four E4M3 weights per TMEM column: 32 keys in 8 columns
-            uint32_t pk[8];
-  #pragma unroll
-            for (int i = 0; i < 8; i++)
-              pk[i] = pack_e4m3x4(pf[4 * i], pf[4 * i + 1], pf[4 * i + 2], pf[4 * i + 3]);
-            tmem_st_32x8(t_s + 8 * q, pk);
+          if constexpr (kHalfSm) {
+            uint32_t ph[16];
+            uint32_t pk[kDt == kDtE4m3 ? 8 : 16];
+            exp2_half_chunk<kDt>(r[q], sc2, nm2, ph, pk, sp2[q & 1]);
+            if constexpr (kDt == kDtE4m3)
+              tmem_st_32x8(t_s + 8 * q, pk);
+            else
+              tmem_st_32x16(t_s + 16 * q, pk);
           } else {
-            uint32_t pk[16];
+            float pf[32];
   #pragma unroll
-            for (int i = 0; i < 16; i++) pk[i] = pack_x2<kDt == kDtFp16>(pf[2 * i], pf[2 * i + 1]);
-            tmem_st_32x16(t_s + 16 * q, pk);
+            for (int i = 0; i < 16; i++) {
+              // masked scores are -inf and ex2(-inf) = +0
+              float x0, x1;
+              f2_unpack(f2_fma(f2_pack(__uint_as_float(r[q][2 * i]),
+                                       __uint_as_float(r[q][2 * i + 1])),
+                               sc2, nm2),
+                        x0, x1);
+              pf[2 * i] = fast_exp2(x0);
+              pf[2 * i + 1] = fast_exp2(x1);
+              sp2[i & 1] = f2_add(sp2[i & 1], f2_pack(pf[2 * i], pf[2 * i + 1]));
+            }
+            if constexpr (kDt == kDtE4m3) {
+              // four E4M3 weights per TMEM column: 32 keys in 8 columns
+              uint32_t pk[8];
+  #pragma unroll
+              for (int i = 0; i < 8; i++)
+                pk[i] = pack_e4m3x4(pf[4 * i], pf[4 * i + 1], pf[4 * i + 2], pf[4 * i + 3]);
+              tmem_st_32x8(t_s + 8 * q, pk);
+            } else {
+              uint32_t pk[16];
+  #pragma unroll
+              for (int i = 0; i < 16; i++)
+                pk[i] = pack_x2<kDt == kDtFp16>(pf[2 * i], pf[2 * i + 1]);
+              tmem_st_32x16(t_s + 16 * q, pk);
+            }
           }
         }
         float s0, s1, s2, s3;
@@ -1184,7 +1250,7 @@ __device__ void run_epilogue(const FwdParams& p, Bars* bars, uint32_t tmem, int3
   if (bad && p.dev_status) atomicOr(p.dev_status, bad);
 }
 
-template <bool kHalves, int kDt>
+template <bool kHalves, int kDt, bool kHalfSm>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                const __grid_constant__ CUtensorMap map_v, const FwdParams p) {
@@ -1224,6 +1290,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->kv_empty[i], 1);
     }
     mbar_init(&bars->drain, 1);
+    bars->wait_limit_ns = p.wait_limit_ns;
     bars->abort = 0;
     fence_mbar_init();
   }
@@ -1238,7 +1305,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < 8) {
     setmaxnreg_inc<regs_softmax<kHalves>()>();
-    run_softmax<kHalves, kDt>(p, bars, tmem, warp >> 2, n_units, off_unit, off_item, off_list);
+    run_softmax<kHalves, kDt, kHalfSm>(p, bars, tmem, warp >> 2, n_units, off_unit, off_item,
+                                       off_list);
   } else if (warp < 12) {
     setmaxnreg_dec<kRegsEpilogue>();
     run_epilogue<kHalves, kDt>(p, bars, tmem, n_units, off_unit, off_item);
@@ -1341,13 +1409,17 @@ cudaError_t launch_forward(const CUtensorMap& map_q, const CUtensorMap& map_k,
                            int32_t num_pages, int32_t tile_tokens, int32_t rows_per_unit,
                            int32_t win_left, int32_t return_lse, float scale_log2,
                            int32_t num_ctas, int64_t comb_cap, bool one_tile_blocks,
-                           int32_t dtype, float out_scale, cudaStream_t stream) {
+                           int32_t dtype, bool half_softmax, float out_scale,
+                           uint64_t wait_limit_ns, cudaStream_t stream) {
   using Kernel = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const FwdParams);
-  // [element type][one_tile_blocks]
-  static const Kernel kernels[3][2] = {
-      {fwd_kernel<false, kDtBf16>, fwd_kernel<true, kDtBf16>},
-      {fwd_kernel<false, kDtFp16>, fwd_kernel<true, kDtFp16>},
-      {fwd_kernel<false, kDtE4m3>, fwd_kernel<true, kDtE4m3>}};
+  // [element type][softmax precision][one_tile_blocks]
+  static const Kernel kernels[3][2][2] = {
+      {{fwd_kernel<false, kDtBf16, false>, fwd_kernel<true, kDtBf16, false>},
+       {fwd_kernel<false, kDtBf16, true>, fwd_kernel<true, kDtBf16, true>}},
+      {{fwd_kernel<false, kDtFp16, false>, fwd_kernel<true, kDtFp16, false>},
+       {fwd_kernel<false, kDtFp16, true>, fwd_kernel<true, kDtFp16, true>}},
+      {{fwd_kernel<false, kDtE4m3, false>, fwd_kernel<true, kDtE4m3, false>},
+       {fwd_kernel<false, kDtE4m3, true>, fwd_kernel<true, kDtE4m3, true>}}};
   if (dtype < 0 || dtype > 2) return cudaErrorInvalidValue;
   static int configured_device = -1;
   int dev = 0;
@@ -1356,8 +1428,8 @@ cudaError_t launch_forward(const CUtensorMap& map_q, const CUtensorMap& map_k,
   if (configured_device != dev) {
     // The register re-split is only safe if the kernel launches with exactly
     // the registers the split was computed for.
-    for (int i = 0; i < 6; i++) {
-      const void* fn = reinterpret_cast<const void*>(kernels[i / 2][i % 2]);
+    for (int i = 0; i < 12; i++) {
+      const void* fn = reinterpret_cast<const void*>(kernels[i / 4][(i / 2) % 2][i % 2]);
       cudaFuncAttributes attr;
       e = cudaFuncGetAttributes(&attr, fn);
       if (e != cudaSuccess) return e;
@@ -1390,10 +1462,15 @@ cudaError_t launch_forward(const CUtensorMap& map_q, const CUtensorMap& map_k,
   p.return_lse = return_lse;
   p.scale_log2 = scale_log2;
   p.out_scale = out_scale;
+  p.wait_limit_ns = wait_limit_ns;
   // every Q block in one tile (decode-like): the instantiation with units in
   // halves; the element type picks the MMA kind, P's format and the output type
-  e = launch_dependent(kernels[dtype][one_tile_blocks ? 1 : 0], dim3(num_ctas), dim3(kThreads),
-                       kSmemBytes, stream, map_q, map_k, map_v, p);
+  {
+    NvtxRange range("gbsa_forward");
+    e = launch_dependent(kernels[dtype][half_softmax ? 1 : 0][one_tile_blocks ? 1 : 0],
+                         dim3(num_ctas),
+                         dim3(kThreads), kSmemBytes, stream, map_q, map_k, map_v, p);
+  }
   if (e != cudaSuccess || comb_cap <= 0) return e;
   CombineParams c;
   c.meta = meta;
@@ -1411,6 +1488,7 @@ cudaError_t launch_forward(const CUtensorMap& map_q, const CUtensorMap& map_k,
   c.rows_per_unit = rows_per_unit;
   c.return_lse = return_lse;
   c.fp16 = dtype == kDtFp16 ? 1 : 0;
+  NvtxRange range("gbsa_combine");
   return launch_dependent(combine_kernel, dim3((unsigned)comb_cap), dim3(256), 0, stream, c);
 }
 

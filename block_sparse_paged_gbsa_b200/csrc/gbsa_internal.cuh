@@ -28,8 +28,32 @@
 #ifdef __CUDACC__
 #include <cuda_runtime.h>
 #endif
+#include <nvtx3/nvToolsExt.h>
 
 namespace gbsa {
+
+// An NVTX range in the "gbsa" domain around the host code that enqueues one
+// launch group (metadata, forward, combine), so that a profiler's timeline
+// names them.  Header-only NVTX: without a tool attached it costs a branch.
+class NvtxRange {
+ public:
+  explicit NvtxRange(const char* name) {
+    static const nvtxDomainHandle_t domain = nvtxDomainCreateA("gbsa");
+    domain_ = domain;
+    nvtxEventAttributes_t a = {};
+    a.version = NVTX_VERSION;
+    a.size = NVTX_EVENT_ATTRIB_STRUCT_SIZE;
+    a.messageType = NVTX_MESSAGE_TYPE_ASCII;
+    a.message.ascii = name;
+    nvtxDomainRangePushEx(domain_, &a);
+  }
+  ~NvtxRange() { nvtxDomainRangePop(domain_); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+
+ private:
+  nvtxDomainHandle_t domain_;
+};
 
 constexpr int kPage = 128;        // keys per KV block = page size (blockShapeY)
 constexpr int kHeadDim = 128;     // D

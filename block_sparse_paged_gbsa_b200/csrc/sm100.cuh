@@ -60,6 +60,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// The same probe, suspending the thread at most `hint_ns` nanoseconds while
+// the phase is incomplete (the thread resumes as soon as it completes).
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity,
+                                                   uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // ---------------------------------------------------------------------------
 // TMA (bulk tensor copies global -> shared, completion counted in bytes on
 // an mbarrier).  Coordinates are element indices, innermost first.
@@ -425,6 +440,37 @@ __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Two base-2 exponentials in half precision: the f16 pair `h` (low half
+// first) to 2^h per half, one instruction for both.
+__device__ __forceinline__ uint32_t exp2_f16x2(uint32_t h) {
+  uint32_t r;
+  asm("ex2.approx.f16x2 %0, %1;" : "=r"(r) : "r"(h));
+  return r;
+}
+
+// The two halves of an f16 pair widened to fp32 (exact).
+__device__ __forceinline__ void f16x2_to_f32(uint32_t h, float& lo, float& hi) {
+  asm("{\n\t.reg .b16 l, h;\n\t"
+      "mov.b32 {l, h}, %2;\n\t"
+      "cvt.f32.f16 %0, l;\n\t"
+      "cvt.f32.f16 %1, h;\n\t}"
+      : "=f"(lo), "=f"(hi)
+      : "r"(h));
+}
+
+// Two f16 pairs (four values, a's low half first) to four E4M3 codes, round
+// to nearest even, saturating to +-448; byte k holds value k.
+__device__ __forceinline__ uint32_t pack_e4m3x4_f16(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 lo, hi;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f16x2 lo, %1;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f16x2 hi, %2;\n\t"
+      "mov.b32 %0, {lo, hi};\n\t}"
+      : "=r"(r)
+      : "r"(a), "r"(b));
+  return r;
 }
 
 }  // namespace sm100

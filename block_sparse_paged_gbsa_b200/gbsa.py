@@ -58,7 +58,8 @@ class _Problem(ctypes.Structure):
                 ("max_blocks_per_split", ctypes.c_int32), ("dtype", ctypes.c_int32),
                 ("softmax_precision", ctypes.c_int32), ("kv_layout", ctypes.c_int32),
                 ("T_kv", ctypes.c_int32), ("q_scale", ctypes.c_double),
-                ("k_scale", ctypes.c_double), ("v_scale", ctypes.c_double)]
+                ("k_scale", ctypes.c_double), ("v_scale", ctypes.c_double),
+                ("wait_limit_ns", ctypes.c_int64)]
 
 
 class _Tensors(ctypes.Structure):
@@ -92,12 +93,13 @@ class Problem:
     max_blocks_per_split: int = 0
     block_y: int = 128
     dtype: int = 0              # 0 = bf16, 1 = fp16, 2 = E4M3 (q, k, v; out bf16 for E4M3)
-    softmax_precision: int = 0  # 0 or 1; both run the fp32 online softmax
+    softmax_precision: int = 0  # 0: fp32 softmax; 1: f16 exponentials, fp32 rescale and sums
     kv_layout: int = 0          # 0 = paged pool + block_table, 1 = TND + cu_seqlens_kv
     T_kv: int = 0               # TND: rows of k and v
     q_scale: float = 1.0        # E4M3: per-tensor dequantization scales
     k_scale: float = 1.0
     v_scale: float = 1.0
+    wait_limit_ns: int = 0      # bound of a pipeline wait of the forward kernel; 0 = 1 s
 
     def as_c(self) -> _Problem:
         p = _Problem()
@@ -106,7 +108,7 @@ class Problem:
         return p
 
 
-ABI_VERSION = 4
+ABI_VERSION = 5
 DTYPE_BF16, DTYPE_FP16, DTYPE_FP8_E4M3 = 0, 1, 2
 
 
@@ -229,7 +231,7 @@ def metadata(sparse_block_idx, sparse_block_count, num_heads_q: int, num_heads_k
              seqused_q=None, num_tokens: int = 0, is_packed_gqa: bool = True, mask_mode: int = 1,
              win_left: int = -1, win_right: int = -1, num_ctas: int = 0,
              max_blocks_per_split: int = 0, dev_status=None, out=None,
-             softmax_precision: int = 1, cu_seqlens_kv=None, max_seqlen_q: int = -1,
+             softmax_precision: int = 0, cu_seqlens_kv=None, max_seqlen_q: int = -1,
              max_seqlen_kv: int = -1, layout_q: str = "TND", layout_kv: str = "PA_BBND",
              quant_mode: int = 0):
     """Builds the work list (int32 tensor) on the device of the inputs.
@@ -239,8 +241,8 @@ def metadata(sparse_block_idx, sparse_block_count, num_heads_q: int, num_heads_k
     checked; cu_seqlens_kv and max_seqlen_q / max_seqlen_kv do not enter the
     work list (it depends on seqused_kv and the Q lengths only).
 
-    softmax_precision: the article's softmaxPrecision (default 1, as in its
-    PyTorch API); 0 and 1 are accepted and both run the fp32 softmax.
+    softmax_precision: the article's softmaxPrecision; accepted here so that
+    its calls run unchanged (the work list does not depend on it).
 
     num_tokens: T if known (enables the device check cu_seqlens_q[B] == T); 0 skips it.
     out: optional preallocated int32 buffer of at least metadata_size() bytes.
@@ -286,7 +288,7 @@ def make_problem(q, k, sparse_block_idx, block_shape, block_table, cu_seqlens_q,
                  softmax_scale=0.0, mask_mode=1, win_left=-1, win_right=-1, is_packed_gqa=True,
                  return_softmax_lse=False, has_seqused_q=False, num_ctas=0,
                  max_blocks_per_split=0, dequant_scales=(1.0, 1.0, 1.0),
-                 softmax_precision=1) -> Problem:
+                 softmax_precision=0, wait_limit_ns=0) -> Problem:
     """The gbsa_problem a forward call with these tensors describes.  A 4-d k
     is the page pool (block_table given); a 3-d k is TND [T_kv, N2, D]."""
     T, N1, D = q.shape
@@ -306,7 +308,8 @@ def make_problem(q, k, sparse_block_idx, block_shape, block_table, cu_seqlens_q,
                    has_seqused_q=int(bool(has_seqused_q)), num_ctas=num_ctas,
                    max_blocks_per_split=max_blocks_per_split, dtype=_dtype_code(q),
                    q_scale=float(dequant_scales[0]), k_scale=float(dequant_scales[1]),
-                   v_scale=float(dequant_scales[2]), softmax_precision=int(softmax_precision))
+                   v_scale=float(dequant_scales[2]), softmax_precision=int(softmax_precision),
+                   wait_limit_ns=int(wait_limit_ns))
 
 
 def forward(q, k, v, sparse_block_idx, sparse_block_count, block_shape: Sequence[int], *,
@@ -316,9 +319,9 @@ def forward(q, k, v, sparse_block_idx, sparse_block_count, block_shape: Sequence
             win_right: int = -1, is_packed_gqa: bool = True, return_softmax_lse: bool = False,
             num_ctas: int = 0, max_blocks_per_split: int = 0, out=None, lse=None, workspace=None,
             dev_status=None, q_dequant_scale=None, k_dequant_scale=None, v_dequant_scale=None,
-            softmax_precision: int = 1, attn_mask=None, p_quant_scale=None,
+            softmax_precision: int = 0, attn_mask=None, p_quant_scale=None,
             layout_q: str = "TND", layout_kv=None, quant_mode=None, dst_type_max: float = 0.0,
-            attention_out_dtype=None):
+            attention_out_dtype=None, wait_limit_ns: int = 0):
     """Block-sparse paged GQA attention.  q, k and v share one element type,
     bf16, fp16 or float8_e4m3fn.  K/V come as the page pool [num_pages, 128,
     N2, D] with ``block_table`` (PA_BBND), or, when ``cu_seqlens_kv`` is given,
@@ -328,8 +331,12 @@ def forward(q, k, v, sparse_block_idx, sparse_block_count, block_shape: Sequence
     host floats (default 1.0; ignored for the 16-bit types) and give a bf16
     out.  Returns (out [T,N1,D] in q's type -- bf16 for E4M3 --, lse [T,N1,1]
     fp32, an empty tensor unless return_softmax_lse).  softmax_precision is the
-    article's softmaxPrecision (default 1, as in its PyTorch API); 0 and 1 are
-    accepted and both run the fp32 online softmax.
+    article's softmaxPrecision: 0 (the default here) is the fp32 online
+    softmax; 1 forms the exponentials in half precision (an f16 exponent, one
+    f16x2 exponential per pair of weights) with the running max, the O
+    rescale and the row sums in fp32.  The article's PyTorch API defaults to
+    1; this binding defaults to 0, the more accurate mode and the only one
+    the article allows for bf16 on the hardware it names.
 
     The article's remaining arguments: attn_mask must be None (only the
     built-in causal mask, mask_mode 1, exists); layout_q is 'TND'; layout_kv,
@@ -338,7 +345,11 @@ def forward(q, k, v, sparse_block_idx, sparse_block_count, block_shape: Sequence
     type (0: bf16 / fp16, 5: float8_e4m3fn); p_quant_scale must be None (the
     weights are cast with the fixed factor 2^8); attention_out_dtype, when
     given, must be the type of out (q's, bf16 for E4M3); dst_type_max is not
-    used."""
+    used.
+
+    wait_limit_ns bounds every pipeline wait of the forward kernel (0: 1 s);
+    a wait that runs out sets the TIMEOUT device-status bit and the results
+    are not valid."""
     import torch
     if q is None or q.dtype not in (torch.bfloat16, torch.float16, torch.float8_e4m3fn):
         raise ValueError("q: expected a bf16, fp16 or float8_e4m3fn tensor")
@@ -389,7 +400,7 @@ def forward(q, k, v, sparse_block_idx, sparse_block_count, block_shape: Sequence
                         is_packed_gqa=is_packed_gqa, return_softmax_lse=return_softmax_lse,
                         has_seqused_q=squ is not None, num_ctas=num_ctas,
                         max_blocks_per_split=max_blocks_per_split, dequant_scales=scales,
-                        softmax_precision=softmax_precision)
+                        softmax_precision=softmax_precision, wait_limit_ns=wait_limit_ns)
     T, N1, D = q.shape
     with torch.cuda.device(dev):
         if out is None:

@@ -61,7 +61,7 @@
 extern "C" {
 #endif
 
-#define GBSA_ABI_VERSION 4
+#define GBSA_ABI_VERSION 5
 
 /* Symbols of the C ABI are exported; everything else in libgbsa is hidden. */
 #if defined(__GNUC__)
@@ -91,7 +91,7 @@ typedef enum gbsa_status {
 #define GBSA_DEV_BAD_COUNT 0x04       /* sparse_count outside [0, top_k]; clamped                       */
 #define GBSA_DEV_BAD_PAGE 0x08        /* block_table entry outside [0, num_pages); the page reads as 0  */
 #define GBSA_DEV_META_MISMATCH 0x10   /* metadata built for another problem; forward did nothing         */
-#define GBSA_DEV_TIMEOUT 0x20         /* a pipeline wait gave up (about 1 s); results are not valid       */
+#define GBSA_DEV_TIMEOUT 0x20         /* a pipeline wait gave up (wait_limit_ns); results are not valid   */
 #define GBSA_DEV_CAPACITY 0x40        /* a work-list capacity bound was exceeded; forward did nothing    */
 
 /* Host-known description of one call.  No field is read from the device.
@@ -131,6 +131,10 @@ typedef struct gbsa_problem {
   double q_scale;             /* GBSA_DTYPE_FP8_E4M3: per-tensor dequantization scales, each */
   double k_scale;             /*   finite and > 0 (q = q_scale * code, ...); the other dtypes */
   double v_scale;             /*   ignore them                                                 */
+  int64_t wait_limit_ns;      /* bound of every pipeline wait of the forward kernel, in ns;
+                                 0 = 1 s.  A wait that runs out sets GBSA_DEV_TIMEOUT, and the
+                                 kernel drains the copies and MMAs it issued and returns
+                                 (results invalid).  >= 0; ABI version 5                      */
 } gbsa_problem;
 
 /* K/V layouts (GBSA article, "Constraints: layouts": PA_BBND page pool, or

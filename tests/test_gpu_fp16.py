@@ -80,25 +80,3 @@ def test_fp16_and_bf16_agree_on_values_both_hold():
     assert torch.equal(fin, torch.isfinite(lh))
     assert (lb[fin] - lh[fin]).abs().max().item() < 2e-3
     assert (ob.float() - oh.float()).abs().max().item() < 2e-2
-
-
-def test_softmax_precision_one_runs_the_fp32_softmax():
-    # softmaxPrecision 1 (the article's PyTorch default) is accepted and
-    # computed with the fp32 softmax: bit-identical to mode 0
-    import block_sparse_paged_gbsa_b200 as gbsa
-    from block_sparse_paged_gbsa_b200.workloads import pool_view
-    from tests.gpu_helpers import device_tensors, run_metadata
-    w = workload("tiny")
-    q, kf, vf = _values(w)
-    t = device_tensors(w)
-    res = []
-    for mode in (0, 1):
-        meta = run_metadata(w, t)
-        res.append(gbsa.forward(q, pool_view(w, kf), pool_view(w, vf), t["idx"], t["cnt"],
-                                [w.block_x, 128], metadata=meta, cu_seqlens_q=t["cu"],
-                                seqused_q=t["squ"], seqused_kv=t["sku"], block_table=t["bt"],
-                                softmax_scale=w.scale, return_softmax_lse=True,
-                                softmax_precision=mode))
-    torch.cuda.synchronize()
-    assert torch.equal(res[0][0], res[1][0]) and torch.equal(res[0][1], res[1][1])
-    _check(w, q, kf, vf, res[1][0], res[1][1])
