@@ -965,21 +965,27 @@ __device__ void run_softmax(const FwdParams& p, Bars* bars, uint32_t tmem, int s
         reg_fence(r[1]);
         reg_fence(r[2]);
         reg_fence(r[3]);
-        // visible key columns of this block for this row: [clo, chi]; the
-        // element mask runs only in warps that hold a row needing it
+        // visible key columns of this block for this row: [clo, chi].  A row
+        // whose output is never written (padding rows of a tile, rows past
+        // seqused_q) is left unmasked: its softmax only feeds its own row of
+        // P and O, which no output reads, and it never rescales O (below).
+        // The element mask runs per 32-column chunk, only in warps where some
+        // row needs it there.
         int32_t clo = 0, chi = kPage - 1;
-        if (!ri.used) {
-          clo = kPage;
-          chi = -1;
-        } else if (entry & kEntryMask) {
+        if (ri.used && (entry & kEntryMask)) {
           const int32_t base = (entry & kEntryLbMask) * kPage;
           clo = key_lo == INT32_MIN ? 0 : max(key_lo - base, 0);
           chi = min(key_hi - base, kPage - 1);
         }
         if (__any_sync(0xffffffffu, clo > 0 || chi < kPage - 1)) {
   #pragma unroll
-          for (int c = 0; c < 128; c++)
-            if (c < clo || c > chi) r[c >> 5][c & 31] = __float_as_uint(-INFINITY);
+          for (int q = 0; q < 4; q++) {
+            if (__any_sync(0xffffffffu, clo > 32 * q || chi < 32 * q + 31)) {
+  #pragma unroll
+              for (int c = 0; c < 32; c++)
+                if (32 * q + c < clo || 32 * q + c > chi) r[q][c] = __float_as_uint(-INFINITY);
+            }
+          }
         }
         // row max: eight independent partial maxima, then a tree
         float mp[8];
@@ -993,9 +999,10 @@ __device__ void run_softmax(const FwdParams& p, Bars* bars, uint32_t tmem, int s
                                fmaxf(mp[6], mp[7]));
         const float m_blk = mx * p.scale_log2;
         const float m_new = fmaxf(m, m_blk);
-        // lazy rescale: keep the old reference max unless it grew past the threshold
-        const bool rescale =
-            m_new != -INFINITY && (m == -INFINITY || m_new > m + rescale_threshold<kDt>());
+        // lazy rescale: keep the old reference max unless it grew past the
+        // threshold (rows whose output is never written keep m = -inf)
+        const bool rescale = ri.used && m_new != -INFINITY &&
+                             (m == -INFINITY || m_new > m + rescale_threshold<kDt>());
         const bool fix_o = rescale && m != -INFINITY;
         const float factor = fix_o ? fast_exp2(m - m_new) : 1.f;
         if (rescale) {
