@@ -134,7 +134,9 @@ typedef struct gbsa_problem {
   int64_t wait_limit_ns;      /* bound of every pipeline wait of the forward kernel, in ns;
                                  0 = 1 s.  A wait that runs out sets GBSA_DEV_TIMEOUT, and the
                                  kernel drains the copies and MMAs it issued and returns
-                                 (results invalid).  >= 0; ABI version 5                      */
+                                 (results invalid).  The clock starts after the wait's first
+                                 barrier probe, which the hardware may hold for tens of us:
+                                 a wait gives up no earlier than the bound.  >= 0; ABI 5      */
 } gbsa_problem;
 
 /* K/V layouts (GBSA article, "Constraints: layouts": PA_BBND page pool, or
