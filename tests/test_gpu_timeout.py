@@ -1,7 +1,7 @@
 """Failure detection on the GPU without a fault: every pipeline wait of the
 forward kernel is bounded (gbsa_problem.wait_limit_ns, 1 s by default).  The
-cases have long units (up to 128 blocks on a few CTAs, or decode pieces of
-tens of blocks), so the epilogue waits a unit's whole run for its output,
+cases have long units (up to 128 prefill blocks, or 256 decode blocks, on 8
+CTAs), so the epilogue waits a unit's whole run for its output,
 far longer than the hardware may hold the first barrier probe on its own;
 with a bound of 1 us that wait runs out.  The kernel must set the TIMEOUT
 status
@@ -32,9 +32,9 @@ CASES = {
     # on 8 CTAs (the split length grows with the work per CTA: no splits)
     "causal_16k_8ctas": (lambda: generate(name="to", seed=95, q_storage=[16384], N1=8, N2=2,
                                           block_x=128, top_k=128, selection="all_causal"), 8),
-    # the one-tile instantiation (units in halves, narrow tiles) with split-KV
-    # pieces of tens of blocks and the combine
-    "decode_s4": (lambda: workload("decode", scale_down=4), 0),
+    # the one-tile instantiation (units in halves, narrow tiles): decode
+    # lists of up to 256 blocks on 8 CTAs (no splits)
+    "decode_s2_8ctas": (lambda: workload("decode", scale_down=2), 8),
 }
 
 
