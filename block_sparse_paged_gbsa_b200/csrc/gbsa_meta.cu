@@ -248,15 +248,15 @@ __device__ __forceinline__ PieceShape piece_shape(int32_t U, int32_t n, int32_t 
   PieceShape s;
   s.U = U;
   s.n = n;
-  s.k = s.n <= L ? 1 : (s.n + L - 1) / L;
-  s.a = s.n / s.k;
+  s.k = s.n <= L ? 1 : (int32_t)(((uint32_t)s.n + (uint32_t)L - 1u) / (uint32_t)L);
+  s.a = (int32_t)((uint32_t)s.n / (uint32_t)s.k);
   s.cA = s.n - s.k * s.a;
   s.cB = s.k - s.cA;
   return s;
 }
 
 // Block-wide exclusive scans of NV int64 values per thread in one pass (one
-// set of barriers).  `scratch` holds 32 * NV int64.  res[v] gets the
+// set of barriers).  `scratch` holds 32 * (NV + 1) int64.  res[v] gets the
 // exclusive prefix of v[v], total[v] the block sum.
 template <int NV>
 __device__ void block_exclusive_scan_n(const int64_t (&v)[NV], int64_t* scratch, int64_t (&res)[NV],
@@ -302,67 +302,79 @@ __device__ void block_exclusive_scan_n(const int64_t (&v)[NV], int64_t* scratch,
   __syncthreads();
 }
 
-// Item fields (tile pairs, live blocks) of the first kPlanCache chunks of
-// blockDim items stay in registers across the three passes; further items
-// are re-read from the item table.
-constexpr int kPlanCache = 4;
+// Item fields (tile pairs U, live blocks n) of the first kPlanSmemItems items
+// are staged in dynamic shared memory; later items are re-read from the item
+// table.
+constexpr int kPlanSmemItems = 24576;
+constexpr int kKeyBits = 9;          // piece lengths 0..256 (and 257 as a query)
+constexpr int32_t kNoKey = 511;      // lanes past the warp's items
 
-__global__ void __launch_bounds__(kPlanThreads) plan_kernel(const MetaParams p) {
-  __shared__ int64_t scratch[32 * 4];
-  __shared__ int32_t hist[kNumKeys];
+size_t plan_smem_bytes(int64_t n_items) {
+  const int64_t c = n_items < kPlanSmemItems ? n_items : kPlanSmemItems;
+  return (size_t)(c * 6 + 16);
+}
+
+// The piece order is a stable counting sort of all pieces by length, longest
+// first; inside a length, pieces follow their item, then tile pair, then
+// their place in the item's split.  Warp w owns the contiguous item range
+// [w R, (w + 1) R) (R = ceil(items / 32)) and walks it 32 items at a time, so
+// item order is (warp, step, lane) order:
+//   pass 2  per (warp, length) piece counts, per-warp unit / slot / combine
+//           totals;
+//   scan    bucket starts (lengths descending), per-(warp, length) offsets
+//           (warps ascending), per-warp slot and combine bases;
+//   pass 3  each warp places its pieces with no block barrier: a piece's
+//           rank inside its length is the warp's running cursor for that
+//           length plus the weights of earlier lanes of the same step with
+//           that length, taken by pointer jumping over lanes of equal keys.
+__global__ void __launch_bounds__(kPlanThreads) plan_kernel(const MetaParams p, int32_t cached) {
+  extern __shared__ __align__(16) unsigned char plan_dyn[];
+  __shared__ int64_t scratch[32 * 5];
+  __shared__ int64_t part[kPlanWarps][3];          // per warp: units, slots, combine records
   __shared__ int32_t bucket_start[kNumKeys];
-  __shared__ int32_t key_run[kNumKeys];
-  __shared__ int32_t warp_key[kPlanWarps][kNumKeys];
-  __shared__ int32_t split_len_sh;
+  __shared__ int32_t warp_key[kPlanWarps][kNumKeys];  // counts, then running cursors
+  __shared__ int64_t cost_sh[kPlanWarps];
   __shared__ int32_t abort_sh;
+  int32_t* sU = reinterpret_cast<int32_t*>(plan_dyn);
+  uint16_t* sN = reinterpret_cast<uint16_t*>(sU + cached);
 
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int i = tid; i < kPlanWarps * kNumKeys; i += blockDim.x) (&warp_key[0][0])[i] = 0;
   allow_dependents();
   grid_dependency_wait();  // the item table and live lists
   const Geometry& g = p.geo;
   int32_t* meta = p.meta;
   const int32_t* items = meta + g.off_item;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int64_t n_items = g.n_items;
-  const int64_t chunks = (n_items + blockDim.x - 1) / blockDim.x;
+  const int32_t n_items = g.n_items;
 
-  for (int i = tid; i < kNumKeys; i += blockDim.x) {
-    hist[i] = 0;
-    key_run[i] = 0;
-  }
-  for (int i = tid; i < kPlanWarps * kNumKeys; i += blockDim.x) (&warp_key[0][0])[i] = 0;
-  if (tid == 0) abort_sh = (meta[H_STATUS] & kDevBadSeqlen) ? 1 : 0;
-
-  // the item fields of this thread's items (chunk k: item k * blockDim + tid)
-  int32_t cU[kPlanCache], cn[kPlanCache];
-#pragma unroll
-  for (int k = 0; k < kPlanCache; k++) {
-    const int64_t i = (int64_t)k * blockDim.x + tid;
-    cU[k] = 0;
-    cn[k] = 0;
-    if (i < n_items) {
-      // item rows are 8 words on a 16-byte boundary: (.., n, n_tiles, ..)
-      const int4 r = *reinterpret_cast<const int4*>(items + 8 * i);
-      cn[k] = r.y;
-      cU[k] = (r.z + 1) / 2;
-    }
-  }
-  auto fields = [&](int64_t k, int32_t& U, int32_t& n) {
-    U = 0;
-    n = 0;
-#pragma unroll
-    for (int c = 0; c < kPlanCache; c++)
-      if (c == k) {
-        U = cU[c];
-        n = cn[c];
-      }
-    if (k >= kPlanCache) {
-      const int64_t i = k * blockDim.x + tid;
-      if (i < n_items) {
-        n = items[8 * i + 1];
-        U = (items[8 * i + 2] + 1) / 2;
-      }
+  auto fields = [&](int32_t i, int32_t& U, int32_t& n) {
+    if (i < cached) {
+      U = sU[i];
+      n = sN[i];
+    } else {
+      const int4 r = *reinterpret_cast<const int4*>(items + 8 * (int64_t)i);
+      n = r.y;
+      U = (r.z + 1) / 2;
     }
   };
+
+  // stage the fields, total cost
+  if (tid == 0) abort_sh = (meta[H_STATUS] & kDevBadSeqlen) ? 1 : 0;
+  int64_t cost = 0;
+#pragma unroll 4
+  for (int32_t i = tid; i < n_items; i += kPlanThreads) {
+    // item rows are 8 words on a 16-byte boundary: (.., n, n_tiles, ..)
+    const int4 r = *reinterpret_cast<const int4*>(items + 8 * (int64_t)i);
+    const int32_t U = (r.z + 1) / 2;
+    if (i < cached) {
+      sU[i] = U;
+      sN[i] = (uint16_t)r.y;
+    }
+    cost += (int64_t)U * r.y;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) cost += __shfl_xor_sync(0xffffffffu, cost, o);
+  if (lane == 0) cost_sh[warp] = cost;
   __syncthreads();
   if (abort_sh) {
     if (tid == 0) {
@@ -375,166 +387,194 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const MetaParams p) 
     }
     return;
   }
-
-  // pass 1: total cost
-  int64_t cost = 0;
-  for (int64_t k = 0; k < chunks; k++) {
-    int32_t U, n;
-    fields(k, U, n);
-    cost += (int64_t)U * n;
+  cost = 0;
+  for (int w = 0; w < kPlanWarps; w++) cost += cost_sh[w];
+  int64_t L64;
+  if (p.forced_split > 0) {
+    L64 = p.forced_split;
+  } else {
+    L64 = cdiv64(cost, 4LL * p.num_ctas);
+    if (L64 < kMinSplitLen) L64 = kMinSplitLen;
   }
-  {
-    const int64_t v[1] = {cost};
-    int64_t r[1], t[1];
-    block_exclusive_scan_n<1>(v, scratch, r, t);
-    cost = t[0];
-  }
+  if (L64 > 0x7fffffffLL) L64 = 0x7fffffffLL;
+  const int32_t L = (int32_t)L64;
   if (tid == 0) {
-    int64_t L;
-    if (p.forced_split > 0) {
-      L = p.forced_split;
-    } else {
-      L = cdiv64(cost, 4LL * p.num_ctas);
-      if (L < kMinSplitLen) L = kMinSplitLen;
-    }
-    if (L > 0x7fffffffLL) L = 0x7fffffffLL;
-    split_len_sh = (int32_t)L;
-    meta[H_SPLIT_LEN] = (int32_t)L;
+    meta[H_SPLIT_LEN] = L;
     meta[H_COST_LO] = (int32_t)(uint32_t)(cost & 0xffffffffLL);
     meta[H_COST_HI] = (int32_t)(uint32_t)((uint64_t)cost >> 32);
   }
-  __syncthreads();
-  const int32_t L = split_len_sh;
 
-  // pass 2: histogram of piece lengths (weighted), totals
-  int64_t pieces = 0, slots = 0, combs = 0;
-  for (int64_t k = 0; k < chunks; k++) {
-    int32_t U, n;
-    fields(k, U, n);
-    if (k * blockDim.x + tid >= n_items) continue;
-    const PieceShape s = piece_shape(U, n, L);
-    if (s.cA) atomicAdd(&hist[s.a + 1], s.U * s.cA);
-    if (s.cB) atomicAdd(&hist[s.a], s.U * s.cB);
-    pieces += (int64_t)s.U * s.k;
-    if (s.k > 1) {
-      slots += (int64_t)s.U * s.k;
-      combs += s.U;
+  const int32_t R = (n_items + kPlanWarps - 1) / kPlanWarps;
+  const int32_t lo = warp * R < n_items ? warp * R : n_items;
+  const int32_t hi = lo + R < n_items ? lo + R : n_items;
+
+  // pass 2: per (warp, length) counts and per-warp totals
+  {
+    int64_t units = 0, slots = 0, combs = 0;
+    for (int32_t i = lo + lane; i < hi; i += 32) {
+      int32_t U, n;
+      fields(i, U, n);
+      const PieceShape s = piece_shape(U, n, L);
+      atomicAdd(&warp_key[warp][s.a], s.U * s.cB);  // cB >= 1
+      if (s.cA) atomicAdd(&warp_key[warp][s.a + 1], s.U * s.cA);
+      units += (int64_t)s.U * s.k;
+      if (s.k > 1) {
+        slots += (int64_t)s.U * s.k;
+        combs += s.U;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      units += __shfl_xor_sync(0xffffffffu, units, o);
+      slots += __shfl_xor_sync(0xffffffffu, slots, o);
+      combs += __shfl_xor_sync(0xffffffffu, combs, o);
+    }
+    if (lane == 0) {
+      part[warp][0] = units;
+      part[warp][1] = slots;
+      part[warp][2] = combs;
     }
   }
+  __syncthreads();
+
+  // per length: offsets over warps (in place) and the length's total;
+  // thread j holds length kNumKeys - 1 - j so that one scan over threads
+  // gives the bucket starts longest first.  Threads 0..31 also carry warp
+  // j's unit / slot / combine totals.
   int64_t n_units, n_slots, n_comb;
   {
-    const int64_t v[3] = {pieces, slots, combs};
-    int64_t r[3], t[3];
-    block_exclusive_scan_n<3>(v, scratch, r, t);  // its barriers also publish hist
-    n_units = t[0];
-    n_slots = t[1];
-    n_comb = t[2];
-  }
-  // bucket starts, longest first: an exclusive scan over the keys in
-  // descending order (thread j holds key kNumKeys - 1 - j)
-  {
     const int key = kNumKeys - 1 - tid;
-    const int64_t v[1] = {tid < kNumKeys ? (int64_t)hist[key] : 0};
-    int64_t r[1], t[1];
-    block_exclusive_scan_n<1>(v, scratch, r, t);
+    int64_t v[4] = {0, 0, 0, 0};
+    if (tid < kNumKeys) {
+      int32_t acc = 0;
+      for (int w = 0; w < kPlanWarps; w++) {
+        const int32_t c = warp_key[w][key];
+        warp_key[w][key] = acc;
+        acc += c;
+      }
+      v[0] = acc;
+    }
+    if (tid < kPlanWarps) {
+      v[1] = part[tid][0];
+      v[2] = part[tid][1];
+      v[3] = part[tid][2];
+    }
+    int64_t r[4], t[4];
+    block_exclusive_scan_n<4>(v, scratch, r, t);
     if (tid < kNumKeys) bucket_start[key] = (int32_t)r[0];
+    if (tid < kPlanWarps) {
+      part[tid][1] = r[2];
+      part[tid][2] = r[3];
+    }
+    n_units = t[1];
+    n_slots = t[2];
+    n_comb = t[3];
   }
   if (tid == 0) {
     const bool over = n_units > g.unit_cap || n_slots > g.slot_cap || n_comb > g.comb_cap;
-    abort_sh = over ? 1 : 0;
     meta[H_NUNITS] = over ? 0 : (int32_t)n_units;
     meta[H_NSLOTS] = over ? 0 : (int32_t)n_slots;
     meta[H_NCOMB] = over ? 0 : (int32_t)n_comb;
     if (over) raise_status(p, kDevCapacity);
   }
   __syncthreads();
-  if (abort_sh) return;
+  if (n_units > g.unit_cap || n_slots > g.slot_cap || n_comb > g.comb_cap) return;
 
-  // pass 3: place every piece (stable within a length), chunk by chunk
-  int32_t* units = meta + g.off_unit;
-  int32_t* comb = meta + g.off_comb;
-  int64_t slot_run = 0, comb_run = 0;
-  for (int64_t k = 0; k < chunks; k++) {
-    const int64_t i = k * blockDim.x + tid;
+  // pass 3: place the pieces, warp by warp
+  int4* units = reinterpret_cast<int4*>(meta + g.off_unit);
+  int4* comb = reinterpret_cast<int4*>(meta + g.off_comb);
+  int32_t slot_cur = (int32_t)part[warp][1], comb_cur = (int32_t)part[warp][2];
+  const uint32_t lt = (1u << lane) - 1u, gt = ~lt & ~(1u << lane);
+  for (int32_t base = lo; base < hi; base += 32) {
+    const int32_t i = base + lane;
+    const bool valid = i < hi;
     PieceShape s{0, 0, 1, 0, 0, 0};
-    const bool valid = i < n_items;
     if (valid) {
       int32_t U, n;
-      fields(k, U, n);
+      fields(i, U, n);
       s = piece_shape(U, n, L);
     }
-    const int32_t kA = (valid && s.cA) ? s.a + 1 : -1;
-    const int32_t wA = (valid && s.cA) ? s.U * s.cA : 0;
-    const int32_t kB = (valid && s.cB) ? s.a : -1;
-    const int32_t wB = (valid && s.cB) ? s.U * s.cB : 0;
-    // per-key exclusive prefix inside the warp, in lane order
-    int32_t preA = 0, preB = 0;
-    for (int src = 0; src < 31; src++) {
-      const int32_t ska = __shfl_sync(0xffffffffu, kA, src);
-      const int32_t swa = __shfl_sync(0xffffffffu, wA, src);
-      const int32_t skb = __shfl_sync(0xffffffffu, kB, src);
-      const int32_t swb = __shfl_sync(0xffffffffu, wB, src);
-      if (src < lane) {
-        if (kA >= 0) preA += (ska == kA ? swa : 0) + (skb == kA ? swb : 0);
-        if (kB >= 0) preB += (ska == kB ? swa : 0) + (skb == kB ? swb : 0);
+    const int32_t a = valid ? s.a : kNoKey;
+    const int32_t wA = s.U * s.cA, wB = s.U * s.cB;  // 0 for lanes past the range
+    // key-equality masks from the bits of a: eq(x) = lanes whose a == x
+    uint32_t bal[kKeyBits];
+#pragma unroll
+    for (int b = 0; b < kKeyBits; b++) bal[b] = __ballot_sync(0xffffffffu, (a >> b) & 1);
+    auto eq = [&](int32_t x) {
+      uint32_t m = 0xffffffffu;
+#pragma unroll
+      for (int b = 0; b < kKeyBits; b++) m &= ((x >> b) & 1) ? bal[b] : ~bal[b];
+      return m;
+    };
+    const uint32_t same = eq(a);
+    // inclusive sums of wA and wB over the lanes <= this one with the same a
+    int32_t sA = wA, sB = wB;
+    int32_t ptr = (same & lt) ? 31 - __clz(same & lt) : -1;
+    while (__any_sync(0xffffffffu, ptr >= 0)) {
+      const int32_t src = ptr >= 0 ? ptr : lane;
+      const int32_t tA = __shfl_sync(0xffffffffu, sA, src);
+      const int32_t tB = __shfl_sync(0xffffffffu, sB, src);
+      const int32_t tp = __shfl_sync(0xffffffffu, ptr, src);
+      if (ptr >= 0) {
+        sA += tA;
+        sB += tB;
+        ptr = tp;
       }
     }
-    if (kA >= 0) atomicAdd(&warp_key[warp][kA], wA);
-    if (kB >= 0) atomicAdd(&warp_key[warp][kB], wB);
-    const int64_t my_slots = (valid && s.k > 1) ? (int64_t)s.U * s.k : 0;
-    const int64_t my_combs = (valid && s.k > 1) ? s.U : 0;
-    int64_t slot_base, comb_base;
-    {
-      const int64_t v[2] = {my_slots, my_combs};
-      int64_t r[2], t[2];
-      block_exclusive_scan_n<2>(v, scratch, r, t);  // its barriers also publish warp_key
-      slot_base = slot_run + r[0];
-      comb_base = comb_run + r[1];
-      slot_run += t[0];
-      comb_run += t[1];
-    }
-    // per key: exclusive prefix over warps, plus the run of earlier chunks
-    for (int key = tid; key < kNumKeys; key += blockDim.x) {
-      int32_t acc = key_run[key];
-      for (int w = 0; w < kPlanWarps; w++) {
-        const int32_t c = warp_key[w][key];
-        warp_key[w][key] = acc;
-        acc += c;
+    // length a gets the short pieces of lanes with a and the long pieces of
+    // lanes with a - 1; length a + 1 the long pieces of lanes with a and the
+    // short pieces of lanes with a + 1
+    const uint32_t prev = (valid && a > 0) ? eq(a - 1) & lt : 0u;
+    const uint32_t next = valid ? eq(a + 1) & lt : 0u;
+    const int32_t xA = __shfl_sync(0xffffffffu, sA, prev ? 31 - __clz(prev) : lane);
+    const int32_t xB = __shfl_sync(0xffffffffu, sB, next ? 31 - __clz(next) : lane);
+    const int32_t preB = sB - wB + (prev ? xA : 0);
+    const int32_t preA = sA - wA + (next ? xB : 0);
+    // slots and combine records in item order
+    int32_t my_slots = s.k > 1 ? s.U * s.k : 0, my_combs = s.k > 1 ? s.U : 0;
+    int32_t iS = my_slots, iC = my_combs;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t ns = __shfl_up_sync(0xffffffffu, iS, o);
+      const int32_t nc = __shfl_up_sync(0xffffffffu, iC, o);
+      if (lane >= o) {
+        iS += ns;
+        iC += nc;
       }
-      key_run[key] = acc;
     }
-    __syncthreads();
+    const int32_t slot_base = slot_cur + iS - my_slots;
+    const int32_t comb_base = comb_cur + iC - my_combs;
+    slot_cur += __shfl_sync(0xffffffffu, iS, 31);
+    comb_cur += __shfl_sync(0xffffffffu, iC, 31);
+    int32_t startA = 0, startB = 0;
     if (valid) {
-      const int32_t startA = kA >= 0 ? bucket_start[kA] + warp_key[warp][kA] + preA : 0;
-      const int32_t startB = kB >= 0 ? bucket_start[kB] + warp_key[warp][kB] + preB : 0;
-      for (int32_t tp = 0; tp < s.U; tp++) {
-        if (s.k > 1) {
-          int32_t* c = comb + 4 * (comb_base + tp);
-          c[0] = (int32_t)i;
-          c[1] = tp;
-          c[2] = (int32_t)(slot_base + (int64_t)tp * s.k);
-          c[3] = s.k;
-        }
-        for (int32_t q = 0; q < s.k; q++) {
-          const int32_t j0 = (int32_t)((int64_t)q * s.n / s.k);
-          const int32_t j1 = (int32_t)((int64_t)(q + 1) * s.n / s.k);
-          const int32_t longs_before = j0 - q * s.a;  // long pieces before q in this pair
-          int32_t pos;
-          if (j1 - j0 == s.a + 1 && s.cA)
-            pos = startA + tp * s.cA + longs_before;
-          else
-            pos = startB + tp * s.cB + (q - longs_before);
-          int32_t* u = units + 4 * (int64_t)pos;
-          u[0] = (int32_t)i;
-          u[1] = tp;
-          u[2] = j0 | (j1 << 16);
-          u[3] = s.k > 1 ? (int32_t)(slot_base + (int64_t)tp * s.k + q) : -1;
-        }
+      startB = bucket_start[a] + warp_key[warp][a] + preB;
+      if (s.cA) startA = bucket_start[a + 1] + warp_key[warp][a + 1] + preA;
+    }
+    __syncwarp();
+    // the last lane of each key group advances the warp's cursors
+    if (valid && !(same & gt)) {
+      atomicAdd(&warp_key[warp][a], sB);
+      if (sA) atomicAdd(&warp_key[warp][a + 1], sA);
+    }
+    __syncwarp();
+    if (valid) {
+      if (s.k > 1)
+        for (int32_t tp = 0; tp < s.U; tp++)
+          comb[comb_base + tp] = make_int4(i, tp, slot_base + tp * s.k, s.k);
+      int32_t j0 = 0, longs = 0;
+      for (int32_t q = 0; q < s.k; q++) {
+        const int32_t j1 = (int32_t)((uint32_t)((q + 1) * s.n) / (uint32_t)s.k);
+        const bool is_long = j1 - j0 == s.a + 1 && s.cA;
+        const int32_t first = is_long ? startA + longs : startB + (q - longs);
+        const int32_t stride = is_long ? s.cA : s.cB;
+        for (int32_t tp = 0; tp < s.U; tp++)
+          units[first + tp * stride] =
+              make_int4(i, tp, j0 | (j1 << 16), s.k > 1 ? slot_base + tp * s.k + q : -1);
+        longs += is_long ? 1 : 0;
+        j0 = j1;
       }
     }
-    __syncthreads();
-    for (int t = tid; t < kPlanWarps * kNumKeys; t += blockDim.x) (&warp_key[0][0])[t] = 0;
-    __syncthreads();
   }
 }
 
@@ -547,7 +587,19 @@ cudaError_t launch_metadata(const MetaParams& p, cudaStream_t stream) {
   const int64_t blocks = (p.geo.n_items + kItemWarps - 1) / kItemWarps;
   e = launch_dependent(item_kernel, dim3((unsigned)blocks), dim3(kItemWarps * 32), 0, stream, p);
   if (e != cudaSuccess) return e;
-  return launch_dependent(plan_kernel, dim3(1), dim3(kPlanThreads), 0, stream, p);
+  const int32_t cached = p.geo.n_items < kPlanSmemItems ? p.geo.n_items : kPlanSmemItems;
+  const size_t smem = plan_smem_bytes(p.geo.n_items);
+  static int configured_device = -1;
+  int dev = 0;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (configured_device != dev) {
+    e = cudaFuncSetAttribute(plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)plan_smem_bytes(kPlanSmemItems));
+    if (e != cudaSuccess) return e;
+    configured_device = dev;
+  }
+  return launch_dependent(plan_kernel, dim3(1), dim3(kPlanThreads), smem, stream, p, cached);
 }
 
 }  // namespace gbsa

@@ -95,6 +95,33 @@ def test_metadata_bit_exact(name):
         assert int(status.item()) == 0
 
 
+LARGE_META = {
+    **{n: (lambda n=n: workload(n)) for n in ("dense", "long", "decode", "ragged")},
+    # 50500 items: past the items whose fields the plan kernel stages in
+    # shared memory, so the rest are re-read from the item table
+    "many_items": lambda: generate(name="many", seed=81, q_storage=[60000, 41000], N1=16, N2=4,
+                                   block_x=8, top_k=3, selection="random_causal"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(LARGE_META))
+def test_metadata_bit_exact_full_size(name):
+    """The work list of the full-size workloads (the launch configuration the
+    benchmark uses, and forced split lengths that give long and short pieces
+    of many lengths) is word for word the sequential rebuild's."""
+    w = LARGE_META[name]()
+    t = device_tensors(w)
+    for ctas, forced in ((0, 0), (148, 3), (64, 2)):
+        status = torch.zeros(1, dtype=torch.int32, device="cuda")
+        meta = run_metadata(w, t, ctas, forced, status).cpu().numpy()
+        ref = scheduler.build(problem_dict(w, ctas or sm_count(), forced), w.sparse_idx,
+                              w.sparse_count, w.cu_seqlens_q, w.q_used, w.kv_used)
+        assert meta.size == ref.size
+        mask = scheduler.defined_mask(ref)
+        assert np.array_equal(meta[mask], ref[mask]), _first_diffs(meta, ref, mask)
+        assert int(status.item()) == int(ref[15])
+
+
 @pytest.mark.parametrize("name", sorted(SMALL))
 def test_forward_matches_oracle(name):
     w = SMALL[name]()
