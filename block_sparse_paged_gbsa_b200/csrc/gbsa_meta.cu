@@ -9,8 +9,10 @@
 // follows seqused, and values are not validated on the host (here the
 // kernels record GBSA_DEV_* bits instead).
 //
-// Three launches on the caller's stream:
-//   1. seq_kernel   (1 CTA):  per-sequence lengths, Q-block bases, header;
+// Launches on the caller's stream:
+//   1. seq_kernel   (1 CTA, only for more than 1024 sequences): per-sequence
+//                   lengths, Q-block bases, header; with fewer sequences every
+//                   item CTA derives them itself and CTA 0 writes them;
 //   2. item_kernel  (1 warp per item): liveness of every list entry, the
 //                   compacted live list with mask / partial-page flags;
 //   3. plan_kernel  (1 CTA):  split length, pieces, longest-first order
@@ -40,8 +42,9 @@ __device__ __forceinline__ void raise_status(const MetaParams& p, int32_t bits) 
 }
 
 // Block-wide exclusive scan of one int64 per thread (blockDim.x threads,
-// a multiple of 32, at most 1024).  `scratch` holds 32 int64.  Returns the
-// exclusive prefix; *total gets the block sum.
+// a multiple of 32, at most 1024).  `scratch` holds 33 int64: the warps'
+// prefixes and, apart from them, the block sum.  Returns the exclusive
+// prefix; *total gets the block sum.
 __device__ int64_t block_exclusive_scan(int64_t v, int64_t* scratch, int64_t* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
   int64_t incl = v;
@@ -62,11 +65,11 @@ __device__ int64_t block_exclusive_scan(int64_t v, int64_t* scratch, int64_t* to
       if (lane >= o) wi += n;
     }
     if (lane < nwarps) scratch[lane] = wi - w;
-    if (lane == 31) scratch[31] = wi;  // lanes >= nwarps add 0, so lane 31 holds the sum
+    if (lane == 31) scratch[32] = wi;  // lanes >= nwarps add 0, so lane 31 holds the sum
   }
   __syncthreads();
   const int64_t res = scratch[warp] + incl - v;
-  *total = scratch[31];
+  *total = scratch[32];
   __syncthreads();
   return res;
 }
@@ -74,13 +77,52 @@ __device__ int64_t block_exclusive_scan(int64_t v, int64_t* scratch, int64_t* to
 // ---------------------------------------------------------------------------
 // 1. sequences
 // ---------------------------------------------------------------------------
+// Header fields known before the plan, the sequence status, and the (at most
+// 3) padding words between the live lists and the unit table.
+__device__ void write_header(const MetaParams& p, int32_t status) {
+  const Geometry& g = p.geo;
+  int32_t* meta = p.meta;
+  meta[H_MAGIC] = (int32_t)kMagic;
+  meta[H_VERSION] = kFormatVersion;
+  meta[H_SIGNATURE] = (int32_t)p.signature;
+  meta[H_B] = p.B;
+  meta[H_NITEMS] = g.n_items;
+  meta[H_TILE_TOKENS] = g.tile_tokens;
+  meta[H_TILES_MAX] = g.tiles_max;
+  meta[H_NUM_CTAS] = p.num_ctas;
+  meta[H_UNIT_CAP] = (int32_t)g.unit_cap;
+  meta[H_SLOT_CAP] = (int32_t)g.slot_cap;
+  meta[H_COMB_CAP] = (int32_t)g.comb_cap;
+  meta[H_STATUS] = status;
+  meta[H_OFF_SEQ] = (int32_t)g.off_seq;
+  meta[H_OFF_ITEM] = (int32_t)g.off_item;
+  meta[H_OFF_LIST] = (int32_t)g.off_list;
+  meta[H_OFF_UNIT] = (int32_t)g.off_unit;
+  meta[H_OFF_COMB] = (int32_t)g.off_comb;
+  meta[H_TOTAL] = (int32_t)g.total_words;
+  meta[H_ROWS_PER_UNIT] = g.rows_per_unit;
+  meta[H_G] = g.G;
+  for (int64_t w = g.off_list + (int64_t)g.n_items * p.top_k; w < g.off_unit; w++) meta[w] = 0;
+  if (status && p.dev_status) atomicOr(p.dev_status, status);
+}
+
+int32_t seq_threads(int32_t B) {
+  const int32_t t = (B + 31) / 32 * 32;
+  return t < kSeqThreads ? t : kSeqThreads;
+}
+
 __global__ void __launch_bounds__(kSeqThreads) seq_kernel(const MetaParams p) {
-  __shared__ int64_t scratch[32];
+  __shared__ int64_t scratch[33];
+  __shared__ int64_t ends_sh[2];  // cu_seqlens_q[0], cu_seqlens_q[B]
   __shared__ int32_t bad_sh;
   const Geometry& g = p.geo;
   int32_t* meta = p.meta;
   allow_dependents();
-  if (threadIdx.x == 0) bad_sh = 0;
+  if (threadIdx.x == 0) {
+    ends_sh[0] = p.cu_seqlens_q[0];
+    ends_sh[1] = p.cu_seqlens_q[p.B];
+    bad_sh = 0;
+  }
   if (threadIdx.x < kHeaderWords) meta[threadIdx.x] = 0;
   __syncthreads();
   int32_t bad = 0;
@@ -99,50 +141,22 @@ __global__ void __launch_bounds__(kSeqThreads) seq_kernel(const MetaParams p) {
     int64_t total;
     const int64_t excl = block_exclusive_scan(nqb, scratch, &total);
     if (b < p.B) {
-      int32_t* row = meta + g.off_seq + 8 * b;
-      row[0] = (int32_t)qs;
-      row[1] = (int32_t)qu;
-      row[2] = (int32_t)ku;
-      row[3] = (int32_t)nqb;
-      row[4] = (int32_t)(running + excl);
-      row[5] = (int32_t)tok;
-      row[6] = 0;
-      row[7] = 0;
+      int4* row = reinterpret_cast<int4*>(meta + g.off_seq + 8 * b);
+      row[0] = make_int4((int32_t)qs, (int32_t)qu, (int32_t)ku, (int32_t)nqb);
+      row[1] = make_int4((int32_t)(running + excl), (int32_t)tok, 0, 0);
     }
     running += total;
   }
   if (bad) atomicOr(&bad_sh, 1);
   __syncthreads();
   if (threadIdx.x == 0) {
-    const int64_t c0 = p.cu_seqlens_q[0], cB = p.cu_seqlens_q[p.B];
+    const int64_t c0 = ends_sh[0], cB = ends_sh[1];
     if (bad_sh || c0 != 0 || running != p.total_q_blocks || (p.T > 0 && cB != p.T) ||
         cB > 0x7fffffffLL)
       bad = kDevBadSeqlen;
     else
       bad = 0;
-    meta[H_MAGIC] = (int32_t)kMagic;
-    meta[H_VERSION] = kFormatVersion;
-    meta[H_SIGNATURE] = (int32_t)p.signature;
-    meta[H_B] = p.B;
-    meta[H_NITEMS] = g.n_items;
-    meta[H_TILE_TOKENS] = g.tile_tokens;
-    meta[H_TILES_MAX] = g.tiles_max;
-    meta[H_NUM_CTAS] = p.num_ctas;
-    meta[H_UNIT_CAP] = (int32_t)g.unit_cap;
-    meta[H_SLOT_CAP] = (int32_t)g.slot_cap;
-    meta[H_COMB_CAP] = (int32_t)g.comb_cap;
-    meta[H_STATUS] = bad;
-    meta[H_OFF_SEQ] = (int32_t)g.off_seq;
-    meta[H_OFF_ITEM] = (int32_t)g.off_item;
-    meta[H_OFF_LIST] = (int32_t)g.off_list;
-    meta[H_OFF_UNIT] = (int32_t)g.off_unit;
-    meta[H_OFF_COMB] = (int32_t)g.off_comb;
-    meta[H_TOTAL] = (int32_t)g.total_words;
-    meta[H_ROWS_PER_UNIT] = g.rows_per_unit;
-    meta[H_G] = g.G;
-    // the (at most 3) padding words between the live lists and the unit table
-    for (int64_t w = g.off_list + (int64_t)g.n_items * p.top_k; w < g.off_unit; w++) meta[w] = 0;
-    if (bad && p.dev_status) atomicOr(p.dev_status, bad);
+    write_header(p, bad);
   }
 }
 
@@ -150,29 +164,147 @@ __global__ void __launch_bounds__(kSeqThreads) seq_kernel(const MetaParams p) {
 // 2. items: one warp per (Q block, KV head)
 // ---------------------------------------------------------------------------
 constexpr int kItemWarps = 8;
+constexpr int kItemThreads = kItemWarps * 32;
+constexpr int kItemSmemSeqs = 2048;  // sequences whose Q-block bases are staged
+constexpr int kOwnSeqMax = 1024;     // up to this many sequences, every item CTA
+                                     // derives the sequence table itself
+constexpr int kOwnSeqPer = kOwnSeqMax / kItemThreads;
+constexpr int kListChunks = kMaxTopK / 32;
 
-__global__ void __launch_bounds__(kItemWarps * 32) item_kernel(const MetaParams p) {
+// Status bits of item i go to word i of the unit table (rows there are
+// undefined until the plan kernel writes them); the plan kernel ORs them
+// into the header.  No word of the buffer has to be zeroed first.
+__device__ __forceinline__ int32_t* item_status_word(const MetaParams& p, int64_t item) {
+  return p.meta + p.geo.off_unit + item;
+}
+
+// kOwnSeq: the first kernel of the call; each CTA computes the per-sequence
+// fields and Q-block bases of all B <= kOwnSeqMax sequences into shared
+// memory, and CTA 0 writes the sequence table and the header.  Otherwise the
+// sequence kernel ran before and the bases are read back from its table.
+template <bool kOwnSeq>
+__global__ void __launch_bounds__(kItemThreads) item_kernel(const MetaParams p) {
+  constexpr int kCap = kOwnSeq ? kOwnSeqMax : kItemSmemSeqs;
+  __shared__ int32_t base_sh[kCap];                    // first Q block of each sequence
+  __shared__ int32_t nqb_sh[kCap];                     // its Q-block count
+  __shared__ int4 row_sh[kOwnSeq ? kOwnSeqMax : 1];    // (qs, qu, ku, first token)
+  __shared__ int64_t scratch[33];
+  __shared__ int32_t bad_sh;
   allow_dependents();
-  grid_dependency_wait();  // the sequence table
   const Geometry& g = p.geo;
   const int lane = threadIdx.x & 31;
   const int64_t item = (int64_t)blockIdx.x * kItemWarps + (threadIdx.x >> 5);
-  if (item >= g.n_items) return;
-  const int32_t* meta_c = p.meta;
+  const bool active = item < g.n_items;
   const int32_t qb = (int32_t)(item / p.N2);
   const int32_t kvh = (int32_t)(item % p.N2);
-  const int32_t* seq = meta_c + g.off_seq;
+
+  // The selection list and count are inputs of the call, complete before the
+  // first kernel of the call started: read them before any wait.
+  int64_t n = 0;
+  int32_t pre[kListChunks];
+  const int32_t* list = p.sparse_idx + ((int64_t)kvh * p.total_q_blocks + qb) * p.top_k;
+  if (active) n = p.sparse_count[(int64_t)kvh * p.total_q_blocks + qb];
+#pragma unroll
+  for (int c = 0; c < kListChunks; c++) {
+    const int32_t j = 32 * c + lane;
+    pre[c] = (active && j < p.top_k) ? list[j] : 0;
+  }
+
+  const int32_t* seq = p.meta + g.off_seq;
+  bool staged = true;
+  if constexpr (kOwnSeq) {
+    const int t = threadIdx.x;
+    if (t == 0) bad_sh = 0;
+    int64_t nq[kOwnSeqPer];
+    int64_t sum = 0;
+    int32_t bad = 0;
+#pragma unroll
+    for (int r = 0; r < kOwnSeqPer; r++) {
+      const int32_t b = kOwnSeqPer * t + r;
+      nq[r] = 0;
+      if (b < p.B) {
+        const int64_t tok = p.cu_seqlens_q[b];
+        const int64_t qs = p.cu_seqlens_q[b + 1] - tok;
+        const int64_t qu = p.has_seqused_q ? (int64_t)p.seqused_q[b] : qs;
+        const int64_t ku = p.seqused_kv[b];
+        if (qs < 0 || qu < 0 || qu > qs || ku < 0) bad = 1;
+        nq[r] = qs > 0 ? cdiv64(qs, p.block_x) : 0;
+        row_sh[b] = make_int4((int32_t)qs, (int32_t)qu, (int32_t)ku, (int32_t)tok);
+        nqb_sh[b] = (int32_t)nq[r];
+      }
+      sum += nq[r];
+    }
+    int64_t total;
+    int64_t run = block_exclusive_scan(sum, scratch, &total);  // its barriers publish row_sh
+#pragma unroll
+    for (int r = 0; r < kOwnSeqPer; r++) {
+      const int32_t b = kOwnSeqPer * t + r;
+      if (b < p.B) base_sh[b] = (int32_t)run;
+      run += nq[r];
+    }
+    if (bad) atomicOr(&bad_sh, 1);
+    if (blockIdx.x == 0) {
+      int32_t* meta = p.meta;
+      if (t < kHeaderWords) meta[t] = 0;
+#pragma unroll
+      for (int r = 0; r < kOwnSeqPer; r++) {
+        const int32_t b = kOwnSeqPer * t + r;
+        if (b < p.B) {
+          const int4 q = row_sh[b];
+          int4* row = reinterpret_cast<int4*>(meta + g.off_seq + 8 * (int64_t)b);
+          row[0] = make_int4(q.x, q.y, q.z, nqb_sh[b]);
+          row[1] = make_int4(base_sh[b], q.w, 0, 0);
+        }
+      }
+      __syncthreads();  // bad_sh complete; the zeroed header before its fields
+      if (t == 0) {
+        const int64_t c0 = p.cu_seqlens_q[0], cB = p.cu_seqlens_q[p.B];
+        const int32_t st = (bad_sh || c0 != 0 || total != p.total_q_blocks ||
+                            (p.T > 0 && cB != p.T) || cB > 0x7fffffffLL)
+                               ? kDevBadSeqlen
+                               : 0;
+        write_header(p, st);
+      }
+    }
+    __syncthreads();
+  } else {
+    grid_dependency_wait();  // the sequence table
+    staged = p.B <= kItemSmemSeqs;
+    if (staged) {
+      for (int32_t b = threadIdx.x; b < p.B; b += kItemThreads) {
+        nqb_sh[b] = seq[8 * b + 3];
+        base_sh[b] = seq[8 * b + 4];
+      }
+    }
+    __syncthreads();
+  }
+  if (!active) return;
+  auto seq_base = [&](int32_t b) { return staged ? base_sh[b] : seq[8 * b + 4]; };
+  auto seq_nqb = [&](int32_t b) { return staged ? nqb_sh[b] : seq[8 * b + 3]; };
 
   // sequence holding Q block qb: the last b with a block starting at or before qb
   int32_t lo = 0, hi = p.B - 1;
   while (lo < hi) {
     const int32_t mid = (lo + hi + 1) >> 1;
-    if (seq[8 * mid + 4] <= qb) lo = mid; else hi = mid - 1;
+    if (seq_base(mid) <= qb) lo = mid; else hi = mid - 1;
   }
   int32_t b = lo;
-  while (b > 0 && seq[8 * b + 3] == 0) b--;
-  const int64_t qs = seq[8 * b + 0], qu = seq[8 * b + 1], ku = seq[8 * b + 2];
-  const int64_t qbl = (int64_t)qb - seq[8 * b + 4];
+  while (b > 0 && seq_nqb(b) == 0) b--;
+  int64_t qs, qu, ku, tok0;
+  if constexpr (kOwnSeq) {
+    const int4 r = row_sh[b];
+    qs = r.x;
+    qu = r.y;
+    ku = r.z;
+    tok0 = r.w;
+  } else {
+    const int4 r = *reinterpret_cast<const int4*>(seq + 8 * b);  // qs, qu, ku, nqb
+    qs = r.x;
+    qu = r.y;
+    ku = r.z;
+    tok0 = seq[8 * b + 5];
+  }
+  const int64_t qbl = (int64_t)qb - seq_base(b);
   const int64_t bx = p.block_x;
   int64_t n_store = qs - qbl * bx;
   if (n_store > bx) n_store = bx;
@@ -187,20 +319,20 @@ __global__ void __launch_bounds__(kItemWarps * 32) item_kernel(const MetaParams 
   const int64_t wl = p.win_left;
 
   int32_t bits = 0;
-  int64_t n = p.sparse_count[(int64_t)kvh * p.total_q_blocks + qb];
   if (n < 0 || n > p.top_k) {
     bits |= kDevBadCount;
     n = n < 0 ? 0 : p.top_k;
   }
-  const int32_t* list = p.sparse_idx + ((int64_t)kvh * p.total_q_blocks + qb) * p.top_k;
   int32_t* out_list = p.meta + g.off_list + item * p.top_k;
   int32_t n_live = 0;
-  for (int64_t j0 = 0; j0 < p.top_k; j0 += 32) {
-    const int64_t j = j0 + lane;
+#pragma unroll
+  for (int c = 0; c < kListChunks; c++) {
+    if (32 * c >= p.top_k) break;
+    const int64_t j = 32 * c + lane;
     int32_t entry = 0;
     bool live = false;
     if (j < n) {
-      const int64_t lb = list[j];
+      const int64_t lb = pre[c];
       if (lb < 0 || lb >= nblk) {
         bits |= kDevBadBlockIdx;
       } else if (n_used > 0) {
@@ -218,19 +350,14 @@ __global__ void __launch_bounds__(kItemWarps * 32) item_kernel(const MetaParams 
     n_live += __popc(ballot);
   }
   for (int64_t j = n_live + lane; j < p.top_k; j += 32) out_list[j] = 0;
-  if (lane == 0) {
-    int32_t* row = p.meta + g.off_item + 8 * item;
-    row[0] = b;
-    row[1] = n_live;
-    row[2] = (int32_t)n_tiles;
-    row[3] = (int32_t)(seq[8 * b + 5] + qbl * bx);
-    row[4] = (int32_t)n_store;
-    row[5] = (int32_t)n_used;
-    row[6] = (int32_t)pos0;
-    row[7] = (int32_t)ku;
-  }
   bits = __reduce_or_sync(0xffffffffu, bits);
-  if (lane == 0) raise_status(p, bits);
+  if (lane == 0) {
+    int4* row = reinterpret_cast<int4*>(p.meta + g.off_item + 8 * item);
+    row[0] = make_int4(b, n_live, (int32_t)n_tiles, (int32_t)(tok0 + qbl * bx));
+    row[1] = make_int4((int32_t)n_store, (int32_t)n_used, (int32_t)pos0, (int32_t)ku);
+    *item_status_word(p, item) = bits;
+    if (bits && p.dev_status) atomicOr(p.dev_status, bits);
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -248,58 +375,27 @@ __device__ __forceinline__ PieceShape piece_shape(int32_t U, int32_t n, int32_t 
   PieceShape s;
   s.U = U;
   s.n = n;
-  s.k = s.n <= L ? 1 : (int32_t)(((uint32_t)s.n + (uint32_t)L - 1u) / (uint32_t)L);
-  s.a = (int32_t)((uint32_t)s.n / (uint32_t)s.k);
-  s.cA = s.n - s.k * s.a;
-  s.cB = s.k - s.cA;
+  if (n <= L) {
+    s.k = 1;
+    s.a = n;
+    s.cA = 0;
+    s.cB = 1;
+  } else {
+    s.k = (int32_t)(((uint32_t)n + (uint32_t)L - 1u) / (uint32_t)L);
+    s.a = (int32_t)((uint32_t)n / (uint32_t)s.k);
+    s.cA = n - s.k * s.a;
+    s.cB = s.k - s.cA;
+  }
   return s;
 }
 
-// Block-wide exclusive scans of NV int64 values per thread in one pass (one
-// set of barriers).  `scratch` holds 32 * (NV + 1) int64.  res[v] gets the
-// exclusive prefix of v[v], total[v] the block sum.
-template <int NV>
-__device__ void block_exclusive_scan_n(const int64_t (&v)[NV], int64_t* scratch, int64_t (&res)[NV],
-                                       int64_t (&total)[NV]) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-  int64_t incl[NV];
-#pragma unroll
-  for (int c = 0; c < NV; c++) incl[c] = v[c];
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-#pragma unroll
-    for (int c = 0; c < NV; c++) {
-      const int64_t n = __shfl_up_sync(0xffffffffu, incl[c], o);
-      if (lane >= o) incl[c] += n;
-    }
-  }
-  __syncthreads();
-  if (lane == 31) {
-#pragma unroll
-    for (int c = 0; c < NV; c++) scratch[32 * c + warp] = incl[c];
-  }
-  __syncthreads();
-  if (warp < NV) {
-    int64_t w = lane < nwarps ? scratch[32 * warp + lane] : 0;
-    int64_t wi = w;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int64_t n = __shfl_up_sync(0xffffffffu, wi, o);
-      if (lane >= o) wi += n;
-    }
-    // lanes >= nwarps add 0, so lane 31's inclusive sum is the total; write
-    // it after every lane has read its own slot
-    __syncwarp();
-    if (lane < nwarps) scratch[32 * warp + lane] = wi - w;
-    if (lane == 31) scratch[32 * NV + warp] = wi;
-  }
-  __syncthreads();
-#pragma unroll
-  for (int c = 0; c < NV; c++) {
-    res[c] = scratch[32 * c + warp] + incl[c] - v[c];
-    total[c] = scratch[32 * NV + c];
-  }
-  __syncthreads();
+// Warp sum of non-negative int64 values, exact while each is below 2^30; a
+// value at or above 2^30 makes the sum at least 2^30, past every capacity.
+__device__ __forceinline__ int64_t warp_sum_sat(int64_t v) {
+  const uint32_t c = v < (1LL << 30) ? (uint32_t)v : (1u << 30);
+  const uint32_t lo = __reduce_add_sync(0xffffffffu, c & 0xffffu);
+  const uint32_t hi = __reduce_add_sync(0xffffffffu, c >> 16);
+  return ((int64_t)hi << 16) + lo;
 }
 
 // Item fields (tile pairs U, live blocks n) of the first kPlanSmemItems items
@@ -329,12 +425,12 @@ size_t plan_smem_bytes(int64_t n_items) {
 //           that length, taken by pointer jumping over lanes of equal keys.
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const MetaParams p, int32_t cached) {
   extern __shared__ __align__(16) unsigned char plan_dyn[];
-  __shared__ int64_t scratch[32 * 5];
-  __shared__ int64_t part[kPlanWarps][3];          // per warp: units, slots, combine records
+  __shared__ int64_t part[kPlanWarps][3];  // per warp: units, slots, combine records
+  __shared__ int64_t totals[3];
   __shared__ int32_t bucket_start[kNumKeys];
   __shared__ int32_t warp_key[kPlanWarps][kNumKeys];  // counts, then running cursors
   __shared__ int64_t cost_sh[kPlanWarps];
-  __shared__ int32_t abort_sh;
+  __shared__ int32_t status_sh, item_bits_sh;
   int32_t* sU = reinterpret_cast<int32_t*>(plan_dyn);
   uint16_t* sN = reinterpret_cast<uint16_t*>(sU + cached);
 
@@ -358,13 +454,20 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const MetaParams p, 
     }
   };
 
-  // stage the fields, total cost
-  if (tid == 0) abort_sh = (meta[H_STATUS] & kDevBadSeqlen) ? 1 : 0;
+  // stage the fields, total cost; the items' status bits (left in the unit
+  // table's first words) go into the header
+  if (tid == 0) {
+    status_sh = meta[H_STATUS];
+    item_bits_sh = 0;
+  }
   int64_t cost = 0;
+  int32_t ibits = 0;
+  const int32_t* item_bits = meta + g.off_unit;
 #pragma unroll 4
   for (int32_t i = tid; i < n_items; i += kPlanThreads) {
     // item rows are 8 words on a 16-byte boundary: (.., n, n_tiles, ..)
     const int4 r = *reinterpret_cast<const int4*>(items + 8 * (int64_t)i);
+    ibits |= item_bits[i];
     const int32_t U = (r.z + 1) / 2;
     if (i < cached) {
       sU[i] = U;
@@ -374,9 +477,14 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const MetaParams p, 
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) cost += __shfl_xor_sync(0xffffffffu, cost, o);
-  if (lane == 0) cost_sh[warp] = cost;
+  ibits = __reduce_or_sync(0xffffffffu, ibits);
+  if (lane == 0) {
+    cost_sh[warp] = cost;
+    if (ibits) atomicOr(&item_bits_sh, ibits);
+  }
   __syncthreads();
-  if (abort_sh) {
+  if (tid == 0) meta[H_STATUS] = status_sh | item_bits_sh;
+  if (status_sh & kDevBadSeqlen) {
     if (tid == 0) {
       meta[H_NUNITS] = 0;
       meta[H_NSLOTS] = 0;
@@ -423,62 +531,87 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const MetaParams p, 
         combs += s.U;
       }
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      units += __shfl_xor_sync(0xffffffffu, units, o);
-      slots += __shfl_xor_sync(0xffffffffu, slots, o);
-      combs += __shfl_xor_sync(0xffffffffu, combs, o);
-    }
+    const int64_t u = warp_sum_sat(units);
+    const int64_t sl = __any_sync(0xffffffffu, slots != 0) ? warp_sum_sat(slots) : 0;
+    const int64_t cb = sl ? warp_sum_sat(combs) : 0;
     if (lane == 0) {
-      part[warp][0] = units;
-      part[warp][1] = slots;
-      part[warp][2] = combs;
+      part[warp][0] = u;
+      part[warp][1] = sl;
+      part[warp][2] = cb;
     }
   }
   __syncthreads();
 
-  // per length: offsets over warps (in place) and the length's total;
-  // thread j holds length kNumKeys - 1 - j so that one scan over threads
-  // gives the bucket starts longest first.  Threads 0..31 also carry warp
-  // j's unit / slot / combine totals.
-  int64_t n_units, n_slots, n_comb;
-  {
-    const int key = kNumKeys - 1 - tid;
-    int64_t v[4] = {0, 0, 0, 0};
-    if (tid < kNumKeys) {
-      int32_t acc = 0;
-      for (int w = 0; w < kPlanWarps; w++) {
-        const int32_t c = warp_key[w][key];
-        warp_key[w][key] = acc;
-        acc += c;
-      }
-      v[0] = acc;
+  // per length: offsets over warps, in place (threads 0..256); per warp:
+  // slot and combine bases (the last warp)
+  if (tid < kNumKeys) {
+    int32_t acc = 0;
+    for (int w = 0; w < kPlanWarps; w++) {
+      const int32_t c = warp_key[w][tid];
+      warp_key[w][tid] = acc;
+      acc += c;
     }
-    if (tid < kPlanWarps) {
-      v[1] = part[tid][0];
-      v[2] = part[tid][1];
-      v[3] = part[tid][2];
-    }
-    int64_t r[4], t[4];
-    block_exclusive_scan_n<4>(v, scratch, r, t);
-    if (tid < kNumKeys) bucket_start[key] = (int32_t)r[0];
-    if (tid < kPlanWarps) {
-      part[tid][1] = r[2];
-      part[tid][2] = r[3];
-    }
-    n_units = t[1];
-    n_slots = t[2];
-    n_comb = t[3];
+    bucket_start[tid] = acc;  // the length's total until the scan below
   }
-  if (tid == 0) {
-    const bool over = n_units > g.unit_cap || n_slots > g.slot_cap || n_comb > g.comb_cap;
-    meta[H_NUNITS] = over ? 0 : (int32_t)n_units;
-    meta[H_NSLOTS] = over ? 0 : (int32_t)n_slots;
-    meta[H_NCOMB] = over ? 0 : (int32_t)n_comb;
-    if (over) raise_status(p, kDevCapacity);
+  if (warp == kPlanWarps - 1) {
+    const int64_t u = part[lane][0], sl = part[lane][1], cb = part[lane][2];
+    int64_t iu = u, is = sl, ic = cb;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int64_t nu = __shfl_up_sync(0xffffffffu, iu, o);
+      const int64_t ns = __shfl_up_sync(0xffffffffu, is, o);
+      const int64_t nc = __shfl_up_sync(0xffffffffu, ic, o);
+      if (lane >= o) {
+        iu += nu;
+        is += ns;
+        ic += nc;
+      }
+    }
+    __syncwarp();
+    part[lane][1] = is - sl;
+    part[lane][2] = ic - cb;
+    if (lane == 31) {
+      totals[0] = iu;
+      totals[1] = is;
+      totals[2] = ic;
+    }
   }
   __syncthreads();
-  if (n_units > g.unit_cap || n_slots > g.slot_cap || n_comb > g.comb_cap) return;
+  // bucket starts, longest first: lane l of warp 0 takes lengths
+  // 256 - 9 l - j (j = 0..8), a serial prefix over its nine, then a warp scan
+  if (warp == 0) {
+    constexpr int kPer = (kNumKeys + 31) / 32;
+    int32_t loc[kPer];
+    int64_t sum = 0;
+#pragma unroll
+    for (int j = 0; j < kPer; j++) {
+      const int key = kNumKeys - 1 - kPer * lane - j;
+      loc[j] = (int32_t)sum;
+      sum += key >= 0 ? bucket_start[key] : 0;
+    }
+    int64_t incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int64_t n = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += n;
+    }
+    const int32_t excl = (int32_t)(incl - sum);
+#pragma unroll
+    for (int j = 0; j < kPer; j++) {
+      const int key = kNumKeys - 1 - kPer * lane - j;
+      if (key >= 0) bucket_start[key] = excl + loc[j];
+    }
+    if (lane == 0) {
+      const int64_t n_units = totals[0], n_slots = totals[1], n_comb = totals[2];
+      const bool over = n_units > g.unit_cap || n_slots > g.slot_cap || n_comb > g.comb_cap;
+      meta[H_NUNITS] = over ? 0 : (int32_t)n_units;
+      meta[H_NSLOTS] = over ? 0 : (int32_t)n_slots;
+      meta[H_NCOMB] = over ? 0 : (int32_t)n_comb;
+      if (over) raise_status(p, kDevCapacity);
+    }
+  }
+  __syncthreads();
+  if (totals[0] > g.unit_cap || totals[1] > g.slot_cap || totals[2] > g.comb_cap) return;
 
   // pass 3: place the pieces, warp by warp
   int4* units = reinterpret_cast<int4*>(meta + g.off_unit);
@@ -495,6 +628,20 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const MetaParams p, 
       s = piece_shape(U, n, L);
     }
     const int32_t a = valid ? s.a : kNoKey;
+    const int32_t U0 = __shfl_sync(0xffffffffu, s.U, 0);  // lane 0 is always valid
+    if (__all_sync(0xffffffffu, !valid || (s.k == 1 && s.U == U0))) {
+      // no split and equal tile pairs: one piece of length n per tile pair,
+      // rank = U0 x (earlier lanes with the same n)
+      const uint32_t same = __match_any_sync(0xffffffffu, a);
+      int32_t start = 0;
+      if (valid) start = bucket_start[a] + warp_key[warp][a] + U0 * __popc(same & lt);
+      __syncwarp();
+      if (valid && !(same & gt)) warp_key[warp][a] += U0 * __popc(same);
+      __syncwarp();
+      if (valid)
+        for (int32_t tp = 0; tp < U0; tp++) units[start + tp] = make_int4(i, tp, s.n << 16, -1);
+      continue;
+    }
     const int32_t wA = s.U * s.cA, wB = s.U * s.cB;  // 0 for lanes past the range
     // key-equality masks from the bits of a: eq(x) = lanes whose a == x
     uint32_t bal[kKeyBits];
@@ -530,22 +677,25 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const MetaParams p, 
     const int32_t xB = __shfl_sync(0xffffffffu, sB, next ? 31 - __clz(next) : lane);
     const int32_t preB = sB - wB + (prev ? xA : 0);
     const int32_t preA = sA - wA + (next ? xB : 0);
-    // slots and combine records in item order
-    int32_t my_slots = s.k > 1 ? s.U * s.k : 0, my_combs = s.k > 1 ? s.U : 0;
-    int32_t iS = my_slots, iC = my_combs;
+    // slots and combine records in item order (only split items have any)
+    int32_t slot_base = 0, comb_base = 0;
+    if (__any_sync(0xffffffffu, s.k > 1)) {
+      const int32_t my_slots = s.k > 1 ? s.U * s.k : 0, my_combs = s.k > 1 ? s.U : 0;
+      int32_t iS = my_slots, iC = my_combs;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int32_t ns = __shfl_up_sync(0xffffffffu, iS, o);
-      const int32_t nc = __shfl_up_sync(0xffffffffu, iC, o);
-      if (lane >= o) {
-        iS += ns;
-        iC += nc;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int32_t ns = __shfl_up_sync(0xffffffffu, iS, o);
+        const int32_t nc = __shfl_up_sync(0xffffffffu, iC, o);
+        if (lane >= o) {
+          iS += ns;
+          iC += nc;
+        }
       }
+      slot_base = slot_cur + iS - my_slots;
+      comb_base = comb_cur + iC - my_combs;
+      slot_cur += __shfl_sync(0xffffffffu, iS, 31);
+      comb_cur += __shfl_sync(0xffffffffu, iC, 31);
     }
-    const int32_t slot_base = slot_cur + iS - my_slots;
-    const int32_t comb_base = comb_cur + iC - my_combs;
-    slot_cur += __shfl_sync(0xffffffffu, iS, 31);
-    comb_cur += __shfl_sync(0xffffffffu, iC, 31);
     int32_t startA = 0, startB = 0;
     if (valid) {
       startB = bucket_start[a] + warp_key[warp][a] + preB;
@@ -580,24 +730,28 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const MetaParams p, 
 
 }  // namespace
 
+// Up to kOwnSeqMax sequences: two launches (items with their own sequence
+// phase, then the plan); more: the sequence kernel first.  The later kernels
+// start early (programmatic dependent launch) and wait for their inputs.
 cudaError_t launch_metadata(const MetaParams& p, cudaStream_t stream) {
-  seq_kernel<<<1, kSeqThreads, 0, stream>>>(p);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
   const int64_t blocks = (p.geo.n_items + kItemWarps - 1) / kItemWarps;
-  e = launch_dependent(item_kernel, dim3((unsigned)blocks), dim3(kItemWarps * 32), 0, stream, p);
+  cudaError_t e;
+  if (p.B <= kOwnSeqMax) {
+    item_kernel<true><<<(unsigned)blocks, kItemThreads, 0, stream>>>(p);
+    e = cudaGetLastError();
+  } else {
+    seq_kernel<<<1, seq_threads(p.B), 0, stream>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    e = launch_dependent(item_kernel<false>, dim3((unsigned)blocks), dim3(kItemThreads), 0,
+                         stream, p);
+  }
   if (e != cudaSuccess) return e;
   const int32_t cached = p.geo.n_items < kPlanSmemItems ? p.geo.n_items : kPlanSmemItems;
   const size_t smem = plan_smem_bytes(p.geo.n_items);
-  static int configured_device = -1;
-  int dev = 0;
-  e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (configured_device != dev) {
-    e = cudaFuncSetAttribute(plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)plan_smem_bytes(kPlanSmemItems));
+  if (smem > 8192) {
+    e = cudaFuncSetAttribute(plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    configured_device = dev;
   }
   return launch_dependent(plan_kernel, dim3(1), dim3(kPlanThreads), smem, stream, p, cached);
 }

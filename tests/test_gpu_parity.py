@@ -101,7 +101,19 @@ LARGE_META = {
     # shared memory, so the rest are re-read from the item table
     "many_items": lambda: generate(name="many", seed=81, q_storage=[60000, 41000], N1=16, N2=4,
                                    block_x=8, top_k=3, selection="random_causal"),
+    # sequence counts around the paths of the sequence phase: derived in
+    # every item CTA (up to 1024), a sequence kernel with the bases staged
+    # in shared memory (up to 2048), and read from its table (beyond)
+    **{f"decode_b{B}": (lambda B=B: _decode_batch(B)) for B in (1024, 1500, 2500)},
 }
+
+
+def _decode_batch(B, seed=82):
+    rng = np.random.default_rng(seed + B)
+    kv = rng.integers(1, 3000, size=B).astype(np.int32)
+    return generate(name=f"db{B}", seed=seed, q_storage=[1] * B, q_used=[1] * B, kv_used=kv,
+                    N1=8, N2=2, block_x=1, top_k=16, selection="decode", count_range=(1, 16),
+                    has_seqused_q=False)
 
 
 @pytest.mark.parametrize("name", sorted(LARGE_META))
@@ -206,6 +218,31 @@ def test_device_status_bits():
     bits = int(status.item())
     assert bits & 0x02 and bits & 0x04 and not bits & ~0x06
     _compare(w, q, kf, vf, out, lse)
+    # the work list, header status word included, is still the rebuild's
+    m = meta.cpu().numpy()
+    ref = scheduler.build(problem_dict(w, sm_count()), w.sparse_idx, w.sparse_count,
+                          w.cu_seqlens_q, w.q_used, w.kv_used)
+    mask = scheduler.defined_mask(ref)
+    assert int(m[15]) == int(ref[15]) == bits
+    assert np.array_equal(m[mask], ref[mask]), _first_diffs(m, ref, mask)
+
+
+@pytest.mark.parametrize("case", ["tiny", "decode_b1100"])
+def test_bad_seqlen_status_matches_rebuild(case):
+    """A negative seqused_kv: the header carries the sequence bit (and the
+    plan is empty) on both paths of the sequence phase (2 and 1100
+    sequences)."""
+    w = _decode_batch(1100) if case == "decode_b1100" else workload("tiny")
+    w.kv_used[1] = -1
+    t = device_tensors(w)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    m = run_metadata(w, t, 0, 0, status).cpu().numpy()
+    ref = scheduler.build(problem_dict(w, sm_count()), w.sparse_idx, w.sparse_count,
+                          w.cu_seqlens_q, w.q_used if w.has_seqused_q else None, w.kv_used)
+    assert int(ref[15]) & 0x01
+    assert int(m[15]) == int(ref[15]) == int(status.item())
+    mask = scheduler.defined_mask(ref)
+    assert np.array_equal(m[mask], ref[mask]), _first_diffs(m, ref, mask)
 
 
 def test_metadata_mismatch_leaves_output_untouched():
