@@ -214,6 +214,11 @@ __global__ void __launch_bounds__(kItemThreads) item_kernel(const MetaParams p) 
   bool staged = true;
   if constexpr (kOwnSeq) {
     const int t = threadIdx.x;
+    int64_t c0 = 0, cB = 0;  // the header's checks, loaded early
+    if (blockIdx.x == 0 && t == 0) {
+      c0 = p.cu_seqlens_q[0];
+      cB = p.cu_seqlens_q[p.B];
+    }
     if (t == 0) bad_sh = 0;
     int64_t nq[kOwnSeqPer];
     int64_t sum = 0;
@@ -258,7 +263,6 @@ __global__ void __launch_bounds__(kItemThreads) item_kernel(const MetaParams p) 
       }
       __syncthreads();  // bad_sh complete; the zeroed header before its fields
       if (t == 0) {
-        const int64_t c0 = p.cu_seqlens_q[0], cB = p.cu_seqlens_q[p.B];
         const int32_t st = (bad_sh || c0 != 0 || total != p.total_q_blocks ||
                             (p.T > 0 && cB != p.T) || cB > 0x7fffffffLL)
                                ? kDevBadSeqlen
@@ -404,6 +408,7 @@ __device__ __forceinline__ int64_t warp_sum_sat(int64_t v) {
 constexpr int kPlanSmemItems = 24576;
 constexpr int kKeyBits = 9;          // piece lengths 0..256 (and 257 as a query)
 constexpr int32_t kNoKey = 511;      // lanes past the warp's items
+constexpr int kKeyWarps = (kNumKeys + 31) / 32;  // warps holding one length per thread
 
 size_t plan_smem_bytes(int64_t n_items) {
   const int64_t c = n_items < kPlanSmemItems ? n_items : kPlanSmemItems;
@@ -427,6 +432,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const MetaParams p, 
   extern __shared__ __align__(16) unsigned char plan_dyn[];
   __shared__ int64_t part[kPlanWarps][3];  // per warp: units, slots, combine records
   __shared__ int64_t totals[3];
+  __shared__ int64_t key_warp_sum[kKeyWarps];
   __shared__ int32_t bucket_start[kNumKeys];
   __shared__ int32_t warp_key[kPlanWarps][kNumKeys];  // counts, then running cursors
   __shared__ int64_t cost_sh[kPlanWarps];
@@ -495,13 +501,20 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const MetaParams p, 
     }
     return;
   }
-  cost = 0;
-  for (int w = 0; w < kPlanWarps; w++) cost += cost_sh[w];
+  cost = cost_sh[lane];  // kPlanWarps == 32: one warp total per lane
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) cost += __shfl_xor_sync(0xffffffffu, cost, o);
   int64_t L64;
   if (p.forced_split > 0) {
     L64 = p.forced_split;
   } else {
-    L64 = cdiv64(cost, 4LL * p.num_ctas);
+    const int64_t d = 4LL * p.num_ctas;
+    if (cost <= 0xffffffffLL && d <= 0xffffffffLL) {  // a 32-bit division
+      const uint32_t q = (uint32_t)cost / (uint32_t)d;
+      L64 = (int64_t)q + ((uint32_t)cost - q * (uint32_t)d != 0u ? 1 : 0);
+    } else {
+      L64 = cdiv64(cost, d);
+    }
     if (L64 < kMinSplitLen) L64 = kMinSplitLen;
   }
   if (L64 > 0x7fffffffLL) L64 = 0x7fffffffLL;
@@ -512,12 +525,15 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const MetaParams p, 
     meta[H_COST_HI] = (int32_t)(uint32_t)((uint64_t)cost >> 32);
   }
 
-  const int32_t R = (n_items + kPlanWarps - 1) / kPlanWarps;
+  // each warp's range is a whole number of 32-item steps: fewer, fuller warps
+  const int32_t R = ((n_items + kPlanWarps - 1) / kPlanWarps + 31) / 32 * 32;
   const int32_t lo = warp * R < n_items ? warp * R : n_items;
   const int32_t hi = lo + R < n_items ? lo + R : n_items;
 
   // pass 2: per (warp, length) counts and per-warp totals
-  {
+  if (lo >= hi) {
+    if (lane == 0) part[warp][0] = part[warp][1] = part[warp][2] = 0;
+  } else {
     int64_t units = 0, slots = 0, combs = 0;
     for (int32_t i = lo + lane; i < hi; i += 32) {
       int32_t U, n;
@@ -542,16 +558,37 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const MetaParams p, 
   }
   __syncthreads();
 
-  // per length: offsets over warps, in place (threads 0..256); per warp:
-  // slot and combine bases (the last warp)
-  if (tid < kNumKeys) {
+  // per length: offsets over warps, in place, and the length's total; thread
+  // t < 257 takes length 256 - t, so the bucket starts (longest first) are an
+  // exclusive scan over threads: inside each of the 9 warps here, across them
+  // after the barrier.  The last warp scans the per-warp slot and combine
+  // counts.
+  int64_t key_excl = 0;
+  if (tid < kKeyWarps * 32) {
     int32_t acc = 0;
-    for (int w = 0; w < kPlanWarps; w++) {
-      const int32_t c = warp_key[w][tid];
-      warp_key[w][tid] = acc;
-      acc += c;
+    if (tid < kNumKeys) {
+      const int key = kNumKeys - 1 - tid;
+      // idle warps' counts are zero; loads batched ahead of the stores
+#pragma unroll
+      for (int w0 = 0; w0 < kPlanWarps; w0 += 16) {
+        int32_t c[16];
+#pragma unroll
+        for (int w = 0; w < 16; w++) c[w] = warp_key[w0 + w][key];
+#pragma unroll
+        for (int w = 0; w < 16; w++) {
+          warp_key[w0 + w][key] = acc;
+          acc += c[w];
+        }
+      }
     }
-    bucket_start[tid] = acc;  // the length's total until the scan below
+    int64_t incl = acc;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int64_t n = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += n;
+    }
+    key_excl = incl - acc;
+    if (lane == 31) key_warp_sum[warp] = incl;
   }
   if (warp == kPlanWarps - 1) {
     const int64_t u = part[lane][0], sl = part[lane][1], cb = part[lane][2];
@@ -577,38 +614,19 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const MetaParams p, 
     }
   }
   __syncthreads();
-  // bucket starts, longest first: lane l of warp 0 takes lengths
-  // 256 - 9 l - j (j = 0..8), a serial prefix over its nine, then a warp scan
-  if (warp == 0) {
-    constexpr int kPer = (kNumKeys + 31) / 32;
-    int32_t loc[kPer];
-    int64_t sum = 0;
+  if (tid < kNumKeys) {
 #pragma unroll
-    for (int j = 0; j < kPer; j++) {
-      const int key = kNumKeys - 1 - kPer * lane - j;
-      loc[j] = (int32_t)sum;
-      sum += key >= 0 ? bucket_start[key] : 0;
-    }
-    int64_t incl = sum;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int64_t n = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += n;
-    }
-    const int32_t excl = (int32_t)(incl - sum);
-#pragma unroll
-    for (int j = 0; j < kPer; j++) {
-      const int key = kNumKeys - 1 - kPer * lane - j;
-      if (key >= 0) bucket_start[key] = excl + loc[j];
-    }
-    if (lane == 0) {
-      const int64_t n_units = totals[0], n_slots = totals[1], n_comb = totals[2];
-      const bool over = n_units > g.unit_cap || n_slots > g.slot_cap || n_comb > g.comb_cap;
-      meta[H_NUNITS] = over ? 0 : (int32_t)n_units;
-      meta[H_NSLOTS] = over ? 0 : (int32_t)n_slots;
-      meta[H_NCOMB] = over ? 0 : (int32_t)n_comb;
-      if (over) raise_status(p, kDevCapacity);
-    }
+    for (int w = 0; w < kKeyWarps - 1; w++)
+      if (w < warp) key_excl += key_warp_sum[w];
+    bucket_start[kNumKeys - 1 - tid] = (int32_t)key_excl;
+  }
+  if (tid == 0) {
+    const int64_t n_units = totals[0], n_slots = totals[1], n_comb = totals[2];
+    const bool over = n_units > g.unit_cap || n_slots > g.slot_cap || n_comb > g.comb_cap;
+    meta[H_NUNITS] = over ? 0 : (int32_t)n_units;
+    meta[H_NSLOTS] = over ? 0 : (int32_t)n_slots;
+    meta[H_NCOMB] = over ? 0 : (int32_t)n_comb;
+    if (over) raise_status(p, kDevCapacity);
   }
   __syncthreads();
   if (totals[0] > g.unit_cap || totals[1] > g.slot_cap || totals[2] > g.comb_cap) return;
@@ -712,10 +730,15 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const MetaParams p, 
       if (s.k > 1)
         for (int32_t tp = 0; tp < s.U; tp++)
           comb[comb_base + tp] = make_int4(i, tp, slot_base + tp * s.k, s.k);
-      int32_t j0 = 0, longs = 0;
+      // piece q covers [floor(q n / k), floor((q + 1) n / k)); with n = a k + cA
+      // the bound advances by a, plus 1 when (q + 1) cA mod k wraps: the
+      // long pieces
+      int32_t j0 = 0, longs = 0, rem = 0;
       for (int32_t q = 0; q < s.k; q++) {
-        const int32_t j1 = (int32_t)((uint32_t)((q + 1) * s.n) / (uint32_t)s.k);
-        const bool is_long = j1 - j0 == s.a + 1 && s.cA;
+        rem += s.cA;
+        const bool is_long = rem >= s.k;
+        if (is_long) rem -= s.k;
+        const int32_t j1 = j0 + s.a + (is_long ? 1 : 0);
         const int32_t first = is_long ? startA + longs : startB + (q - longs);
         const int32_t stride = is_long ? s.cA : s.cB;
         for (int32_t tp = 0; tp < s.U; tp++)
