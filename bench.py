@@ -431,7 +431,10 @@ def measure(name, args, dev, world, rank, sampler, dist, headline):
     torch.cuda.synchronize()
     meta_host = meta_buf[:32].cpu().numpy()
     comb_cap = int(meta_host[10])
-    launches_per_step = 3 + 1 + (1 if comb_cap > 0 else 0)
+    # metadata (two kernels up to METADATA_FUSED_MAX_B sequences, else three),
+    # the forward, and the combine when the work list can hold split pieces
+    meta_launches = 2 if w.B <= gbsa.gbsa.METADATA_FUSED_MAX_B else 3
+    launches_per_step = meta_launches + 1 + (1 if comb_cap > 0 else 0)
 
     events = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     if world > 1:

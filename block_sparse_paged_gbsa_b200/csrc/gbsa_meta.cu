@@ -21,6 +21,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "gbsa.h"
 #include "gbsa_internal.cuh"
 
 namespace gbsa {
@@ -166,9 +167,10 @@ __global__ void __launch_bounds__(kSeqThreads) seq_kernel(const MetaParams p) {
 constexpr int kItemWarps = 8;
 constexpr int kItemThreads = kItemWarps * 32;
 constexpr int kItemSmemSeqs = 2048;  // sequences whose Q-block bases are staged
-constexpr int kOwnSeqMax = 1024;     // up to this many sequences, every item CTA
-                                     // derives the sequence table itself
+constexpr int kOwnSeqMax = GBSA_METADATA_FUSED_MAX_B;  // up to this many sequences,
+                                     // every item CTA derives the sequence table itself
 constexpr int kOwnSeqPer = kOwnSeqMax / kItemThreads;
+static_assert(kOwnSeqMax % kItemThreads == 0, "whole sequences per item thread");
 constexpr int kListChunks = kMaxTopK / 32;
 
 // Status bits of item i go to word i of the unit table (rows there are

@@ -109,6 +109,9 @@ class Problem:
 
 
 ABI_VERSION = 5
+# GBSA_METADATA_FUSED_MAX_B: up to this many sequences the metadata call is
+# two kernel launches, above it three.
+METADATA_FUSED_MAX_B = 1024
 DTYPE_BF16, DTYPE_FP16, DTYPE_FP8_E4M3 = 0, 1, 2
 
 

@@ -188,10 +188,16 @@ GBSA_API const char* gbsa_status_string(gbsa_status status);
  * Returns GBSA_ERR_NO_DEVICE if num_ctas == 0 and no device can be queried. */
 GBSA_API gbsa_status gbsa_metadata_size(const gbsa_problem* problem, size_t* bytes);
 
+/* Up to this many sequences (B) gbsa_metadata() launches two kernels on the
+ * stream (items with their own sequence phase, then the plan); above it,
+ * three (a sequence kernel first).  The bytes written are the same. */
+#define GBSA_METADATA_FUSED_MAX_B 1024
+
 /* Builds the work list for `problem` into the caller's device buffer `meta`
  * (16-byte aligned, meta_bytes >= gbsa_metadata_size()).  Reads
  * sparse_idx, sparse_count, cu_seqlens_q, seqused_q and seqused_kv; other
  * tensor fields may be NULL.  Deterministic: equal inputs give equal bytes.
+ * The buffer's previous content is irrelevant (nothing has to be zeroed).
  * GBSA article, "two-phase call" step 2 and "Constraints: metadata first". */
 GBSA_API gbsa_status gbsa_metadata(const gbsa_problem* problem, const gbsa_tensors* tensors,
                           void* meta, size_t meta_bytes, int32_t* dev_status, void* stream);

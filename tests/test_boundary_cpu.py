@@ -51,6 +51,14 @@ def _problem(**kw):
     return Problem(**base), w
 
 
+def test_header_constants_match_the_binding():
+    text = open(HEADER).read()
+    abi = int(re.search(r"#define GBSA_ABI_VERSION (\d+)", text).group(1))
+    fused = int(re.search(r"#define GBSA_METADATA_FUSED_MAX_B (\d+)", text).group(1))
+    assert abi == gbsa.gbsa.ABI_VERSION
+    assert fused == gbsa.gbsa.METADATA_FUSED_MAX_B
+
+
 def test_metadata_size_matches_format(lib):
     for ctas, forced in ((148, 0), (7, 3)):
         p, w = _problem(num_ctas=ctas, max_blocks_per_split=forced)
