@@ -364,6 +364,12 @@ def roofline(acc, fwd_ms, peaks, fp8, traffic):
         achieved = nbytes / (fwd_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": round(achieved, 3), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4)}
+    if tensor:
+        # the same rate against the seconds-long, power-capped GEMM figure, the
+        # fitting denominator when the timed region itself runs under the cap
+        t_sus = peaks["bf16_tflops_sustained"] * (2.0 if fp8 else 1.0)
+        roof["peak_sustained"] = round(t_sus, 3)
+        roof["frac_sustained"] = round(achieved / t_sus, 4)
     roof["traffic"] = traffic
     roof["kernel"] = "gbsa forward (attention + split-KV combine launch)"
     roof["peak_source"] = peaks["source"] + " (burst)" + (
