@@ -411,6 +411,8 @@ constexpr int kPlanSmemItems = 24576;
 constexpr int kKeyBits = 9;          // piece lengths 0..256 (and 257 as a query)
 constexpr int32_t kNoKey = 511;      // lanes past the warp's items
 constexpr int kKeyWarps = (kNumKeys + 31) / 32;  // warps holding one length per thread
+constexpr int kKeyRow = 36;                      // words per length in the (length, warp) table
+static_assert(kPlanWarps == 32 && kKeyRow % 4 == 0 && kKeyRow >= kPlanWarps, "table rows");
 
 size_t plan_smem_bytes(int64_t n_items) {
   const int64_t c = n_items < kPlanSmemItems ? n_items : kPlanSmemItems;
@@ -436,14 +438,18 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const MetaParams p, 
   __shared__ int64_t totals[3];
   __shared__ int64_t key_warp_sum[kKeyWarps];
   __shared__ int32_t bucket_start[kNumKeys];
-  __shared__ int32_t warp_key[kPlanWarps][kNumKeys];  // counts, then running cursors
+  // per (length, warp): counts, then running cursors.  A length's row is
+  // 36 words: its 32 warps in 8 aligned int4, rows 16 B apart modulo 128 B
+  // so that 8 lanes of a vector access reach 8 different bank groups.
+  __shared__ __align__(16) int32_t key_warp[kNumKeys][kKeyRow];
+  __shared__ int32_t split_len_sh;
   __shared__ int64_t cost_sh[kPlanWarps];
   __shared__ int32_t status_sh, item_bits_sh;
   int32_t* sU = reinterpret_cast<int32_t*>(plan_dyn);
   uint16_t* sN = reinterpret_cast<uint16_t*>(sU + cached);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  for (int i = tid; i < kPlanWarps * kNumKeys; i += blockDim.x) (&warp_key[0][0])[i] = 0;
+  for (int i = tid; i < kNumKeys * kKeyRow; i += blockDim.x) (&key_warp[0][0])[i] = 0;
   allow_dependents();
   grid_dependency_wait();  // the item table and live lists
   const Geometry& g = p.geo;
@@ -503,29 +509,34 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const MetaParams p, 
     }
     return;
   }
-  cost = cost_sh[lane];  // kPlanWarps == 32: one warp total per lane
+  // the split length, once (warp 0)
+  if (warp == 0) {
+    cost = cost_sh[lane];  // kPlanWarps == 32: one warp total per lane
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) cost += __shfl_xor_sync(0xffffffffu, cost, o);
-  int64_t L64;
-  if (p.forced_split > 0) {
-    L64 = p.forced_split;
-  } else {
-    const int64_t d = 4LL * p.num_ctas;
-    if (cost <= 0xffffffffLL && d <= 0xffffffffLL) {  // a 32-bit division
-      const uint32_t q = (uint32_t)cost / (uint32_t)d;
-      L64 = (int64_t)q + ((uint32_t)cost - q * (uint32_t)d != 0u ? 1 : 0);
-    } else {
-      L64 = cdiv64(cost, d);
+    for (int o = 16; o > 0; o >>= 1) cost += __shfl_xor_sync(0xffffffffu, cost, o);
+    if (lane == 0) {
+      int64_t L64;
+      if (p.forced_split > 0) {
+        L64 = p.forced_split;
+      } else {
+        const int64_t d = 4LL * p.num_ctas;
+        if (cost <= 0xffffffffLL && d <= 0xffffffffLL) {  // a 32-bit division
+          const uint32_t q = (uint32_t)cost / (uint32_t)d;
+          L64 = (int64_t)q + ((uint32_t)cost - q * (uint32_t)d != 0u ? 1 : 0);
+        } else {
+          L64 = cdiv64(cost, d);
+        }
+        if (L64 < kMinSplitLen) L64 = kMinSplitLen;
+      }
+      if (L64 > 0x7fffffffLL) L64 = 0x7fffffffLL;
+      split_len_sh = (int32_t)L64;
+      meta[H_SPLIT_LEN] = (int32_t)L64;
+      meta[H_COST_LO] = (int32_t)(uint32_t)(cost & 0xffffffffLL);
+      meta[H_COST_HI] = (int32_t)(uint32_t)((uint64_t)cost >> 32);
     }
-    if (L64 < kMinSplitLen) L64 = kMinSplitLen;
   }
-  if (L64 > 0x7fffffffLL) L64 = 0x7fffffffLL;
-  const int32_t L = (int32_t)L64;
-  if (tid == 0) {
-    meta[H_SPLIT_LEN] = L;
-    meta[H_COST_LO] = (int32_t)(uint32_t)(cost & 0xffffffffLL);
-    meta[H_COST_HI] = (int32_t)(uint32_t)((uint64_t)cost >> 32);
-  }
+  __syncthreads();
+  const int32_t L = split_len_sh;
 
   // each warp's range is a whole number of 32-item steps: fewer, fuller warps
   const int32_t R = ((n_items + kPlanWarps - 1) / kPlanWarps + 31) / 32 * 32;
@@ -541,8 +552,8 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const MetaParams p, 
       int32_t U, n;
       fields(i, U, n);
       const PieceShape s = piece_shape(U, n, L);
-      atomicAdd(&warp_key[warp][s.a], s.U * s.cB);  // cB >= 1
-      if (s.cA) atomicAdd(&warp_key[warp][s.a + 1], s.U * s.cA);
+      atomicAdd(&key_warp[s.a][warp], s.U * s.cB);  // cB >= 1
+      if (s.cA) atomicAdd(&key_warp[s.a + 1][warp], s.U * s.cA);
       units += (int64_t)s.U * s.k;
       if (s.k > 1) {
         slots += (int64_t)s.U * s.k;
@@ -570,17 +581,21 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const MetaParams p, 
     int32_t acc = 0;
     if (tid < kNumKeys) {
       const int key = kNumKeys - 1 - tid;
-      // idle warps' counts are zero; loads batched ahead of the stores
+      // the length's 32 warp counts (idle warps' are zero) in 8 vector loads
+      int4* row = reinterpret_cast<int4*>(&key_warp[key][0]);
+      int4 c[kPlanWarps / 4];
 #pragma unroll
-      for (int w0 = 0; w0 < kPlanWarps; w0 += 16) {
-        int32_t c[16];
+      for (int v = 0; v < kPlanWarps / 4; v++) c[v] = row[v];
 #pragma unroll
-        for (int w = 0; w < 16; w++) c[w] = warp_key[w0 + w][key];
-#pragma unroll
-        for (int w = 0; w < 16; w++) {
-          warp_key[w0 + w][key] = acc;
-          acc += c[w];
-        }
+      for (int v = 0; v < kPlanWarps / 4; v++) {
+        const int4 x = c[v];
+        int4 e;
+        e.x = acc;
+        e.y = acc + x.x;
+        e.z = e.y + x.y;
+        e.w = e.z + x.z;
+        acc = e.w + x.w;
+        row[v] = e;
       }
     }
     int64_t incl = acc;
@@ -654,9 +669,9 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const MetaParams p, 
       // rank = U0 x (earlier lanes with the same n)
       const uint32_t same = __match_any_sync(0xffffffffu, a);
       int32_t start = 0;
-      if (valid) start = bucket_start[a] + warp_key[warp][a] + U0 * __popc(same & lt);
+      if (valid) start = bucket_start[a] + key_warp[a][warp] + U0 * __popc(same & lt);
       __syncwarp();
-      if (valid && !(same & gt)) warp_key[warp][a] += U0 * __popc(same);
+      if (valid && !(same & gt)) key_warp[a][warp] += U0 * __popc(same);
       __syncwarp();
       if (valid)
         for (int32_t tp = 0; tp < U0; tp++) units[start + tp] = make_int4(i, tp, s.n << 16, -1);
@@ -718,14 +733,14 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const MetaParams p, 
     }
     int32_t startA = 0, startB = 0;
     if (valid) {
-      startB = bucket_start[a] + warp_key[warp][a] + preB;
-      if (s.cA) startA = bucket_start[a + 1] + warp_key[warp][a + 1] + preA;
+      startB = bucket_start[a] + key_warp[a][warp] + preB;
+      if (s.cA) startA = bucket_start[a + 1] + key_warp[a + 1][warp] + preA;
     }
     __syncwarp();
     // the last lane of each key group advances the warp's cursors
     if (valid && !(same & gt)) {
-      atomicAdd(&warp_key[warp][a], sB);
-      if (sA) atomicAdd(&warp_key[warp][a + 1], sA);
+      atomicAdd(&key_warp[a][warp], sB);
+      if (sA) atomicAdd(&key_warp[a + 1][warp], sA);
     }
     __syncwarp();
     if (valid) {
