@@ -422,16 +422,19 @@ size_t plan_smem_bytes(int64_t n_items) {
 // The piece order is a stable counting sort of all pieces by length, longest
 // first; inside a length, pieces follow their item, then tile pair, then
 // their place in the item's split.  Warp w owns the contiguous item range
-// [w R, (w + 1) R) (R = ceil(items / 32)) and walks it 32 items at a time, so
+// [w R, (w + 1) R), R = ceil(items / 32) rounded up to a multiple of 32 (so
+// small lists use fewer, fuller warps), and walks it 32 items at a time, so
 // item order is (warp, step, lane) order:
-//   pass 2  per (warp, length) piece counts, per-warp unit / slot / combine
+//   pass 2  per (length, warp) piece counts, per-warp unit / slot / combine
 //           totals;
-//   scan    bucket starts (lengths descending), per-(warp, length) offsets
+//   scan    bucket starts (lengths descending), per-(length, warp) offsets
 //           (warps ascending), per-warp slot and combine bases;
 //   pass 3  each warp places its pieces with no block barrier: a piece's
 //           rank inside its length is the warp's running cursor for that
 //           length plus the weights of earlier lanes of the same step with
-//           that length, taken by pointer jumping over lanes of equal keys.
+//           that length -- by match_any and a popcount when no lane splits
+//           and all have equal tile pairs, else by pointer jumping over
+//           lanes of equal keys.
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const MetaParams p, int32_t cached) {
   extern __shared__ __align__(16) unsigned char plan_dyn[];
   __shared__ int64_t part[kPlanWarps][3];  // per warp: units, slots, combine records
