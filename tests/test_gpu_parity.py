@@ -290,3 +290,15 @@ def test_full_size_sampled_rows(name):
     assert torch.isfinite(out.float()).all()
     rows = _sample_rows(w, 3000, seed=1)
     _compare(w, q, kf, vf, out, lse, rows)
+
+
+@pytest.mark.parametrize("B,forced", [(1500, 0), (1500, 3), (2500, 0)])
+def test_forward_with_many_sequences(B, forced):
+    """Above 1024 sequences the sequence table comes from its own kernel (and
+    above 2048 the item kernel looks it up in global memory): the forward on
+    that work list matches the oracle on every row."""
+    w = _decode_batch(B)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    q, kf, vf, meta, out, lse = run_gpu(w, forced=forced, dev_status=status)
+    assert int(status.item()) == 0
+    _compare(w, q, kf, vf, out, lse)
