@@ -190,6 +190,8 @@ def generate(*, name="custom", seed=0, q_storage, q_used=None, kv_used=None, N1,
                     elif selection == "sink_diag_random":
                         if nc <= top_k:
                             chosen = list(range(nc))
+                        elif top_k == 1:            # room for the diagonal block only
+                            chosen = [diag]
                         else:
                             chosen = [0, diag] + list(_choose(rng, np.arange(1, diag), top_k - 2))
                     elif selection == "random_causal":

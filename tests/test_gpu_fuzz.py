@@ -1,0 +1,114 @@
+"""Seeded random problems across the parameter space: group sizes 1..16, Q
+block sizes from 1 to 200 tokens (several tiles, one tile, narrow tiles),
+empty and partly used sequences, KV lengths with partial last pages or no
+keys at all, sliding windows, every selection kind and list order, garbage
+past each count, forced split lengths, CTA counts from 1 to 148, bf16, fp16
+and E4M3, strided page pools.  For each: the work list is word for word the
+sequential rebuild's (device status included), and sampled rows of out and
+lse match the fp64 oracle: bf16 and fp16 under the output rule (raw 1e-2
+where |exact| < 2, plus half a 16-bit ulp above) and the 1e-3 lse rule, E4M3
+under its bound (R22, as in test_gpu_fp8)."""
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_paged_gbsa_b200 as gbsa
+from block_sparse_paged_gbsa_b200.workloads import PAGE, generate, make_values, pool_view
+from oracle import scheduler
+from tests.gpu_helpers import device_tensors, problem_dict, run_forward, run_metadata, sm_count
+from tests.helpers import assert_lse_close, assert_out_close, oracle_rows, oracle_rows_fp8
+
+pytestmark = pytest.mark.gpu
+
+N_CASES = 150
+FP8_SCALES = (0.37, 1.9, 0.61)  # q, k, v dequantization scales
+
+
+def fuzz_case(k: int):
+    """(workload, dtype, num_ctas, forced split length) of case k."""
+    rng = np.random.default_rng(7000 + k)
+    N2 = int(rng.choice([1, 2, 4]))
+    G = int(rng.choice([1, 2, 3, 4, 5, 7, 8, 16]))
+    block_x = int(rng.choice([1, 5, 16, 32, 64, 128, 200]))
+    B = int(rng.integers(1, 5))
+    qs = rng.integers(0, 600, size=B)
+    if qs.sum() == 0:
+        qs[0] = 1
+    qu = np.array([int(rng.integers(0, q + 1)) if rng.random() < 0.3 else int(q) for q in qs])
+    ku = np.array([max(0, int(u) + int(rng.integers(-50, 400))) if rng.random() < 0.85
+                   else int(rng.integers(0, 3)) for u in qu])
+    selection = str(rng.choice(["random_causal", "random_any", "all_causal", "sink_diag_random"]))
+    window = rng.random() < 0.4
+    w = generate(name=f"fuzz{k}", seed=5000 + k, q_storage=qs, q_used=qu, kv_used=ku,
+                 N1=N2 * G, N2=N2, block_x=block_x, top_k=int(rng.integers(1, 25)),
+                 selection=selection, win_left=int(rng.integers(0, 500)) if window else -1,
+                 win_right=0 if window else -1,
+                 page_stride_factor=float(rng.choice([1.0, 1.0, 1.5])),
+                 list_order=str(rng.choice(["ascending", "descending", "shuffled"])))
+    r = rng.random()
+    dtype = torch.float8_e4m3fn if r < 0.2 else (torch.float16 if r < 0.45 else torch.bfloat16)
+    ctas = int(rng.choice([0, 1, 7, 148]))
+    forced = int(rng.choice([0, 0, 1, 2, 3]))
+    return w, dtype, ctas, forced
+
+
+def _rows(w, n=1500, seed=0):
+    rng = np.random.default_rng(seed)
+    ends = np.concatenate([w.cu_seqlens_q[:-1], w.cu_seqlens_q[1:] - 1])
+    tok = np.concatenate([rng.integers(0, w.T, n), ends[(ends >= 0) & (ends < w.T)]])
+    return np.stack([tok, rng.integers(0, w.N1, tok.size)], 1).astype(np.int64)
+
+
+@pytest.mark.parametrize("k", range(N_CASES))
+def test_fuzz_case(k):
+    w, dtype, ctas, forced = fuzz_case(k)
+    t = device_tensors(w)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    meta = run_metadata(w, t, ctas, forced, status)
+    ref = scheduler.build(problem_dict(w, ctas or sm_count(), forced), w.sparse_idx,
+                          w.sparse_count, w.cu_seqlens_q, w.q_used if w.has_seqused_q else None,
+                          w.kv_used)
+    m = meta.cpu().numpy()
+    mask = scheduler.defined_mask(ref)
+    assert m.size == ref.size and np.array_equal(m[mask], ref[mask])
+    assert int(status.item()) == int(ref[15])
+    q, kf, vf = make_values(w, "cuda", dtype=dtype)
+    rows = _rows(w, seed=k)
+    if dtype == torch.float8_e4m3fn:
+        out, lse = gbsa.forward(q, pool_view(w, kf), pool_view(w, vf), t["idx"], t["cnt"],
+                                [w.block_x, 128], metadata=meta, cu_seqlens_q=t["cu"],
+                                seqused_q=t["squ"], seqused_kv=t["sku"], block_table=t["bt"],
+                                softmax_scale=w.scale, win_left=w.win_left,
+                                win_right=w.win_right, return_softmax_lse=True, num_ctas=ctas,
+                                max_blocks_per_split=forced, q_dequant_scale=FP8_SCALES[0],
+                                k_dequant_scale=FP8_SCALES[1], v_dequant_scale=FP8_SCALES[2])
+        torch.cuda.synchronize()
+        _check_e4m3(w, q, kf, vf, out, lse, rows)
+        return
+    out, lse = run_forward(w, q, kf, vf, t, meta, num_ctas=ctas, forced=forced)
+    torch.cuda.synchronize()
+    assert out.dtype == dtype
+    ro, rl = oracle_rows(w, q.cpu(), kf.cpu(), vf.cpu(), rows)
+    o = out.float().cpu().numpy().astype(np.float64)[rows[:, 0], rows[:, 1]]
+    l = lse.float().cpu().numpy()[..., 0].astype(np.float64)[rows[:, 0], rows[:, 1]]
+    assert_out_close(o, ro)
+    assert_lse_close(l, rl)
+
+
+def _check_e4m3(w, q, kf, vf, out, lse, rows):
+    """The E4M3 bound of test_gpu_fp8 (the weights' E4M3 cast: 2^-4 of
+    out_abs, 2^-10 of the smallest weights; bf16 out; fp32 sums); the mean
+    error condition only where enough rows see a key."""
+    assert out.dtype == torch.bfloat16
+    ro, rl, ra = oracle_rows_fp8(w, q.cpu(), kf.cpu(), vf.cpu(), FP8_SCALES, rows)
+    o = out.float().cpu().numpy().astype(np.float64)[rows[:, 0], rows[:, 1]]
+    l = lse.float().cpu().numpy()[..., 0].astype(np.float64)[rows[:, 0], rows[:, 1]]
+    assert_lse_close(l, rl)
+    fin = np.isfinite(rl)
+    assert (o[~fin] == 0).all()
+    vmax = float(vf.float().nan_to_num(0.0).abs().max()) * abs(FP8_SCALES[2])
+    bound = (2.0 ** -4 + 1e-5) * ra + 2.0 ** -9 * np.abs(ro) + 2.0 ** -18 * w.top_k * PAGE * vmax
+    err = np.abs(o - ro)
+    assert (err <= bound).all(), f"max excess {np.max(err - bound):.3g}"
+    if fin.sum() >= 100:
+        assert err[fin].mean() <= 0.25 * ((2.0 ** -4) * ra[fin]).mean()
