@@ -7,15 +7,16 @@ and E4M3, strided page pools.  For each: the work list is word for word the
 sequential rebuild's (device status included), and sampled rows of out and
 lse match the fp64 oracle: bf16 and fp16 under the output rule (raw 1e-2
 where |exact| < 2, plus half a 16-bit ulp above) and the 1e-3 lse rule, E4M3
-under its bound (R22, as in test_gpu_fp8)."""
+under its bound (R22, as in test_gpu_fp8).  The same keys in the non-paged
+TND layout (NaN rows between the sequences) give bit-identical out and lse."""
 import numpy as np
 import pytest
 import torch
 
 import block_sparse_paged_gbsa_b200 as gbsa
-from block_sparse_paged_gbsa_b200.workloads import PAGE, generate, make_values, pool_view
+from block_sparse_paged_gbsa_b200.workloads import PAGE, generate, make_values, pool_view, tnd_kv
 from oracle import scheduler
-from tests.gpu_helpers import device_tensors, problem_dict, run_forward, run_metadata, sm_count
+from tests.gpu_helpers import device_tensors, problem_dict, run_metadata, sm_count
 from tests.helpers import assert_lse_close, assert_out_close, oracle_rows, oracle_rows_fp8
 
 pytestmark = pytest.mark.gpu
@@ -74,19 +75,27 @@ def test_fuzz_case(k):
     assert int(status.item()) == int(ref[15])
     q, kf, vf = make_values(w, "cuda", dtype=dtype)
     rows = _rows(w, seed=k)
-    if dtype == torch.float8_e4m3fn:
-        out, lse = gbsa.forward(q, pool_view(w, kf), pool_view(w, vf), t["idx"], t["cnt"],
-                                [w.block_x, 128], metadata=meta, cu_seqlens_q=t["cu"],
-                                seqused_q=t["squ"], seqused_kv=t["sku"], block_table=t["bt"],
-                                softmax_scale=w.scale, win_left=w.win_left,
-                                win_right=w.win_right, return_softmax_lse=True, num_ctas=ctas,
-                                max_blocks_per_split=forced, q_dequant_scale=FP8_SCALES[0],
-                                k_dequant_scale=FP8_SCALES[1], v_dequant_scale=FP8_SCALES[2])
+    fp8 = dtype == torch.float8_e4m3fn
+    scales = dict(q_dequant_scale=FP8_SCALES[0], k_dequant_scale=FP8_SCALES[1],
+                  v_dequant_scale=FP8_SCALES[2]) if fp8 else {}
+
+    def forward(k_, v_, **layout):
+        o_, l_ = gbsa.forward(q, k_, v_, t["idx"], t["cnt"], [w.block_x, 128], metadata=meta,
+                              cu_seqlens_q=t["cu"], seqused_q=t["squ"], seqused_kv=t["sku"],
+                              softmax_scale=w.scale, win_left=w.win_left, win_right=w.win_right,
+                              return_softmax_lse=True, num_ctas=ctas,
+                              max_blocks_per_split=forced, **scales, **layout)
         torch.cuda.synchronize()
+        return o_, l_
+
+    out, lse = forward(pool_view(w, kf), pool_view(w, vf), block_table=t["bt"])
+    kt, vt, cu_kv = tnd_kv(w, kf, vf, seed=k)
+    if cu_kv[-1] > 0:  # a TND K/V array needs at least one row
+        to, tl = forward(kt, vt, cu_seqlens_kv=torch.as_tensor(cu_kv, device="cuda"))
+        assert torch.equal(out, to) and torch.equal(lse, tl)
+    if fp8:
         _check_e4m3(w, q, kf, vf, out, lse, rows)
         return
-    out, lse = run_forward(w, q, kf, vf, t, meta, num_ctas=ctas, forced=forced)
-    torch.cuda.synchronize()
     assert out.dtype == dtype
     ro, rl = oracle_rows(w, q.cpu(), kf.cpu(), vf.cpu(), rows)
     o = out.float().cpu().numpy().astype(np.float64)[rows[:, 0], rows[:, 1]]
