@@ -211,6 +211,35 @@ def keys_bound(w, rows):
     return cnt.astype(np.float64) * PAGE
 
 
+def r24_lse_bound(n_keys, ref_lse):
+    """Per-row bound of |lse - exact| under R24 (softmaxPrecision 1).  lse =
+    ln2 * (m + log2 l) with l the fp32 sum of the f16 weights P_p = 2^x_p; a
+    weight's relative error is at most 2^-9.9 (ex2.approx.f16) plus
+    ln2 * 2^-11 * |x_p| (the f16 rounding of x_p), |x_p| <= 8 (the reference
+    lag) + log2(e) (M - S_p).  The error of l relative to l is the weighted
+    mean of those, and the softmax-weighted mean of M - S_p is at most ln n
+    (the weights' entropy ln Z + E[M - S] is at most ln n, with Z >= 1), so
+    |ln(l' / l)| <= (1 + 2^-8) (2^-9.9 + ln2 2^-11 (8 + log2 n)); weights
+    below the f16 range lose at most n 2^-24 of l >= 1; fp32 arithmetic
+    adds 1e-5 |lse|."""
+    n = np.maximum(np.asarray(n_keys, np.float64), 1.0)
+    rel = (1.0 + 2.0 ** -8) * (2.0 ** -9.9 + math.log(2.0) * 2.0 ** -11 * (8.0 + np.log2(n)))
+    r = np.asarray(ref_lse, np.float64)
+    return rel + n * 2.0 ** -24 + 1e-5 * np.abs(np.where(np.isfinite(r), r, 0.0))
+
+
+def assert_lse_close_r24(gpu_lse, ref_lse, n_keys):
+    """lse under r24_lse_bound, with the same -inf pattern."""
+    g = np.asarray(gpu_lse, np.float64)
+    r = np.asarray(ref_lse, np.float64)
+    inf_r = np.isneginf(r)
+    assert np.array_equal(np.isneginf(g), inf_r), "lse: -inf pattern differs"
+    fin = ~inf_r
+    if fin.any():
+        excess = np.abs(g[fin] - r[fin]) - r24_lse_bound(np.asarray(n_keys)[fin], r[fin])
+        assert (excess <= 0).all(), f"lse: max excess over the R24 bound {excess.max():.3g}"
+
+
 def r24_bound(dtype, ref, out_abs, gap_abs, n_keys, vmax):
     """The per-element bound of reading R24 (softmaxPrecision 1; derivation in
     tests/test_gpu_softmax_precision.py): the f16 exponent and exponential

@@ -8,7 +8,11 @@ sequential rebuild's (device status included), and sampled rows of out and
 lse match the fp64 oracle: bf16 and fp16 under the output rule (raw 1e-2
 where |exact| < 2, plus half a 16-bit ulp above) and the 1e-3 lse rule, E4M3
 under its bound (R22, as in test_gpu_fp8).  The same keys in the non-paged
-TND layout (NaN rows between the sequences) give bit-identical out and lse."""
+TND layout (NaN rows between the sequences) give bit-identical out and lse.
+softmaxPrecision 1 on the same inputs stays within its R24 bound (as in
+test_gpu_softmax_precision)."""
+import math
+
 import numpy as np
 import pytest
 import torch
@@ -17,7 +21,9 @@ import block_sparse_paged_gbsa_b200 as gbsa
 from block_sparse_paged_gbsa_b200.workloads import PAGE, generate, make_values, pool_view, tnd_kv
 from oracle import scheduler
 from tests.gpu_helpers import device_tensors, problem_dict, run_metadata, sm_count
-from tests.helpers import assert_lse_close, assert_out_close, oracle_rows, oracle_rows_fp8
+from tests.helpers import (assert_lse_close, assert_lse_close_r24, assert_out_close, keys_bound,
+                           oracle_rows, oracle_rows_fp8, r24_bound)
+from tests.test_gpu_softmax_precision import _oracle as oracle_mode1
 
 pytestmark = pytest.mark.gpu
 
@@ -79,14 +85,18 @@ def test_fuzz_case(k):
     scales = dict(q_dequant_scale=FP8_SCALES[0], k_dequant_scale=FP8_SCALES[1],
                   v_dequant_scale=FP8_SCALES[2]) if fp8 else {}
 
-    def forward(k_, v_, **layout):
+    def forward(k_, v_, mode=0, **layout):
         o_, l_ = gbsa.forward(q, k_, v_, t["idx"], t["cnt"], [w.block_x, 128], metadata=meta,
                               cu_seqlens_q=t["cu"], seqused_q=t["squ"], seqused_kv=t["sku"],
                               softmax_scale=w.scale, win_left=w.win_left, win_right=w.win_right,
                               return_softmax_lse=True, num_ctas=ctas,
-                              max_blocks_per_split=forced, **scales, **layout)
+                              max_blocks_per_split=forced, softmax_precision=mode, **scales,
+                              **layout)
         torch.cuda.synchronize()
         return o_, l_
+
+    o1, l1 = forward(pool_view(w, kf), pool_view(w, vf), mode=1, block_table=t["bt"])
+    _check_mode1(w, q, kf, vf, o1, l1, rows, dtype)
 
     out, lse = forward(pool_view(w, kf), pool_view(w, vf), block_table=t["bt"])
     kt, vt, cu_kv = tnd_kv(w, kf, vf, seed=k)
@@ -121,3 +131,24 @@ def _check_e4m3(w, q, kf, vf, out, lse, rows):
     assert (err <= bound).all(), f"max excess {np.max(err - bound):.3g}"
     if fin.sum() >= 100:
         assert err[fin].mean() <= 0.25 * ((2.0 ** -4) * ra[fin]).mean()
+
+
+def _check_mode1(w, q, kf, vf, out, lse, rows, dtype):
+    """softmaxPrecision 1 under R24 (per element; the mean error condition
+    only where enough rows see a key)."""
+    name = {torch.bfloat16: "bf16", torch.float16: "fp16", torch.float8_e4m3fn: "e4m3"}[dtype]
+    scales = FP8_SCALES if name == "e4m3" else (1.0, 1.0, 1.0)
+    ro, rl, oa, ga = oracle_mode1(w, q, kf, vf, rows, scales)
+    o = out.float().cpu().numpy().astype(np.float64)[rows[:, 0], rows[:, 1]]
+    l = lse.float().cpu().numpy()[..., 0].astype(np.float64)[rows[:, 0], rows[:, 1]]
+    assert_lse_close_r24(l, rl, keys_bound(w, rows))
+    fin = np.isfinite(rl)
+    assert (o[~fin] == 0).all()
+    vmax = float(vf.float().nan_to_num(0.0).abs().max()) * abs(scales[2])
+    bound = r24_bound(name, ro, oa, ga, keys_bound(w, rows), vmax)
+    err = np.abs(o - ro)
+    assert (err <= bound).all(), f"mode 1: max excess {np.max(err - bound):.3g}"
+    if fin.sum() >= 100:
+        mean_scale = (2.0 ** -4 * oa if name == "e4m3" else
+                      2.0 * ((2.0 ** -9.9 + 8 * math.log(2) * 2.0 ** -11) * oa + 2.0 ** -11 * ga))
+        assert err[fin].mean() <= 0.25 * mean_scale[fin].mean()

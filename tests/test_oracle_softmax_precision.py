@@ -4,9 +4,11 @@ is attainable: a numpy emulation of the mode's arithmetic -- keys in list
 order, blocks of 128, the running reference max with the lazy threshold of 8,
 the exponent rounded to f16 and its exponential rounded to f16, fp32 row sums
 of those weights, P rounded to the element type for the product -- stays
-within the bound against the fp64 oracle, with a mean error well below it.
-And the bound has teeth: the same emulation with the two weights of each f16
-pair swapped (a plausible packing mistake) breaks it on the same rows."""
+within the bound against the fp64 oracle, with a mean error well below it,
+and its lse within the R24 lse bound.  And the bounds have teeth: the same
+emulation with the two weights of each f16 pair swapped (a plausible packing
+mistake) breaks the output bound on the same rows, and its lse left in log2
+units breaks the lse bound."""
 import math
 
 import numpy as np
@@ -14,7 +16,8 @@ import pytest
 import torch
 
 from block_sparse_paged_gbsa_b200.workloads import PAGE, bf16_bits, workload
-from tests.helpers import keys_bound, logical_kv, r24_bound, to_f64
+from tests.helpers import (assert_lse_close_r24, keys_bound, logical_kv, r24_bound,
+                           r24_lse_bound, to_f64)
 
 LOG2E = 1.0 / math.log(2.0)
 
@@ -28,13 +31,14 @@ def _f16(x):
     return np.asarray(x, np.float32).astype(np.float16).astype(np.float64)
 
 
-def _emulate(w, q, kf, vf, rows, dtype, round_exponent=_f16, swap_pairs=False):
+def _emulate(w, q, kf, vf, rows, dtype, round_exponent=_f16, swap_pairs=False, with_lse=False):
     dt = "bf16" if q.dtype == torch.bfloat16 else "fp16"
     qd = to_f64(bf16_bits(q), dt)
     kb, vb = bf16_bits(kf), bf16_bits(vf)
     qbase = np.concatenate([[0], np.cumsum(-(-np.diff(w.cu_seqlens_q) // w.block_x))])
     scale_log2 = np.float32(w.scale * LOG2E)
     out = np.zeros((rows.shape[0], w.D))
+    lse = np.full(rows.shape[0], -np.inf)
     cache = {}
     for i, (tg, h) in enumerate(rows):
         b = int(np.searchsorted(w.cu_seqlens_q, tg, side="right") - 1)
@@ -85,7 +89,8 @@ def _emulate(w, q, kf, vf, rows, dtype, round_exponent=_f16, swap_pairs=False):
             acc = acc + Pu @ V[p, kvh, :]
         if lsum > 0:
             out[i] = acc / float(lsum)
-    return out
+            lse[i] = (m + math.log2(float(lsum))) * math.log(2.0)
+    return (out, lse) if with_lse else out
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "fp16"])
@@ -108,7 +113,7 @@ def test_r24_bound_attainable_by_emulation(name, dtype):
         seqused_kv=w.kv_used, block_table=w.block_table, block_x=w.block_x, scale=w.scale,
         win_left=w.win_left, win_right=w.win_right, rows=rows, dtype=dtype, out_abs=oa,
         gap_abs=ga)
-    em = _emulate(w, q, kf, vf, rows, dtype)
+    em, em_lse = _emulate(w, q, kf, vf, rows, dtype, with_lse=True)
     vmax = float(vf.float().nan_to_num(0.0).abs().max())
     bound = r24_bound(dtype, ro, oa, ga, keys_bound(w, rows), vmax)
     err = np.abs(em - ro)
@@ -119,3 +124,10 @@ def test_r24_bound_attainable_by_emulation(name, dtype):
     # swapped pair halves break the bound on these rows
     bad = _emulate(w, q, kf, vf, rows, dtype, swap_pairs=True)
     assert (np.abs(bad - ro) > bound).any()
+    # the lse bound of R24 holds for the same arithmetic, and an lse left in
+    # log2 units (the running max is kept in log2 units) breaks it
+    n_keys = keys_bound(w, rows)
+    assert_lse_close_r24(em_lse, rl, n_keys)
+    fin = np.isfinite(rl)
+    bad_lse = em_lse[fin] / math.log(2.0)
+    assert (np.abs(bad_lse - rl[fin]) > r24_lse_bound(n_keys[fin], rl[fin])).any()
