@@ -8,7 +8,8 @@ sequential rebuild's (device status included), and sampled rows of out and
 lse match the fp64 oracle: bf16 and fp16 under the output rule (raw 1e-2
 where |exact| < 2, plus half a 16-bit ulp above) and the 1e-3 lse rule, E4M3
 under its bound (R22, as in test_gpu_fp8).  The same keys in the non-paged
-TND layout (NaN rows between the sequences) give bit-identical out and lse.
+TND layout (NaN rows between the sequences) give bit-identical out and lse,
+and so does a call without the lse output (out).
 softmaxPrecision 1 on the same inputs stays within its R24 bound (as in
 test_gpu_softmax_precision)."""
 import math
@@ -85,11 +86,11 @@ def test_fuzz_case(k):
     scales = dict(q_dequant_scale=FP8_SCALES[0], k_dequant_scale=FP8_SCALES[1],
                   v_dequant_scale=FP8_SCALES[2]) if fp8 else {}
 
-    def forward(k_, v_, mode=0, **layout):
+    def forward(k_, v_, mode=0, with_lse=True, **layout):
         o_, l_ = gbsa.forward(q, k_, v_, t["idx"], t["cnt"], [w.block_x, 128], metadata=meta,
                               cu_seqlens_q=t["cu"], seqused_q=t["squ"], seqused_kv=t["sku"],
                               softmax_scale=w.scale, win_left=w.win_left, win_right=w.win_right,
-                              return_softmax_lse=True, num_ctas=ctas,
+                              return_softmax_lse=with_lse, num_ctas=ctas,
                               max_blocks_per_split=forced, softmax_precision=mode, **scales,
                               **layout)
         torch.cuda.synchronize()
@@ -99,6 +100,9 @@ def test_fuzz_case(k):
     _check_mode1(w, q, kf, vf, o1, l1, rows, dtype)
 
     out, lse = forward(pool_view(w, kf), pool_view(w, vf), block_table=t["bt"])
+    # without the lse output, out is the same
+    o_nl, _ = forward(pool_view(w, kf), pool_view(w, vf), with_lse=False, block_table=t["bt"])
+    assert torch.equal(out, o_nl)
     kt, vt, cu_kv = tnd_kv(w, kf, vf, seed=k)
     if cu_kv[-1] > 0:  # a TND K/V array needs at least one row
         to, tl = forward(kt, vt, cu_seqlens_kv=torch.as_tensor(cu_kv, device="cuda"))
