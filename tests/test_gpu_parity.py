@@ -12,8 +12,7 @@ import torch
 import block_sparse_paged_gbsa_b200 as gbsa
 from block_sparse_paged_gbsa_b200.workloads import generate, make_values, pool_view, workload
 from oracle import scheduler
-from tests.gpu_helpers import (device_tensors, problem_dict, run_forward, run_gpu, run_metadata,
-                               sm_count)
+from tests.gpu_helpers import device_tensors, problem_dict, run_gpu, run_metadata, sm_count
 from tests.helpers import assert_lse_close, assert_out_close, oracle_all, oracle_rows
 
 pytestmark = pytest.mark.gpu
