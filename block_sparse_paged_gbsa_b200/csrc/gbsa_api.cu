@@ -21,7 +21,7 @@ namespace gbsa {
 cudaError_t launch_metadata(const MetaParams& p, cudaStream_t stream);
 size_t forward_smem_bytes();
 cudaError_t launch_forward(const CUtensorMap& map_q, const CUtensorMap& map_k,
-                           const CUtensorMap& map_v, const int32_t* meta,
+                           const CUtensorMap& map_v, int32_t* meta,
                            const int32_t* block_table, const int64_t* cu_seqlens_kv, void* out,
                            float* lse, float* ws_o,
                            float* ws_lse, int32_t* dev_status, uint32_t signature, int32_t N1,
@@ -299,7 +299,7 @@ gbsa_status gbsa_metadata(const gbsa_problem* problem, const gbsa_tensors* t, vo
   return GBSA_OK;
 }
 
-gbsa_status gbsa_forward(const gbsa_problem* problem, const gbsa_tensors* t, const void* meta,
+gbsa_status gbsa_forward(const gbsa_problem* problem, const gbsa_tensors* t, void* meta,
                          void* workspace, size_t ws_bytes, int32_t* dev_status, void* stream) {
   gbsa_status st = validate(problem, false);
   if (st != GBSA_OK) return st;
@@ -349,7 +349,7 @@ gbsa_status gbsa_forward(const gbsa_problem* problem, const gbsa_tensors* t, con
   float* ws_o = static_cast<float*>(workspace);
   float* ws_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + wl.lse_off);
   const cudaError_t e = launch_forward(
-      map_q, map_k, map_v, static_cast<const int32_t*>(meta), tnd ? nullptr : t->block_table,
+      map_q, map_k, map_v, static_cast<int32_t*>(meta), tnd ? nullptr : t->block_table,
       tnd ? t->cu_seqlens_kv : nullptr, t->out,
       problem->return_lse ? t->lse : nullptr, ws_o, ws_lse, dev_status,
       problem_signature(problem, ctas), problem->N1, problem->N2, problem->T, problem->top_k,

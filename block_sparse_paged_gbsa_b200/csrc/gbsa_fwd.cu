@@ -22,8 +22,9 @@
 // the first columns of its S (two 16-bit or four E4M3 weights per column).
 // Element types (kDt): bf16, fp16 (kind::f16 MMAs) and E4M3 (kind::f8f6f4,
 // per-tensor dequantization scales folded into the score scale and 1 / l).
-// Units come from the metadata work list, longest first; the CTAs take them
-// wave by wave, in reverse CTA order on odd waves (unit_of).  Every wait is
+// Units come from the metadata work list, longest first: CTA c starts with
+// unit c and then takes the next untaken unit from a counter in the work
+// list's header, so SMs that run faster take more units.  Every wait is
 // bounded (by FwdParams::wait_limit_ns, 1 s unless the caller sets another):
 // after it the kernel sets GBSA_DEV_TIMEOUT, drains its own copies and MMAs
 // (each drain bounded by 1 s), frees TMEM and returns.
@@ -126,6 +127,7 @@ __device__ __forceinline__ float as_float(uint32_t x) { return __uint_as_float(x
 
 struct FwdParams {
   const int32_t* meta;
+  int32_t* work;  // meta + H_UNIT_NEXT: the unit counter, then the finished-CTA count
   const int32_t* block_table;  // paged K/V
   const int64_t* cu_kv;        // TND K/V: first row of each sequence (block_table unused)
   uint16_t* out;  // fp16 for fp16 inputs, else bf16
@@ -141,7 +143,22 @@ struct FwdParams {
   uint64_t wait_limit_ns;  // bound of every pipeline wait
 };
 
+// The units a CTA takes after its first come from a counter shared by the
+// grid (in list order, so a fast SM takes more units than a slow one).  Its
+// producer warp fetches each one and hands the unit's record (its unit-table
+// row and its item's row) to the other roles through a ring of kUnitQ entries.
+constexpr uint32_t kUnitQ = 4;
+constexpr uint32_t kUnitReaders = 13;  // warps 0..12: softmax 8, epilogue 4, MMA 1
+struct UnitRec {
+  int4 rec;   // unit row: item, tile pair, blocks [j0, j1), split slot
+  int4 a, c;  // item row, words 0..3 and 4..7
+};
+
 struct Bars {
+  UnitRec uq[kUnitQ];
+  int32_t uq_id[kUnitQ];      // unit index, or -1: no more units
+  uint64_t uq_full[kUnitQ];   // entry written (producer)
+  uint64_t uq_empty[kUnitQ];  // entry read (one arrival per reading warp)
   uint64_t q_full[2], q_empty[2];
   uint64_t kv_full[kMaxStages], kv_empty[kMaxStages];
   uint64_t s_full[2];      // S of a block ready (MMA commit)
@@ -159,15 +176,6 @@ struct Bars {
 constexpr int kSmemBytes = kSmemBars + (int)sizeof(Bars);
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
-// The k-th unit of this CTA.  Units are sorted longest first; wave k covers
-// units [k * gridDim.x, (k + 1) * gridDim.x) and hands them to the CTAs in
-// reverse order on odd waves, which evens out the per-CTA sums of a sorted
-// list far better than plain round robin.  Increasing in k.
-__device__ __forceinline__ int32_t unit_of(int32_t k) {
-  const int32_t c = (k & 1) ? (int32_t)(gridDim.x - 1 - blockIdx.x) : (int32_t)blockIdx.x;
-  return k * (int32_t)gridDim.x + c;
-}
-
 struct Unit {
   int32_t item, tp, j0, j1, slot;
   int32_t b, n_tiles, tok_begin, n_store, n_used, pos0, ku;
@@ -176,18 +184,25 @@ struct Unit {
                     // and odd blocks (two partial softmaxes, merged at the end)
 };
 
+// The record of unit u, read from the work list in global memory.
+__device__ __forceinline__ UnitRec fetch_unit(const int32_t* meta, int64_t off_unit,
+                                              int64_t off_item, int32_t u) {
+  UnitRec r;
+  r.rec = *reinterpret_cast<const int4*>(meta + off_unit + 4 * (int64_t)u);
+  r.a = *reinterpret_cast<const int4*>(meta + off_item + 8 * (int64_t)r.rec.x);
+  r.c = *reinterpret_cast<const int4*>(meta + off_item + 8 * (int64_t)r.rec.x + 4);
+  return r;
+}
+
 template <bool kHalves>
-__device__ __forceinline__ Unit load_unit(const int32_t* meta, int64_t off_unit, int64_t off_item,
-                                          int32_t u, int32_t N2) {
+__device__ __forceinline__ Unit decode_unit(const UnitRec& r, int32_t N2) {
   Unit x;
-  const int4 rec = *reinterpret_cast<const int4*>(meta + off_unit + 4 * (int64_t)u);
+  const int4 rec = r.rec, a = r.a, c = r.c;
   x.item = rec.x;
   x.tp = rec.y;
   x.j0 = rec.z & 0xffff;
   x.j1 = (int32_t)((uint32_t)rec.z >> 16);
   x.slot = rec.w;
-  const int4 a = *reinterpret_cast<const int4*>(meta + off_item + 8 * (int64_t)x.item);
-  const int4 c = *reinterpret_cast<const int4*>(meta + off_item + 8 * (int64_t)x.item + 4);
   x.b = a.x;
   x.n_tiles = a.z;
   x.tok_begin = a.w;
@@ -220,6 +235,37 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Bars* b
       return false;
     }
   }
+}
+
+// The k-th entry of the unit queue, read by a whole warp: waits until the
+// producer wrote it, copies it, and (lane 0, once every lane has read it)
+// releases it.  False when the queue has ended (unit < 0) or a wait gave up.
+struct UnitCursor {
+  uint32_t k = 0;
+  __device__ __forceinline__ bool next(Bars* bars, UnitRec& r) {
+    const uint32_t s = k % kUnitQ;
+    if (!wait_bar(&bars->uq_full[s], (k / kUnitQ) & 1, bars)) return false;
+    const int32_t u = bars->uq_id[s];
+    r = bars->uq[s];
+    __syncwarp();
+    if (lane_id() == 0) mbar_arrive(&bars->uq_empty[s]);
+    k++;
+    return u >= 0;
+  }
+};
+
+// Producer side: writes unit u (u < 0: the end) as the k-th entry once every
+// reader has released the entry's previous use.  Whole warp; lane 0 writes.
+__device__ __forceinline__ bool push_unit(Bars* bars, uint32_t k, int32_t u, const UnitRec& r,
+                                          uint32_t lane) {
+  const uint32_t s = k % kUnitQ;
+  if (k >= kUnitQ && !wait_bar(&bars->uq_empty[s], ((k / kUnitQ) & 1) ^ 1, bars)) return false;
+  if (lane == 0) {
+    bars->uq[s] = r;
+    bars->uq_id[s] = u;
+    mbar_arrive(&bars->uq_full[s]);
+  }
+  return true;
 }
 
 // Operand layouts in shared memory (128-byte swizzle, tiles 1 KiB aligned):
@@ -301,6 +347,63 @@ __device__ __forceinline__ bool produce_q(const FwdParams& p, const CUtensorMap*
   return true;
 }
 
+// The copies of one unit with n > 0 blocks (whole warp; lane 0 issues).
+template <bool kHalves, int kDt>
+__device__ __forceinline__ void produce_unit(const FwdParams& p, const CUtensorMap* map_q,
+                                             const CUtensorMap* map_k, const CUtensorMap* map_v,
+                                             uint8_t* smem, Bars* bars, const Unit& x,
+                                             int64_t off_list, uint32_t& kv_iter,
+                                             uint32_t& q_iter0, uint32_t& q_iter1, int32_t& bad,
+                                             bool& ok, uint32_t lane) {
+  const int32_t n = x.j1 - x.j0;
+  const int32_t* list = p.meta + off_list + (int64_t)x.item * p.top_k + x.j0;
+  const bool tnd = p.cu_kv != nullptr;
+  const int32_t* bt = tnd ? nullptr : p.block_table + (int64_t)x.b * p.max_pages;
+  const int64_t row0 = tnd ? p.cu_kv[x.b] : 0;  // TND: first row of the sequence
+  // order: Q0, K_0, Q1, V_0, K_1, V_1, ... (Q1 of a unit waits for the
+  // previous unit's last S1, which comes later than its last S0); a unit
+  // in halves: Q0, then per block pair K_j, K_j+1, V_j, V_j+1
+  // pages of the first 32 entries: the loads overlap the wait for the Q slot
+  // per lane: the page of an entry (paged), or its first row (TND); live
+  // entries lie inside the sequence, so a TND row stays inside k / v
+  int32_t page = 0;
+  if ((int32_t)lane < n) {
+    const int32_t lb = list[lane] & kEntryLbMask;
+    page = tnd ? (int32_t)(row0 + (int64_t)lb * kPage) : (lb < p.max_pages ? bt[lb] : -1);
+  }
+  ok = produce_q<kDt>(p, map_q, smem, bars, q_iter0, x, 0, lane);
+  for (int32_t c0 = 0; c0 < n && ok; c0 += 32) {
+    if (c0 > 0 && c0 + (int32_t)lane < n) {
+      const int32_t lb = list[c0 + lane] & kEntryLbMask;
+      page = tnd ? (int32_t)(row0 + (int64_t)lb * kPage) : (lb < p.max_pages ? bt[lb] : -1);
+    }
+    if (!tnd && c0 + (int32_t)lane < n && (page < 0 || page >= p.num_pages)) {
+      bad |= kDevBadPage;
+      page = 0;
+    }
+    const int32_t cn = min(32, n - c0);
+    if (x.halves) {
+      // blocks c0 + jj (even) and c0 + jj + 1 share a 32-entry chunk
+      for (int32_t jj = 0; jj < cn && ok; jj += 2) {
+        const bool has1 = jj + 1 < cn;
+        const int32_t pg0 = __shfl_sync(0xffffffffu, page, jj);
+        const int32_t pg1 = __shfl_sync(0xffffffffu, page, (jj + 1) & 31);
+        ok = produce_kv<kDt>(map_k, smem, bars, kv_iter, x.kvh, pg0, tnd, lane);
+        if (ok && has1) ok = produce_kv<kDt>(map_k, smem, bars, kv_iter, x.kvh, pg1, tnd, lane);
+        if (ok) ok = produce_kv<kDt>(map_v, smem, bars, kv_iter, x.kvh, pg0, tnd, lane);
+        if (ok && has1) ok = produce_kv<kDt>(map_v, smem, bars, kv_iter, x.kvh, pg1, tnd, lane);
+      }
+      continue;
+    }
+    for (int32_t jj = 0; jj < cn && ok; jj++) {
+      const int32_t pg = __shfl_sync(0xffffffffu, page, jj);
+      ok = produce_kv<kDt>(map_k, smem, bars, kv_iter, x.kvh, pg, tnd, lane);
+      if (ok && c0 + jj == 0 && x.nt == 2) ok = produce_q<kDt>(p, map_q, smem, bars, q_iter1, x, 1, lane);
+      if (ok) ok = produce_kv<kDt>(map_v, smem, bars, kv_iter, x.kvh, pg, tnd, lane);
+    }
+  }
+}
+
 template <bool kHalves, int kDt>
 __device__ void run_producer(const FwdParams& p, const CUtensorMap* map_q, const CUtensorMap* map_k,
                              const CUtensorMap* map_v, uint8_t* smem, Bars* bars, int32_t n_units,
@@ -312,55 +415,35 @@ __device__ void run_producer(const FwdParams& p, const CUtensorMap* map_q, const
   uint32_t kv_iter = 0, q_iter0 = 0, q_iter1 = 0;
   int32_t bad = 0;
   bool ok = true;
-  for (int32_t wave = 0, u = unit_of(0); u < n_units && ok; u = unit_of(++wave)) {
-    const Unit x = load_unit<kHalves>(p.meta, off_unit, off_item, u, p.N2);
+  // the first unit of CTA c is unit c; the next ones come from the counter
+  int32_t u = (int32_t)blockIdx.x;
+  for (uint32_t kq = 0; ok; kq++) {
+    const bool live = u < n_units;
+    UnitRec r{};
+    if (live) r = fetch_unit(p.meta, off_unit, off_item, u);
+    const Unit x = decode_unit<kHalves>(r, p.N2);
     const int32_t n = x.j1 - x.j0;
-    if (n <= 0) continue;
-    const int32_t* list = p.meta + off_list + (int64_t)x.item * p.top_k + x.j0;
-    const bool tnd = p.cu_kv != nullptr;
-    const int32_t* bt = tnd ? nullptr : p.block_table + (int64_t)x.b * p.max_pages;
-    const int64_t row0 = tnd ? p.cu_kv[x.b] : 0;  // TND: first row of the sequence
-    // order: Q0, K_0, Q1, V_0, K_1, V_1, ... (Q1 of a unit waits for the
-    // previous unit's last S1, which comes later than its last S0); a unit
-    // in halves: Q0, then per block pair K_j, K_j+1, V_j, V_j+1
-    // pages of the first 32 entries: the loads overlap the wait for the Q slot
-    // per lane: the page of an entry (paged), or its first row (TND); live
-    // entries lie inside the sequence, so a TND row stays inside k / v
-    int32_t page = 0;
-    if ((int32_t)lane < n) {
-      const int32_t lb = list[lane] & kEntryLbMask;
-      page = tnd ? (int32_t)(row0 + (int64_t)lb * kPage) : (lb < p.max_pages ? bt[lb] : -1);
-    }
-    ok = produce_q<kDt>(p, map_q, smem, bars, q_iter0, x, 0, lane);
-    for (int32_t c0 = 0; c0 < n && ok; c0 += 32) {
-      if (c0 > 0 && c0 + (int32_t)lane < n) {
-        const int32_t lb = list[c0 + lane] & kEntryLbMask;
-        page = tnd ? (int32_t)(row0 + (int64_t)lb * kPage) : (lb < p.max_pages ? bt[lb] : -1);
-      }
-      if (!tnd && c0 + (int32_t)lane < n && (page < 0 || page >= p.num_pages)) {
-        bad |= kDevBadPage;
-        page = 0;
-      }
-      const int32_t cn = min(32, n - c0);
-      if (x.halves) {
-        // blocks c0 + jj (even) and c0 + jj + 1 share a 32-entry chunk
-        for (int32_t jj = 0; jj < cn && ok; jj += 2) {
-          const bool has1 = jj + 1 < cn;
-          const int32_t pg0 = __shfl_sync(0xffffffffu, page, jj);
-          const int32_t pg1 = __shfl_sync(0xffffffffu, page, (jj + 1) & 31);
-          ok = produce_kv<kDt>(map_k, smem, bars, kv_iter, x.kvh, pg0, tnd, lane);
-          if (ok && has1) ok = produce_kv<kDt>(map_k, smem, bars, kv_iter, x.kvh, pg1, tnd, lane);
-          if (ok) ok = produce_kv<kDt>(map_v, smem, bars, kv_iter, x.kvh, pg0, tnd, lane);
-          if (ok && has1) ok = produce_kv<kDt>(map_v, smem, bars, kv_iter, x.kvh, pg1, tnd, lane);
-        }
-        continue;
-      }
-      for (int32_t jj = 0; jj < cn && ok; jj++) {
-        const int32_t pg = __shfl_sync(0xffffffffu, page, jj);
-        ok = produce_kv<kDt>(map_k, smem, bars, kv_iter, x.kvh, pg, tnd, lane);
-        if (ok && c0 + jj == 0 && x.nt == 2) ok = produce_q<kDt>(p, map_q, smem, bars, q_iter1, x, 1, lane);
-        if (ok) ok = produce_kv<kDt>(map_v, smem, bars, kv_iter, x.kvh, pg, tnd, lane);
-      }
+    if (!(ok = push_unit(bars, kq, live ? u : -1, r, lane))) break;
+    if (!live) break;
+    // the unit after this one; the atomic's latency overlaps this unit's
+    // copies, and its value is always read (below) so that it has completed
+    // before the CTA counts itself finished
+    int32_t nxt = 0;
+    if (lane == 0) nxt = (int32_t)gridDim.x + atomicAdd(p.work, 1);
+    if (n > 0) produce_unit<kHalves, kDt>(p, map_q, map_k, map_v, smem, bars, x, off_list, kv_iter,
+                                          q_iter0, q_iter1, bad, ok, lane);
+    u = __shfl_sync(0xffffffffu, nxt, 0);
+  }
+  if (lane == 0) {
+    // This CTA fetches no more units (after an abort too): it counts itself,
+    // and the last CTA to do so puts both counters back to zero for the next
+    // launch on this work list.  Every CTA counts itself only after the value
+    // of its last fetch came back, so no fetch follows the reset.  (Counting
+    // here, not at the CTA's exit, keeps the atomics off the exit path.)
+    __threadfence();
+    if (atomicAdd(p.work + 1, 1) == min((int32_t)gridDim.x, n_units) - 1) {
+      atomicExch(p.work, 0);
+      atomicExch(p.work + 1, 0);
     }
   }
   bad = __reduce_or_sync(0xffffffffu, bad);
@@ -492,7 +575,7 @@ __device__ __forceinline__ void zero_v_tail(uint8_t* smem, uint32_t vs, int32_t 
 
 template <bool kHalves, int kDt>
 __device__ void run_mma(const FwdParams& p, uint8_t* smem, Bars* bars, uint32_t tmem,
-                        int32_t n_units, int32_t off_unit, int32_t off_item, int32_t off_list) {
+                        int64_t off_list) {
   const uint32_t lane = lane_id();
   uint32_t q_iter0 = 0, q_iter1 = 0;
   uint32_t blk0 = 0, blk1 = 0;      // blocks per tile slot (p_full phases)
@@ -510,11 +593,11 @@ __device__ void run_mma(const FwdParams& p, uint8_t* smem, Bars* bars, uint32_t 
   const uint32_t v_lo0 = (uint32_t)smem_desc_sw128(ring_addr, kHalfBytes, 1024);
   constexpr uint32_t kStageLo = stage_bytes<kDt>() >> 4;
 
-  for (int32_t wave = 0, u = unit_of(0); u < n_units && ok; u = unit_of(++wave)) {
-    const int4 rec = *reinterpret_cast<const int4*>(p.meta + off_unit + 4 * (int64_t)u);
+  UnitRec ur;
+  for (UnitCursor cur; ok && cur.next(bars, ur);) {
+    const int4 rec = ur.rec, irow = ur.a;
     const int32_t item = rec.x, j0 = rec.z & 0xffff, n = (int32_t)((uint32_t)rec.z >> 16) - j0;
-    const int4 irow = *reinterpret_cast<const int4*>(p.meta + off_item + 8 * (int64_t)item);
-    const int32_t ku = p.meta[off_item + 8 * (int64_t)item + 7];
+    const int32_t ku = ur.c.w;
     const bool two = irow.z - 2 * rec.y >= 2;
     const bool halves = kHalves && irow.z == 1 && n >= kHalvesMinBlocks;
     if (halves) {
@@ -911,7 +994,7 @@ __device__ __forceinline__ uint8_t* dyn_smem() {
 
 template <bool kHalves, int kDt, bool kHalfSm>
 __device__ void run_softmax(const FwdParams& p, Bars* bars, uint32_t tmem, int slot,
-                            int32_t n_units, int64_t off_unit, int64_t off_item, int64_t off_list) {
+                            int64_t off_list) {
   const int row = threadIdx.x & 127;
   const uint32_t lane_sel = (uint32_t)(threadIdx.x & 96) << 16;  // warp's 32-lane quarter
   const uint32_t t_s = tmem + 128 * slot + lane_sel;
@@ -919,8 +1002,9 @@ __device__ void run_softmax(const FwdParams& p, Bars* bars, uint32_t tmem, int s
   // narrow tiles (the one-tile instantiation only: the second Q slot is free)
   const bool narrow = kHalves && p.tile_tokens * p.G <= kNarrowRows;
   uint32_t blk = 0, units = 0;
-  for (int32_t wave = 0, u = unit_of(0); u < n_units; u = unit_of(++wave)) {
-    const Unit x = load_unit<kHalves>(p.meta, off_unit, off_item, u, p.N2);
+  UnitRec ur;
+  for (UnitCursor cur; cur.next(bars, ur);) {
+    const Unit x = decode_unit<kHalves>(ur, p.N2);
     const int32_t nblk = x.j1 - x.j0;
     if ((slot >= x.nt && !x.halves) || nblk <= 0) continue;
     // a unit in halves: both slots hold the rows of its one tile, slot s
@@ -1111,16 +1195,16 @@ __device__ __forceinline__ float out_numerator(const FwdParams& p) {
 }
 
 template <bool kHalves, int kDt>
-__device__ void run_epilogue(const FwdParams& p, Bars* bars, uint32_t tmem, int32_t n_units,
-                             int64_t off_unit, int64_t off_item) {
+__device__ void run_epilogue(const FwdParams& p, Bars* bars, uint32_t tmem) {
   const int row = threadIdx.x & 127;
   const uint32_t lane_sel = (uint32_t)(threadIdx.x & 96) << 16;
   const int rows_in_tile = p.tile_tokens * p.G;
   uint32_t units_stats[2] = {0, 0}, units_final[2] = {0, 0};
   int32_t bad = 0;
   bool ok = true;
-  for (int32_t wave = 0, u = unit_of(0); u < n_units && ok; u = unit_of(++wave)) {
-    const Unit x = load_unit<kHalves>(p.meta, off_unit, off_item, u, p.N2);
+  UnitRec ur;
+  for (UnitCursor cur; ok && cur.next(bars, ur);) {
+    const Unit x = decode_unit<kHalves>(ur, p.N2);
     const int32_t nblk = x.j1 - x.j0;
     if (x.halves) {
       // two partial softmaxes over the even and odd blocks of one tile:
@@ -1281,6 +1365,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   Bars* bars = reinterpret_cast<Bars*>(smem + kSmemBars);
   if (threadIdx.x == 0) {
+    for (uint32_t i = 0; i < kUnitQ; i++) {
+      mbar_init(&bars->uq_full[i], 1);
+      mbar_init(&bars->uq_empty[i], kUnitReaders);
+    }
     for (int i = 0; i < 2; i++) {
       mbar_init(&bars->q_full[i], 1);
       mbar_init(&bars->q_empty[i], 1);
@@ -1311,15 +1399,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < 8) {
     setmaxnreg_inc<regs_softmax<kHalves>()>();
-    run_softmax<kHalves, kDt, kHalfSm>(p, bars, tmem, warp >> 2, n_units, off_unit, off_item,
-                                       off_list);
+    run_softmax<kHalves, kDt, kHalfSm>(p, bars, tmem, warp >> 2, off_list);
   } else if (warp < 12) {
     setmaxnreg_dec<kRegsEpilogue>();
-    run_epilogue<kHalves, kDt>(p, bars, tmem, n_units, off_unit, off_item);
+    run_epilogue<kHalves, kDt>(p, bars, tmem);
   } else {
     setmaxnreg_dec<regs_control<kHalves>()>();
     if (warp == kWarpMma) {
-      run_mma<kHalves, kDt>(p, smem, bars, tmem, n_units, (int32_t)off_unit, (int32_t)off_item, (int32_t)off_list);
+      run_mma<kHalves, kDt>(p, smem, bars, tmem, off_list);
     } else if (warp == kWarpProducer) {
       if (lane_id() == 0) {
         tma_prefetch_map(&map_q);
@@ -1407,7 +1494,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const CombineParams p) {
 size_t forward_smem_bytes() { return kSmemBytes; }
 
 cudaError_t launch_forward(const CUtensorMap& map_q, const CUtensorMap& map_k,
-                           const CUtensorMap& map_v, const int32_t* meta,
+                           const CUtensorMap& map_v, int32_t* meta,
                            const int32_t* block_table, const int64_t* cu_seqlens_kv, void* out,
                            float* lse, float* ws_o,
                            float* ws_lse, int32_t* dev_status, uint32_t signature, int32_t N1,
@@ -1447,6 +1534,7 @@ cudaError_t launch_forward(const CUtensorMap& map_q, const CUtensorMap& map_k,
   }
   FwdParams p;
   p.meta = meta;
+  p.work = meta + H_UNIT_NEXT;
   p.block_table = block_table;
   p.cu_kv = cu_seqlens_kv;
   p.out = static_cast<uint16_t*>(out);

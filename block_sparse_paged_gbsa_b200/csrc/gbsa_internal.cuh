@@ -71,7 +71,11 @@ enum HdrField : int {
   H_MAGIC = 0, H_VERSION, H_SIGNATURE, H_B, H_NITEMS, H_TILE_TOKENS, H_TILES_MAX, H_NUM_CTAS,
   H_UNIT_CAP, H_SLOT_CAP, H_COMB_CAP, H_NUNITS, H_NSLOTS, H_NCOMB, H_SPLIT_LEN, H_STATUS,
   H_COST_LO, H_COST_HI, H_OFF_SEQ, H_OFF_ITEM, H_OFF_LIST, H_OFF_UNIT, H_OFF_COMB, H_TOTAL,
-  H_ROWS_PER_UNIT, H_G
+  H_ROWS_PER_UNIT, H_G,
+  // Work counters of the forward (zero when the metadata is built; each
+  // forward launch fetches units through H_UNIT_NEXT and counts finished CTAs
+  // in H_CTAS_DONE, and its last CTA puts both back to zero).
+  H_UNIT_NEXT, H_CTAS_DONE
 };
 
 // Device-status bits (mirrors GBSA_DEV_* in include/gbsa.h).

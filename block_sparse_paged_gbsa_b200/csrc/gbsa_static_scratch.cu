@@ -98,7 +98,7 @@ gbsa_status scratch_address(void** out) {
 }  // namespace
 
 extern "C" gbsa_status gbsa_forward_static_scratch(const gbsa_problem* problem,
-                                                   const gbsa_tensors* tensors, const void* meta,
+                                                   const gbsa_tensors* tensors, void* meta,
                                                    int32_t* dev_status, void* stream) {
   size_t need = 0;
   gbsa_status st = gbsa_workspace_size(problem, &need);

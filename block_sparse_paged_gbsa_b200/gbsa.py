@@ -108,7 +108,7 @@ class Problem:
         return p
 
 
-ABI_VERSION = 5
+ABI_VERSION = 6
 # GBSA_METADATA_FUSED_MAX_B: up to this many sequences the metadata call is
 # two kernel launches, above it three.
 METADATA_FUSED_MAX_B = 1024

@@ -61,7 +61,7 @@
 extern "C" {
 #endif
 
-#define GBSA_ABI_VERSION 5
+#define GBSA_ABI_VERSION 6
 
 /* Symbols of the C ABI are exported; everything else in libgbsa is hidden. */
 #if defined(__GNUC__)
@@ -211,11 +211,18 @@ GBSA_API gbsa_status gbsa_workspace_size(const gbsa_problem* problem, size_t* by
  * work list in `meta`.  `workspace` (16-byte aligned, ws_bytes >=
  * gbsa_workspace_size()) is caller-owned scratch, overwritten.  If `meta`
  * was built for a different problem the kernels set GBSA_DEV_META_MISMATCH
- * and leave out/lse untouched.  Deterministic for a fixed num_ctas
+ * and leave out/lse (and `meta`) untouched.
+ * The forward writes to `meta` (ABI 6): the CTAs take work units through a
+ * counter in its header (words 26 and 27), which gbsa_metadata() leaves at
+ * zero and every forward call puts back to zero before it finishes, so the
+ * same metadata serves any number of calls, CUDA graph replays included.
+ * Calls that share one metadata buffer must therefore not overlap on the GPU
+ * (other streams, other host threads): order them on one stream or with
+ * events, or give each its own copy.  Deterministic for a fixed num_ctas
  * (GBSA article, "Constraints: determinism").  Rows past seqused_q, and rows
  * with no visible key, get out = 0 and lse = -inf. */
 GBSA_API gbsa_status gbsa_forward(const gbsa_problem* problem, const gbsa_tensors* tensors,
-                         const void* meta, void* workspace, size_t ws_bytes,
+                         void* meta, void* workspace, size_t ws_bytes,
                          int32_t* dev_status, void* stream);
 
 /* Size of the device scratch that gbsa_forward_static_scratch() uses. */
@@ -251,7 +258,7 @@ GBSA_API gbsa_status gbsa_forward(const gbsa_problem* problem, const gbsa_tensor
  * Everything else -- arguments, layouts, errors, dev_status -- is as for
  * gbsa_forward(). */
 GBSA_API gbsa_status gbsa_forward_static_scratch(const gbsa_problem* problem,
-                                                 const gbsa_tensors* tensors, const void* meta,
+                                                 const gbsa_tensors* tensors, void* meta,
                                                  int32_t* dev_status, void* stream);
 
 #ifdef __cplusplus

@@ -19,7 +19,8 @@ Header, 32 words:
   15 status bits           16/17 total_cost lo/hi 18 off_seq
   19 off_item              20 off_list            21 off_unit
   22 off_combine           23 total_words         24 rows_per_unit
-  25 G                     26..31 zero
+  25 G                     26..31 zero (26, 27: the forward's unit counters,
+                                           back at zero after every call)
 Sequence table (B x 8):   qs, qu, ku, n_qblocks, qblock_base, tok_begin, 0, 0
 Item table (n_items x 8): b, n_live, n_tiles, tok_begin, n_store, n_used, pos0, ku
   item i = qb * N2 + kvh  (Q-block major, then KV head)

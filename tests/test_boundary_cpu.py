@@ -36,7 +36,7 @@ def test_exports_every_declared_symbol(lib):
             "gbsa_workspace_size"} <= set(names)
     for n in names:
         assert hasattr(lib, n), n
-    assert lib.gbsa_abi_version() == 5
+    assert lib.gbsa_abi_version() == gbsa.gbsa.ABI_VERSION == 6
     for code in range(0, 9):
         assert lib.gbsa_status_string(code).decode().startswith("GBSA_")
 

@@ -4,10 +4,10 @@ cases have long units (up to 128 prefill blocks, or 256 decode blocks, on 8
 CTAs), so the epilogue waits a unit's whole run for its output,
 far longer than the hardware may hold the first barrier probe on its own;
 with a bound of 1 us that wait runs out.  The kernel must set the TIMEOUT
-status
-bit, drain the copies and MMAs it issued, release its tensor memory and
-return, and the next call on the same stream, with the default bound, must
-be correct."""
+status bit, drain the copies and MMAs it issued, release its tensor memory,
+put the work list's unit counters back to zero and return, and the next
+call on the same stream and work list, with the default bound, must be
+correct."""
 import numpy as np
 import pytest
 import torch
@@ -52,6 +52,8 @@ def test_wait_limit_runs_out_then_next_call_is_correct(name):
                  num_ctas=ctas, dev_status=status, wait_limit_ns=1000)
     torch.cuda.synchronize()               # the call returned
     assert int(status.item()) & TIMEOUT_BIT
+    # its work counters (header words 26, 27) are back at zero for the next call
+    assert int(meta[26].item()) == 0 and int(meta[27].item()) == 0
     for _ in range(2):
         status2 = torch.zeros(1, dtype=torch.int32, device="cuda")
         out, lse = run_forward(w, q, kf, vf, t, meta, num_ctas=ctas, dev_status=status2)
