@@ -611,11 +611,17 @@ __device__ void run_mma(const FwdParams& p, uint8_t* smem, Bars* bars, uint32_t 
       if (!(ok = warp_wait(&bars->q_full[0], q_iter0 & 1, bars))) break;
       q_iter0++;
       const int32_t n0 = (n + 1) >> 1, n1 = n >> 1;
+      // blocks of these 32 whose V tile has rows past seqused_kv (bit j & 31):
+      // a register test per block instead of a shuffle of the entry
+      uint32_t partial = __ballot_sync(0xffffffffu, entries & kEntryPartial);
       uint32_t pv1 = 0;  // ring stage of V of the pending odd block
       for (int32_t i = 0; i < n0 && ok; i++) {
         const int32_t j = 2 * i;
         const bool has1 = j + 1 < n;
-        if (i > 0 && (j & 31) == 0) entries = j + (int32_t)lane < n ? list[j + lane] : 0;
+        if (i > 0 && (j & 31) == 0) {
+          entries = j + (int32_t)lane < n ? list[j + lane] : 0;
+          partial = __ballot_sync(0xffffffffu, entries & kEntryPartial);
+        }
         // ---- S0_i = Q K_j
         if (!(ok = warp_wait(&bars->kv_full[rp.stage], rp.phase, bars))) break;
         if (lane == 0) {
@@ -653,7 +659,8 @@ __device__ void run_mma(const FwdParams& p, uint8_t* smem, Bars* bars, uint32_t 
         // ---- V_j, then PV0_i = P0 V_j
         const Ring rv0 = rp.ahead(has1 ? 2 : 1);
         if (!(ok = warp_wait(&bars->kv_full[rv0.stage], rv0.phase, bars))) break;
-        zero_v_tail<kDt>(smem, rv0.stage, __shfl_sync(0xffffffffu, entries, j & 31), ku, lane);
+        if ((partial >> (j & 31)) & 1u)
+          zero_v_tail<kDt>(smem, rv0.stage, __shfl_sync(0xffffffffu, entries, j & 31), ku, lane);
         if (i == 0 && units0 > 0)
           if (!(ok = warp_wait(&bars->o_free[0], (units0 - 1) & 1, bars))) break;
         if (!(ok = warp_wait(&bars->p_full[0], blk0 & 1, bars))) break;
@@ -668,7 +675,9 @@ __device__ void run_mma(const FwdParams& p, uint8_t* smem, Bars* bars, uint32_t 
         if (has1) {
           const Ring rv1 = rp.ahead(3);
           if (!(ok = warp_wait(&bars->kv_full[rv1.stage], rv1.phase, bars))) break;
-          zero_v_tail<kDt>(smem, rv1.stage, __shfl_sync(0xffffffffu, entries, (j + 1) & 31), ku, lane);
+          if ((partial >> ((j + 1) & 31)) & 1u)
+            zero_v_tail<kDt>(smem, rv1.stage, __shfl_sync(0xffffffffu, entries, (j + 1) & 31), ku,
+                             lane);
           pv1 = rv1.stage;
         }
         rp = rp.ahead(has1 ? 4 : 2);
