@@ -89,3 +89,30 @@ def test_graph_replays_bit_identical():
         assert _counters(meta) == (0, 0)
         assert torch.equal(out, ref_out) and torch.equal(lse, ref_lse)
     del graph
+
+
+def test_separate_work_lists_run_concurrently():
+    """Calls on two streams with their own work lists may overlap: each list
+    has its own counters.  Each result equals the same call run alone."""
+    cases = [(workload("ragged", scale_down=8), 7), (workload("dense", scale_down=4), 0)]
+    prepared = []
+    for w, ctas in cases:
+        q, kf, vf = make_values(w, "cuda")
+        t = device_tensors(w)
+        meta = run_metadata(w, t, ctas)
+        alone = run_forward(w, q, kf, vf, t, meta, ctas)
+        torch.cuda.synchronize()
+        prepared.append((w, ctas, q, kf, vf, t, meta, (alone[0].clone(), alone[1].clone())))
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    results = [[], []]
+    for s in streams:
+        s.wait_stream(torch.cuda.current_stream())
+    for _ in range(3):
+        for k, (w, ctas, q, kf, vf, t, meta, _) in enumerate(prepared):
+            with torch.cuda.stream(streams[k]):
+                results[k].append(run_forward(w, q, kf, vf, t, meta, ctas))
+    torch.cuda.synchronize()
+    for k, (w, ctas, q, kf, vf, t, meta, (ref_out, ref_lse)) in enumerate(prepared):
+        assert _counters(meta) == (0, 0)
+        for out, lse in results[k]:
+            assert torch.equal(out, ref_out) and torch.equal(lse, ref_lse)
