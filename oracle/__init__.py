@@ -1,4 +1,5 @@
-"""fp64 CPU oracle for block-sparse paged GQA attention (forward).
+"""fp64 CPU oracle for block-sparse paged GQA attention (forward, and the
+gradients of its output).
 
 TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
 CPU-baseline leg of ``bench.py`` may import this package.  It shares no code
@@ -11,7 +12,8 @@ What the oracle computes is stated at the top of ``gbsa_oracle.c``; it follows
 the GenericBlockSparseAttention article (cf-1.com/news/4865651), "Function /
 sparse attention mechanism" and "Constraints", and the FlashAttention blog
 post on CANN ops-transformer (ai6s.net), "three steps" (the online softmax is
-exactly the two-pass softmax).  Pins: tests/test_oracle_pins.py.
+exactly the two-pass softmax).  Pins: tests/test_oracle_pins.py (forward),
+tests/test_oracle_backward.py (gradients: finite differences, closed forms).
 """
 from __future__ import annotations
 
@@ -61,6 +63,11 @@ def load_library(path: str):
     w = lib.gbsa_oracle_widen
     w.argtypes = [i32, ptr, i64, ptr]
     w.restype = ctypes.c_int
+    g = lib.gbsa_oracle_attention_backward
+    g.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, i32, i32, i64, dbl, i32, i32, i32,
+                  ptr, ptr, ptr, ptr, ptr, ptr, ptr, ptr, ptr, ptr, ptr, ptr, ptr, ptr, ptr, ptr,
+                  ptr]
+    g.restype = ctypes.c_int
     return lib
 
 
@@ -163,3 +170,54 @@ def attention(*, q_bits, rows=None, **kw):
     all_rows = np.stack([tt.reshape(-1), hh.reshape(-1)], axis=1)
     out, lse = attention_rows(q_bits=q_bits, rows=all_rows, **kw)
     return out.reshape(T, N1, D), lse.reshape(T, N1)
+
+
+def attention_backward(*, q_bits, k_bits, v_bits, dout_bits, kv_page_stride, num_pages, sparse_idx,
+                       sparse_count, cu_seqlens_q, seqused_q, seqused_kv, block_table, block_x,
+                       scale, win_left=-1, win_right=-1, dtype="bf16", cu_seqlens_kv=None,
+                       with_abs=False, lib=None):
+    """Reference gradients of out (fp64) for an incoming gradient ``dout_bits``
+    (uint16 [T, N1, D], the type of q).  Arguments as for ``attention_rows``.
+
+    Returns (dq [T, N1, D], dk, dv), dk and dv flat float64 arrays laid out
+    like k_bits and v_bits (the page pool with ``kv_page_stride``, or TND);
+    with ``with_abs`` also (dq_abs, dk_abs, dv_abs), the same sums of the
+    absolute values of their terms.
+    """
+    q_bits = _as(q_bits, np.uint16)
+    dout_bits = _as(dout_bits, np.uint16)
+    k_bits = _as(k_bits, np.uint16).reshape(-1)
+    v_bits = _as(v_bits, np.uint16).reshape(-1)
+    T, N1, D = q_bits.shape
+    if dout_bits.shape != q_bits.shape:
+        raise ValueError("dout: expected the shape of q")
+    sparse_idx = _as(sparse_idx, np.int32)
+    N2, tqb, top_k = sparse_idx.shape
+    sparse_count = _as(sparse_count, np.int32)
+    cu = _as(cu_seqlens_q, np.int64)
+    squ = _as(seqused_q, np.int32)
+    sku = _as(seqused_kv, np.int32)
+    cukv = _as(cu_seqlens_kv, np.int64)
+    B = cu.shape[0] - 1
+    if cukv is None:
+        bt = _as(block_table, np.int32)
+        max_pages = bt.shape[1]
+        need = (num_pages - 1) * kv_page_stride + 128 * N2 * D
+    else:
+        bt, max_pages, num_pages, kv_page_stride = None, 0, 0, 0
+        need = int(cukv[-1]) * N2 * D
+    if k_bits.size < need or v_bits.size < need:
+        raise ValueError("page pool arrays are shorter than num_pages pages")
+    dq = np.zeros((T, N1, D), np.float64)
+    dk = np.zeros(k_bits.size, np.float64)
+    dv = np.zeros(v_bits.size, np.float64)
+    absv = [np.zeros_like(dq), np.zeros_like(dk), np.zeros_like(dv)] if with_abs else [None] * 3
+    rc = (lib or _load()).gbsa_oracle_attention_backward(
+        B, T, N1, N2, D, block_x, tqb, top_k, max_pages, num_pages, kv_page_stride, float(scale),
+        win_left, win_right, DTYPES[dtype], _ptr(q_bits), _ptr(k_bits), _ptr(v_bits),
+        _ptr(dout_bits), _ptr(sparse_idx), _ptr(sparse_count), _ptr(cu), _ptr(squ), _ptr(sku),
+        _ptr(bt), _ptr(cukv), _ptr(dq), _ptr(dk), _ptr(dv), *(_ptr(a) for a in absv))
+    if rc != 0:
+        raise ValueError(f"oracle rejected the inputs (code {rc})")
+    return (dq, dk, dv, *absv) if with_abs else (dq, dk, dv)
+

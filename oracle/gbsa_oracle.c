@@ -1,6 +1,7 @@
 /*
  * gbsa_oracle.c -- plain fp64 CPU reference for block-sparse paged GQA
- * attention (forward).  TEST INFRASTRUCTURE ONLY: the tests, the smoke check
+ * attention (forward, and the gradients of its output at the end).  TEST
+ * INFRASTRUCTURE ONLY: the tests, the smoke check
  * and the benchmark's CPU-baseline leg may call it; the product path never
  * does.  It shares no code, header or constant with the CUDA library.
  *
@@ -314,3 +315,150 @@ int gbsa_oracle_attention_rows(int32_t B, int32_t T, int32_t N1, int32_t N2, int
   free(c.q_block_base);
   return c.failed;
 }
+
+/*
+ * Gradients of the attention output (training).  The GBSA article's
+ * overview says the operator serves inference and training but gives no
+ * backward; this is the gradient of the function computed above, taken
+ * analytically and written out plainly.  For a row (tg, h) with visible
+ * keys p (the same enumeration as one_row), weights w_p = exp(s_p - lse),
+ * output O = sum_p w_p v_p and incoming gradient g = dout[tg][h]:
+ *
+ *   dv_p   += w_p g                                (dO / dv_p)
+ *   dlt     = sum_d g[d] O[d]
+ *   ds_p    = w_p (g . v_p - dlt)                  (softmax Jacobian)
+ *   dq     += scale sum_p ds_p k_p
+ *   dk_p   += scale ds_p q
+ *
+ * Rows with no key or past seqused_q contribute nothing.  dq is
+ * [T][N1][D]; dk and dv have the layout of k and v (the paged pool
+ * [num_pages][128][N2][D] with kv_page_stride, or TND [T_kv][N2][D]) and
+ * are accumulated over every row and list entry that reads a key (a block
+ * listed twice counts twice, as in the forward).  The *_abs outputs
+ * (optional) get the same sums with every term replaced by its absolute
+ * value: the scale of the rounding error of any evaluation order.
+ * Single-threaded.  Returns 0 on success.
+ */
+int gbsa_oracle_attention_backward(int32_t B, int32_t T, int32_t N1, int32_t N2, int32_t D,
+                                   int32_t block_x, int32_t total_q_blocks, int32_t top_k,
+                                   int32_t max_pages_per_seq, int32_t num_pages,
+                                   int64_t kv_page_stride, double scale, int32_t win_left,
+                                   int32_t win_right, int32_t dtype, const uint16_t* q,
+                                   const uint16_t* k, const uint16_t* v, const uint16_t* dout,
+                                   const int32_t* sparse_idx, const int32_t* sparse_count,
+                                   const int64_t* cu_seqlens_q, const int32_t* seqused_q,
+                                   const int32_t* seqused_kv, const int32_t* block_table,
+                                   const int64_t* cu_seqlens_kv, double* dq, double* dk,
+                                   double* dv, double* dq_abs, double* dk_abs, double* dv_abs) {
+  if (B < 1 || T < 1 || N2 < 1 || N1 < N2 || N1 % N2 || D < 1 || block_x < 1 || top_k < 1 ||
+      total_q_blocks < 1 || (dtype != 0 && dtype != 1))
+    return 10;
+  if (!cu_seqlens_kv && (max_pages_per_seq < 1 || num_pages < 1)) return 10;
+  if (cu_seqlens_kv) {
+    if (cu_seqlens_kv[0] != 0) return 14;
+    for (int32_t b = 0; b < B; b++)
+      if (seqused_kv[b] < 0 || seqused_kv[b] > cu_seqlens_kv[b + 1] - cu_seqlens_kv[b]) return 14;
+    kv_page_stride = (int64_t)N2 * D;
+  }
+  oracle_ctx c;
+  memset(&c, 0, sizeof c);
+  c.B = B; c.T = T; c.N1 = N1; c.N2 = N2; c.D = D; c.block_x = block_x;
+  c.total_q_blocks = total_q_blocks; c.top_k = top_k;
+  c.max_pages_per_seq = max_pages_per_seq; c.num_pages = num_pages;
+  c.kv_page_stride = kv_page_stride; c.scale = scale;
+  c.win_left = win_left; c.win_right = win_right;
+  c.widen = dtype ? widen_fp16 : widen_bf16;
+  c.q = q; c.k = k; c.v = v; c.sparse_idx = sparse_idx; c.sparse_count = sparse_count;
+  c.cu_seqlens_q = cu_seqlens_q; c.seqused_q = seqused_q; c.seqused_kv = seqused_kv;
+  c.block_table = block_table; c.cu_seqlens_kv = cu_seqlens_kv;
+  c.q_block_base = (int64_t*)malloc(sizeof(int64_t) * (size_t)B);
+  if (!c.q_block_base) return 11;
+  int64_t acc = 0;
+  for (int32_t b = 0; b < B; b++) {
+    c.q_block_base[b] = acc;
+    const int64_t qs = cu_seqlens_q[b + 1] - cu_seqlens_q[b];
+    if (qs < 0) { free(c.q_block_base); return 12; }
+    acc += (qs + block_x - 1) / block_x;
+  }
+  if (acc != total_q_blocks || cu_seqlens_q[0] != 0 || cu_seqlens_q[B] != T) {
+    free(c.q_block_base);
+    return 13;
+  }
+  const int64_t cap = (int64_t)top_k * ORACLE_PAGE;
+  double* score = (double*)malloc(sizeof(double) * (size_t)cap);
+  int64_t* key_page = (int64_t*)malloc(sizeof(int64_t) * (size_t)cap);
+  int32_t* key_row = (int32_t*)malloc(sizeof(int32_t) * (size_t)cap);
+  double* out = (double*)malloc(sizeof(double) * (size_t)D);
+  int rc = (!score || !key_page || !key_row || !out) ? 11 : 0;
+  const int32_t G = N1 / N2;
+  for (int64_t tg = 0; tg < T && !rc; tg++) {
+    for (int32_t h = 0; h < N1 && !rc; h++) {
+      double lse;
+      /* the keys of (tg, h) in key_page / key_row and their scores, then O */
+      rc = one_row(&c, tg, h, out, &lse, NULL, NULL, score, key_page, key_row);
+      if (rc || lse == -INFINITY) continue;
+      /* the key count: one_row leaves it implicit, so enumerate again the way
+         it does (visible positions of every in-range entry, in list order) */
+      const int32_t b = find_sequence(&c, tg);
+      const int64_t t = tg - cu_seqlens_q[b];
+      const int64_t qs = cu_seqlens_q[b + 1] - cu_seqlens_q[b];
+      const int64_t qu = seqused_q ? (int64_t)seqused_q[b] : qs;
+      const int64_t ku = seqused_kv[b];
+      const int32_t kvh = h / G;
+      const int64_t qb = c.q_block_base[b] + t / block_x;
+      int64_t n = sparse_count[(int64_t)kvh * total_q_blocks + qb];
+      if (n < 0) n = 0;
+      if (n > top_k) n = top_k;
+      const int64_t pos = t + (ku - qu);
+      const int64_t blocks_in_seq = (ku + ORACLE_PAGE - 1) / ORACLE_PAGE;
+      const int32_t* list = sparse_idx + ((int64_t)kvh * total_q_blocks + qb) * top_k;
+      int64_t nk = 0;
+      for (int64_t j = 0; j < n; j++) {
+        const int64_t lb = list[j];
+        if (lb < 0 || lb >= blocks_in_seq) continue;
+        for (int32_t r = 0; r < ORACLE_PAGE; r++) {
+          const int64_t p = lb * ORACLE_PAGE + r;
+          if (p >= ku || p > pos) continue;
+          if (win_left >= 0 && p < pos - win_left) continue;
+          if (win_right >= 0 && p > pos + win_right) continue;
+          nk++;
+        }
+      }
+      const uint16_t* qrow = q + (tg * N1 + h) * (int64_t)D;
+      const uint16_t* grow = dout + (tg * N1 + h) * (int64_t)D;
+      double dlt = 0.0, dlt_abs = 0.0;
+      for (int32_t d = 0; d < D; d++) {
+        dlt += c.widen(grow[d]) * out[d];
+        dlt_abs += fabs(c.widen(grow[d]) * out[d]);
+      }
+      double* dqr = dq + (tg * N1 + h) * (int64_t)D;
+      double* dqa = dq_abs ? dq_abs + (tg * N1 + h) * (int64_t)D : NULL;
+      for (int64_t i = 0; i < nk; i++) {
+        const int64_t base = key_page[i] * kv_page_stride + ((int64_t)key_row[i] * N2 + kvh) * D;
+        const uint16_t* krow = k + base;
+        const uint16_t* vrow = v + base;
+        const double w = exp(score[i] - lse);
+        double gv = 0.0, gv_abs = 0.0;
+        for (int32_t d = 0; d < D; d++) {
+          gv += c.widen(grow[d]) * c.widen(vrow[d]);
+          gv_abs += fabs(c.widen(grow[d]) * c.widen(vrow[d]));
+        }
+        const double ds = w * (gv - dlt);
+        const double ds_abs = w * (gv_abs + dlt_abs);
+        for (int32_t d = 0; d < D; d++) {
+          const double g = c.widen(grow[d]);
+          dv[base + d] += w * g;
+          dqr[d] += scale * ds * c.widen(krow[d]);
+          dk[base + d] += scale * ds * c.widen(qrow[d]);
+          if (dv_abs) dv_abs[base + d] += w * fabs(g);
+          if (dqa) dqa[d] += scale * ds_abs * fabs(c.widen(krow[d]));
+          if (dk_abs) dk_abs[base + d] += scale * ds_abs * fabs(c.widen(qrow[d]));
+        }
+      }
+    }
+  }
+  free(score); free(key_page); free(key_row); free(out);
+  free(c.q_block_base);
+  return rc;
+}
+
