@@ -114,10 +114,12 @@ static int32_t find_sequence(const oracle_ctx* c, int64_t tg) {
   return lo;
 }
 
-/* Computes one (tg, h) row; scratch holds room for top_k*128 keys. */
+/* Computes one (tg, h) row; scratch holds room for top_k*128 keys.  When
+ * n_keys / kv_head are given they get the number of visible keys (their
+ * scores, pages and rows are in score, key_page, key_row) and the KV head. */
 static int one_row(const oracle_ctx* c, int64_t tg, int32_t h, double* out, double* lse,
                    double* out_abs, double* gap_abs, double* score, int64_t* key_page,
-                   int32_t* key_row) {
+                   int32_t* key_row, int64_t* n_keys, int32_t* kv_head) {
   const int32_t D = c->D;
   for (int32_t d = 0; d < D; d++) out[d] = 0.0;
   if (out_abs)
@@ -125,6 +127,7 @@ static int one_row(const oracle_ctx* c, int64_t tg, int32_t h, double* out, doub
   if (gap_abs)
     for (int32_t d = 0; d < D; d++) gap_abs[d] = 0.0;
   *lse = -INFINITY;
+  if (n_keys) *n_keys = 0;
   if (tg < 0 || tg >= c->T || h < 0 || h >= c->N1) return 1;
 
   const int32_t b = find_sequence(c, tg);
@@ -173,6 +176,8 @@ static int one_row(const oracle_ctx* c, int64_t tg, int32_t h, double* out, doub
       nk++;
     }
   }
+  if (n_keys) *n_keys = nk;
+  if (kv_head) *kv_head = kvh;
   if (nk == 0) return 0;
 
   const uint16_t* qrow = c->q + (tg * c->N1 + h) * (int64_t)D;
@@ -203,6 +208,28 @@ static int one_row(const oracle_ctx* c, int64_t tg, int32_t h, double* out, doub
   return 0;
 }
 
+/* c->q_block_base[b] = Q blocks of the sequences before b, counted over
+ * storage lengths ("Constraints: block split"); checks the prefix sums.
+ * Allocates the array (the caller frees it) and returns 0, or an error code
+ * with nothing allocated. */
+static int q_block_bases(oracle_ctx* c) {
+  c->q_block_base = (int64_t*)malloc(sizeof(int64_t) * (size_t)c->B);
+  if (!c->q_block_base) return 11;
+  const int64_t block_x = c->block_x;
+  int64_t acc = 0;
+  for (int32_t b = 0; b < c->B; b++) {
+    c->q_block_base[b] = acc;
+    const int64_t qs = c->cu_seqlens_q[b + 1] - c->cu_seqlens_q[b];
+    if (qs < 0) { free(c->q_block_base); return 12; }
+    acc += (qs + block_x - 1) / block_x;
+  }
+  if (acc != c->total_q_blocks || c->cu_seqlens_q[0] != 0 || c->cu_seqlens_q[c->B] != c->T) {
+    free(c->q_block_base);
+    return 13;
+  }
+  return 0;
+}
+
 typedef struct {
   oracle_ctx* c;
   int64_t begin, end;
@@ -221,7 +248,8 @@ static void* run_job(void* arg) {
     for (int64_t i = job->begin; i < job->end; i++) {
       const int rc = one_row(c, c->rows[2 * i], (int32_t)c->rows[2 * i + 1], c->out + i * c->D,
                              c->lse + i, c->out_abs ? c->out_abs + i * c->D : NULL,
-                             c->gap_abs ? c->gap_abs + i * c->D : NULL, score, key_page, key_row);
+                             c->gap_abs ? c->gap_abs + i * c->D : NULL, score, key_page, key_row,
+                             NULL, NULL);
       if (rc) c->failed = rc;
     }
   }
@@ -284,20 +312,8 @@ int gbsa_oracle_attention_rows(int32_t B, int32_t T, int32_t N1, int32_t N2, int
   c.out_abs = out_abs;
   c.gap_abs = gap_abs;
 
-  /* Q blocks are counted over storage lengths ("Constraints: block split"). */
-  c.q_block_base = (int64_t*)malloc(sizeof(int64_t) * (size_t)B);
-  if (!c.q_block_base) return 11;
-  int64_t acc = 0;
-  for (int32_t b = 0; b < B; b++) {
-    c.q_block_base[b] = acc;
-    const int64_t qs = cu_seqlens_q[b + 1] - cu_seqlens_q[b];
-    if (qs < 0) { free(c.q_block_base); return 12; }
-    acc += (qs + block_x - 1) / block_x;
-  }
-  if (acc != total_q_blocks || cu_seqlens_q[0] != 0 || cu_seqlens_q[B] != T) {
-    free(c.q_block_base);
-    return 13;
-  }
+  const int qrc = q_block_bases(&c);
+  if (qrc) return qrc;
 
   if (n_threads < 1) n_threads = 1;
   if (n_threads > 256) n_threads = 256;
@@ -371,59 +387,22 @@ int gbsa_oracle_attention_backward(int32_t B, int32_t T, int32_t N1, int32_t N2,
   c.q = q; c.k = k; c.v = v; c.sparse_idx = sparse_idx; c.sparse_count = sparse_count;
   c.cu_seqlens_q = cu_seqlens_q; c.seqused_q = seqused_q; c.seqused_kv = seqused_kv;
   c.block_table = block_table; c.cu_seqlens_kv = cu_seqlens_kv;
-  c.q_block_base = (int64_t*)malloc(sizeof(int64_t) * (size_t)B);
-  if (!c.q_block_base) return 11;
-  int64_t acc = 0;
-  for (int32_t b = 0; b < B; b++) {
-    c.q_block_base[b] = acc;
-    const int64_t qs = cu_seqlens_q[b + 1] - cu_seqlens_q[b];
-    if (qs < 0) { free(c.q_block_base); return 12; }
-    acc += (qs + block_x - 1) / block_x;
-  }
-  if (acc != total_q_blocks || cu_seqlens_q[0] != 0 || cu_seqlens_q[B] != T) {
-    free(c.q_block_base);
-    return 13;
-  }
+  const int qrc = q_block_bases(&c);
+  if (qrc) return qrc;
   const int64_t cap = (int64_t)top_k * ORACLE_PAGE;
   double* score = (double*)malloc(sizeof(double) * (size_t)cap);
   int64_t* key_page = (int64_t*)malloc(sizeof(int64_t) * (size_t)cap);
   int32_t* key_row = (int32_t*)malloc(sizeof(int32_t) * (size_t)cap);
   double* out = (double*)malloc(sizeof(double) * (size_t)D);
   int rc = (!score || !key_page || !key_row || !out) ? 11 : 0;
-  const int32_t G = N1 / N2;
   for (int64_t tg = 0; tg < T && !rc; tg++) {
     for (int32_t h = 0; h < N1 && !rc; h++) {
       double lse;
-      /* the keys of (tg, h) in key_page / key_row and their scores, then O */
-      rc = one_row(&c, tg, h, out, &lse, NULL, NULL, score, key_page, key_row);
-      if (rc || lse == -INFINITY) continue;
-      /* the key count: one_row leaves it implicit, so enumerate again the way
-         it does (visible positions of every in-range entry, in list order) */
-      const int32_t b = find_sequence(&c, tg);
-      const int64_t t = tg - cu_seqlens_q[b];
-      const int64_t qs = cu_seqlens_q[b + 1] - cu_seqlens_q[b];
-      const int64_t qu = seqused_q ? (int64_t)seqused_q[b] : qs;
-      const int64_t ku = seqused_kv[b];
-      const int32_t kvh = h / G;
-      const int64_t qb = c.q_block_base[b] + t / block_x;
-      int64_t n = sparse_count[(int64_t)kvh * total_q_blocks + qb];
-      if (n < 0) n = 0;
-      if (n > top_k) n = top_k;
-      const int64_t pos = t + (ku - qu);
-      const int64_t blocks_in_seq = (ku + ORACLE_PAGE - 1) / ORACLE_PAGE;
-      const int32_t* list = sparse_idx + ((int64_t)kvh * total_q_blocks + qb) * top_k;
       int64_t nk = 0;
-      for (int64_t j = 0; j < n; j++) {
-        const int64_t lb = list[j];
-        if (lb < 0 || lb >= blocks_in_seq) continue;
-        for (int32_t r = 0; r < ORACLE_PAGE; r++) {
-          const int64_t p = lb * ORACLE_PAGE + r;
-          if (p >= ku || p > pos) continue;
-          if (win_left >= 0 && p < pos - win_left) continue;
-          if (win_right >= 0 && p > pos + win_right) continue;
-          nk++;
-        }
-      }
+      int32_t kvh = 0;
+      /* the visible keys of (tg, h) (pages, rows, scores), its KV head and O */
+      rc = one_row(&c, tg, h, out, &lse, NULL, NULL, score, key_page, key_row, &nk, &kvh);
+      if (rc || lse == -INFINITY) continue;
       const uint16_t* qrow = q + (tg * N1 + h) * (int64_t)D;
       const uint16_t* grow = dout + (tg * N1 + h) * (int64_t)D;
       double dlt = 0.0, dlt_abs = 0.0;
