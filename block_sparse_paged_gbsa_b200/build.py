@@ -15,7 +15,7 @@ import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
-SOURCES = ["gbsa_api.cu", "gbsa_meta.cu", "gbsa_fwd.cu", "gbsa_static_scratch.cu"]
+SOURCES = ["gbsa_api.cu", "gbsa_meta.cu", "gbsa_fwd.cu", "gbsa_bwd.cu", "gbsa_static_scratch.cu"]
 HEADERS = ["gbsa_internal.cuh", "sm100.cuh"]
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 OUT = os.path.join(HERE, "libgbsa.so")

@@ -31,6 +31,16 @@ cudaError_t launch_forward(const CUtensorMap& map_q, const CUtensorMap& map_k,
                            int32_t num_ctas, int64_t comb_cap, bool one_tile_blocks,
                            int32_t dtype, bool half_softmax, float out_scale,
                            uint64_t wait_limit_ns, cudaStream_t stream);
+size_t backward_smem_bytes();
+cudaError_t launch_backward(const int32_t* meta, const void* q, const void* k, const void* v,
+                            const void* out, const void* dout, const float* lse,
+                            const int32_t* block_table, const int64_t* cu_seqlens_kv, float* dq,
+                            float* dk, float* dv, size_t dk_bytes, float* delta,
+                            int32_t* dev_status, uint32_t signature, int32_t N1, int32_t N2,
+                            int32_t T, int32_t T_kv, int32_t top_k, int32_t max_pages,
+                            int32_t num_pages, int64_t kv_page_stride, int32_t tile_tokens,
+                            int32_t tiles_max, int32_t n_items, int32_t win_left, float scale,
+                            int32_t dtype, cudaStream_t stream);
 }  // namespace gbsa
 
 using namespace gbsa;
@@ -358,6 +368,53 @@ gbsa_status gbsa_forward(const gbsa_problem* problem, const gbsa_tensors* t, voi
       g.comb_cap, g.tiles_max == 1, problem->dtype, problem->softmax_precision == 1,
       fp8 ? (float)problem->v_scale : 1.f,
       problem->wait_limit_ns > 0 ? (uint64_t)problem->wait_limit_ns : kDefaultWaitLimitNs,
+      static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return GBSA_ERR_CUDA;
+  }
+  return GBSA_OK;
+}
+
+gbsa_status gbsa_backward_workspace_size(const gbsa_problem* problem, size_t* bytes) {
+  if (!bytes) return GBSA_ERR_INVALID_ARG;
+  const gbsa_status st = validate(problem, false);
+  if (st != GBSA_OK) return st;
+  *bytes = (size_t)(((int64_t)problem->T * problem->N1 * 4 + 15) / 16 * 16);
+  return GBSA_OK;
+}
+
+gbsa_status gbsa_backward(const gbsa_problem* problem, const gbsa_tensors* t, const void* dout,
+                          const void* meta, float* dq, float* dk, float* dv, void* workspace,
+                          size_t ws_bytes, int32_t* dev_status, void* stream) {
+  gbsa_status st = validate(problem, false);
+  if (st != GBSA_OK) return st;
+  if (problem->dtype == GBSA_DTYPE_FP8_E4M3) return GBSA_ERR_UNSUPPORTED;
+  const bool tnd = problem->kv_layout == GBSA_KV_TND;
+  if (!t || !meta || !dout || !dq || !dk || !dv || !t->q || !t->k || !t->v || !t->out || !t->lse ||
+      !t->sparse_idx || !t->sparse_count || !t->cu_seqlens_q || !t->seqused_kv ||
+      (tnd ? !t->cu_seqlens_kv : !t->block_table) || (problem->has_seqused_q && !t->seqused_q))
+    return GBSA_ERR_INVALID_ARG;
+  if (!aligned16(t->q) || !aligned16(t->k) || !aligned16(t->v) || !aligned16(t->out) ||
+      !aligned16(dout) || !aligned16(meta) || !aligned16(dq) || !aligned16(dk) ||
+      !aligned16(dv) || (reinterpret_cast<uintptr_t>(t->lse) & 3u))
+    return GBSA_ERR_ALIGNMENT;
+  size_t need = 0;
+  if ((st = gbsa_backward_workspace_size(problem, &need)) != GBSA_OK) return st;
+  if (ws_bytes < need || !workspace || !aligned16(workspace)) return GBSA_ERR_WORKSPACE_TOO_SMALL;
+  int32_t ctas;
+  if ((st = resolve_ctas(problem, &ctas)) != GBSA_OK) return st;
+  const Geometry g = make_geometry(problem, ctas);
+  const int64_t kv_rows = tnd ? (int64_t)problem->T_kv : (int64_t)problem->num_pages * kPage;
+  const size_t dk_bytes = (size_t)(kv_rows * problem->N2 * kHeadDim) * sizeof(float);
+  const double scale = problem->scale > 0.0 ? problem->scale : 1.0 / sqrt((double)problem->D);
+  const cudaError_t e = launch_backward(
+      static_cast<const int32_t*>(meta), t->q, t->k, t->v, t->out, dout, t->lse,
+      tnd ? nullptr : t->block_table, tnd ? t->cu_seqlens_kv : nullptr, dq, dk, dv, dk_bytes,
+      static_cast<float*>(workspace), dev_status, problem_signature(problem, ctas), problem->N1,
+      problem->N2, problem->T, tnd ? problem->T_kv : 0, problem->top_k,
+      problem->max_pages_per_seq, problem->num_pages, tnd ? 0 : problem->kv_page_stride,
+      g.tile_tokens, g.tiles_max, g.n_items, problem->win_left, (float)scale, problem->dtype,
       static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) {
     cudaGetLastError();

@@ -156,6 +156,10 @@ def _load():
         lib.gbsa_metadata.restype = ctypes.c_int
         lib.gbsa_forward.argtypes = [P, Tn, vp, vp, sz, vp, vp]
         lib.gbsa_forward.restype = ctypes.c_int
+        lib.gbsa_backward_workspace_size.argtypes = [P, ctypes.POINTER(sz)]
+        lib.gbsa_backward_workspace_size.restype = ctypes.c_int
+        lib.gbsa_backward.argtypes = [P, Tn, vp, vp, vp, vp, vp, vp, sz, vp, vp]
+        lib.gbsa_backward.restype = ctypes.c_int
         if lib.gbsa_abi_version() != ABI_VERSION:
             raise RuntimeError("libgbsa ABI version mismatch")
         _lib = lib
@@ -442,3 +446,79 @@ def forward(q, k, v, sparse_block_idx, sparse_block_count, block_shape: Sequence
 
 def decode_dev_status(word: int) -> list:
     return [name for bit, name in DEV_BITS.items() if word & bit]
+
+
+def backward(dout, q, k, v, out, lse, sparse_block_idx, sparse_block_count,
+             block_shape: Sequence[int], *, metadata, cu_seqlens_q, seqused_kv, block_table=None,
+             seqused_q=None, cu_seqlens_kv=None, softmax_scale: float = 0.0, win_left: int = -1,
+             win_right: int = -1, num_ctas: int = 0, max_blocks_per_split: int = 0, dq=None,
+             dk=None, dv=None, workspace=None, dev_status=None):
+    """Gradients of out for the incoming gradient ``dout`` ([T, N1, D], the type
+    of q): returns (dq, dk, dv) in fp32 -- dq [T, N1, D]; dk, dv compact
+    [num_pages, 128, N2, D] for the page pool (whatever its page stride), or
+    [T_kv, N2, D] for TND.  ``out`` and ``lse`` are the forward's results for
+    the same inputs (lse [T, N1, 1] or [T, N1]); the other arguments, and
+    ``metadata``, ``num_ctas`` and ``max_blocks_per_split``, are those of that
+    forward call.  bf16 and fp16 only.  The pages give no backward: this is
+    the exact gradient of the forward's function (a library addition)."""
+    import torch
+    q = _need(q, "q", q.dtype, 3)
+    dev = q.device
+    if q.dtype not in (torch.bfloat16, torch.float16):
+        raise ValueError("backward: bf16 or fp16 inputs only")
+    tnd = cu_seqlens_kv is not None
+    for name, t in (("k", k), ("v", v)):
+        if t is None or t.dtype != q.dtype or t.device != dev or t.dim() != (3 if tnd else 4):
+            raise ValueError(f"{name}: expected {q.dtype} on {dev}, "
+                             f"{'[T_kv, N2, D]' if tnd else '[num_pages, 128, N2, D]'}")
+        if tnd and not t.is_contiguous():
+            raise ValueError(f"{name}: TND k / v must be contiguous")
+        if not tnd and t.stride()[1:] != (t.shape[2] * t.shape[3], t.shape[3], 1):
+            raise ValueError(f"{name}: only dim0 (the page axis) may be strided")
+    if k.shape != v.shape or k.stride() != v.stride():
+        raise ValueError("k and v must have the same shape and strides")
+    dout = _need(dout, "dout", q.dtype, 3, dev)
+    out = _need(out, "out", q.dtype, 3, dev)
+    if dout.shape != q.shape or out.shape != q.shape:
+        raise ValueError("dout, out: expected the shape of q")
+    T, N1, D = q.shape
+    lse = _need(lse.reshape(T, N1) if lse is not None else None, "lse", torch.float32, 2, dev)
+    idx = _need(sparse_block_idx, "sparse_block_idx", torch.int32, 3, dev)
+    cnt = _need(sparse_block_count, "sparse_block_count", torch.int32, 2, dev)
+    cu = _need(cu_seqlens_q, "cu_seqlens_q", torch.int64, 1, dev)
+    sku = _need(seqused_kv, "seqused_kv", torch.int32, 1, dev)
+    bt = None if tnd else _need(block_table, "block_table", torch.int32, 2, dev)
+    cukv = _need(cu_seqlens_kv, "cu_seqlens_kv", torch.int64, 1, dev) if tnd else None
+    squ = None if seqused_q is None else _need(seqused_q, "seqused_q", torch.int32, 1, dev)
+    meta = _need(metadata, "metadata", torch.int32, 1, dev)
+    prob = make_problem(q, k, idx, block_shape, bt, cu, softmax_scale=softmax_scale,
+                        win_left=win_left, win_right=win_right, has_seqused_q=squ is not None,
+                        num_ctas=num_ctas, max_blocks_per_split=max_blocks_per_split)
+    kv_shape = (k.shape[0], k.shape[1], k.shape[2], k.shape[3]) if not tnd else tuple(k.shape)
+    with torch.cuda.device(dev):
+        dq = torch.empty((T, N1, D), dtype=torch.float32, device=dev) if dq is None else \
+            _need(dq, "dq", torch.float32, 3, dev)
+        dk = torch.empty(kv_shape, dtype=torch.float32, device=dev) if dk is None else dk
+        dv = torch.empty(kv_shape, dtype=torch.float32, device=dev) if dv is None else dv
+        for name, t in (("dk", dk), ("dv", dv)):
+            if t.dtype != torch.float32 or tuple(t.shape) != kv_shape or not t.is_contiguous():
+                raise ValueError(f"{name}: expected a contiguous fp32 tensor of shape {kv_shape}")
+        n = ctypes.c_size_t(0)
+        _check(_load().gbsa_backward_workspace_size(ctypes.byref(prob.as_c()), ctypes.byref(n)),
+               "gbsa_backward_workspace_size")
+        if workspace is None:
+            workspace = torch.empty((max(int(n.value), 16),), dtype=torch.uint8, device=dev)
+        if dev_status is not None:
+            dev_status = _need(dev_status, "dev_status", torch.int32, 1, dev)
+        ten = _Tensors(q=_ptr(q), k=_ptr(k), v=_ptr(v), sparse_idx=_ptr(idx),
+                       sparse_count=_ptr(cnt), cu_seqlens_q=_ptr(cu), seqused_q=_ptr(squ),
+                       seqused_kv=_ptr(sku), block_table=_ptr(bt), out=_ptr(out), lse=_ptr(lse),
+                       cu_seqlens_kv=_ptr(cukv))
+        _check(_load().gbsa_backward(ctypes.byref(prob.as_c()), ctypes.byref(ten), _ptr(dout),
+                                     meta.data_ptr(), _ptr(dq), _ptr(dk), _ptr(dv),
+                                     workspace.data_ptr(),
+                                     workspace.numel() * workspace.element_size(),
+                                     _ptr(dev_status), _stream_handle()),
+               "gbsa_backward")
+    return dq, dk, dv
+

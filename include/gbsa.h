@@ -261,6 +261,40 @@ GBSA_API gbsa_status gbsa_forward_static_scratch(const gbsa_problem* problem,
                                                  const gbsa_tensors* tensors, void* meta,
                                                  int32_t* dev_status, void* stream);
 
+/* Bytes of device scratch gbsa_backward() needs: one fp32 per (token, query
+ * head), T * N1 * 4 rounded up to 16. */
+GBSA_API gbsa_status gbsa_backward_workspace_size(const gbsa_problem* problem, size_t* bytes);
+
+/* Gradients of the attention output, for training (the GBSA article's
+ * overview names training as a use of the operator but specifies no
+ * backward; this is the exact gradient of the forward's function, a
+ * library addition).  Given dout (the gradient of the loss with respect to
+ * out: [T][N1][D], the element type of q) it computes
+ *   dq [T][N1][D]                       fp32, every row written (0 where a
+ *                                       row has no visible key or lies past
+ *                                       seqused_q);
+ *   dk, dv                              fp32, compact: [num_pages][128][N2][D]
+ *                                       for the paged pool (page p's rows at
+ *                                       p * 128 * N2 * D, whatever the pool's
+ *                                       kv_page_stride), or [T_kv][N2][D] for
+ *                                       TND; zeroed by the call, then summed
+ *                                       over every row and list entry that
+ *                                       reads a key (a block listed twice
+ *                                       counts twice, as in the forward).
+ * Inputs are those of the forward call plus its results: tensors->out and
+ * tensors->lse (lse required, whatever problem->return_lse says) for the
+ * same q, k, v and lists; `meta` is the work list gbsa_metadata() built for
+ * this problem (read only here).  bf16 and fp16 only (E4M3:
+ * GBSA_ERR_UNSUPPORTED); softmax_precision is ignored (the gradient of the
+ * exact softmax).  `workspace` (16-byte aligned, ws_bytes >=
+ * gbsa_backward_workspace_size()) is overwritten.  All pointers 16-byte
+ * aligned except lse (4).  Errors as for gbsa_forward(); a page index out of
+ * range sets GBSA_DEV_BAD_PAGE and skips the block. */
+GBSA_API gbsa_status gbsa_backward(const gbsa_problem* problem, const gbsa_tensors* tensors,
+                                   const void* dout, const void* meta, float* dq, float* dk,
+                                   float* dv, void* workspace, size_t ws_bytes,
+                                   int32_t* dev_status, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
