@@ -82,6 +82,9 @@ def parse_args():
     ap.add_argument("--softmax-precision", type=int, default=0, choices=[0, 1],
                     help="the article's softmaxPrecision (0: fp32 online softmax; 1: "
                          "half-precision exponentials with fp32 rescale and row sums)")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the gradient computation (gbsa.backward) of one workload "
+                         "(dense unless --workload names another) instead of the forward")
     ap.add_argument("--scale-down", type=int, default=1,
                     help="shrink the workload's sequence lengths by this factor (same "
                          "structure); for profiler captures that must stay small")
@@ -566,6 +569,83 @@ def measure(name, args, dev, world, rank, sampler, dist, headline):
     return res, e2e, cpu
 
 
+def measure_backward(name, args, dev, sampler):
+    """Times gbsa.backward on one workload: the forward runs once first (out and
+    lse are its inputs), then args.steps backward calls with CUDA events and
+    the L2 flushed between them.  FLOPs: the five products per (tile, block)
+    against the forward's two, block-granular."""
+    import torch
+
+    import block_sparse_paged_gbsa_b200 as gbsa
+    from block_sparse_paged_gbsa_b200.accounting import work
+    from block_sparse_paged_gbsa_b200.workloads import make_values, pool_view, workload
+
+    w = workload(name, scale_down=args.scale_down)
+    tdt = {"bf16": torch.bfloat16, "fp16": torch.float16}[args.dtype]
+    acc = work(w, in_bytes=2)
+    q, kf, vf = make_values(w, dev, dtype=tdt)
+    to = lambda a, dt: torch.as_tensor(np.ascontiguousarray(a), dtype=dt, device=dev)
+    idx, cnt = to(w.sparse_idx, torch.int32), to(w.sparse_count, torch.int32)
+    cu, sku, bt = to(w.cu_seqlens_q, torch.int64), to(w.kv_used, torch.int32), to(w.block_table, torch.int32)
+    squ = to(w.q_used, torch.int32) if w.has_seqused_q else None
+    k, v = pool_view(w, kf), pool_view(w, vf)
+    bs = [w.block_x, 128]
+    meta = gbsa.metadata(idx, cnt, w.N1, w.N2, w.D, bs, cu_seqlens_q=cu, seqused_q=squ,
+                         seqused_kv=sku, num_tokens=w.T, win_left=w.win_left,
+                         win_right=w.win_right)
+    kw = dict(metadata=meta, cu_seqlens_q=cu, seqused_q=squ, seqused_kv=sku, block_table=bt,
+              softmax_scale=w.scale, win_left=w.win_left, win_right=w.win_right)
+    out, lse = gbsa.forward(q, k, v, idx, cnt, bs, return_softmax_lse=True, **kw)
+    g = torch.Generator(device=dev).manual_seed(99)
+    dout = torch.randn(q.shape, generator=g, device=dev, dtype=torch.float32).to(tdt)
+    dq = torch.empty(q.shape, dtype=torch.float32, device=dev)
+    dk = torch.empty(k.shape, dtype=torch.float32, device=dev)
+    dv = torch.empty(k.shape, dtype=torch.float32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step():
+        gbsa.backward(dout, q, k, v, out, lse, idx, cnt, bs, dq=dq, dk=dk, dv=dv,
+                      dev_status=status, **kw)
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    t_wall0 = time.time()
+    for e in events:
+        flush.zero_()
+        e[0].record()
+        step()
+        e[1].record()
+    torch.cuda.synchronize()
+    clocks = sampler.window(t_wall0, time.time())
+    ms = float(np.mean([e[0].elapsed_time(e[1]) for e in events]))
+    flops = 2.5 * acc["flops_block"]
+    peaks = load_peaks()
+    achieved = flops / (ms * 1e-3) / 1e12
+    sm_clock = 1.965e9
+    fma_peak = 148 * 128 * 2 * sm_clock / 1e12  # fp32 FMA pipes, nominal clock
+    return {
+        "metric": "effective backward TFLOPS (dQ, dK, dV; block-granular FLOPs = 2.5 x the forward's)",
+        "value": round(achieved, 4), "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": round(ms, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": args.dtype, "data": "synthetic",
+        "config": {"workload": describe(name, args) + " -- backward",
+                   "l2": "flushed between timed steps (256 MiB write)"},
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 3),
+                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": round(achieved / peaks["bf16_tflops"], 4), "traffic": None,
+                     "kernel": "gbsa backward (delta + gradient kernels; fp32 FMA products)",
+                     "peak_source": peaks["source"] + " (burst)",
+                     "fp32_fma_peak_tflops": round(fma_peak, 1),
+                     "frac_of_fp32_fma_peak": round(achieved / fma_peak, 4)},
+        "clocks": clocks, "gpu_launches": 2 * args.steps, "dev_status": int(status.item()),
+        "e2e": None, "cpu_baseline": None,
+    }
+
+
 def main():
     args = parse_args()
     world, rank, local = dist_info()
@@ -584,6 +664,19 @@ def main():
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
+
+    if args.backward:
+        if world > 1:
+            raise SystemExit("--backward runs on one GPU")
+        sampler = ClockSampler(local)
+        sampler.start()
+        try:
+            line = measure_backward("dense" if args.workload == "all" else args.workload, args,
+                                    dev, sampler)
+        finally:
+            sampler.stop()
+        print(json.dumps(line), flush=True)
+        return
 
     names = ORDER if args.workload == "all" else [args.workload]
     head = headline_name(args)
