@@ -625,8 +625,6 @@ def measure_backward(name, args, dev, sampler):
     flops = 2.5 * acc["flops_block"]
     peaks = load_peaks()
     achieved = flops / (ms * 1e-3) / 1e12
-    sm_clock = 1.965e9
-    fma_peak = 148 * 128 * 2 * sm_clock / 1e12  # fp32 FMA pipes, nominal clock
     return {
         "metric": "effective backward TFLOPS (dQ, dK, dV; block-granular FLOPs = 2.5 x the forward's)",
         "value": round(achieved, 4), "unit": UNIT, "n_gpus": 1, "steps": args.steps,
@@ -637,10 +635,8 @@ def measure_backward(name, args, dev, sampler):
         "roofline": {"bound": "tensor", "achieved": round(achieved, 3),
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": round(achieved / peaks["bf16_tflops"], 4), "traffic": None,
-                     "kernel": "gbsa backward (delta + gradient kernels; fp32 FMA products)",
-                     "peak_source": peaks["source"] + " (burst)",
-                     "fp32_fma_peak_tflops": round(fma_peak, 1),
-                     "frac_of_fp32_fma_peak": round(achieved / fma_peak, 4)},
+                     "kernel": "gbsa backward (delta + gradient kernels; mma.sync products)",
+                     "peak_source": peaks["source"] + " (burst)"},
         "clocks": clocks, "gpu_launches": 2 * args.steps, "dev_status": int(status.item()),
         "e2e": None, "cpu_baseline": None,
     }

@@ -14,10 +14,11 @@
 // dQ of its rows stays in registers and is written once, dK and dV of each
 // key are added to fp32 outputs with vector atomics (many tiles read a key).
 //
-// This first version does its five 128 x 128 x 128 products per block with
-// fp32 FMAs from shared memory (16-bit tiles, rows padded to 65 words so
-// that the rows a warp reads fall in distinct banks); the tensor-core form
-// (tcgen05 products with dK / dV accumulated per KV block) is the next step.
+// The five 128 x 128 x 128 products per block run on the tensor cores as
+// warp-level mma.sync (m16n8k16, fp32 accumulators) fed by ldmatrix from
+// padded shared tiles; P and dS enter them in the element type of q.  Each
+// of the 8 warps owns a 32 x 64 tile of every product.  (The tcgen05 form,
+// with dK / dV accumulated per KV block in TMEM, is the next step.)
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -33,12 +34,13 @@ using namespace sm100;
 
 namespace {
 
-constexpr int kBwdThreads = 256;
-constexpr int kRowWords = 65;  // 128 16-bit elements + one padding word per row
-constexpr int kTileWords = 128 * kRowWords;
-constexpr size_t kBwdSmem = 4 * kTileWords * 4     // Q, dO, K, V (16-bit pairs)
-                            + 128 * 128 * 4         // P, then dS (fp32)
-                            + 3 * 128 * 4;          // per row: lse (log2 units), delta, position
+constexpr int kBwdThreads = 256;  // 8 warps, each a 32 x 64 tile of every product
+// 16-bit tiles of 128 rows x 128 elements; rows padded to 136 elements (272 B)
+// so that the 8 rows an ldmatrix reads start in distinct bank groups
+constexpr int kRowElems = 136;
+constexpr int kTileElems = 128 * kRowElems;
+constexpr size_t kBwdSmem = 6 * kTileElems * 2  // Q, dO, K, V, P, dS
+                            + 3 * 128 * 4;      // per row: lse (log2 units), delta, position
 static_assert(kBwdSmem <= 232448, "shared memory budget");
 
 struct BwdParams {
@@ -87,31 +89,111 @@ __global__ void __launch_bounds__(256) delta_kernel(const BwdParams p) {
 }
 
 // 128 rows of 128 16-bit elements from global rows at `src(r)` (nullptr: a
-// row of zeros) into a padded shared tile.  Whole CTA.
+// row of zeros) into a padded shared tile (row stride kRowElems).  Whole CTA.
 template <typename F>
-__device__ __forceinline__ void load_tile(uint32_t* tile, F src) {
+__device__ __forceinline__ void load_tile(uint16_t* tile, F src) {
   for (int i = threadIdx.x; i < 128 * 16; i += kBwdThreads) {
     const int r = i >> 4, c = i & 15;  // row, 16-byte chunk
     const uint16_t* s = src(r);
     uint4 v = make_uint4(0, 0, 0, 0);
     if (s) v = reinterpret_cast<const uint4*>(s)[c];
-    uint32_t* d = tile + r * kRowWords + 4 * c;
-    d[0] = v.x;
-    d[1] = v.y;
-    d[2] = v.z;
-    d[3] = v.w;
+    *reinterpret_cast<uint4*>(tile + r * kRowElems + 8 * c) = v;
   }
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const uint16_t* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_u32(p)));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], const uint16_t* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_u32(p)));
+}
+
+// D += A B for one m16 n8 k16 tile, fp32 accumulators.
+template <int kDt>
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+  if constexpr (kDt == 1)
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  else
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// One warp's 32 x 64 tile of C = A B over K = 128, from shared 16-bit
+// tiles with row stride kRowElems:
+//   A: kATrans ? stored [k][m] (A = stored^T) : stored [m][k];
+//   B: kBTrans ? stored [k][n]               : stored [n][k] (B = stored^T).
+// The warp's rows are m0 .. m0 + 31, its columns n0 .. n0 + 63;
+// acc[tm][tn] is the m16 n8 fragment at (m0 + 16 tm, n0 + 8 tn).
+template <int kDt, bool kATrans, bool kBTrans>
+__device__ __forceinline__ void warp_gemm(float (&acc)[2][8][4], const uint16_t* A,
+                                          const uint16_t* B, int m0, int n0) {
+  const int lane = threadIdx.x & 31;
+  const int i8 = lane >> 3, j8 = lane & 7;
+#pragma unroll 1
+  for (int k0 = 0; k0 < 128; k0 += 16) {
+    uint32_t a[2][4];
+#pragma unroll
+    for (int tm = 0; tm < 2; tm++) {
+      const int mb = m0 + 16 * tm;
+      if constexpr (kATrans)  // matrices (m, k), (m+8, k), (m, k+8), (m+8, k+8)
+        ldsm_x4_t(a[tm], A + (k0 + (i8 >> 1) * 8 + j8) * kRowElems + mb + (i8 & 1) * 8);
+      else
+        ldsm_x4(a[tm], A + (mb + (lane & 15)) * kRowElems + k0 + (lane >> 4) * 8);
+    }
+#pragma unroll
+    for (int tp = 0; tp < 4; tp++) {  // pairs of n8 tiles
+      const int nb = n0 + 16 * tp;
+      uint32_t b[4];  // b0, b1 of tile nb, then of tile nb + 8
+      if constexpr (kBTrans)  // matrices (k, n), (k+8, n), (k, n+8), (k+8, n+8)
+        ldsm_x4_t(b, B + (k0 + (i8 & 1) * 8 + j8) * kRowElems + nb + (i8 >> 1) * 8);
+      else
+        ldsm_x4(b, B + (nb + (i8 >> 1) * 8 + j8) * kRowElems + k0 + (i8 & 1) * 8);
+#pragma unroll
+      for (int tm = 0; tm < 2; tm++) {
+        mma16816<kDt>(acc[tm][2 * tp], a[tm], b[0], b[1]);
+        mma16816<kDt>(acc[tm][2 * tp + 1], a[tm], b[2], b[3]);
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void zero_acc(float (&acc)[2][8][4]) {
+#pragma unroll
+  for (int tm = 0; tm < 2; tm++)
+#pragma unroll
+    for (int tn = 0; tn < 8; tn++)
+#pragma unroll
+      for (int e = 0; e < 4; e++) acc[tm][tn][e] = 0.f;
+}
+
+// Two floats as a 16-bit pair of the element type (the lower first).
+template <int kDt>
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+  return kDt == 1 ? pack_f16x2(lo, hi) : pack_bf16x2(lo, hi);
 }
 
 template <int kDt>
 __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kernel(const BwdParams p) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
-  uint32_t* sQ = reinterpret_cast<uint32_t*>(smem_raw);
-  uint32_t* sG = sQ + kTileWords;  // dO
-  uint32_t* sK = sG + kTileWords;
-  uint32_t* sV = sK + kTileWords;
-  float* sP = reinterpret_cast<float*>(sV + kTileWords);  // [128 rows][128 keys]
-  float* sL = sP + 128 * 128;                              // lse * log2(e), -inf: no weight
+  uint16_t* sQ = reinterpret_cast<uint16_t*>(smem_raw);
+  uint16_t* sG = sQ + kTileElems;  // dO
+  uint16_t* sK = sG + kTileElems;
+  uint16_t* sV = sK + kTileElems;
+  uint16_t* sP = sV + kTileElems;   // P [row][key], in the element type
+  uint16_t* sS = sP + kTileElems;   // dS [row][key]
+  float* sL = reinterpret_cast<float*>(sS + kTileElems);  // lse * log2(e), -inf: no weight
   float* sD = sL + 128;                                    // delta
   int32_t* sPos = reinterpret_cast<int32_t*>(sD + 128);   // query position
 
@@ -133,9 +215,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kernel(const BwdParams p) 
   const int32_t kvh = item % p.N2;
   const int32_t rows_in_tile = p.tile_tokens * p.G;
 
-  // rows of this tile: token offset r / G in the tile, head r % G
-  // (a token past T, which only inconsistent lengths give, is left alone:
-  // the metadata status has flagged them)
+  // rows of this tile: token offset r / G in the tile, head r % G (a token
+  // past T, which only inconsistent lengths give, is left alone: the
+  // metadata status has flagged them)
   auto row_tok = [&](int r) { return s * p.tile_tokens + r / p.G; };
   auto in_t = [&](int r) { return tok_begin + row_tok(r) < p.T; };
   auto row_valid = [&](int r) { return r < rows_in_tile && row_tok(r) < n_store && in_t(r); };
@@ -154,13 +236,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kernel(const BwdParams p) 
     sPos[r] = pos0 + row_tok(r);
   }
 
-  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
-  // ownership: rows / keys ty + 16 i and tx + 16 j; head-dim pairs tx + 16 j
-  float dq[8][8];
-#pragma unroll
-  for (int i = 0; i < 8; i++)
-#pragma unroll
-    for (int j = 0; j < 8; j++) dq[i][j] = 0.f;
+  // warp w owns rows (or keys) 32 (w >> 1) .. + 31 and columns 64 (w & 1) .. + 63
+  // of every 128 x 128 product; a fragment element e of tile (tm, tn) sits at
+  // row m0 + 16 tm + lane / 4 + 8 (e >> 1), column n0 + 8 tn + 2 (lane % 4) + (e & 1)
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = 32 * (warp >> 1), n0 = 64 * (warp & 1);
+  const int fr = lane >> 2, fc = 2 * (lane & 3);
+  float dq[2][8][4];
+  zero_acc(dq);
 
   const int32_t* list = meta + off_list + (int64_t)item * p.top_k;
   const bool tnd = p.cu_kv != nullptr;
@@ -194,174 +277,101 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kernel(const BwdParams p) 
     });
     __syncthreads();
 
-    // ---- S and P = exp(s - lse) on visible (row, key) pairs
-    {
-      float acc[8][8];
+    float acc[2][8][4];
+    // ---- S = Q K^T, then P = exp(s - lse) on visible (row, key) pairs
+    zero_acc(acc);
+    warp_gemm<kDt, false, false>(acc, sQ, sK, m0, n0);
 #pragma unroll
-      for (int i = 0; i < 8; i++)
+    for (int tm = 0; tm < 2; tm++)
 #pragma unroll
-        for (int j = 0; j < 8; j++) acc[i][j] = 0.f;
-#pragma unroll 2
-      for (int dp = 0; dp < 64; dp++) {
-        float2 qv[8], kv[8];
-#pragma unroll
-        for (int i = 0; i < 8; i++) qv[i] = widen2<kDt>(sQ[(ty + 16 * i) * kRowWords + dp]);
-#pragma unroll
-        for (int j = 0; j < 8; j++) kv[j] = widen2<kDt>(sK[(tx + 16 * j) * kRowWords + dp]);
-#pragma unroll
-        for (int i = 0; i < 8; i++)
-#pragma unroll
-          for (int j = 0; j < 8; j++) acc[i][j] += qv[i].x * kv[j].x + qv[i].y * kv[j].y;
-      }
-#pragma unroll
-      for (int i = 0; i < 8; i++) {
-        const int r = ty + 16 * i;
+      for (int h = 0; h < 2; h++) {
+        const int r = m0 + 16 * tm + fr + 8 * h;
         const int32_t pos = sPos[r];
         const float l2 = sL[r];
 #pragma unroll
-        for (int j = 0; j < 8; j++) {
-          const int c = tx + 16 * j;
-          const int32_t key = lb * kPage + c;
-          const bool vis = l2 != -INFINITY && key < ku && key <= pos &&
-                           (p.win_left < 0 || key >= pos - p.win_left);
-          sP[r * 128 + c] = vis ? fast_exp2(acc[i][j] * p.scale_log2 - l2) : 0.f;
+        for (int tn = 0; tn < 8; tn++) {
+          const int c = n0 + 8 * tn + fc;
+          float pv[2];
+#pragma unroll
+          for (int u = 0; u < 2; u++) {
+            const int32_t key = lb * kPage + c + u;
+            const bool vis = l2 != -INFINITY && key < ku && key <= pos &&
+                             (p.win_left < 0 || key >= pos - p.win_left);
+            pv[u] = vis ? fast_exp2(acc[tm][tn][2 * h + u] * p.scale_log2 - l2) : 0.f;
+          }
+          *reinterpret_cast<uint32_t*>(sP + r * kRowElems + c) = pack2<kDt>(pv[0], pv[1]);
         }
       }
-    }
     __syncthreads();
 
-    // ---- dV[key][d] += sum_r P[r][key] dO[r][d]   (keys ty + 16 i, d pairs tx + 16 j)
-    {
-      float2 acc[8][4];
+    // ---- dV = P^T dO   (rows: keys, columns: head dim)
+    zero_acc(acc);
+    warp_gemm<kDt, true, true>(acc, sP, sG, m0, n0);
 #pragma unroll
-      for (int i = 0; i < 8; i++)
+    for (int tm = 0; tm < 2; tm++)
 #pragma unroll
-        for (int j = 0; j < 4; j++) acc[i][j] = make_float2(0.f, 0.f);
-#pragma unroll 2
-      for (int r = 0; r < 128; r++) {
-        float pv[8];
-        float2 gv[4];
-#pragma unroll
-        for (int i = 0; i < 8; i++) pv[i] = sP[r * 128 + ty + 16 * i];
-#pragma unroll
-        for (int j = 0; j < 4; j++) gv[j] = widen2<kDt>(sG[r * kRowWords + tx + 16 * j]);
-#pragma unroll
-        for (int i = 0; i < 8; i++)
-#pragma unroll
-          for (int j = 0; j < 4; j++) {
-            acc[i][j].x += pv[i] * gv[j].x;
-            acc[i][j].y += pv[i] * gv[j].y;
-          }
-      }
-#pragma unroll
-      for (int i = 0; i < 8; i++) {
-        const int c = ty + 16 * i;
+      for (int h = 0; h < 2; h++) {
+        const int c = m0 + 16 * tm + fr + 8 * h;
         if (!key_ok(c)) continue;
-        float* dst = p.dv + ((grow0 + c) * p.N2 + kvh) * kHeadDim;
+        float2* dst = reinterpret_cast<float2*>(p.dv + ((grow0 + c) * p.N2 + kvh) * kHeadDim);
 #pragma unroll
-        for (int j = 0; j < 4; j++)
-          atomicAdd(reinterpret_cast<float2*>(dst) + tx + 16 * j, acc[i][j]);
+        for (int tn = 0; tn < 8; tn++)
+          atomicAdd(dst + ((n0 + 8 * tn + fc) >> 1),
+                    make_float2(acc[tm][tn][2 * h], acc[tm][tn][2 * h + 1]));
       }
-    }
 
-    // ---- dS = P (dO . V - delta), in place of P (rows ty + 16 i, keys tx + 16 j)
-    {
-      float acc[8][8];
+    // ---- dS = P (dO V^T - delta)   (P as the products use it: 16-bit)
+    zero_acc(acc);
+    warp_gemm<kDt, false, false>(acc, sG, sV, m0, n0);
 #pragma unroll
-      for (int i = 0; i < 8; i++)
+    for (int tm = 0; tm < 2; tm++)
 #pragma unroll
-        for (int j = 0; j < 8; j++) acc[i][j] = 0.f;
-#pragma unroll 2
-      for (int dp = 0; dp < 64; dp++) {
-        float2 gv[8], vv[8];
-#pragma unroll
-        for (int i = 0; i < 8; i++) gv[i] = widen2<kDt>(sG[(ty + 16 * i) * kRowWords + dp]);
-#pragma unroll
-        for (int j = 0; j < 8; j++) vv[j] = widen2<kDt>(sV[(tx + 16 * j) * kRowWords + dp]);
-#pragma unroll
-        for (int i = 0; i < 8; i++)
-#pragma unroll
-          for (int j = 0; j < 8; j++) acc[i][j] += gv[i].x * vv[j].x + gv[i].y * vv[j].y;
-      }
-      __syncthreads();  // every thread has read P for dV
-#pragma unroll
-      for (int i = 0; i < 8; i++) {
-        const int r = ty + 16 * i;
+      for (int h = 0; h < 2; h++) {
+        const int r = m0 + 16 * tm + fr + 8 * h;
         const float dlt = sD[r];
 #pragma unroll
-        for (int j = 0; j < 8; j++) {
-          const int c = tx + 16 * j;
-          sP[r * 128 + c] = sP[r * 128 + c] * (acc[i][j] - dlt);
+        for (int tn = 0; tn < 8; tn++) {
+          const int c = n0 + 8 * tn + fc;
+          const float2 pv = widen2<kDt>(*reinterpret_cast<const uint32_t*>(sP + r * kRowElems + c));
+          *reinterpret_cast<uint32_t*>(sS + r * kRowElems + c) =
+              pack2<kDt>(pv.x * (acc[tm][tn][2 * h] - dlt), pv.y * (acc[tm][tn][2 * h + 1] - dlt));
         }
       }
-    }
     __syncthreads();
 
-    // ---- dQ[r][d] += scale sum_key dS[r][key] K[key][d]   (rows ty + 16 i, d pairs tx + 16 j)
-#pragma unroll 2
-    for (int c = 0; c < 128; c++) {
-      float sv[8];
-      float2 kv[4];
-#pragma unroll
-      for (int i = 0; i < 8; i++) sv[i] = sP[(ty + 16 * i) * 128 + c];
-#pragma unroll
-      for (int j = 0; j < 4; j++) kv[j] = widen2<kDt>(sK[c * kRowWords + tx + 16 * j]);
-#pragma unroll
-      for (int i = 0; i < 8; i++)
-#pragma unroll
-        for (int j = 0; j < 4; j++) {
-          dq[i][2 * j] += sv[i] * kv[j].x;
-          dq[i][2 * j + 1] += sv[i] * kv[j].y;
-        }
-    }
+    // ---- dQ += dS K   (rows: queries, columns: head dim)
+    warp_gemm<kDt, false, true>(dq, sS, sK, m0, n0);
 
-    // ---- dK[key][d] += scale sum_r dS[r][key] Q[r][d]   (keys ty + 16 i, d pairs tx + 16 j)
-    {
-      float2 acc[8][4];
+    // ---- dK = scale dS^T Q   (rows: keys, columns: head dim)
+    zero_acc(acc);
+    warp_gemm<kDt, true, true>(acc, sS, sQ, m0, n0);
 #pragma unroll
-      for (int i = 0; i < 8; i++)
+    for (int tm = 0; tm < 2; tm++)
 #pragma unroll
-        for (int j = 0; j < 4; j++) acc[i][j] = make_float2(0.f, 0.f);
-#pragma unroll 2
-      for (int r = 0; r < 128; r++) {
-        float sv[8];
-        float2 qv[4];
-#pragma unroll
-        for (int i = 0; i < 8; i++) sv[i] = sP[r * 128 + ty + 16 * i];
-#pragma unroll
-        for (int j = 0; j < 4; j++) qv[j] = widen2<kDt>(sQ[r * kRowWords + tx + 16 * j]);
-#pragma unroll
-        for (int i = 0; i < 8; i++)
-#pragma unroll
-          for (int j = 0; j < 4; j++) {
-            acc[i][j].x += sv[i] * qv[j].x;
-            acc[i][j].y += sv[i] * qv[j].y;
-          }
-      }
-#pragma unroll
-      for (int i = 0; i < 8; i++) {
-        const int c = ty + 16 * i;
+      for (int h = 0; h < 2; h++) {
+        const int c = m0 + 16 * tm + fr + 8 * h;
         if (!key_ok(c)) continue;
-        float* dst = p.dk + ((grow0 + c) * p.N2 + kvh) * kHeadDim;
+        float2* dst = reinterpret_cast<float2*>(p.dk + ((grow0 + c) * p.N2 + kvh) * kHeadDim);
 #pragma unroll
-        for (int j = 0; j < 4; j++)
-          atomicAdd(reinterpret_cast<float2*>(dst) + tx + 16 * j,
-                    make_float2(acc[i][j].x * p.scale, acc[i][j].y * p.scale));
+        for (int tn = 0; tn < 8; tn++)
+          atomicAdd(dst + ((n0 + 8 * tn + fc) >> 1),
+                    make_float2(acc[tm][tn][2 * h] * p.scale, acc[tm][tn][2 * h + 1] * p.scale));
       }
-    }
   }
 
   // dQ of the tile's stored rows (0 for rows past seqused_q or with no key)
 #pragma unroll
-  for (int i = 0; i < 8; i++) {
-    const int r = ty + 16 * i;
-    if (!row_valid(r)) continue;
-    float* dst = p.dq + row_index(r) * kHeadDim;
+  for (int tm = 0; tm < 2; tm++)
 #pragma unroll
-    for (int j = 0; j < 4; j++)
-      reinterpret_cast<float2*>(dst)[tx + 16 * j] =
-          make_float2(dq[i][2 * j] * p.scale, dq[i][2 * j + 1] * p.scale);
-  }
+    for (int h = 0; h < 2; h++) {
+      const int r = m0 + 16 * tm + fr + 8 * h;
+      if (!row_valid(r)) continue;
+      float2* dst = reinterpret_cast<float2*>(p.dq + row_index(r) * kHeadDim);
+#pragma unroll
+      for (int tn = 0; tn < 8; tn++)
+        dst[(n0 + 8 * tn + fc) >> 1] =
+            make_float2(dq[tm][tn][2 * h] * p.scale, dq[tm][tn][2 * h + 1] * p.scale);
+    }
   if (bad && p.dev_status) atomicOr(p.dev_status, bad);
 }
 

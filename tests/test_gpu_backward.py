@@ -1,15 +1,17 @@
 """Gradients of the attention output on the GPU (gbsa.backward) against the
 fp64 oracle's (oracle.attention_backward, pinned in test_oracle_backward).
 
-Tolerance, from the arithmetic of the CUDA path: the products run in fp32
-from the exact 16-bit inputs, and P = exp(s - lse) uses the forward's fp32
-lse; the delta D = dO . O uses the forward's 16-bit out, whose rounding
-(2^-9 relative for bf16, 2^-11 for fp16) moves every dS by at most
-2^-9 * P * sum_d |dO_d O_d|.  So per element |dq - dq_ref| and
-|dk - dk_ref| stay within 2^-9 of the oracle's sum of absolute terms, plus
-fp32 rounding and the lse error; the test allows 2^-8.  dv has no delta
-term: 2^-12 of its absolute sum.  Keys nobody sees get exactly 0, and so do
-dq rows with no key or past seqused_q."""
+Tolerance, from the arithmetic of the CUDA path: the products take the
+exact 16-bit inputs with fp32 accumulation, and P = exp(s - lse) uses the
+forward's fp32 lse.  Three roundings reach the result: the delta D = dO . O
+uses the forward's 16-bit out (2^-9 relative for bf16, 2^-11 for fp16),
+which moves every dS by at most 2^-9 * P * sum_d |dO_d O_d|; P and dS enter
+the products rounded to the element type (2^-9 of each term); fp32 sums and
+the lse error stay far below.  So per element |dq - dq_ref| and
+|dk - dk_ref| stay within 2^-8 of the oracle's sum of absolute terms, and
+|dv - dv_ref| (no delta term) within 2^-9 of its own; the test allows twice
+that, 2^-7 and 2^-8.  Keys nobody sees get exactly 0, and so do dq rows with
+no key or past seqused_q."""
 import numpy as np
 import pytest
 import torch
@@ -106,9 +108,9 @@ def _run(w, dtype, tnd=False, seed=0):
 
 def _check(got, ref):
     dq_ref, dk_ref, dv_ref, dq_abs, dk_abs, dv_abs = ref
-    for name, g, r, a, rel in (("dq", got[0], dq_ref, dq_abs, 2.0 ** -8),
-                               ("dk", got[1], dk_ref, dk_abs, 2.0 ** -8),
-                               ("dv", got[2], dv_ref, dv_abs, 2.0 ** -12)):
+    for name, g, r, a, rel in (("dq", got[0], dq_ref, dq_abs, 2.0 ** -7),
+                               ("dk", got[1], dk_ref, dk_abs, 2.0 ** -7),
+                               ("dv", got[2], dv_ref, dv_abs, 2.0 ** -8)):
         g = g.double().cpu().numpy()
         assert g.shape == r.shape, name
         assert np.isfinite(g).all(), name
