@@ -66,14 +66,15 @@ def _compact(w, flat):
     return a.reshape(w.num_pages, PAGE, w.N2, w.D)
 
 
-def _run(w, dtype, tnd=False, seed=0):
+def _run(w, dtype, tnd=False, seed=0, ctas=0, forced=0):
     q, kf, vf = make_values(w, "cuda", dtype=dtype)
     t = device_tensors(w)
-    meta = run_metadata(w, t)
+    meta = run_metadata(w, t, ctas, forced)
     g = torch.Generator(device="cuda").manual_seed(1234 + seed)
     dout = torch.randn(q.shape, generator=g, device="cuda", dtype=torch.float32).to(dtype)
     kw = dict(metadata=meta, cu_seqlens_q=t["cu"], seqused_q=t["squ"], seqused_kv=t["sku"],
-              softmax_scale=w.scale, win_left=w.win_left, win_right=w.win_right)
+              softmax_scale=w.scale, win_left=w.win_left, win_right=w.win_right,
+              num_ctas=ctas, max_blocks_per_split=forced)
     if tnd:
         kt, vt, cu_kv = tnd_kv(w, kf, vf, seed=seed)
         kvkw = dict(cu_seqlens_kv=torch.as_tensor(cu_kv, device="cuda"))
@@ -136,6 +137,35 @@ def test_backward_fp16():
 def test_backward_tnd():
     got, ref = _run(_cases()["g5_window"](), torch.bfloat16, tnd=True, seed=2)
     _check(got, ref)
+
+
+def test_backward_with_split_work_list():
+    """A work list built with forced splits and 7 CTAs: the backward reads
+    only its item table and live lists, and takes the same problem (the
+    list's signature covers num_ctas and the split length)."""
+    got, ref = _run(_cases()["g5_window"](), torch.bfloat16, seed=3, ctas=7, forced=2)
+    _check(got, ref)
+
+
+def test_backward_metadata_of_another_problem_is_refused():
+    """A work list built for other CTA settings: the kernel sets the
+    mismatch bit and leaves dq alone."""
+    w = _cases()["tiny"]()
+    q, kf, vf = make_values(w, "cuda")
+    t = device_tensors(w)
+    meta = run_metadata(w, t, 7, 0)
+    kw = dict(cu_seqlens_q=t["cu"], seqused_q=t["squ"], seqused_kv=t["sku"],
+              block_table=t["bt"], softmax_scale=w.scale)
+    out, lse = gbsa.forward(q, pool_view(w, kf), pool_view(w, vf), t["idx"], t["cnt"],
+                            [w.block_x, 128], metadata=meta, num_ctas=7, return_softmax_lse=True,
+                            **kw)
+    dq = torch.full(q.shape, 7.0, dtype=torch.float32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    gbsa.backward(q, q, pool_view(w, kf), pool_view(w, vf), out, lse, t["idx"], t["cnt"],
+                  [w.block_x, 128], metadata=meta, num_ctas=5, dq=dq, dev_status=status, **kw)
+    torch.cuda.synchronize()
+    assert int(status.item()) & 0x10
+    assert bool((dq == 7.0).all())
 
 
 def test_backward_rejects_e4m3():
