@@ -11,7 +11,9 @@ under its bound (R22, as in test_gpu_fp8).  The same keys in the non-paged
 TND layout (NaN rows between the sequences) give bit-identical out and lse,
 and so does a call without the lse output (out).
 softmaxPrecision 1 on the same inputs stays within its R24 bound (as in
-test_gpu_softmax_precision)."""
+test_gpu_softmax_precision).  Every tenth case also runs the backward
+(16-bit types) against the oracle's gradients under the bound of
+test_gpu_backward (R25)."""
 import math
 
 import numpy as np
@@ -156,3 +158,40 @@ def _check_mode1(w, q, kf, vf, out, lse, rows, dtype):
         mean_scale = (2.0 ** -4 * oa if name == "e4m3" else
                       2.0 * ((2.0 ** -9.9 + 8 * math.log(2) * 2.0 ** -11) * oa + 2.0 ** -11 * ga))
         assert err[fin].mean() <= 0.25 * mean_scale[fin].mean()
+
+
+@pytest.mark.parametrize("k", range(0, N_CASES, 10))
+def test_fuzz_backward(k):
+    """The gradients of every tenth random problem (16-bit element types)
+    against the oracle's, under the bound of test_gpu_backward (R25)."""
+    from tests.test_gpu_backward import _check, _compact
+    import oracle
+    from tests.helpers import bf16_bits, elem_dtype
+
+    w, dtype, ctas, forced = fuzz_case(k)
+    if dtype == torch.float8_e4m3fn:
+        dtype = torch.bfloat16
+    t = device_tensors(w)
+    meta = run_metadata(w, t, ctas, forced)
+    q, kf, vf = make_values(w, "cuda", dtype=dtype)
+    g = torch.Generator(device="cuda").manual_seed(9000 + k)
+    dout = torch.randn(q.shape, generator=g, device="cuda", dtype=torch.float32).to(dtype)
+    kw = dict(metadata=meta, cu_seqlens_q=t["cu"], seqused_q=t["squ"], seqused_kv=t["sku"],
+              block_table=t["bt"], softmax_scale=w.scale, win_left=w.win_left,
+              win_right=w.win_right, num_ctas=ctas, max_blocks_per_split=forced)
+    kp, vp = pool_view(w, kf), pool_view(w, vf)
+    out, lse = gbsa.forward(q, kp, vp, t["idx"], t["cnt"], [w.block_x, 128],
+                            return_softmax_lse=True, **kw)
+    dq, dk, dv = gbsa.backward(dout, q, kp, vp, out, lse, t["idx"], t["cnt"], [w.block_x, 128],
+                               **kw)
+    torch.cuda.synchronize()
+    ref = oracle.attention_backward(
+        q_bits=bf16_bits(q), k_bits=bf16_bits(kf), v_bits=bf16_bits(vf), dout_bits=bf16_bits(dout),
+        kv_page_stride=w.kv_page_stride, num_pages=w.num_pages, sparse_idx=w.sparse_idx,
+        sparse_count=w.sparse_count, cu_seqlens_q=w.cu_seqlens_q, seqused_q=w.seqused_q,
+        seqused_kv=w.kv_used, block_table=w.block_table, block_x=w.block_x, scale=w.scale,
+        win_left=w.win_left, win_right=w.win_right, dtype=elem_dtype(q), with_abs=True)
+    ref = [r if i % 3 == 0 else _compact(w, r) for i, r in enumerate(ref)]
+    if np.abs(ref[0]).max() == 0 and np.abs(ref[2]).max() == 0:
+        pytest.skip("no row sees a key")
+    _check((dq, dk, dv), ref)
