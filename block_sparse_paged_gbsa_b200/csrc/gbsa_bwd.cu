@@ -39,6 +39,7 @@ constexpr int kBwdThreads = 256;  // 8 warps, each a 32 x 64 tile of every produ
 // so that the 8 rows an ldmatrix reads start in distinct bank groups
 constexpr int kRowElems = 136;
 constexpr int kTileElems = 128 * kRowElems;
+static_assert(128 * 16 % kBwdThreads == 0, "whole 16-byte chunks per thread");
 constexpr size_t kBwdSmem = 6 * kTileElems * 2  // Q, dO, K, V, P, dS
                             + 3 * 128 * 4;      // per row: lse (log2 units), delta, position
 static_assert(kBwdSmem <= 232448, "shared memory budget");
@@ -88,16 +89,29 @@ __global__ void __launch_bounds__(256) delta_kernel(const BwdParams p) {
   if (lane == 0) p.delta[row] = s;
 }
 
-// 128 rows of 128 16-bit elements from global rows at `src(r)` (nullptr: a
-// row of zeros) into a padded shared tile (row stride kRowElems).  Whole CTA.
-template <typename F>
-__device__ __forceinline__ void load_tile(uint16_t* tile, F src) {
-  for (int i = threadIdx.x; i < 128 * 16; i += kBwdThreads) {
+// Two tiles of 128 rows x 128 16-bit elements from global rows at `src0(r)`
+// and `src1(r)` (nullptr: a row of zeros) into padded shared tiles (row
+// stride kRowElems).  Whole CTA; every thread issues all 16 of its loads
+// before its first store, so their latencies overlap.
+constexpr int kChunksPerThread = 128 * 16 / kBwdThreads;  // 16-byte chunks of a tile
+template <typename F0, typename F1>
+__device__ __forceinline__ void load_tiles(uint16_t* t0, uint16_t* t1, F0 src0, F1 src1) {
+  uint4 v0[kChunksPerThread], v1[kChunksPerThread];
+#pragma unroll
+  for (int it = 0; it < kChunksPerThread; it++) {
+    const int i = threadIdx.x + it * kBwdThreads;
     const int r = i >> 4, c = i & 15;  // row, 16-byte chunk
-    const uint16_t* s = src(r);
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (s) v = reinterpret_cast<const uint4*>(s)[c];
-    *reinterpret_cast<uint4*>(tile + r * kRowElems + 8 * c) = v;
+    const uint16_t* a = src0(r);
+    const uint16_t* b = src1(r);
+    v0[it] = a ? reinterpret_cast<const uint4*>(a)[c] : make_uint4(0, 0, 0, 0);
+    v1[it] = b ? reinterpret_cast<const uint4*>(b)[c] : make_uint4(0, 0, 0, 0);
+  }
+#pragma unroll
+  for (int it = 0; it < kChunksPerThread; it++) {
+    const int i = threadIdx.x + it * kBwdThreads;
+    const int r = i >> 4, c = i & 15;
+    *reinterpret_cast<uint4*>(t0 + r * kRowElems + 8 * c) = v0[it];
+    *reinterpret_cast<uint4*>(t1 + r * kRowElems + 8 * c) = v1[it];
   }
 }
 
@@ -225,8 +239,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kernel(const BwdParams p) 
   auto row_index = [&](int r) {  // (token, head) row of q / dq
     return ((int64_t)(tok_begin + row_tok(r)) * p.N1 + kvh * p.G + r % p.G);
   };
-  load_tile(sQ, [&](int r) { return row_used(r) ? p.q + row_index(r) * kHeadDim : nullptr; });
-  load_tile(sG, [&](int r) { return row_used(r) ? p.dout + row_index(r) * kHeadDim : nullptr; });
+  load_tiles(sQ, sG, [&](int r) { return row_used(r) ? p.q + row_index(r) * kHeadDim : nullptr; },
+             [&](int r) { return row_used(r) ? p.dout + row_index(r) * kHeadDim : nullptr; });
   if (threadIdx.x < 128) {
     const int r = threadIdx.x;
     const bool used = row_used(r);
@@ -269,12 +283,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kernel(const BwdParams p) 
       return key < ku && (!tnd || row0 + c < p.T_kv);
     };
     __syncthreads();  // the previous block's tiles are no longer read
-    load_tile(sK, [&](int c) {
-      return key_ok(c) ? p.k + ((row0 + c) * p.N2 + kvh) * kHeadDim : nullptr;
-    });
-    load_tile(sV, [&](int c) {
-      return key_ok(c) ? p.v + ((row0 + c) * p.N2 + kvh) * kHeadDim : nullptr;
-    });
+    load_tiles(sK, sV,
+               [&](int c) { return key_ok(c) ? p.k + ((row0 + c) * p.N2 + kvh) * kHeadDim : nullptr; },
+               [&](int c) { return key_ok(c) ? p.v + ((row0 + c) * p.N2 + kvh) * kHeadDim : nullptr; });
     __syncthreads();
 
     float acc[2][8][4];
