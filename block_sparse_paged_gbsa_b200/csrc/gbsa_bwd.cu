@@ -115,6 +115,17 @@ __device__ __forceinline__ void load_tiles(uint16_t* t0, uint16_t* t1, F0 src0, 
   }
 }
 
+// 16 bytes global -> shared without registers (zero-filled past src_bytes)
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const uint16_t* p) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
@@ -262,30 +273,62 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kernel(const BwdParams p) 
   const int32_t* list = meta + off_list + (int64_t)item * p.top_k;
   const bool tnd = p.cu_kv != nullptr;
   int32_t bad = 0;
-  for (int32_t e = 0; e < n_live; e++) {
-    const int32_t lb = list[e] & kEntryLbMask;
-    // first row of the block in k / v (rows of N2 * D elements; a page is
-    // kv_page_stride elements) and in the compact dk / dv
+  // block e of the list: its first row in k / v (rows of N2 * D elements; a
+  // page is kv_page_stride elements) and in the compact dk / dv; ok = false
+  // for a page index out of range (the block then gets no weight)
+  struct Blk {
+    int32_t lb;
     int64_t row0, grow0;
+    bool ok;
+  };
+  const int64_t page_rows = tnd ? 0 : p.kv_page_stride / ((int64_t)p.N2 * kHeadDim);
+  auto block_of = [&](int32_t e) {
+    Blk x;
+    x.lb = list[e] & kEntryLbMask;
+    x.ok = true;
     if (tnd) {
-      row0 = grow0 = p.cu_kv[b] + (int64_t)lb * kPage;
+      x.row0 = x.grow0 = p.cu_kv[b] + (int64_t)x.lb * kPage;
     } else {
-      const int32_t page = lb < p.max_pages ? p.block_table[(int64_t)b * p.max_pages + lb] : -1;
-      if (page < 0 || page >= p.num_pages) {  // uniform over the CTA
-        bad |= kDevBadPage;
-        continue;
-      }
-      row0 = (int64_t)page * (p.kv_page_stride / ((int64_t)p.N2 * kHeadDim));
-      grow0 = (int64_t)page * kPage;
+      const int32_t page =
+          x.lb < p.max_pages ? p.block_table[(int64_t)b * p.max_pages + x.lb] : -1;
+      x.ok = page >= 0 && page < p.num_pages;
+      x.row0 = x.ok ? (int64_t)page * page_rows : 0;
+      x.grow0 = x.ok ? (int64_t)page * kPage : 0;
     }
-    auto key_ok = [&](int c) {
-      const int64_t key = (int64_t)lb * kPage + c;
-      return key < ku && (!tnd || row0 + c < p.T_kv);
-    };
-    __syncthreads();  // the previous block's tiles are no longer read
-    load_tiles(sK, sV,
-               [&](int c) { return key_ok(c) ? p.k + ((row0 + c) * p.N2 + kvh) * kHeadDim : nullptr; },
-               [&](int c) { return key_ok(c) ? p.v + ((row0 + c) * p.N2 + kvh) * kHeadDim : nullptr; });
+    return x;
+  };
+  auto key_ok = [&](const Blk& x, int c) {
+    const int64_t key = (int64_t)x.lb * kPage + c;
+    return x.ok && key < ku && (!tnd || x.row0 + c < p.T_kv);
+  };
+  // asynchronous copy of block x's K or V tile (rows past seqused_kv, and a
+  // block with no weight, are zero-filled)
+  auto fetch = [&](uint16_t* tile, const uint16_t* src, const Blk& x) {
+#pragma unroll
+    for (int it = 0; it < kChunksPerThread; it++) {
+      const int i = threadIdx.x + it * kBwdThreads;
+      const int r = i >> 4, c = i & 15;
+      const bool ok = key_ok(x, r);
+      cp_async16(tile + r * kRowElems + 8 * c,
+                 ok ? src + ((x.row0 + r) * p.N2 + kvh) * kHeadDim + 8 * c : src, ok ? 16u : 0u);
+    }
+  };
+  if (n_live > 0) {
+    const Blk x0 = block_of(0);
+    fetch(sK, p.k, x0);
+    fetch(sV, p.v, x0);
+    cp_async_commit();
+  }
+  for (int32_t e = 0; e < n_live; e++) {
+    // K and V of block e were fetched during block e - 1 (or above); the
+    // next block's are fetched as soon as each tile is free: V after dP,
+    // K after dQ
+    const Blk x = block_of(e);
+    if (!x.ok) bad |= kDevBadPage;
+    const int32_t lb = x.lb;
+    const bool has_next = e + 1 < n_live;
+    const Blk xn = block_of(has_next ? e + 1 : e);
+    cp_async_wait_all();
     __syncthreads();
 
     float acc[2][8][4];
@@ -306,7 +349,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kernel(const BwdParams p) 
 #pragma unroll
           for (int u = 0; u < 2; u++) {
             const int32_t key = lb * kPage + c + u;
-            const bool vis = l2 != -INFINITY && key < ku && key <= pos &&
+            const bool vis = x.ok && l2 != -INFINITY && key < ku && key <= pos &&
                              (p.win_left < 0 || key >= pos - p.win_left);
             pv[u] = vis ? fast_exp2(acc[tm][tn][2 * h + u] * p.scale_log2 - l2) : 0.f;
           }
@@ -323,8 +366,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kernel(const BwdParams p) 
 #pragma unroll
       for (int h = 0; h < 2; h++) {
         const int c = m0 + 16 * tm + fr + 8 * h;
-        if (!key_ok(c)) continue;
-        float2* dst = reinterpret_cast<float2*>(p.dv + ((grow0 + c) * p.N2 + kvh) * kHeadDim);
+        if (!key_ok(x, c)) continue;
+        float2* dst = reinterpret_cast<float2*>(p.dv + ((x.grow0 + c) * p.N2 + kvh) * kHeadDim);
 #pragma unroll
         for (int tn = 0; tn < 8; tn++)
           atomicAdd(dst + ((n0 + 8 * tn + fc) >> 1),
@@ -348,10 +391,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kernel(const BwdParams p) 
               pack2<kDt>(pv.x * (acc[tm][tn][2 * h] - dlt), pv.y * (acc[tm][tn][2 * h + 1] - dlt));
         }
       }
-    __syncthreads();
+    __syncthreads();  // dS is complete and V no longer read
+    if (has_next) {
+      fetch(sV, p.v, xn);
+      cp_async_commit();
+    }
 
     // ---- dQ += dS K   (rows: queries, columns: head dim)
     warp_gemm<kDt, false, true>(dq, sS, sK, m0, n0);
+    __syncthreads();  // K no longer read
+    if (has_next) {
+      fetch(sK, p.k, xn);
+      cp_async_commit();
+    }
 
     // ---- dK = scale dS^T Q   (rows: keys, columns: head dim)
     zero_acc(acc);
@@ -361,8 +413,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_kernel(const BwdParams p) 
 #pragma unroll
       for (int h = 0; h < 2; h++) {
         const int c = m0 + 16 * tm + fr + 8 * h;
-        if (!key_ok(c)) continue;
-        float2* dst = reinterpret_cast<float2*>(p.dk + ((grow0 + c) * p.N2 + kvh) * kHeadDim);
+        if (!key_ok(x, c)) continue;
+        float2* dst = reinterpret_cast<float2*>(p.dk + ((x.grow0 + c) * p.N2 + kvh) * kHeadDim);
 #pragma unroll
         for (int tn = 0; tn < 8; tn++)
           atomicAdd(dst + ((n0 + 8 * tn + fc) >> 1),
