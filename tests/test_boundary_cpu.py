@@ -146,6 +146,32 @@ def test_forward_pointer_rules(lib):
     assert _call_forward(lib, p, _fake_tensors(), ws_bytes=0) == 5        # workspace too small
 
 
+def _call_backward(lib, p, tensors, dout=11 << 20, meta=16, dq=12 << 20, dk=13 << 20,
+                   dv=14 << 20, ws=16, ws_bytes=1 << 30):
+    return lib.gbsa_backward(ctypes.byref(p.as_c()), ctypes.byref(tensors), dout, meta, dq, dk, dv,
+                             ws, ws_bytes, None, None)
+
+
+def test_backward_host_rules(lib):
+    """gbsa_backward checks its arguments before any launch (these cases never
+    reach the device)."""
+    p, w = _problem()
+    s = lambda rc: lib.gbsa_status_string(rc).decode()
+    assert s(_call_backward(lib, p, _fake_tensors(), dout=None)) == "GBSA_ERR_INVALID_ARG"
+    assert s(_call_backward(lib, p, _fake_tensors(), dk=None)) == "GBSA_ERR_INVALID_ARG"
+    # lse is an input here, whatever return_lse says
+    assert s(_call_backward(lib, _problem(return_lse=0)[0], _fake_tensors(lse=None))) == \
+        "GBSA_ERR_INVALID_ARG"
+    assert s(_call_backward(lib, p, _fake_tensors(), dq=(12 << 20) + 8)) == "GBSA_ERR_ALIGNMENT"
+    assert s(_call_backward(lib, p, _fake_tensors(), dout=(11 << 20) + 2)) == "GBSA_ERR_ALIGNMENT"
+    assert s(_call_backward(lib, p, _fake_tensors(), ws_bytes=16)) == "GBSA_ERR_WORKSPACE_TOO_SMALL"
+    p8, _ = _problem(dtype=2, q_scale=1.0, k_scale=1.0, v_scale=1.0)
+    assert s(_call_backward(lib, p8, _fake_tensors())) == "GBSA_ERR_UNSUPPORTED"
+    n = ctypes.c_size_t(0)
+    assert lib.gbsa_backward_workspace_size(ctypes.byref(p.as_c()), ctypes.byref(n)) == 0
+    assert n.value == (w.T * w.N1 * 4 + 15) // 16 * 16
+
+
 def test_no_device_means_no_default_cta_count(lib):
     import torch
     if torch.cuda.is_available():

@@ -10,6 +10,9 @@ It is pinned here against quantities that do not use that formula:
   dout); the weights of a row sum to 1 (the dv of all keys sums to the dout
   of the rows that see a key) and the score gradients of a row sum to 0 (the
   dk of all keys sums to 0).
+
+Five planted mistakes in the gradient code (test_mutant_is_caught) each
+fail at least one of these pins.
 """
 import numpy as np
 import pytest
@@ -34,14 +37,14 @@ def _problem(seed, window=False, D=8, N1=4, N2=2):
     return w
 
 
-def _kw(w, D, dtype="fp16"):
+def _kw(w, D, dtype="fp16", lib=None):
     npages = w.num_pages
     stride = PAGE * w.N2 * D
     return dict(kv_page_stride=stride, num_pages=npages, sparse_idx=w.sparse_idx,
                 sparse_count=w.sparse_count, cu_seqlens_q=w.cu_seqlens_q,
                 seqused_q=w.q_used if w.has_seqused_q else None, seqused_kv=w.kv_used,
                 block_table=w.block_table, block_x=w.block_x, scale=D ** -0.5,
-                win_left=w.win_left, win_right=w.win_right, dtype=dtype)
+                win_left=w.win_left, win_right=w.win_right, dtype=dtype, lib=lib)
 
 
 def _bits(x):
@@ -66,10 +69,10 @@ def _values(w, D, seed):
 
 
 @pytest.mark.parametrize("window", [False, True])
-def test_gradients_match_finite_differences(window):
+def test_gradients_match_finite_differences(window, lib=None):
     D = 8
     w = _problem(11 + window, window, D)
-    kw = _kw(w, D)
+    kw = _kw(w, D, lib=lib)
     q, k, v, g = _values(w, D, 3)
     dq, dk, dv = oracle.attention_backward(q_bits=_bits(q), k_bits=_bits(k), v_bits=_bits(v),
                                            dout_bits=_bits(g), **kw)
@@ -104,10 +107,10 @@ def test_gradients_match_finite_differences(window):
     assert checked >= 60
 
 
-def test_constant_values_give_no_query_or_key_gradient():
+def test_constant_values_give_no_query_or_key_gradient(lib=None):
     D = 8
     w = _problem(21, True, D)
-    kw = _kw(w, D)
+    kw = _kw(w, D, lib=lib)
     q, k, v, g = _values(w, D, 4)
     c = _grid_values(np.random.default_rng(9), (w.N2, D))
     v = np.broadcast_to(c, (v.size // (w.N2 * D), w.N2, D)).reshape(-1).copy()  # one vector per head
@@ -117,13 +120,13 @@ def test_constant_values_give_no_query_or_key_gradient():
     assert np.abs(dv).max() > 1e-3  # v still gets a gradient
 
 
-def test_single_key_rows():
+def test_single_key_rows(lib=None):
     """block_x = 1, one-token rows at position 0 of their sequences: each
     row sees exactly key 0, with weight 1."""
     D = 8
     w = generate(name="one", seed=31, q_storage=[1, 1, 1], q_used=[1, 1, 1], kv_used=[1, 1, 1],
                  N1=4, N2=2, block_x=1, top_k=2, selection="all_causal")
-    kw = _kw(w, D)
+    kw = _kw(w, D, lib=lib)
     q, k, v, g = _values(w, D, 6)
     dq, dk, dv = oracle.attention_backward(q_bits=_bits(q), k_bits=_bits(k), v_bits=_bits(v),
                                            dout_bits=_bits(g), **kw)
@@ -137,12 +140,12 @@ def test_single_key_rows():
             assert np.array_equal(dv4[page, 0, kvh], expect)
 
 
-def test_row_sums():
+def test_row_sums(lib=None):
     """sum over keys of dv = sum of dout over rows that see a key; sum over
     keys of dk = 0 (the score gradients of each row sum to zero)."""
     D = 8
     w = _problem(41, True, D)
-    kw = _kw(w, D)
+    kw = _kw(w, D, lib=lib)
     q, k, v, g = _values(w, D, 8)
     dq, dk, dv = oracle.attention_backward(q_bits=_bits(q), k_bits=_bits(k), v_bits=_bits(v),
                                            dout_bits=_bits(g), **kw)
@@ -157,3 +160,36 @@ def test_row_sums():
         assert np.allclose(dv_h[kvh], expect, rtol=0, atol=1e-12)
         assert np.abs(dk_h[kvh]).max() <= 1e-12
     assert sees.any() and (~sees).any()
+
+
+# Planted mistakes in the oracle's gradient code: every one must fail a pin.
+MUTANTS = {
+    "delta_dropped": ("const double ds = w * (gv - dlt);", "const double ds = w * gv;"),
+    "dk_unscaled": ("dk[base + d] += scale * ds * c.widen(qrow[d]);",
+                    "dk[base + d] += ds * c.widen(qrow[d]);"),
+    "dv_unweighted": ("dv[base + d] += w * g;", "dv[base + d] += g;"),
+    "dq_from_v": ("dqr[d] += scale * ds * c.widen(krow[d]);",
+                  "dqr[d] += scale * ds * c.widen(vrow[d]);"),
+    "weight_without_lse": ("const double w = exp(score[i] - lse);", "const double w = exp(score[i]);"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(oracle._SRC).read()
+    assert src.count(old) == 1, f"mutation anchor for {name} not found exactly once"
+    path = tmp_path / f"{name}.c"
+    path.write_text(src.replace(old, new))
+    lib = oracle.load_library(oracle.compile_to(str(path), str(tmp_path / f"{name}.so")))
+    pins = (lambda: test_gradients_match_finite_differences(True, lib=lib),
+            lambda: test_constant_values_give_no_query_or_key_gradient(lib=lib),
+            lambda: test_single_key_rows(lib=lib), lambda: test_row_sums(lib=lib))
+    caught = 0
+    for pin in pins:
+        try:
+            pin()
+        except AssertionError:
+            caught += 1
+    assert caught > 0, f"{name} passes every pin"
+
