@@ -352,7 +352,9 @@ int gbsa_oracle_attention_rows(int32_t B, int32_t T, int32_t N1, int32_t N2, int
  * are accumulated over every row and list entry that reads a key (a block
  * listed twice counts twice, as in the forward).  The *_abs outputs
  * (optional) get the same sums with every term replaced by its absolute
- * value: the scale of the rounding error of any evaluation order.
+ * value, the term g.O of ds by sum_d |g[d]| sum_p w_p |v_p[d]|: the scale of
+ * the rounding error of any evaluation order that forms the delta from a
+ * computed O.
  * Single-threaded.  Returns 0 on success.
  */
 int gbsa_oracle_attention_backward(int32_t B, int32_t T, int32_t N1, int32_t N2, int32_t D,
@@ -394,21 +396,24 @@ int gbsa_oracle_attention_backward(int32_t B, int32_t T, int32_t N1, int32_t N2,
   int64_t* key_page = (int64_t*)malloc(sizeof(int64_t) * (size_t)cap);
   int32_t* key_row = (int32_t*)malloc(sizeof(int32_t) * (size_t)cap);
   double* out = (double*)malloc(sizeof(double) * (size_t)D);
-  int rc = (!score || !key_page || !key_row || !out) ? 11 : 0;
+  double* oabs = (double*)malloc(sizeof(double) * (size_t)D);
+  int rc = (!score || !key_page || !key_row || !out || !oabs) ? 11 : 0;
   for (int64_t tg = 0; tg < T && !rc; tg++) {
     for (int32_t h = 0; h < N1 && !rc; h++) {
       double lse;
       int64_t nk = 0;
       int32_t kvh = 0;
       /* the visible keys of (tg, h) (pages, rows, scores), its KV head and O */
-      rc = one_row(&c, tg, h, out, &lse, NULL, NULL, score, key_page, key_row, &nk, &kvh);
+      rc = one_row(&c, tg, h, out, &lse, oabs, NULL, score, key_page, key_row, &nk, &kvh);
       if (rc || lse == -INFINITY) continue;
       const uint16_t* qrow = q + (tg * N1 + h) * (int64_t)D;
       const uint16_t* grow = dout + (tg * N1 + h) * (int64_t)D;
+      /* dlt_abs scales the error of a delta formed from a computed O: every
+         O[d] errs in proportion to sum_p w_p |v_p[d]| (oabs), not to |O[d]| */
       double dlt = 0.0, dlt_abs = 0.0;
       for (int32_t d = 0; d < D; d++) {
         dlt += c.widen(grow[d]) * out[d];
-        dlt_abs += fabs(c.widen(grow[d]) * out[d]);
+        dlt_abs += fabs(c.widen(grow[d])) * oabs[d];
       }
       double* dqr = dq + (tg * N1 + h) * (int64_t)D;
       double* dqa = dq_abs ? dq_abs + (tg * N1 + h) * (int64_t)D : NULL;
@@ -436,7 +441,7 @@ int gbsa_oracle_attention_backward(int32_t B, int32_t T, int32_t N1, int32_t N2,
       }
     }
   }
-  free(score); free(key_page); free(key_row); free(out);
+  free(score); free(key_page); free(key_row); free(out); free(oabs);
   free(c.q_block_base);
   return rc;
 }
