@@ -3,17 +3,18 @@ fp64 oracle's (oracle.attention_backward, pinned in test_oracle_backward).
 
 Tolerance, from the arithmetic of the CUDA path: the products take the
 exact 16-bit inputs with fp32 accumulation, and P = exp(s - lse) uses the
-forward's fp32 lse.  Two roundings reach the result.  The delta D = dO . O
-uses the forward's computed out, which errs per element by at most
-2^-8 sum_p w_p |v_p| (its own 16-bit weights, then its 16-bit output), so D
-errs by at most 2^-8 A with A = sum_d |dO_d| sum_p w_p |v_p[d]|; and P and
-dS enter the products rounded to the element type (2^-9 of each term).
-Every dS then errs by at most 2^-8 P A + 2^-9 |dS| <= 1.5 * 2^-8 of the
-oracle's absolute-term sum for it, P (|dO| . |V| + A); fp32 sums and the lse
-error stay far below.  So |dq - dq_ref| and |dk - dk_ref| stay within
-1.5 * 2^-8 of the oracle's absolute-term sums, and |dv - dv_ref| (no delta
-term) within 2^-9; the test allows 2^-7 and 2^-8.  Keys nobody sees get
-exactly 0, and so do dq rows with no key or past seqused_q."""
+forward's fp32 lse.  Rounding to the element type errs by at most u = 2^-8
+relative for bf16 (8 significant bits) and 2^-11 for fp16.  The delta
+D = dO . O uses the forward's computed out, which errs per element by at
+most 2u sum_p w_p |v_p| (its own 16-bit weights, then its 16-bit output), so
+D errs by at most 2u A with A = sum_d |dO_d| sum_p w_p |v_p[d]|; P and dS
+enter the products rounded (u of each term).  Every dS then errs by at most
+2u P A + u |dS| <= 3u of the oracle's absolute-term sum for it,
+P (|dO| . |V| + A); fp32 sums and the lse error stay far below.  So
+|dq - dq_ref| and |dk - dk_ref| stay within 3u = 1.5 * 2^-7 of the oracle's
+absolute-term sums and |dv - dv_ref| (no delta term) within u = 2^-8; the
+test allows 2^-6 and 2^-7.  Keys nobody sees get exactly 0, and so do dq
+rows with no key or past seqused_q."""
 import numpy as np
 import pytest
 import torch
@@ -111,9 +112,9 @@ def _run(w, dtype, tnd=False, seed=0, ctas=0, forced=0):
 
 def _check(got, ref):
     dq_ref, dk_ref, dv_ref, dq_abs, dk_abs, dv_abs = ref
-    for name, g, r, a, rel in (("dq", got[0], dq_ref, dq_abs, 2.0 ** -7),
-                               ("dk", got[1], dk_ref, dk_abs, 2.0 ** -7),
-                               ("dv", got[2], dv_ref, dv_abs, 2.0 ** -8)):
+    for name, g, r, a, rel in (("dq", got[0], dq_ref, dq_abs, 2.0 ** -6),
+                               ("dk", got[1], dk_ref, dk_abs, 2.0 ** -6),
+                               ("dv", got[2], dv_ref, dv_abs, 2.0 ** -7)):
         g = g.double().cpu().numpy()
         assert g.shape == r.shape, name
         assert np.isfinite(g).all(), name
