@@ -248,9 +248,12 @@ def r24_bound(dtype, ref, out_abs, gap_abs, n_keys, vmax):
     to bf16, E4M3 the R22 bound of the weights' E4M3 cast."""
     d0 = 2.0 ** -9.9 + 8.0 * math.log(2.0) * 2.0 ** -11
     b = 2.0 * (1.0 + 2.0 ** -8) * (d0 * out_abs + 2.0 ** -11 * gap_abs)
-    b = b + 2.0 * n_keys[:, None] * 2.0 ** -24 * vmax + 2.0 ** -9 * np.abs(ref) + 1e-5 * out_abs
+    # the 16-bit output: u |exact|, u = 2^-8 for a bf16 out (8 significant
+    # bits; E4M3 inputs give a bf16 out too), 2^-11 for fp16 (kept at 2^-9)
+    u_out = 2.0 ** -9 if dtype == "fp16" else 2.0 ** -8
+    b = b + 2.0 * n_keys[:, None] * 2.0 ** -24 * vmax + u_out * np.abs(ref) + 1e-5 * out_abs
     if dtype == "bf16":
-        b = b + 2.0 ** -9 * out_abs
+        b = b + 2.0 ** -8 * out_abs  # P rounded to bf16 for the product
     if dtype == "e4m3":
         # the weights' E4M3 cast (R22): 2^-4 relative, 2^-10 below 2^-6
         b = b + 2.0 ** -4 * out_abs + 2.0 ** -18 * n_keys[:, None] * vmax

@@ -19,9 +19,11 @@ Tolerance (reading R24), per element, with S_p the natural-log scores:
   oracle;
 * weights below the f16 range (2^-24) are lost: at most n 2^-24 |v|max over
   the n visible keys;
-* bf16: P rounded to bf16 in the product only, 2^-9 out_abs; E4M3: the R22
+* bf16: P rounded to bf16 in the product only, 2^-8 out_abs (bf16 keeps 8
+  significant bits: u = 2^-8); E4M3: the R22
   bound of the weights' E4M3 cast on top;
-* the 16-bit output: 2^-9 |exact|; fp32 accumulation: 1e-5 out_abs.
+* the 16-bit output: u |exact| (2^-8 for a bf16 out, E4M3 included; fp16,
+  u = 2^-11, keeps 2^-9); fp32 accumulation: 1e-5 out_abs.
 The rounding errors have no common sign, so the mean error must also stay a
 small part of the mean bound (a systematic mistake would not)."""
 import math
