@@ -132,7 +132,7 @@ def _check_e4m3(w, q, kf, vf, out, lse, rows):
     fin = np.isfinite(rl)
     assert (o[~fin] == 0).all()
     vmax = float(vf.float().nan_to_num(0.0).abs().max()) * abs(FP8_SCALES[2])
-    bound = (2.0 ** -4 + 1e-5) * ra + 2.0 ** -9 * np.abs(ro) + 2.0 ** -18 * w.top_k * PAGE * vmax
+    bound = (2.0 ** -4 + 1e-5) * ra + 2.0 ** -8 * np.abs(ro) + 2.0 ** -18 * w.top_k * PAGE * vmax
     err = np.abs(o - ro)
     assert (err <= bound).all(), f"max excess {np.max(err - bound):.3g}"
     if fin.sum() >= 100:

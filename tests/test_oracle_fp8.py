@@ -143,7 +143,7 @@ def _emulate_e4m3_p(w, q8, k8, v8, scales, rows, threshold=0.5):
 
 def _r22_check(w, ro, ra, got, fin, vmax):
     n_vis = w.top_k * 128
-    bound = (2.0 ** -4 + 1e-5) * ra + 2.0 ** -9 * np.abs(ro) + 2.0 ** -18 * n_vis * vmax
+    bound = (2.0 ** -4 + 1e-5) * ra + 2.0 ** -8 * np.abs(ro) + 2.0 ** -18 * n_vis * vmax
     err = np.abs(got - ro)
     return bool((err <= bound).all()), float(err[fin].mean()), float((2.0 ** -4 * ra[fin]).mean())
 
