@@ -193,3 +193,42 @@ def test_mutant_is_caught(name, tmp_path):
             caught += 1
     assert caught > 0, f"{name} passes every pin"
 
+
+
+def test_tnd_layout_gives_the_paged_gradients():
+    """The same logical keys in the TND layout (with NaN rows between the
+    sequences) and in the paged pool give the same dq, and the same dk / dv
+    at every (sequence, position, head)."""
+    import torch
+
+    from block_sparse_paged_gbsa_b200.workloads import make_values, pool_view, tnd_kv
+    from tests.helpers import bf16_bits
+
+    w = generate(name="bwdtnd", seed=51, q_storage=[40, 70], q_used=[40, 66], kv_used=[300, 150],
+                 N1=4, N2=2, block_x=16, top_k=3, selection="random_causal", win_left=100,
+                 win_right=0, page_stride_factor=1.5, list_order="shuffled")
+    q, kf, vf = make_values(w, "cpu", dtype=torch.float16)
+    g = torch.randn(q.shape, generator=torch.Generator().manual_seed(3)).to(torch.float16)
+    kt, vt, cu_kv = tnd_kv(w, kf, vf, seed=1)
+    common = dict(q_bits=bf16_bits(q), dout_bits=bf16_bits(g), sparse_idx=w.sparse_idx,
+                  sparse_count=w.sparse_count, cu_seqlens_q=w.cu_seqlens_q,
+                  seqused_q=w.seqused_q, seqused_kv=w.kv_used, block_x=w.block_x, scale=w.scale,
+                  win_left=w.win_left, win_right=w.win_right, dtype="fp16")
+    pq, pk, pv = oracle.attention_backward(k_bits=bf16_bits(kf), v_bits=bf16_bits(vf),
+                                           kv_page_stride=w.kv_page_stride,
+                                           num_pages=w.num_pages, block_table=w.block_table,
+                                           **common)
+    tq, tk, tv = oracle.attention_backward(k_bits=bf16_bits(kt), v_bits=bf16_bits(vt),
+                                           kv_page_stride=0, num_pages=0, block_table=None,
+                                           cu_seqlens_kv=cu_kv, **common)
+    assert np.array_equal(pq, tq) and np.abs(pq).max() > 0
+    D = w.D
+    for b in range(w.B):
+        for pos in range(int(w.kv_used[b])):
+            page, r = int(w.block_table[b, pos // PAGE]), pos % PAGE
+            for h in range(w.N2):
+                po = page * w.kv_page_stride + (r * w.N2 + h) * D
+                to = ((int(cu_kv[b]) + pos) * w.N2 + h) * D
+                assert np.array_equal(pk[po:po + D], tk[to:to + D])
+                assert np.array_equal(pv[po:po + D], tv[to:to + D])
+    assert np.abs(tk).max() > 0
